@@ -1,0 +1,93 @@
+"""Dense brute-force entropic OT on a materialised cost matrix (tiny inputs only).
+
+TEST INFRASTRUCTURE ONLY.  An implementation independent of ``oracle.core``
+(numpy broadcasting and ``scipy.special.logsumexp`` instead of streamed C),
+used to pin it.  Also holds the textbook kernel-domain (scaling) form of
+Sinkhorn's algorithm, which reaches the same potentials without any
+log-sum-exp, and the closed-form solution of the 2x2 problem.
+"""
+from __future__ import annotations
+
+import numpy as np
+from scipy.special import logsumexp
+
+
+def cost_matrix(X, Y):
+    """C_ij = |x_i - y_j|^2 from the differences (broadcast, n*m*d doubles)."""
+    diff = np.asarray(X, dtype=np.float64)[:, None, :] - np.asarray(Y, dtype=np.float64)[None, :, :]
+    return np.einsum("ijk,ijk->ij", diff, diff)
+
+
+def update_f(C, logb, g, eps):
+    return -eps * logsumexp((g[None, :] - C) / eps + logb[None, :], axis=1)
+
+
+def update_g(C, loga, f, eps):
+    return -eps * logsumexp((f[:, None] - C) / eps + loga[:, None], axis=0)
+
+
+def solve(C, loga, logb, eps, iters, g0=None):
+    g = np.zeros(C.shape[1]) if g0 is None else np.array(g0, dtype=np.float64)
+    f = np.zeros(C.shape[0])
+    for _ in range(iters):
+        f = update_f(C, logb, g, eps)
+        g = update_g(C, loga, f, eps)
+    return f, g
+
+
+def plan(C, loga, logb, f, g, eps):
+    """P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps)."""
+    return np.exp(loga[:, None] + logb[None, :] + (f[:, None] + g[None, :] - C) / eps)
+
+
+def costs(C, loga, logb, f, g, eps):
+    P = plan(C, loga, logb, f, g, eps)
+    a, b = np.exp(loga), np.exp(logb)
+    sum_p = P.sum()
+    ab = a[:, None] * b[None, :]
+    kl = float(np.sum(P * np.log(P / ab)) - sum_p + 1.0)
+    primal = float(np.sum(P * C))
+    return dict(dual=float(a @ f + b @ g - eps * (sum_p - 1.0)), primal=primal,
+                entropic_primal=primal + eps * kl, sum_p=float(sum_p))
+
+
+def scaling_sinkhorn(C, a, b, eps, iters):
+    """Textbook matrix-scaling Sinkhorn (Cuturi 2013): K = exp(-C/eps),
+    u <- a / (K v), v <- b / (K^T u), starting from v = b.
+
+    The plan is diag(u) K diag(v); in the potentials' parametrisation
+    P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps) this is f = eps log(u/a),
+    g = eps log(v/b).  Only usable where exp(-C/eps) does not underflow.
+    """
+    K = np.exp(-C / eps)
+    v = np.array(b, dtype=np.float64)
+    u = np.ones_like(a)
+    for _ in range(iters):
+        u = a / (K @ v)
+        v = b / (K.T @ u)
+    return eps * np.log(u / a), eps * np.log(v / b)
+
+
+def two_by_two_plan(C, a1, b1, eps):
+    """Exact entropic-OT plan for n = m = 2.
+
+    With both marginals fixed, the plan has one free entry p = P_11:
+    P = [[p, a1-p], [b1-p, 1-a1-b1+p]].  Optimality of the entropic problem
+    (P = diag(u) K diag(v)) forces the cross ratio
+    P_11 P_22 / (P_12 P_21) = K_11 K_22 / (K_12 K_21) = kappa, a quadratic in p
+    whose root inside the feasible interval is the unique optimum.
+    """
+    kappa = np.exp(-(C[0, 0] + C[1, 1] - C[0, 1] - C[1, 0]) / eps)
+    A = 1.0 - kappa
+    B = 1.0 - a1 - b1 + kappa * (a1 + b1)
+    Cc = -kappa * a1 * b1
+    lo, hi = max(0.0, a1 + b1 - 1.0), min(a1, b1)
+    if abs(A) < 1e-300:
+        roots = [-Cc / B]
+    else:
+        disc = np.sqrt(B * B - 4 * A * Cc)
+        roots = [(-B + disc) / (2 * A), (-B - disc) / (2 * A)]
+    p = [r for r in roots if lo - 1e-15 <= r <= hi + 1e-15]
+    assert len(p) >= 1, (roots, lo, hi)
+    p = p[0]
+    return np.array([[p, a1 - p], [b1 - p, 1.0 - a1 - b1 + p]])
