@@ -1,0 +1,179 @@
+/*
+ * flashsinkhorn.h -- C ABI of the B200 (sm_100a) log-domain Sinkhorn library.
+ *
+ * The operation is the stabilised log-domain Sinkhorn iteration for entropic
+ * optimal transport with squared-Euclidean cost, written in attention form
+ * ("FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 1, Proposition 1):
+ *
+ *   C_ij = |x_i|^2 + |y_j|^2 - 2 x_i.y_j
+ *   f-update  f_i = |x_i|^2 - eps * LSE_j [ (2 x_i.y_j + g_j - |y_j|^2)/eps + log b_j ]
+ *   g-update  g_j = |y_j|^2 - eps * LSE_i [ (2 x_i.y_j + f_i - |x_i|^2)/eps + log a_i ]
+ *
+ * i.e. a row (column) LogSumExp of the dot-product score matrix X Y^T shifted
+ * by a per-column (per-row) bias.  The n x m cost or score matrix is never
+ * stored anywhere (section 2 of the same page: streamed tiles, online LSE,
+ * one fused pass per update).
+ *
+ * Conventions shared by every call
+ *  - Pointers named "device" are CUDA device pointers on the device that was
+ *    current at fs_create; "host" pointers are ordinary host memory.
+ *  - Arrays are dense row-major: X [batch][n][d], Y [batch][m][d],
+ *    a/f [batch][n], b/g [batch][m], float32 unless stated.
+ *  - Every call is enqueued on the stream given to fs_create and returns
+ *    without waiting, except the calls documented as synchronising
+ *    (fs_create, fs_marginal_err, fs_ot_cost, fs_sync, fs_solve_host).
+ *  - Errors are return codes; nothing aborts or exits.  fs_last_error gives
+ *    a message.  After FS_ERR_CUDA the handle should be destroyed.
+ *  - One handle per thread / stream.  The library never allocates anything
+ *    of size n*m: handle memory is O(batch (n + m) d).
+ */
+#ifndef FLASHSINKHORN_H
+#define FLASHSINKHORN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FS_API __attribute__((visibility("default")))
+#else
+#define FS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FS_OK = 0,
+    FS_ERR_INVALID_ARG = 1, /* bad sizes, eps, weights, null pointers           */
+    FS_ERR_CUDA = 2,        /* a CUDA runtime call failed                        */
+    FS_ERR_UNSUPPORTED = 3, /* device is not sm_100 (B200) or shape unsupported  */
+    FS_ERR_NONFINITE = 4,   /* a non-finite input or result was detected         */
+    FS_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out                */
+    FS_ERR_OOM = 6          /* device allocation failed                          */
+} fs_status;
+
+typedef enum { FS_F32 = 0, FS_BF16 = 1 } fs_dtype; /* element type of X and Y */
+
+/* Operand precision of the score product X Y^T (accumulation is always fp32). */
+typedef enum {
+    FS_PREC_AUTO = 0,     /* BF16 for bf16 inputs, 3XTF32 for fp32 inputs             */
+    FS_PREC_BF16 = 1,     /* one bf16 tensor-core pass (exact for bf16 inputs)        */
+    FS_PREC_TF32 = 2,     /* one tf32 tensor-core pass                                */
+    FS_PREC_3XTF32 = 3,   /* hi*hi + lo*hi + hi*lo tf32 passes (~fp32 accurate)       */
+    FS_PREC_F32_SIMT = 5  /* plain fp32 FMA on CUDA cores (validation path)           */
+} fs_precision;
+
+typedef enum {
+    FS_SCHED_ALTERNATING = 0, /* f from g, then g from the new f (Gauss-Seidel)   */
+    FS_SCHED_SYMMETRIC = 1    /* f and g both from the previous pair (Jacobi)     */
+} fs_schedule;
+
+typedef struct {
+    int batch;          /* independent problems sharing n, m, d, eps            */
+    int n, m, d;        /* points in X, in Y, and their dimension               */
+    fs_dtype dtype;     /* element type of X and Y                              */
+    fs_precision prec;  /* score-product precision                              */
+    float eps;          /* entropic regularisation, absolute units of C         */
+} fs_desc;
+
+typedef struct fs_handle fs_handle;
+
+/* Resolved configuration of a handle (for logging and benchmarks). */
+typedef struct {
+    int prec;               /* resolved fs_precision                            */
+    int d_pad;              /* padded feature dimension                         */
+    int row_bytes;          /* bytes of one packed operand row                  */
+    int swizzle_bytes;      /* shared-memory swizzle span of the operand tiles  */
+    int stages;             /* column-tile pipeline depth                       */
+    int block_rows, block_cols; /* tile shape of one CTA step                   */
+    int splits_f, splits_g; /* column splits of the f- and g-direction passes   */
+    int launches_update;    /* kernel launches of one fs_update_f / fs_update_g */
+    int launches_solve_iter;/* kernel launches per fs_solve iteration           */
+    size_t device_bytes;    /* device memory owned by the handle                */
+} fs_info;
+
+/*
+ * Create a solver for one (batched) problem: X and Y (device, dtype, row-major
+ * [batch][n|m][d]), weights a (device [batch][n]) and b (device [batch][m]),
+ * NULL meaning uniform 1/n (1/m).  Weights must be positive and sum to 1
+ * within 1e-5 per problem.  X and Y are copied and packed into handle-owned
+ * buffers (fp32 inputs are first shifted by a common per-problem centre,
+ * which leaves every potential unchanged), so the caller may free them
+ * afterwards.  Synchronises `stream` once to validate the inputs.
+ * stream: a cudaStream_t (NULL = legacy default stream).
+ * Errors: FS_ERR_INVALID_ARG (sizes < 1, eps <= 0 or non-finite, bad weights,
+ * null X/Y/out), FS_ERR_NONFINITE (non-finite X or Y), FS_ERR_UNSUPPORTED
+ * (device is not compute capability 10.x), FS_ERR_OOM, FS_ERR_CUDA.
+ * On error *out is set to NULL and nothing is leaked.
+ */
+FS_API fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const float *a,
+                    const float *b, void *stream, fs_handle **out);
+
+/* One f-update (device g [batch][m] -> device f [batch][n]).  Asynchronous.
+ * f and g must not overlap.  Non-finite results are flagged for fs_sync. */
+FS_API fs_status fs_update_f(fs_handle *h, const float *g, float *f);
+
+/* One g-update (device f [batch][n] -> device g [batch][m]).  Asynchronous. */
+FS_API fs_status fs_update_g(fs_handle *h, const float *f, float *g);
+
+/*
+ * `iters` Sinkhorn iterations in place (device f, g).  ALTERNATING: each
+ * iteration is f <- update_f(g) then g <- update_g(f); the incoming f is not
+ * read (the first half-step overwrites it), so only g is an initial value.
+ * SYMMETRIC: (f, g) <- (update_f(g), update_g(f)) from the previous pair;
+ * both are initial values.  iters = 0 is a no-op.  Asynchronous.
+ */
+FS_API fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule schedule);
+
+/*
+ * Marginal errors of the plan P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps) at
+ * device potentials (f, g): err_row[k] = sum_i |r_i - a_i|, err_col[k] =
+ * sum_j |c_j - b_j| for each problem k (host arrays [batch]; either may be
+ * NULL).  Streams the score matrix once per requested direction.
+ * Synchronises the stream.
+ */
+FS_API fs_status fs_marginal_err(fs_handle *h, const float *f, const float *g, double *err_row,
+                          double *err_col);
+
+/*
+ * Objectives at device potentials (f, g), host arrays [batch] (either may be
+ * NULL):  dual[k]   = <a,f> + <b,g> - eps (sum_ij P_ij - 1)
+ *         primal[k] = <P, C>  (transport cost of the plan)
+ * Streams the score matrix once.  Synchronises the stream.
+ */
+FS_API fs_status fs_ot_cost(fs_handle *h, const float *f, const float *g, double *dual,
+                     double *primal);
+
+/* Wait for the handle's stream and report device-side flags raised since the
+ * last check (FS_ERR_NONFINITE, FS_ERR_TIMEOUT). */
+FS_API fs_status fs_sync(fs_handle *h);
+
+/* Resolved configuration of the handle. */
+FS_API fs_status fs_get_info(const fs_handle *h, fs_info *info);
+
+/* Free the handle (waits for its stream first).  NULL is accepted. */
+FS_API fs_status fs_destroy(fs_handle *h);
+
+/* Last error message of the handle; NULL handle -> the last error of any
+ * call on this thread that had no handle to record it in. */
+FS_API const char *fs_last_error(const fs_handle *h);
+
+/*
+ * One-call end-to-end solve from HOST arrays: copies X, Y (dtype), a, b
+ * (NULL = uniform) and the initial g to the current device, creates a
+ * handle, runs `iters` iterations, copies f and g back, and evaluates the
+ * marginal errors and objectives (any of the four result arrays may be
+ * NULL).  Host buffers may be pageable; pinned buffers make the copies
+ * asynchronous.  g_host is read (initial g) and written (final g); f_host
+ * is written.  Synchronises `stream`.  Errors as fs_create / fs_solve.
+ */
+FS_API fs_status fs_solve_host(const fs_desc *desc, const void *X_host, const void *Y_host,
+                        const float *a_host, const float *b_host, float *f_host,
+                        float *g_host, int iters, fs_schedule schedule, double *err_row,
+                        double *err_col, double *dual, double *primal, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHSINKHORN_H */

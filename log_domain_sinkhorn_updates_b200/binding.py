@@ -1,0 +1,246 @@
+"""ctypes binding of the C ABI declared in ``include/flashsinkhorn.h``.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Device arrays are torch CUDA tensors (their data pointers are
+passed through); host arrays are numpy arrays.  If the shared library is
+missing the import fails loudly -- there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libflashsinkhorn.so")
+
+FS_OK, FS_ERR_INVALID_ARG, FS_ERR_CUDA, FS_ERR_UNSUPPORTED, FS_ERR_NONFINITE, FS_ERR_TIMEOUT, FS_ERR_OOM = range(7)
+FS_F32, FS_BF16 = 0, 1
+PRECISIONS = {"auto": 0, "bf16": 1, "tf32": 2, "3xtf32": 3, "f32_simt": 5}
+PRECISION_NAMES = {v: k for k, v in PRECISIONS.items()}
+SCHEDULES = {"alternating": 0, "symmetric": 1}
+STATUS_NAMES = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_CUDA", 3: "FS_ERR_UNSUPPORTED",
+                4: "FS_ERR_NONFINITE", 5: "FS_ERR_TIMEOUT", 6: "FS_ERR_OOM"}
+
+EXPORTS = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_err", "fs_ot_cost",
+           "fs_sync", "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host"]
+
+
+class FsDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("n", ctypes.c_int), ("m", ctypes.c_int), ("d", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("prec", ctypes.c_int), ("eps", ctypes.c_float)]
+
+
+class FsInfo(ctypes.Structure):
+    _fields_ = [("prec", ctypes.c_int), ("d_pad", ctypes.c_int), ("row_bytes", ctypes.c_int),
+                ("swizzle_bytes", ctypes.c_int), ("stages", ctypes.c_int), ("block_rows", ctypes.c_int),
+                ("block_cols", ctypes.c_int), ("splits_f", ctypes.c_int), ("splits_g", ctypes.c_int),
+                ("launches_update", ctypes.c_int), ("launches_solve_iter", ctypes.c_int),
+                ("device_bytes", ctypes.c_size_t)]
+
+    def as_dict(self):
+        d = {k: getattr(self, k) for k, _ in self._fields_}
+        d["prec"] = PRECISION_NAMES.get(d["prec"], d["prec"])
+        return d
+
+
+class FsError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """The loaded C library (ctypes.CDLL); raises ImportError if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"CUDA extension missing: {LIB_PATH} (run log_domain_sinkhorn_updates_b200/build.py)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, dp, fp = ctypes.c_void_p, ctypes.POINTER(ctypes.c_double), ctypes.c_void_p
+        L.fs_create.argtypes = [ctypes.POINTER(FsDesc), vp, vp, vp, vp, vp, ctypes.POINTER(ctypes.c_void_p)]
+        L.fs_update_f.argtypes = [vp, fp, fp]
+        L.fs_update_g.argtypes = [vp, fp, fp]
+        L.fs_solve.argtypes = [vp, fp, fp, ctypes.c_int, ctypes.c_int]
+        L.fs_marginal_err.argtypes = [vp, fp, fp, dp, dp]
+        L.fs_ot_cost.argtypes = [vp, fp, fp, dp, dp]
+        L.fs_sync.argtypes = [vp]
+        L.fs_get_info.argtypes = [vp, ctypes.POINTER(FsInfo)]
+        L.fs_destroy.argtypes = [vp]
+        L.fs_last_error.argtypes = [vp]
+        L.fs_last_error.restype = ctypes.c_char_p
+        L.fs_solve_host.argtypes = [ctypes.POINTER(FsDesc), vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
+                                    dp, dp, dp, dp, vp]
+        for name in EXPORTS:
+            if name != "fs_last_error":
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(status, handle=None):
+    if status != FS_OK:
+        msg = lib().fs_last_error(handle)
+        raise FsError(status, msg.decode() if msg else "")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _f32(t):
+    import torch
+    if t is not None and t.dtype != torch.float32:
+        raise ValueError("potentials and weights must be float32")
+    return _ptr(t)
+
+
+def _stream_ptr(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Handle:
+    """Owns an ``fs_handle*``; freed by ``fs_destroy`` (or when collected)."""
+
+    def __init__(self, ptr, desc, stream):
+        self.ptr = ptr
+        self.desc = desc
+        self.stream = stream
+
+    @property
+    def batch(self):
+        return self.desc.batch
+
+    @property
+    def n(self):
+        return self.desc.n
+
+    @property
+    def m(self):
+        return self.desc.m
+
+    def __del__(self):
+        try:
+            fs_destroy(self)
+        except Exception:
+            pass
+
+
+def fs_create(X, Y, a=None, b=None, eps=0.1, prec="auto", stream=None) -> Handle:
+    """X [batch, n, d] / [n, d], Y likewise (CUDA float32 or bfloat16), a [batch, n], b [batch, m] or None."""
+    import torch
+    if X.dim() == 2:
+        X, Y = X.unsqueeze(0), Y.unsqueeze(0)
+        a = None if a is None else a.reshape(1, -1)
+        b = None if b is None else b.reshape(1, -1)
+    if X.dtype != Y.dtype:
+        raise ValueError("X and Y must share a dtype")
+    dtype = {torch.float32: FS_F32, torch.bfloat16: FS_BF16}.get(X.dtype)
+    if dtype is None:
+        raise ValueError("X, Y must be float32 or bfloat16")
+    B, n, d = X.shape
+    m = Y.shape[1]
+    if Y.shape[0] != B or Y.shape[2] != d:
+        raise ValueError("X and Y shapes disagree")
+    desc = FsDesc(B, n, m, d, dtype, PRECISIONS[prec] if isinstance(prec, str) else int(prec), float(eps))
+    out = ctypes.c_void_p()
+    st = lib().fs_create(ctypes.byref(desc), _ptr(X), _ptr(Y), _f32(a), _f32(b), _stream_ptr(stream),
+                         ctypes.byref(out))
+    _check(st)
+    return Handle(out, desc, stream)
+
+
+def fs_update_f(h: Handle, g, f):
+    _check(lib().fs_update_f(h.ptr, _f32(g), _f32(f)), h.ptr)
+
+
+def fs_update_g(h: Handle, f, g):
+    _check(lib().fs_update_g(h.ptr, _f32(f), _f32(g)), h.ptr)
+
+
+def fs_solve(h: Handle, f, g, iters, schedule="alternating"):
+    _check(lib().fs_solve(h.ptr, _f32(f), _f32(g), int(iters), SCHEDULES[schedule]), h.ptr)
+
+
+def fs_marginal_err(h: Handle, f, g, row=True, col=True):
+    er = np.zeros(h.batch)
+    ec = np.zeros(h.batch)
+    dp = ctypes.POINTER(ctypes.c_double)
+    _check(lib().fs_marginal_err(h.ptr, _f32(f), _f32(g), er.ctypes.data_as(dp) if row else None,
+                                 ec.ctypes.data_as(dp) if col else None), h.ptr)
+    return (er if row else None), (ec if col else None)
+
+
+def fs_ot_cost(h: Handle, f, g):
+    dual = np.zeros(h.batch)
+    primal = np.zeros(h.batch)
+    dp = ctypes.POINTER(ctypes.c_double)
+    _check(lib().fs_ot_cost(h.ptr, _f32(f), _f32(g), dual.ctypes.data_as(dp), primal.ctypes.data_as(dp)), h.ptr)
+    return dual, primal
+
+
+def fs_sync(h: Handle):
+    _check(lib().fs_sync(h.ptr), h.ptr)
+
+
+def fs_get_info(h: Handle) -> dict:
+    info = FsInfo()
+    _check(lib().fs_get_info(h.ptr, ctypes.byref(info)), h.ptr)
+    return info.as_dict()
+
+
+def fs_destroy(h: Handle):
+    if h is not None and h.ptr:
+        p, h.ptr = h.ptr, None
+        lib().fs_destroy(p)
+
+
+def fs_last_error(h: Handle = None) -> str:
+    msg = lib().fs_last_error(h.ptr if h is not None else None)
+    return msg.decode() if msg else ""
+
+
+def fs_solve_host(X, Y, a, b, g0, eps, iters, dtype="f32", prec="auto", schedule="alternating", stream=None,
+                  measure=True, out=None):
+    """End-to-end solve from host (numpy) arrays through ``fs_solve_host``.
+
+    X, Y: [batch, n|m, d] float32 (or uint16 bfloat16 bits with dtype="bf16"),
+    a, b: float32 or None (uniform), g0: [batch, m] float32 initial g.
+    Returns (f, g, err_row, err_col, dual, primal) as numpy arrays.
+    """
+    X = np.ascontiguousarray(X)
+    Y = np.ascontiguousarray(Y)
+    if X.ndim == 2:
+        X, Y = X[None], Y[None]
+    B, n, d = X.shape
+    m = Y.shape[1]
+    desc = FsDesc(B, n, m, d, FS_BF16 if dtype == "bf16" else FS_F32, PRECISIONS[prec], float(eps))
+    if out is None:
+        f = np.empty((B, n), np.float32)
+        g = np.array(g0, dtype=np.float32).reshape(B, m)
+    else:
+        f, g = out
+        g[...] = np.asarray(g0, dtype=np.float32).reshape(B, m)
+    res = [np.zeros(B) for _ in range(4)]
+    dp = ctypes.POINTER(ctypes.c_double)
+    vp = lambda arr: None if arr is None else ctypes.c_void_p(arr.ctypes.data)  # noqa: E731
+    rp = [r.ctypes.data_as(dp) if measure else None for r in res]
+    st = lib().fs_solve_host(ctypes.byref(desc), vp(X), vp(Y),
+                             vp(None if a is None else np.ascontiguousarray(a, np.float32)),
+                             vp(None if b is None else np.ascontiguousarray(b, np.float32)),
+                             vp(f), vp(g), int(iters), SCHEDULES[schedule], *rp,
+                             None if stream is None else ctypes.c_void_p(stream.cuda_stream))
+    _check(st)
+    return (f, g, *res)

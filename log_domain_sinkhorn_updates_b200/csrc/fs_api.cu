@@ -1,0 +1,592 @@
+// C ABI of the library: handle lifetime, layout planning, pass scheduling.
+//
+// Everything the functions below compute runs in the kernels of this
+// directory; the host code only validates arguments, allocates the handle's
+// O(batch (n+m) d) buffers, builds TMA descriptors and enqueues launches on
+// the handle's stream.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "flashsinkhorn.h"
+#include "fs_internal.cuh"
+#include "fs_prep.cuh"
+
+using fs::kBlockCols;
+using fs::kBlockRows;
+
+struct fs_handle {
+    fs_desc desc{};
+    int prec = 0;  // resolved fs_precision
+    cudaStream_t stream = nullptr;
+    int device = 0, sms = 148;
+    // packed operand layout
+    int d_p = 0, planes = 1, elem = 4, row_bytes = 0, swz = 0, plane_bytes = 0, pack_mode = 0, row_elems = 0;
+    int n_pad = 0, m_pad = 0;
+    // device memory (one allocation, carved)
+    void *block = nullptr;
+    size_t bytes = 0;
+    void *packX = nullptr, *packY = nullptr;
+    float *xn = nullptr, *yn = nullptr, *la2 = nullptr, *lb2 = nullptr;
+    float *bias_row = nullptr, *bias_col = nullptr, *center = nullptr;
+    float4 *part = nullptr;
+    unsigned *counters = nullptr;
+    double *stats = nullptr, *red = nullptr, *wstat = nullptr;
+    int *err = nullptr;
+    double *host_red = nullptr;  // pinned
+    int *host_err = nullptr;     // pinned
+    CUtensorMap mapX{}, mapY{};
+    int splits_f = 1, tps_f = 1, splits_g = 1, tps_g = 1;
+    int stages = 2, stages_meas = 2;
+    size_t smem = 0, smem_meas = 0;
+    unsigned long long timeout_ns = 2000000000ull;
+    std::string last_error;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fs_status fail(fs_handle *h, fs_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    if (h)
+        h->last_error = buf;
+    else
+        g_last_error = buf;
+    return st;
+}
+
+#define FS_CUDA(h, call)                                                                                    \
+    do {                                                                                                    \
+        cudaError_t e_ = (call);                                                                            \
+        if (e_ != cudaSuccess)                                                                              \
+            return fail((h), e_ == cudaErrorMemoryAllocation ? FS_ERR_OOM : FS_ERR_CUDA, "%s: %s (%s:%d)", \
+                        #call, cudaGetErrorString(e_), __FILE__, __LINE__);                                 \
+    } while (0)
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+int round_up(int x, int k) { return (x + k - 1) / k * k; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Column split plan for a pass with `row_blocks` CTAs-worth of rows (all
+// problems) and `col_tiles` column tiles: pick the split count S that
+// minimises (waves) x (tiles per CTA + per-CTA overhead), one CTA per SM.
+void plan_splits(int row_blocks, int col_tiles, int sms, int *splits, int *tps) {
+    const double overhead = 6.0;  // per-CTA set-up + epilogue, in tile-equivalents
+    double best = 1e300;
+    *splits = 1;
+    *tps = col_tiles;
+    for (int s = 1; s <= col_tiles && s <= 64; ++s) {
+        const int t = (col_tiles + s - 1) / s;
+        const int se = (col_tiles + t - 1) / t;
+        const long long ctas = (long long)row_blocks * se;
+        const long long waves = (ctas + sms - 1) / sms;
+        const double cost = (double)waves * (t + overhead);
+        if (cost < best - 1e-9) {
+            best = cost;
+            *splits = se;
+            *tps = t;
+        }
+    }
+}
+
+fs_status encode_map(fs_handle *h, CUtensorMap *map, void *base, int rows_total) {
+    auto fn = encode_fn();
+    if (!fn) return fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    const CUtensorMapDataType dt = h->elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    cuuint64_t gdim[2] = {(cuuint64_t)(h->row_bytes / h->elem), (cuuint64_t)rows_total};
+    cuuint64_t gstride[1] = {(cuuint64_t)h->row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)(h->swz / h->elem), (cuuint32_t)kBlockRows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw = h->swz == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : h->swz == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = fn(map, dt, 2, base, gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return FS_OK;
+}
+
+fs::PassParams make_pass(const fs_handle *h, bool fdir, bool measure) {
+    fs::PassParams p{};
+    const fs_desc &D = h->desc;
+    p.rows = fdir ? D.n : D.m;
+    p.rows_pad = fdir ? h->n_pad : h->m_pad;
+    p.cols = fdir ? D.m : D.n;
+    p.cols_pad = fdir ? h->m_pad : h->n_pad;
+    p.row_bytes = h->row_bytes;
+    p.swz = h->swz;
+    p.plane_bytes = h->plane_bytes;
+    p.d = D.d;
+    p.splits = fdir ? h->splits_f : h->splits_g;
+    p.tiles_per_split = fdir ? h->tps_f : h->tps_g;
+    p.col_tiles = p.cols_pad / kBlockCols;
+    p.stages = measure ? h->stages_meas : h->stages;
+    p.eps = (double)D.eps;
+    p.scale2 = (float)(fs::kLog2ed / (double)D.eps);
+    p.col_bias = fdir ? h->bias_col : h->bias_row;
+    p.row_norm = fdir ? h->xn : h->yn;
+    p.row_logw2 = fdir ? h->la2 : h->lb2;
+    p.col_norm = fdir ? h->yn : h->xn;
+    p.part = h->part;
+    p.counters = h->counters;
+    p.stats = h->stats;
+    p.plain_rows = fdir ? h->packX : h->packY;
+    p.plain_cols = fdir ? h->packY : h->packX;
+    p.timeout_ns = h->timeout_ns;
+    p.err = h->err;
+    return p;
+}
+
+cudaError_t run_pass(fs_handle *h, const fs::PassParams &p, bool fdir, bool measure) {
+    if (h->prec == FS_PREC_F32_SIMT) return fs::launch_lse_simt(p, h->desc.batch, measure, h->stream);
+    const CUtensorMap *mr = fdir ? &h->mapX : &h->mapY;
+    const CUtensorMap *mc = fdir ? &h->mapY : &h->mapX;
+    return fs::launch_lse_tc(p, h->desc.batch, measure, h->prec, mr, mc, measure ? h->smem_meas : h->smem,
+                             h->stream);
+}
+
+// Bias of the pass that has `cnt`-side columns, from potential pot of that side.
+cudaError_t run_bias(fs_handle *h, const float *pot, bool col_is_y) {
+    const fs_desc &D = h->desc;
+    const double scale2 = fs::kLog2ed / (double)D.eps;
+    if (col_is_y)
+        return fs::launch_bias(pot, D.batch, D.m, h->m_pad, h->yn, h->lb2, scale2, h->bias_col, h->stream);
+    return fs::launch_bias(pot, D.batch, D.n, h->n_pad, h->xn, h->la2, scale2, h->bias_row, h->stream);
+}
+
+fs_status update(fs_handle *h, const float *in, float *out, bool fdir, bool write_next_bias) {
+    FS_CUDA(h, run_bias(h, in, fdir));
+    fs::PassParams p = make_pass(h, fdir, false);
+    p.pot_out = out;
+    p.next_bias = write_next_bias ? (fdir ? h->bias_row : h->bias_col) : nullptr;
+    FS_CUDA(h, run_pass(h, p, fdir, false));
+    return FS_OK;
+}
+
+fs_status check_flags(fs_handle *h) {
+    FS_CUDA(h, cudaMemcpyAsync(h->host_err, h->err, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
+    FS_CUDA(h, cudaMemsetAsync(h->err, 0, sizeof(int), h->stream));
+    FS_CUDA(h, cudaStreamSynchronize(h->stream));
+    const int e = *h->host_err;
+    if (e & fs::kDevErrTimeout) return fail(h, FS_ERR_TIMEOUT, "a bounded device wait timed out");
+    if (e & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in a result or input");
+    return FS_OK;
+}
+
+// Measure pass in direction fdir at potentials (f, g); results land in
+// h->red[slot][batch][8].
+fs_status measure(fs_handle *h, const float *f, const float *g, bool fdir, int slot, bool want_col_sum) {
+    const fs_desc &D = h->desc;
+    FS_CUDA(h, run_bias(h, fdir ? g : f, fdir));
+    fs::PassParams p = make_pass(h, fdir, true);
+    p.pot_in = fdir ? f : g;
+    FS_CUDA(h, run_pass(h, p, fdir, true));
+    const int row_blocks = p.rows_pad / kBlockRows;
+    FS_CUDA(h, fs::launch_finalize(h->stats, D.batch, row_blocks, want_col_sum ? (fdir ? g : f) : nullptr,
+                                   fdir ? h->lb2 : h->la2, p.cols, p.cols_pad, h->red + (size_t)slot * D.batch * 8,
+                                   h->stream));
+    return FS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *fs_last_error(const fs_handle *h) { return h ? h->last_error.c_str() : g_last_error.c_str(); }
+
+fs_status fs_destroy(fs_handle *h) {
+    if (!h) return FS_OK;
+    cudaSetDevice(h->device);
+    if (h->stream) cudaStreamSynchronize(h->stream);
+    if (h->block) cudaFree(h->block);
+    if (h->host_red) cudaFreeHost(h->host_red);
+    if (h->host_err) cudaFreeHost(h->host_err);
+    delete h;
+    return FS_OK;
+}
+
+fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const float *a, const float *b,
+                    void *stream, fs_handle **out) {
+    if (out) *out = nullptr;
+    if (!desc || !X || !Y || !out) return fail(nullptr, FS_ERR_INVALID_ARG, "null argument");
+    const fs_desc D = *desc;
+    if (D.batch < 1 || D.n < 1 || D.m < 1 || D.d < 1)
+        return fail(nullptr, FS_ERR_INVALID_ARG, "sizes must be >= 1 (batch=%d n=%d m=%d d=%d)", D.batch, D.n, D.m,
+                    D.d);
+    if (!(D.eps > 0.f) || !std::isfinite(D.eps))
+        return fail(nullptr, FS_ERR_INVALID_ARG, "eps must be finite and > 0");
+    if (D.dtype != FS_F32 && D.dtype != FS_BF16) return fail(nullptr, FS_ERR_INVALID_ARG, "unknown dtype");
+    if (D.prec != FS_PREC_AUTO && D.prec != FS_PREC_BF16 && D.prec != FS_PREC_TF32 && D.prec != FS_PREC_3XTF32 &&
+        D.prec != FS_PREC_F32_SIMT)
+        return fail(nullptr, FS_ERR_INVALID_ARG, "unknown precision");
+    if ((long long)D.batch * (D.n + 127) > (1LL << 31) || (long long)D.batch * (D.m + 127) > (1LL << 31))
+        return fail(nullptr, FS_ERR_UNSUPPORTED, "batch * rows exceeds 2^31");
+
+    fs_handle *h = new fs_handle();
+    h->desc = D;
+    h->stream = static_cast<cudaStream_t>(stream);
+    {
+        cudaError_t e = cudaGetDevice(&h->device);
+        cudaDeviceProp prop;
+        if (e == cudaSuccess) e = cudaGetDeviceProperties(&prop, h->device);
+        if (e != cudaSuccess) {
+            fail(nullptr, FS_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
+            delete h;
+            return FS_ERR_CUDA;
+        }
+        if (prop.major != 10) {
+            fail(nullptr, FS_ERR_UNSUPPORTED, "device %s is sm_%d%d; this library is built for sm_100a", prop.name,
+                 prop.major, prop.minor);
+            delete h;
+            return FS_ERR_UNSUPPORTED;
+        }
+        h->sms = prop.multiProcessorCount;
+    }
+    if (const char *env = getenv("FS_WAIT_TIMEOUT_MS")) {
+        const long long ms = atoll(env);
+        if (ms > 0) h->timeout_ns = (unsigned long long)ms * 1000000ull;
+    }
+
+    // ---- precision and packed layout ----
+    int prec = D.prec;
+    if (prec == FS_PREC_AUTO) prec = D.dtype == FS_BF16 ? FS_PREC_BF16 : FS_PREC_3XTF32;
+    h->prec = prec;
+    if (prec == FS_PREC_F32_SIMT) {
+        if (D.d > 256) {
+            fail(nullptr, FS_ERR_UNSUPPORTED, "the fp32 SIMT path supports d <= 256");
+            delete h;
+            return FS_ERR_UNSUPPORTED;
+        }
+        h->elem = 4;
+        h->planes = 1;
+        h->d_p = D.d;
+        h->row_bytes = D.d * 4;
+        h->swz = 0;
+        h->plane_bytes = D.d * 4;
+        h->pack_mode = fs::kPackPlain;
+        h->row_elems = D.d;
+    } else {
+        h->elem = prec == FS_PREC_BF16 ? 2 : 4;
+        h->planes = prec == FS_PREC_3XTF32 ? 2 : 1;
+        const int kstep = prec == FS_PREC_BF16 ? 16 : 8;  // elements per 32-byte MMA K slice
+        h->d_p = round_up(D.d, kstep);
+        h->plane_bytes = h->d_p * h->elem;
+        const int used = h->planes * h->plane_bytes;
+        if (used <= 32) {
+            h->row_bytes = 32;
+            h->swz = 32;
+        } else if (used <= 64) {
+            h->row_bytes = 64;
+            h->swz = 64;
+        } else {
+            h->row_bytes = round_up(used, 128);
+            h->swz = 128;
+        }
+        h->pack_mode = prec == FS_PREC_BF16 ? fs::kPackBf16 : (prec == FS_PREC_TF32 ? fs::kPackTf32 : fs::kPack3xTf32);
+        h->row_elems = h->row_bytes / h->elem;
+        h->stages = fs::tc_max_stages(h->row_bytes, false);
+        h->stages_meas = fs::tc_max_stages(h->row_bytes, true);
+        if (h->stages < 2 || h->stages_meas < 2) {
+            fail(nullptr, FS_ERR_UNSUPPORTED,
+                 "d=%d needs %d-byte operand rows; the tensor-core pass supports rows up to 512 bytes "
+                 "(bf16 d<=256, tf32 d<=128, 3xTF32 d<=64)",
+                 D.d, h->row_bytes);
+            delete h;
+            return FS_ERR_UNSUPPORTED;
+        }
+        h->smem = fs::tc_smem_bytes(h->row_bytes, h->stages, false);
+        h->smem_meas = fs::tc_smem_bytes(h->row_bytes, h->stages_meas, true);
+    }
+    h->n_pad = round_up(D.n, kBlockRows);
+    h->m_pad = round_up(D.m, kBlockRows);
+    plan_splits(D.batch * (h->n_pad / kBlockRows), h->m_pad / kBlockCols, h->sms, &h->splits_f, &h->tps_f);
+    plan_splits(D.batch * (h->m_pad / kBlockRows), h->n_pad / kBlockCols, h->sms, &h->splits_g, &h->tps_g);
+
+    // ---- one device allocation, carved ----
+    const size_t B = (size_t)D.batch;
+    const size_t max_pad = (size_t)(h->n_pad > h->m_pad ? h->n_pad : h->m_pad);
+    const int max_splits = h->splits_f > h->splits_g ? h->splits_f : h->splits_g;
+    const size_t max_rb = max_pad / kBlockRows;
+    size_t off = 0;
+    auto carve = [&](size_t bytes) {
+        size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    const size_t o_packX = carve(B * h->n_pad * h->row_bytes);
+    const size_t o_packY = carve(B * h->m_pad * h->row_bytes);
+    const size_t o_xn = carve(B * h->n_pad * 4), o_yn = carve(B * h->m_pad * 4);
+    const size_t o_la2 = carve(B * h->n_pad * 4), o_lb2 = carve(B * h->m_pad * 4);
+    const size_t o_brow = carve(B * h->n_pad * 4), o_bcol = carve(B * h->m_pad * 4);
+    const size_t o_center = carve(B * D.d * 4);
+    const size_t o_part = carve(max_splits > 1 ? B * max_splits * max_pad * 16 : 16);
+    const size_t o_ctr = carve(B * max_rb * 4);
+    const size_t o_stats = carve(B * max_rb * 4 * 8);
+    const size_t o_red = carve(2 * B * 8 * 8);
+    const size_t o_wstat = carve(2 * B * 2 * 8);
+    const size_t o_err = carve(16);
+    h->bytes = off;
+    {
+        cudaError_t e = cudaMalloc(&h->block, h->bytes);
+        if (e == cudaSuccess) e = cudaMallocHost((void **)&h->host_red, 2 * B * 8 * 8 + 4 * B * 8);
+        if (e == cudaSuccess) e = cudaMallocHost((void **)&h->host_err, 16);
+        if (e != cudaSuccess) {
+            fail(nullptr, e == cudaErrorMemoryAllocation ? FS_ERR_OOM : FS_ERR_CUDA, "allocation of %zu bytes: %s",
+                 h->bytes, cudaGetErrorString(e));
+            fs_destroy(h);
+            return e == cudaErrorMemoryAllocation ? FS_ERR_OOM : FS_ERR_CUDA;
+        }
+    }
+    char *base = static_cast<char *>(h->block);
+    h->packX = base + o_packX;
+    h->packY = base + o_packY;
+    h->xn = reinterpret_cast<float *>(base + o_xn);
+    h->yn = reinterpret_cast<float *>(base + o_yn);
+    h->la2 = reinterpret_cast<float *>(base + o_la2);
+    h->lb2 = reinterpret_cast<float *>(base + o_lb2);
+    h->bias_row = reinterpret_cast<float *>(base + o_brow);
+    h->bias_col = reinterpret_cast<float *>(base + o_bcol);
+    h->center = reinterpret_cast<float *>(base + o_center);
+    h->part = reinterpret_cast<float4 *>(base + o_part);
+    h->counters = reinterpret_cast<unsigned *>(base + o_ctr);
+    h->stats = reinterpret_cast<double *>(base + o_stats);
+    h->red = reinterpret_cast<double *>(base + o_red);
+    h->wstat = reinterpret_cast<double *>(base + o_wstat);
+    h->err = reinterpret_cast<int *>(base + o_err);
+
+    // ---- set-up kernels ----
+    fs_status st = FS_OK;
+    auto run = [&]() -> fs_status {
+        const bool bf16 = D.dtype == FS_BF16;
+        FS_CUDA(h, cudaMemsetAsync(h->counters, 0, B * max_rb * 4, h->stream));
+        FS_CUDA(h, cudaMemsetAsync(h->err, 0, 16, h->stream));
+        const float *t = nullptr;
+        if (!bf16) {
+            FS_CUDA(h, fs::launch_center(X, Y, bf16, D.batch, D.n, D.m, D.d, h->center, h->stream));
+            t = h->center;
+        }
+        FS_CUDA(h, fs::launch_pack(X, bf16, D.n, h->n_pad, D.d, D.batch, t, 1.f, h->pack_mode, h->d_p, h->row_elems,
+                                   h->packX, h->xn, h->err, h->stream));
+        FS_CUDA(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, 2.f, h->pack_mode, h->d_p, h->row_elems,
+                                   h->packY, h->yn, h->err, h->stream));
+        FS_CUDA(h, fs::launch_weights(a, D.batch, D.n, h->n_pad, h->la2, h->wstat, h->stream));
+        FS_CUDA(h, fs::launch_weights(b, D.batch, D.m, h->m_pad, h->lb2, h->wstat + 2 * B, h->stream));
+        FS_CUDA(h, fs::launch_fill(h->bias_row, B * h->n_pad, -INFINITY, h->stream));
+        FS_CUDA(h, fs::launch_fill(h->bias_col, B * h->m_pad, -INFINITY, h->stream));
+        double *hw = h->host_red + 2 * B * 8;
+        FS_CUDA(h, cudaMemcpyAsync(hw, h->wstat, 4 * B * 8, cudaMemcpyDeviceToHost, h->stream));
+        FS_CUDA(h, cudaMemcpyAsync(h->host_err, h->err, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
+        FS_CUDA(h, cudaMemsetAsync(h->err, 0, 16, h->stream));
+        FS_CUDA(h, cudaStreamSynchronize(h->stream));
+        for (size_t k = 0; k < 2 * B; ++k) {
+            const bool is_a = k < B;
+            const double s = hw[2 * k], bad = hw[2 * k + 1];
+            if (bad > 0 || !(std::fabs(s - 1.0) <= 1e-5))
+                return fail(h, FS_ERR_INVALID_ARG, "weights %s of problem %zu must be positive and sum to 1 (sum=%.9g)",
+                            is_a ? "a" : "b", is_a ? k : k - B, s);
+        }
+        if (*h->host_err & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in X or Y");
+        if (prec != FS_PREC_F32_SIMT) {
+            fs_status s2 = encode_map(h, &h->mapX, h->packX, D.batch * h->n_pad);
+            if (s2 != FS_OK) return s2;
+            s2 = encode_map(h, &h->mapY, h->packY, D.batch * h->m_pad);
+            if (s2 != FS_OK) return s2;
+        }
+        return FS_OK;
+    };
+    st = run();
+    if (st != FS_OK) {
+        g_last_error = h->last_error;
+        fs_destroy(h);
+        return st;
+    }
+    *out = h;
+    return FS_OK;
+}
+
+fs_status fs_update_f(fs_handle *h, const float *g, float *f) {
+    if (!h || !g || !f) return fail(h, FS_ERR_INVALID_ARG, "null argument");
+    FS_CUDA(h, cudaSetDevice(h->device));
+    return update(h, g, f, true, false);
+}
+
+fs_status fs_update_g(fs_handle *h, const float *f, float *g) {
+    if (!h || !f || !g) return fail(h, FS_ERR_INVALID_ARG, "null argument");
+    FS_CUDA(h, cudaSetDevice(h->device));
+    return update(h, f, g, false, false);
+}
+
+fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule schedule) {
+    if (!h || !f || !g || iters < 0) return fail(h, FS_ERR_INVALID_ARG, "bad argument");
+    if (schedule != FS_SCHED_ALTERNATING && schedule != FS_SCHED_SYMMETRIC)
+        return fail(h, FS_ERR_INVALID_ARG, "unknown schedule");
+    if (iters == 0) return FS_OK;
+    FS_CUDA(h, cudaSetDevice(h->device));
+    if (schedule == FS_SCHED_ALTERNATING) {
+        // One bias launch from the initial g; afterwards every pass's fused
+        // epilogue writes the bias the next pass reads.
+        FS_CUDA(h, run_bias(h, g, true));
+        for (int it = 0; it < iters; ++it) {
+            fs::PassParams pf = make_pass(h, true, false);
+            pf.pot_out = f;
+            pf.next_bias = h->bias_row;
+            FS_CUDA(h, run_pass(h, pf, true, false));
+            fs::PassParams pg = make_pass(h, false, false);
+            pg.pot_out = g;
+            pg.next_bias = h->bias_col;
+            FS_CUDA(h, run_pass(h, pg, false, false));
+        }
+    } else {
+        for (int it = 0; it < iters; ++it) {
+            FS_CUDA(h, run_bias(h, g, true));
+            FS_CUDA(h, run_bias(h, f, false));
+            fs::PassParams pf = make_pass(h, true, false);
+            pf.pot_out = f;
+            FS_CUDA(h, run_pass(h, pf, true, false));
+            fs::PassParams pg = make_pass(h, false, false);
+            pg.pot_out = g;
+            FS_CUDA(h, run_pass(h, pg, false, false));
+        }
+    }
+    return FS_OK;
+}
+
+fs_status fs_marginal_err(fs_handle *h, const float *f, const float *g, double *err_row, double *err_col) {
+    if (!h || !f || !g) return fail(h, FS_ERR_INVALID_ARG, "null argument");
+    FS_CUDA(h, cudaSetDevice(h->device));
+    const size_t B = (size_t)h->desc.batch;
+    if (err_row) {
+        fs_status s = measure(h, f, g, true, 0, false);
+        if (s != FS_OK) return s;
+    }
+    if (err_col) {
+        fs_status s = measure(h, f, g, false, 1, false);
+        if (s != FS_OK) return s;
+    }
+    FS_CUDA(h, cudaMemcpyAsync(h->host_red, h->red, 2 * B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
+    fs_status s = check_flags(h);
+    if (s != FS_OK) return s;
+    for (size_t k = 0; k < B; ++k) {
+        if (err_row) err_row[k] = h->host_red[k * 8 + 0];
+        if (err_col) err_col[k] = h->host_red[(B + k) * 8 + 0];
+    }
+    return FS_OK;
+}
+
+fs_status fs_ot_cost(fs_handle *h, const float *f, const float *g, double *dual, double *primal) {
+    if (!h || !f || !g) return fail(h, FS_ERR_INVALID_ARG, "null argument");
+    FS_CUDA(h, cudaSetDevice(h->device));
+    const size_t B = (size_t)h->desc.batch;
+    fs_status s = measure(h, f, g, true, 0, true);
+    if (s != FS_OK) return s;
+    FS_CUDA(h, cudaMemcpyAsync(h->host_red, h->red, B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
+    s = check_flags(h);
+    if (s != FS_OK) return s;
+    const double eps = (double)h->desc.eps;
+    for (size_t k = 0; k < B; ++k) {
+        const double *r = h->host_red + k * 8;  // [|r-a|, sum r, sum r*meanC, <a,f>, <b,g>]
+        if (dual) dual[k] = r[3] + r[4] - eps * (r[1] - 1.0);
+        if (primal) primal[k] = r[2];
+    }
+    return FS_OK;
+}
+
+fs_status fs_sync(fs_handle *h) {
+    if (!h) return fail(nullptr, FS_ERR_INVALID_ARG, "null handle");
+    FS_CUDA(h, cudaSetDevice(h->device));
+    return check_flags(h);
+}
+
+fs_status fs_get_info(const fs_handle *h, fs_info *info) {
+    if (!h || !info) return FS_ERR_INVALID_ARG;
+    info->prec = h->prec;
+    info->d_pad = h->d_p;
+    info->row_bytes = h->row_bytes;
+    info->swizzle_bytes = h->swz;
+    info->stages = h->stages;
+    info->block_rows = kBlockRows;
+    info->block_cols = kBlockCols;
+    info->splits_f = h->splits_f;
+    info->splits_g = h->splits_g;
+    info->launches_update = 2;
+    info->launches_solve_iter = 2;
+    info->device_bytes = h->bytes;
+    return FS_OK;
+}
+
+fs_status fs_solve_host(const fs_desc *desc, const void *X_host, const void *Y_host, const float *a_host,
+                        const float *b_host, float *f_host, float *g_host, int iters, fs_schedule schedule,
+                        double *err_row, double *err_col, double *dual, double *primal, void *stream) {
+    if (!desc || !X_host || !Y_host || !f_host || !g_host || iters < 0)
+        return fail(nullptr, FS_ERR_INVALID_ARG, "null or bad argument");
+    const fs_desc D = *desc;
+    if (D.batch < 1 || D.n < 1 || D.m < 1 || D.d < 1)
+        return fail(nullptr, FS_ERR_INVALID_ARG, "sizes must be >= 1");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t B = (size_t)D.batch, es = D.dtype == FS_BF16 ? 2 : 4;
+    const size_t bx = B * D.n * D.d * es, by = B * D.m * D.d * es, bf = B * D.n * 4, bg = B * D.m * 4;
+    const size_t total = align256(bx) + align256(by) + 2 * align256(bf) + 2 * align256(bg);
+    char *blk = nullptr;
+    cudaError_t e = cudaMallocAsync((void **)&blk, total, s);
+    if (e != cudaSuccess)
+        return fail(nullptr, e == cudaErrorMemoryAllocation ? FS_ERR_OOM : FS_ERR_CUDA, "cudaMallocAsync: %s",
+                    cudaGetErrorString(e));
+    char *dX = blk, *dY = dX + align256(bx);
+    float *da = reinterpret_cast<float *>(dY + align256(by));
+    float *df = reinterpret_cast<float *>(reinterpret_cast<char *>(da) + align256(bf));
+    float *db = reinterpret_cast<float *>(reinterpret_cast<char *>(df) + align256(bf));
+    float *dg = reinterpret_cast<float *>(reinterpret_cast<char *>(db) + align256(bg));
+    fs_handle *h = nullptr;
+    fs_status st = FS_OK;
+    auto body = [&]() -> fs_status {
+        FS_CUDA(nullptr, cudaMemcpyAsync(dX, X_host, bx, cudaMemcpyHostToDevice, s));
+        FS_CUDA(nullptr, cudaMemcpyAsync(dY, Y_host, by, cudaMemcpyHostToDevice, s));
+        if (a_host) FS_CUDA(nullptr, cudaMemcpyAsync(da, a_host, bf, cudaMemcpyHostToDevice, s));
+        if (b_host) FS_CUDA(nullptr, cudaMemcpyAsync(db, b_host, bg, cudaMemcpyHostToDevice, s));
+        FS_CUDA(nullptr, cudaMemcpyAsync(dg, g_host, bg, cudaMemcpyHostToDevice, s));
+        fs_status r = fs_create(&D, dX, dY, a_host ? da : nullptr, b_host ? db : nullptr, s, &h);
+        if (r != FS_OK) return r;
+        r = fs_solve(h, df, dg, iters, schedule);
+        if (r == FS_OK && (err_row || err_col)) r = fs_marginal_err(h, df, dg, err_row, err_col);
+        if (r == FS_OK && (dual || primal)) r = fs_ot_cost(h, df, dg, dual, primal);
+        if (r != FS_OK) {
+            g_last_error = h->last_error;
+            return r;
+        }
+        FS_CUDA(h, cudaMemcpyAsync(f_host, df, bf, cudaMemcpyDeviceToHost, s));
+        FS_CUDA(h, cudaMemcpyAsync(g_host, dg, bg, cudaMemcpyDeviceToHost, s));
+        return fs_sync(h);
+    };
+    st = body();
+    if (st != FS_OK && h) g_last_error = h->last_error;
+    fs_destroy(h);
+    cudaFreeAsync(blk, s);
+    cudaStreamSynchronize(s);
+    return st;
+}
+
+}  // extern "C"

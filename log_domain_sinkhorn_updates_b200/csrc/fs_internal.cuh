@@ -1,0 +1,109 @@
+// Internal declarations of the sm_100a log-domain Sinkhorn library.
+//
+// Notation follows "FlashSinkhorn: IO-aware EOT on GPU" (Metodologia,
+// Proposition 1): a pass computes, for every row i of its "row side",
+//
+//   LSE2_i = log2 sum_j 2^( S_ij * log2(e)/eps + beta_j ),   S_ij = <q_i, k_j>
+//
+// where the packed operands are q = x - t and k = 2 (y - t) (t a common
+// centre, zero for bf16 inputs), so S_ij = 2 (x_i - t).(y_j - t), and beta_j
+// is the column bias ((g_j - |y_j - t|^2)/eps + log b_j) * log2(e) in base-2
+// units (-inf on padding columns).  The f-update is then
+//   f_i = |x_i - t|^2 - eps ln2 LSE2_i.
+// The g-update is the same pass with the two sides exchanged (the product is
+// symmetric in q and k: S_ji^T = <k_j, q_i>).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fs {
+
+constexpr int kBlockRows = 128;   // rows of one CTA (one TMEM lane per row)
+constexpr int kBlockCols = 128;   // columns of one streamed tile
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr double kLn2d = 0.69314718055994530942;
+constexpr double kLog2ed = 1.44269504088896340736;
+
+// device error bits (fs_handle::err)
+constexpr int kDevErrNonfinite = 1;
+constexpr int kDevErrTimeout = 2;
+constexpr int kDevErrBadWeights = 4;
+
+// Parameters of one streamed LSE pass (row side R against column side C).
+struct PassParams {
+    int rows, rows_pad;        // valid and padded rows of the row side
+    int cols, cols_pad;        // valid and padded columns
+    int row_bytes;             // bytes of a packed operand row (tensor-core paths)
+    int swz;                   // swizzle span in bytes (32, 64 or 128)
+    int plane_bytes;           // bytes of one operand plane (multiple of 32)
+    int d;                     // feature dim of the plain fp32 layout (SIMT path)
+    int splits;                // column splits (grid.y)
+    int tiles_per_split;       // column tiles handled by one split
+    int col_tiles;             // total column tiles
+    int stages;                // pipeline depth (tensor-core path)
+    float scale2;              // log2(e)/eps
+    double eps;
+    const float *col_bias;     // [batch][cols_pad], base-2, -inf on padding
+    const float *row_norm;     // [batch][rows_pad] |row - t|^2
+    const float *row_logw2;    // [batch][rows_pad] log2 of the row weights
+    const float *col_norm;     // [batch][cols_pad] (measure passes only)
+    const float *pot_in;       // [batch][rows] current row potential (measure passes)
+    float *pot_out;            // [batch][rows] new row potential (update passes)
+    float *next_bias;          // [batch][rows_pad] base-2 bias for the opposite pass, or null
+    float4 *part;              // [batch][splits][rows_pad] split partials (m, l, w, -)
+    unsigned *counters;        // [batch][row_blocks] arrival counters (self-resetting)
+    double *stats;             // [batch][row_blocks][4] measure partial sums
+    const void *plain_rows;    // SIMT path: [batch][rows_pad][d] fp32
+    const void *plain_cols;    // SIMT path: [batch][cols_pad][d] fp32
+    unsigned long long timeout_ns;
+    int *err;
+};
+
+// ---------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Merge two online-LSE states (max m, sum l, weighted sum w) in base 2.
+__device__ __forceinline__ void lse_merge(float &m, float &l, float &w, float m2, float l2, float w2) {
+    float M = fmaxf(m, m2);
+    if (M == -INFINITY) { m = -INFINITY; l = 0.f; w = 0.f; return; }
+    float s1 = exp2f(m - M), s2 = exp2f(m2 - M);
+    l = l * s1 + l2 * s2;
+    w = w * s1 + w2 * s2;
+    m = M;
+}
+
+// Finish 128 rows of a pass.  Called by exactly 128 threads (one per row,
+// row_local = 0..127) that hold the final online state of their row over the
+// CTA's column range.  bar_id/bar_threads name a barrier covering exactly
+// these 128 threads.  Handles the split merge (the last CTA of a row block to
+// arrive merges all splits in fixed order, so results are deterministic),
+// the potential write, the next pass's bias, and measure-mode statistics.
+template <bool MEASURE>
+__device__ void finish_rows(const PassParams &p, int row_local, float m, float l, float w,
+                            int bar_id, double *red_smem /* >= 4*128 doubles */,
+                            int *flag_smem);
+
+}  // namespace fs
+
+// Launchers (defined in the .cu files); all return cudaGetLastError().
+namespace fs {
+cudaError_t launch_lse_simt(const PassParams &p, int batch, bool measure, cudaStream_t s);
+cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec,
+                          const void *map_rows, const void *map_cols, size_t smem_bytes,
+                          cudaStream_t s);
+size_t tc_smem_bytes(int row_bytes, int stages, bool measure);
+int tc_max_stages(int row_bytes, bool measure);
+}  // namespace fs

@@ -1,0 +1,27 @@
+// Launchers of the set-up and helper kernels (fs_prep.cu).
+#pragma once
+
+#include "fs_internal.cuh"
+
+namespace fs {
+
+// Operand packing modes.
+constexpr int kPackBf16 = 0;    // one bf16 plane
+constexpr int kPackTf32 = 1;    // one fp32 plane rounded to tf32
+constexpr int kPack3xTf32 = 2;  // [hi | lo] fp32 planes, hi = tf32(v), lo = v - hi
+constexpr int kPackPlain = 3;   // plain fp32 rows of d values (SIMT path)
+
+cudaError_t launch_center(const void *X, const void *Y, bool bf16, int batch, int n, int m, int d, float *t,
+                          cudaStream_t s);
+cudaError_t launch_pack(const void *src, bool bf16, int rows, int rows_pad, int d, int batch, const float *t,
+                        float scale, int mode, int d_p, int row_elems, void *dst, float *norm, int *err,
+                        cudaStream_t s);
+cudaError_t launch_weights(const float *w, int batch, int cnt, int cnt_pad, float *lw2, double *wstat,
+                           cudaStream_t s);
+cudaError_t launch_fill(float *p, size_t count, float v, cudaStream_t s);
+cudaError_t launch_bias(const float *pot, int batch, int cnt, int cnt_pad, const float *norm, const float *lw2,
+                        double scale2, float *out, cudaStream_t s);
+cudaError_t launch_finalize(const double *stats, int batch, int row_blocks, const float *col_pot,
+                            const float *col_lw2, int cols, int cols_pad, double *out, cudaStream_t s);
+
+}  // namespace fs

@@ -1,0 +1,144 @@
+"""GPU parity against the CPU oracle, through the C ABI.
+
+Single updates: every workload recipe at sizes the oracle finishes in seconds,
+spanning several 128-row/128-column tiles with ragged tails; the bar is
+max |f_gpu - f_oracle| <= 1e-4 * max_ij C_ij (both sides see the same float32
+inputs, the oracle in double).  Full solves: marginal L1 error and dual cost
+after the recipe's iteration count within 1e-3 relative (plus the float32
+noise floor of the marginal error, see test_solve_parity).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import device_inputs, max_cost, make_problem, oracle_arrays, smooth_potential
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": dict(),
+    "middim": dict(n=1000, m=900),
+    "cloud3d": dict(n=1500, m=1100),
+    "highdim": dict(n=700, m=650),
+    "batched": dict(batch=3, n=600, m=520),
+}
+PRECS = ["auto", "f32_simt"]
+
+
+def _fs():
+    import log_domain_sinkhorn_updates_b200 as fs
+    return fs
+
+
+@pytest.mark.parametrize("prec", PRECS)
+@pytest.mark.parametrize("name", list(SMALL))
+def test_single_update_parity(cuda_device, name, prec):
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a, b = device_inputs(prob)
+    h = fs.fs_create(X, Y, a, b, eps=prob.eps, prec=prec)
+    rng = np.random.default_rng(77)
+    tol = 1e-4 * max_cost(prob)
+    g_in = np.stack([smooth_potential(rng, prob.m, 0.5) for _ in range(prob.batch)])
+    f_in = np.stack([smooth_potential(rng, prob.n, 0.5) for _ in range(prob.batch)])
+    f = torch.empty(prob.batch, prob.n, device=cuda_device)
+    g = torch.empty(prob.batch, prob.m, device=cuda_device)
+    fs.fs_update_f(h, torch.from_numpy(g_in).to(cuda_device), f)
+    fs.fs_update_g(h, torch.from_numpy(f_in).to(cuda_device), g)
+    fs.fs_sync(h)
+    f = f.cpu().numpy()
+    g = g.cpu().numpy()
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fo = oracle.update_f(Xo, Yo, logb, g_in[k].astype(np.float64), prob.eps)
+        go = oracle.update_g(Xo, Yo, loga, f_in[k].astype(np.float64), prob.eps)
+        ef = np.abs(f[k] - fo).max()
+        eg = np.abs(g[k] - go).max()
+        assert ef <= tol[k], (name, prec, k, ef, tol[k])
+        assert eg <= tol[k], (name, prec, k, eg, tol[k])
+        if prec == "auto":  # the chosen mode must leave 4x margin to the bar
+            assert max(ef, eg) <= tol[k] / 4, (name, k, ef, eg, tol[k])
+
+
+SOLVE = {
+    "tiny": dict(),
+    "middim": dict(n=1000, m=900),
+    "cloud3d": dict(n=1500, m=1100),
+    "highdim": dict(n=700, m=650),
+    "batched": dict(batch=3, n=600, m=520),
+}
+
+
+def _gauge_fixed_diff(fg, gg, fo, go, a, b):
+    """GPU - oracle potentials after removing the common constant (f + c, g - c leaves P unchanged)."""
+    c = a @ (fg - fo)
+    return fg - fo - c, gg - go + c
+
+
+def _first_order_err_bound(df, dg, a, b, eps):
+    """|d err_row| + |d err_col| <= 2 (sum_i a_i |df_i| + sum_j b_j |dg_j|)/eps to first order
+    (d r_i = sum_j P_ij (df_i + dg_j)/eps and likewise for c_j)."""
+    return 2.0 * (a @ np.abs(df) + b @ np.abs(dg)) / eps
+
+
+@pytest.mark.parametrize("name", list(SOLVE))
+def test_solve_parity(cuda_device, name):
+    """fs_solve from g = 0 for the recipe's iteration count, then the fused measurements,
+    against the oracle's own solve from the same inputs."""
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SOLVE[name])
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    f = torch.zeros(prob.batch, prob.n, device=cuda_device)
+    g = torch.zeros(prob.batch, prob.m, device=cuda_device)
+    fs.fs_solve(h, f, g, prob.iters)
+    er, ec = fs.fs_marginal_err(h, f, g)
+    dual, primal = fs.fs_ot_cost(h, f, g)
+    fg, gg = f.cpu().numpy().astype(np.float64), g.cpu().numpy().astype(np.float64)
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fo, go = oracle.solve(Xo, Yo, loga, logb, prob.eps, prob.iters)
+        eo = oracle.marginal_error(Xo, Yo, loga, logb, fo, go, prob.eps)
+        co = oracle.costs(Xo, Yo, loga, logb, fo, go, prob.eps)
+        df, dg = _gauge_fixed_diff(fg[k], gg[k], fo, go, np.exp(loga), np.exp(logb))
+        tau = _first_order_err_bound(df, dg, np.exp(loga), np.exp(logb), prob.eps)
+        e_gpu, e_o = er[k] + ec[k], eo[0] + eo[1]
+        print(f"{name}[{k}] err gpu={e_gpu:.6e} oracle={e_o:.6e} tau={tau:.3e} "
+              f"dual {dual[k]:.9g} vs {co['dual']:.9g}  primal {primal[k]:.9g} vs {co['primal']:.9g} "
+              f"max|df|={np.abs(df).max():.3e} max|dg|={np.abs(dg).max():.3e}")
+        assert abs(e_gpu - e_o) <= 1e-3 * e_o + tau, (name, k, e_gpu, e_o, tau)
+        assert abs(dual[k] - co["dual"]) <= 1e-3 * abs(co["dual"]), (name, k, dual[k], co["dual"])
+        assert abs(primal[k] - co["primal"]) <= 1e-3 * abs(co["primal"]), (name, k, primal[k], co["primal"])
+
+
+@pytest.mark.parametrize("name", list(SOLVE))
+def test_measure_parity(cuda_device, name):
+    """fs_marginal_err / fs_ot_cost at the oracle's converged potentials (rounded to float32,
+    the same bytes on both sides) against the oracle's measurements at those potentials."""
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SOLVE[name])
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    pots = [oracle.solve(*arr, prob.eps, prob.iters) for arr in oracle_arrays(prob)]
+    f32 = np.stack([p[0] for p in pots]).astype(np.float32)
+    g32 = np.stack([p[1] for p in pots]).astype(np.float32)
+    f = torch.from_numpy(f32).to(cuda_device)
+    g = torch.from_numpy(g32).to(cuda_device)
+    er, ec = fs.fs_marginal_err(h, f, g)
+    dual, primal = fs.fs_ot_cost(h, f, g)
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
+        eo = oracle.marginal_error(Xo, Yo, loga, logb, fk, gk, prob.eps)
+        co = oracle.costs(Xo, Yo, loga, logb, fk, gk, prob.eps)
+        # float32 LSE of each row carries a relative error ~2^-22 of its log-domain
+        # argument (|pot| + max C)/eps; first-order effect on the marginal sums:
+        cmax = co["max_cost"]
+        a, b = np.exp(loga), np.exp(logb)
+        tau = 2.0 ** -21 * (a @ (np.abs(fk) + cmax) + b @ (np.abs(gk) + cmax)) / prob.eps
+        print(f"{name}[{k}] row {er[k]:.6e}/{eo[0]:.6e} col {ec[k]:.6e}/{eo[1]:.6e} tau={tau:.2e} "
+              f"dual {dual[k]:.10g}/{co['dual']:.10g} primal {primal[k]:.10g}/{co['primal']:.10g}")
+        assert abs(er[k] - eo[0]) <= 1e-3 * eo[0] + tau, (name, k, er[k], eo[0], tau)
+        assert abs(ec[k] - eo[1]) <= 1e-3 * eo[1] + tau, (name, k, ec[k], eo[1], tau)
+        assert abs(dual[k] - co["dual"]) <= 1e-3 * abs(co["dual"]), (name, k)
+        assert abs(primal[k] - co["primal"]) <= 1e-3 * abs(co["primal"]), (name, k)
