@@ -151,8 +151,14 @@ FS_API fs_status fs_sync(fs_handle *h);
 /* Resolved configuration of the handle. */
 FS_API fs_status fs_get_info(const fs_handle *h, fs_info *info);
 
-/* Free the handle (waits for its stream first).  NULL is accepted. */
+/* Free the handle.  Its device memory is released in stream order on the
+ * handle's stream (no host wait), so the stream must still exist; work
+ * already enqueued that uses the handle completes first.  NULL is accepted. */
 FS_API fs_status fs_destroy(fs_handle *h);
+
+/* Number of CUDA kernels this library has launched in this process so far
+ * (all handles, all threads).  Host-side counter; never synchronises. */
+FS_API unsigned long long fs_kernel_launches(void);
 
 /* Last error message of the handle; NULL handle -> the last error of any
  * call on this thread that had no handle to record it in. */

@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_CUDA", 3: "FS_ER
                 4: "FS_ERR_NONFINITE", 5: "FS_ERR_TIMEOUT", 6: "FS_ERR_OOM"}
 
 EXPORTS = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_err", "fs_ot_cost",
-           "fs_sync", "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host"]
+           "fs_sync", "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches"]
 
 
 class FsDesc(ctypes.Structure):
@@ -75,8 +75,10 @@ def lib():
         L.fs_last_error.restype = ctypes.c_char_p
         L.fs_solve_host.argtypes = [ctypes.POINTER(FsDesc), vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
                                     dp, dp, dp, dp, vp]
+        L.fs_kernel_launches.argtypes = []
+        L.fs_kernel_launches.restype = ctypes.c_ulonglong
         for name in EXPORTS:
-            if name != "fs_last_error":
+            if name not in ("fs_last_error", "fs_kernel_launches"):
                 getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -210,6 +212,11 @@ def fs_destroy(h: Handle):
 def fs_last_error(h: Handle = None) -> str:
     msg = lib().fs_last_error(h.ptr if h is not None else None)
     return msg.decode() if msg else ""
+
+
+def fs_kernel_launches() -> int:
+    """Kernels the library has launched in this process (host-side count)."""
+    return int(lib().fs_kernel_launches())
 
 
 def fs_solve_host(X, Y, a, b, g0, eps, iters, dtype="f32", prec="auto", schedule="alternating", stream=None,

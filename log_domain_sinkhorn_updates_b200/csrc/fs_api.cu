@@ -12,8 +12,10 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "flashsinkhorn.h"
 #include "fs_internal.cuh"
@@ -40,8 +42,8 @@ struct fs_handle {
     unsigned *counters = nullptr;
     double *stats = nullptr, *red = nullptr, *wstat = nullptr;
     int *err = nullptr;
-    double *host_red = nullptr;  // pinned
-    int *host_err = nullptr;     // pinned
+    std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
+    int host_err[4] = {0, 0, 0, 0};
     CUtensorMap mapX{}, mapY{};
     int splits_f = 1, tps_f = 1, splits_g = 1, tps_g = 1;
     int stages = 2, stages_meas = 2;
@@ -53,6 +55,7 @@ struct fs_handle {
 namespace {
 
 thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_launches{0};  // kernels this library has launched
 
 fs_status fail(fs_handle *h, fs_status st, const char *fmt, ...) {
     char buf[512];
@@ -75,6 +78,13 @@ fs_status fail(fs_handle *h, fs_status st, const char *fmt, ...) {
                         #call, cudaGetErrorString(e_), __FILE__, __LINE__);                                 \
     } while (0)
 
+// FS_CUDA for a call that launches one kernel: also counts the launch.
+#define FS_LAUNCH(h, call)                 \
+    do {                                   \
+        FS_CUDA(h, call);                  \
+        g_launches.fetch_add(1, std::memory_order_relaxed); \
+    } while (0)
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 int round_up(int x, int k) { return (x + k - 1) / k * k; }
 
@@ -89,6 +99,32 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
     });
     return fn;
+}
+
+// Library-owned stream-ordered memory pool of a device.  Handles allocate
+// and free their buffers on their stream from this pool, so creating and
+// destroying handles neither synchronises the device nor returns memory to
+// the driver each time; up to 1 GiB of freed memory stays cached.
+cudaError_t device_pool(int device, cudaMemPool_t *out) {
+    static std::mutex mu;
+    static std::vector<cudaMemPool_t> pools;
+    std::lock_guard<std::mutex> lock(mu);
+    if ((int)pools.size() <= device) pools.resize(device + 1, nullptr);
+    if (!pools[device]) {
+        cudaMemPoolProps props{};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = device;
+        cudaMemPool_t pool;
+        cudaError_t e = cudaMemPoolCreate(&pool, &props);
+        if (e != cudaSuccess) return e;
+        unsigned long long keep = 1ull << 30;
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+        pools[device] = pool;
+    }
+    *out = pools[device];
+    return cudaSuccess;
 }
 
 // Column split plan for a pass with `row_blocks` CTAs-worth of rows (all
@@ -179,11 +215,11 @@ cudaError_t run_bias(fs_handle *h, const float *pot, bool col_is_y) {
 }
 
 fs_status update(fs_handle *h, const float *in, float *out, bool fdir, bool write_next_bias) {
-    FS_CUDA(h, run_bias(h, in, fdir));
+    FS_LAUNCH(h, run_bias(h, in, fdir));
     fs::PassParams p = make_pass(h, fdir, false);
     p.pot_out = out;
     p.next_bias = write_next_bias ? (fdir ? h->bias_row : h->bias_col) : nullptr;
-    FS_CUDA(h, run_pass(h, p, fdir, false));
+    FS_LAUNCH(h, run_pass(h, p, fdir, false));
     return FS_OK;
 }
 
@@ -191,7 +227,7 @@ fs_status check_flags(fs_handle *h) {
     FS_CUDA(h, cudaMemcpyAsync(h->host_err, h->err, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
     FS_CUDA(h, cudaMemsetAsync(h->err, 0, sizeof(int), h->stream));
     FS_CUDA(h, cudaStreamSynchronize(h->stream));
-    const int e = *h->host_err;
+    const int e = h->host_err[0];
     if (e & fs::kDevErrTimeout) return fail(h, FS_ERR_TIMEOUT, "a bounded device wait timed out");
     if (e & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in a result or input");
     return FS_OK;
@@ -201,12 +237,12 @@ fs_status check_flags(fs_handle *h) {
 // h->red[slot][batch][8].
 fs_status measure(fs_handle *h, const float *f, const float *g, bool fdir, int slot, bool want_col_sum) {
     const fs_desc &D = h->desc;
-    FS_CUDA(h, run_bias(h, fdir ? g : f, fdir));
+    FS_LAUNCH(h, run_bias(h, fdir ? g : f, fdir));
     fs::PassParams p = make_pass(h, fdir, true);
     p.pot_in = fdir ? f : g;
-    FS_CUDA(h, run_pass(h, p, fdir, true));
+    FS_LAUNCH(h, run_pass(h, p, fdir, true));
     const int row_blocks = p.rows_pad / kBlockRows;
-    FS_CUDA(h, fs::launch_finalize(h->stats, D.batch, row_blocks, want_col_sum ? (fdir ? g : f) : nullptr,
+    FS_LAUNCH(h, fs::launch_finalize(h->stats, D.batch, row_blocks, want_col_sum ? (fdir ? g : f) : nullptr,
                                    fdir ? h->lb2 : h->la2, p.cols, p.cols_pad, h->red + (size_t)slot * D.batch * 8,
                                    h->stream));
     return FS_OK;
@@ -216,15 +252,14 @@ fs_status measure(fs_handle *h, const float *f, const float *g, bool fdir, int s
 
 extern "C" {
 
+unsigned long long fs_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
 const char *fs_last_error(const fs_handle *h) { return h ? h->last_error.c_str() : g_last_error.c_str(); }
 
 fs_status fs_destroy(fs_handle *h) {
     if (!h) return FS_OK;
     cudaSetDevice(h->device);
-    if (h->stream) cudaStreamSynchronize(h->stream);
-    if (h->block) cudaFree(h->block);
-    if (h->host_red) cudaFreeHost(h->host_red);
-    if (h->host_err) cudaFreeHost(h->host_err);
+    if (h->block) cudaFreeAsync(h->block, h->stream);  // stream-ordered: no device-wide sync
     delete h;
     return FS_OK;
 }
@@ -250,21 +285,21 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     h->desc = D;
     h->stream = static_cast<cudaStream_t>(stream);
     {
+        int major = 0, minor = 0;
         cudaError_t e = cudaGetDevice(&h->device);
-        cudaDeviceProp prop;
-        if (e == cudaSuccess) e = cudaGetDeviceProperties(&prop, h->device);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, h->device);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, h->device);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->device);
         if (e != cudaSuccess) {
             fail(nullptr, FS_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
             delete h;
             return FS_ERR_CUDA;
         }
-        if (prop.major != 10) {
-            fail(nullptr, FS_ERR_UNSUPPORTED, "device %s is sm_%d%d; this library is built for sm_100a", prop.name,
-                 prop.major, prop.minor);
+        if (major != 10) {
+            fail(nullptr, FS_ERR_UNSUPPORTED, "device is sm_%d%d; this library is built for sm_100a", major, minor);
             delete h;
             return FS_ERR_UNSUPPORTED;
         }
-        h->sms = prop.multiProcessorCount;
     }
     if (const char *env = getenv("FS_WAIT_TIMEOUT_MS")) {
         const long long ms = atoll(env);
@@ -351,15 +386,17 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     const size_t o_err = carve(16);
     h->bytes = off;
     {
-        cudaError_t e = cudaMalloc(&h->block, h->bytes);
-        if (e == cudaSuccess) e = cudaMallocHost((void **)&h->host_red, 2 * B * 8 * 8 + 4 * B * 8);
-        if (e == cudaSuccess) e = cudaMallocHost((void **)&h->host_err, 16);
+        cudaMemPool_t pool = nullptr;
+        cudaError_t e = device_pool(h->device, &pool);
+        if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&h->block, h->bytes, pool, h->stream);
         if (e != cudaSuccess) {
+            h->block = nullptr;
             fail(nullptr, e == cudaErrorMemoryAllocation ? FS_ERR_OOM : FS_ERR_CUDA, "allocation of %zu bytes: %s",
                  h->bytes, cudaGetErrorString(e));
             fs_destroy(h);
             return e == cudaErrorMemoryAllocation ? FS_ERR_OOM : FS_ERR_CUDA;
         }
+        h->host_red.assign(2 * B * 8 + 4 * B, 0.0);
     }
     char *base = static_cast<char *>(h->block);
     h->packX = base + o_packX;
@@ -386,18 +423,18 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         FS_CUDA(h, cudaMemsetAsync(h->err, 0, 16, h->stream));
         const float *t = nullptr;
         if (!bf16) {
-            FS_CUDA(h, fs::launch_center(X, Y, bf16, D.batch, D.n, D.m, D.d, h->center, h->stream));
+            FS_LAUNCH(h, fs::launch_center(X, Y, bf16, D.batch, D.n, D.m, D.d, h->center, h->stream));
             t = h->center;
         }
-        FS_CUDA(h, fs::launch_pack(X, bf16, D.n, h->n_pad, D.d, D.batch, t, 1.f, h->pack_mode, h->d_p, h->row_elems,
+        FS_LAUNCH(h, fs::launch_pack(X, bf16, D.n, h->n_pad, D.d, D.batch, t, 1.f, h->pack_mode, h->d_p, h->row_elems,
                                    h->packX, h->xn, h->err, h->stream));
-        FS_CUDA(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, 2.f, h->pack_mode, h->d_p, h->row_elems,
+        FS_LAUNCH(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, 2.f, h->pack_mode, h->d_p, h->row_elems,
                                    h->packY, h->yn, h->err, h->stream));
-        FS_CUDA(h, fs::launch_weights(a, D.batch, D.n, h->n_pad, h->la2, h->wstat, h->stream));
-        FS_CUDA(h, fs::launch_weights(b, D.batch, D.m, h->m_pad, h->lb2, h->wstat + 2 * B, h->stream));
-        FS_CUDA(h, fs::launch_fill(h->bias_row, B * h->n_pad, -INFINITY, h->stream));
-        FS_CUDA(h, fs::launch_fill(h->bias_col, B * h->m_pad, -INFINITY, h->stream));
-        double *hw = h->host_red + 2 * B * 8;
+        FS_LAUNCH(h, fs::launch_weights(a, D.batch, D.n, h->n_pad, h->la2, h->wstat, h->stream));
+        FS_LAUNCH(h, fs::launch_weights(b, D.batch, D.m, h->m_pad, h->lb2, h->wstat + 2 * B, h->stream));
+        FS_LAUNCH(h, fs::launch_fill(h->bias_row, B * h->n_pad, -INFINITY, h->stream));
+        FS_LAUNCH(h, fs::launch_fill(h->bias_col, B * h->m_pad, -INFINITY, h->stream));
+        double *hw = h->host_red.data() + 2 * B * 8;
         FS_CUDA(h, cudaMemcpyAsync(hw, h->wstat, 4 * B * 8, cudaMemcpyDeviceToHost, h->stream));
         FS_CUDA(h, cudaMemcpyAsync(h->host_err, h->err, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
         FS_CUDA(h, cudaMemsetAsync(h->err, 0, 16, h->stream));
@@ -409,7 +446,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
                 return fail(h, FS_ERR_INVALID_ARG, "weights %s of problem %zu must be positive and sum to 1 (sum=%.9g)",
                             is_a ? "a" : "b", is_a ? k : k - B, s);
         }
-        if (*h->host_err & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in X or Y");
+        if (h->host_err[0] & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in X or Y");
         if (prec != FS_PREC_F32_SIMT) {
             fs_status s2 = encode_map(h, &h->mapX, h->packX, D.batch * h->n_pad);
             if (s2 != FS_OK) return s2;
@@ -449,27 +486,27 @@ fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule sche
     if (schedule == FS_SCHED_ALTERNATING) {
         // One bias launch from the initial g; afterwards every pass's fused
         // epilogue writes the bias the next pass reads.
-        FS_CUDA(h, run_bias(h, g, true));
+        FS_LAUNCH(h, run_bias(h, g, true));
         for (int it = 0; it < iters; ++it) {
             fs::PassParams pf = make_pass(h, true, false);
             pf.pot_out = f;
             pf.next_bias = h->bias_row;
-            FS_CUDA(h, run_pass(h, pf, true, false));
+            FS_LAUNCH(h, run_pass(h, pf, true, false));
             fs::PassParams pg = make_pass(h, false, false);
             pg.pot_out = g;
             pg.next_bias = h->bias_col;
-            FS_CUDA(h, run_pass(h, pg, false, false));
+            FS_LAUNCH(h, run_pass(h, pg, false, false));
         }
     } else {
         for (int it = 0; it < iters; ++it) {
-            FS_CUDA(h, run_bias(h, g, true));
-            FS_CUDA(h, run_bias(h, f, false));
+            FS_LAUNCH(h, run_bias(h, g, true));
+            FS_LAUNCH(h, run_bias(h, f, false));
             fs::PassParams pf = make_pass(h, true, false);
             pf.pot_out = f;
-            FS_CUDA(h, run_pass(h, pf, true, false));
+            FS_LAUNCH(h, run_pass(h, pf, true, false));
             fs::PassParams pg = make_pass(h, false, false);
             pg.pot_out = g;
-            FS_CUDA(h, run_pass(h, pg, false, false));
+            FS_LAUNCH(h, run_pass(h, pg, false, false));
         }
     }
     return FS_OK;
@@ -487,7 +524,7 @@ fs_status fs_marginal_err(fs_handle *h, const float *f, const float *g, double *
         fs_status s = measure(h, f, g, false, 1, false);
         if (s != FS_OK) return s;
     }
-    FS_CUDA(h, cudaMemcpyAsync(h->host_red, h->red, 2 * B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
+    FS_CUDA(h, cudaMemcpyAsync(h->host_red.data(), h->red, 2 * B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
     fs_status s = check_flags(h);
     if (s != FS_OK) return s;
     for (size_t k = 0; k < B; ++k) {
@@ -503,12 +540,12 @@ fs_status fs_ot_cost(fs_handle *h, const float *f, const float *g, double *dual,
     const size_t B = (size_t)h->desc.batch;
     fs_status s = measure(h, f, g, true, 0, true);
     if (s != FS_OK) return s;
-    FS_CUDA(h, cudaMemcpyAsync(h->host_red, h->red, B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
+    FS_CUDA(h, cudaMemcpyAsync(h->host_red.data(), h->red, B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
     s = check_flags(h);
     if (s != FS_OK) return s;
     const double eps = (double)h->desc.eps;
     for (size_t k = 0; k < B; ++k) {
-        const double *r = h->host_red + k * 8;  // [|r-a|, sum r, sum r*meanC, <a,f>, <b,g>]
+        const double *r = h->host_red.data() + k * 8;  // [|r-a|, sum r, sum r*meanC, <a,f>, <b,g>]
         if (dual) dual[k] = r[3] + r[4] - eps * (r[1] - 1.0);
         if (primal) primal[k] = r[2];
     }
@@ -551,7 +588,11 @@ fs_status fs_solve_host(const fs_desc *desc, const void *X_host, const void *Y_h
     const size_t bx = B * D.n * D.d * es, by = B * D.m * D.d * es, bf = B * D.n * 4, bg = B * D.m * 4;
     const size_t total = align256(bx) + align256(by) + 2 * align256(bf) + 2 * align256(bg);
     char *blk = nullptr;
-    cudaError_t e = cudaMallocAsync((void **)&blk, total, s);
+    int dev = 0;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = device_pool(dev, &pool);
+    if (e == cudaSuccess) e = cudaMallocFromPoolAsync((void **)&blk, total, pool, s);
     if (e != cudaSuccess)
         return fail(nullptr, e == cudaErrorMemoryAllocation ? FS_ERR_OOM : FS_ERR_CUDA, "cudaMallocAsync: %s",
                     cudaGetErrorString(e));

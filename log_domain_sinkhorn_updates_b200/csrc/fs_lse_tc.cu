@@ -7,8 +7,8 @@
 // `stages`-deep TMA ring.  For every column tile one thread issues the
 // tcgen05.mma chain S = Q K^T into one of two TMEM accumulators (128 lanes x
 // 128 fp32 columns each), so the MMA of tile t+1 overlaps the exponentials of
-// tile t.  Eight "softmax" warps (two per TMEM lane quadrant, each taking 64
-// of the 128 columns) read S with tcgen05.ld, form
+// tile t.  Eight "softmax" warps (two per TMEM lane quadrant; one group of
+// four takes the even tiles, the other the odd ones) read S with tcgen05.ld, form
 //   z_ij = S_ij * log2(e)/eps + beta_j        (beta_j staged next to the K tile)
 // and update a per-row online maximum and sum of 2^(z - max) in registers
 // (online LSE, section 2).  Nothing of size n*m ever leaves the SM: the pass
@@ -31,6 +31,9 @@ namespace fs {
 namespace {
 
 constexpr int kThreads = 320;
+// Largest growth (base 2) of a row's maximum that is absorbed without a
+// rescale: terms up to 2^kLazy stay in the running sum as they are.
+constexpr float kLazy = 12.f;
 constexpr int kTmemCols = 256;  // two 128-column fp32 accumulators
 
 __device__ __forceinline__ uint32_t saddr(const void *p) {
@@ -154,6 +157,24 @@ __device__ __forceinline__ uint32_t make_idesc() {
            ((uint32_t)(kBlockRows >> 4) << 24);
 }
 
+// sum_k 2^(z_k - ref) over a 128-column tile, fp32 pairs.
+__device__ __forceinline__ float sum_exp2_tile(const float (&z)[128], float ref) {
+    const uint64_t rn = pack2(-ref, -ref);
+    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int k = 0; k < 128; k += 2) {
+        float d0, d1;
+        unpack2(add2(pack2(z[k], z[k + 1]), rn), d0, d1);
+        acc[(k / 2) & 3] = add2(acc[(k / 2) & 3], pack2(ex2_approx(d0), ex2_approx(d1)));
+    }
+    float a0, a1, a2, a3, a4, a5, a6, a7;
+    unpack2(acc[0], a0, a1);
+    unpack2(acc[1], a2, a3);
+    unpack2(acc[2], a4, a5);
+    unpack2(acc[3], a6, a7);
+    return ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+}
+
 struct SmemLayout {
     uint32_t q, k, bias, cnorm, merge, red, bars, misc, total;
 };
@@ -211,12 +232,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(empty + s, 1 + 8);  // MMA commit + the eight softmax warps
+            mbar_init(empty + s, 1 + 4);  // MMA commit + the four warps of the tile's group
         }
         mbar_init(qfull, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(sfull + b, 1);
-            mbar_init(sempty + b, 8);
+            mbar_init(sempty + b, 4);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -324,84 +345,158 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ---------------- softmax warps ----------------
+        // Group 0 (warps 2..5) takes the even tiles, which the MMA writes to TMEM
+        // buffer 0; group 1 (warps 6..9) the odd tiles in buffer 1.  The two
+        // warps sharing an SM sub-partition therefore work on different tiles
+        // and their max / exp phases interleave on the MUFU.
         const int q = warp & 3;          // TMEM lane quadrant this warp may access
-        const int h = (warp - 2) >> 2;   // which 64-column half of each tile
+        const int grp = (warp - 2) >> 2; // tile parity handled by this warp
         const int rl = q * 32 + lane;    // row within the block
         const float c = p.scale2;
         const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_pad + rb * kBlockRows + rl] : 0.f;
         float m = -INFINITY, l = 0.f, w = 0.f;
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 64);
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * kBlockCols);
         bool ok = true;
-        for (int t = 0; t < ntiles; ++t) {
+        for (int t = grp; t < ntiles; t += 2) {
             const int s = t % NST;
             const uint32_t ph = (uint32_t)(t / NST) & 1u;
-            const int b = t & 1;
             const uint32_t bph = (uint32_t)(t >> 1) & 1u;
-            if (!mbar_wait(sfull + b, bph, p.timeout_ns)) {
+            if (!mbar_wait(sfull + grp, bph, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            uint32_t r0[32], r1[32];
-            tmem_ld32(taddr + (uint32_t)(b * kBlockCols), r0);
-            tmem_ld32(taddr + (uint32_t)(b * kBlockCols) + 32u, r1);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sempty + b);
-            // The bias slice arrived with the K tile; make its bytes visible here too.
-            if (!mbar_wait(full + s, ph, p.timeout_ns)) {
-                ok = false;
-                break;
-            }
-            const float4 *bq = reinterpret_cast<const float4 *>(sBias + s * kBlockCols + h * 64);
-            const float4 *cq = reinterpret_cast<const float4 *>(sCN + s * kBlockCols + h * 64);
-            float sv[64], z[64];
+            if (!MEASURE) {
+                uint32_t r[128];
+                tmem_ld32(taddr + 0u, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                tmem_ld32(taddr + 32u, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+                tmem_ld32(taddr + 64u, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+                tmem_ld32(taddr + 96u, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sempty + grp);
+                // the bias slice arrived with the K tile; make its bytes visible here too
+                if (!mbar_wait(full + s, ph, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                const float4 *bq = reinterpret_cast<const float4 *>(sBias + s * kBlockCols);
+                const uint64_t cc = pack2(c, c);
+                float z[128];
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                sv[k] = __uint_as_float(r0[k]);
-                sv[32 + k] = __uint_as_float(r1[k]);
-            }
-            float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
+                for (int k = 0; k < 128; k += 4) {
+                    const float4 bb = bq[k / 4];
+                    unpack2(fma2(pack2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), cc, pack2(bb.x, bb.y)),
+                            z[k], z[k + 1]);
+                    unpack2(fma2(pack2(__uint_as_float(r[k + 2]), __uint_as_float(r[k + 3])), cc, pack2(bb.z, bb.w)),
+                            z[k + 2], z[k + 3]);
+                }
+                if (m == -INFINITY) {
+                    // first tile of this warp: two passes (max, then exponentials)
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int k = 0; k < 64; k += 4) {
-                const float4 bb = bq[k / 4];
-                z[k + 0] = fmaf(sv[k + 0], c, bb.x);
-                z[k + 1] = fmaf(sv[k + 1], c, bb.y);
-                z[k + 2] = fmaf(sv[k + 2], c, bb.z);
-                z[k + 3] = fmaf(sv[k + 3], c, bb.w);
-                t0 = fmaxf(t0, z[k + 0]);
-                t1 = fmaxf(t1, z[k + 1]);
-                t2 = fmaxf(t2, z[k + 2]);
-                t3 = fmaxf(t3, z[k + 3]);
-            }
-            const float mnew = fmaxf(m, fmaxf(fmaxf(t0, t1), fmaxf(t2, t3)));
-            if (mnew != -INFINITY) {
-                const float scale = ex2_approx(m - mnew);
-                float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                float w0 = 0.f, w1 = 0.f;
+                    for (int k = 0; k < 128; k += 8) {
+                        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k], z[k + 1]);
+                        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 2], z[k + 3]);
+                        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 4], z[k + 5]);
+                        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 6], z[k + 7]);
+                    }
+                    const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                    if (tmax != -INFINITY) {
+                        l = sum_exp2_tile(z, tmax);
+                        m = tmax;
+                    }
+                } else {
+                    // Later tiles: exponentials relative to the running max as it
+                    // stood, the tile max alongside (no dependency between the two).
+                    // Terms up to 2^kLazy are kept as they are; a larger jump of the
+                    // maximum redoes the tile against the new maximum.
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    const uint64_t mneg = pack2(-m, -m);
+                    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int k = 0; k < 64; k += 4) {
-                    const float e0 = ex2_approx(z[k + 0] - mnew);
-                    const float e1 = ex2_approx(z[k + 1] - mnew);
-                    const float e2 = ex2_approx(z[k + 2] - mnew);
-                    const float e3 = ex2_approx(z[k + 3] - mnew);
-                    a0 += e0;
-                    a1 += e1;
-                    a2 += e2;
-                    a3 += e3;
-                    if (MEASURE) {
-                        // C_ij = |row|^2 + |col|^2 - S_ij
-                        const float4 cn = cq[k / 4];
-                        w0 = fmaf(e0, xn + cn.x - sv[k + 0], w0);
-                        w1 = fmaf(e1, xn + cn.y - sv[k + 1], w1);
-                        w0 = fmaf(e2, xn + cn.z - sv[k + 2], w0);
-                        w1 = fmaf(e3, xn + cn.w - sv[k + 3], w1);
+                    for (int k = 0; k < 128; k += 2) {
+                        float d0, d1;
+                        unpack2(add2(pack2(z[k], z[k + 1]), mneg), d0, d1);
+                        acc[(k / 2) & 3] = add2(acc[(k / 2) & 3], pack2(ex2_approx(d0), ex2_approx(d1)));
+                        mx[(k / 2) & 3] = max3(mx[(k / 2) & 3], z[k], z[k + 1]);
+                    }
+                    const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                    if (tmax > m + kLazy) {
+                        l = l * ex2_approx(m - tmax) + sum_exp2_tile(z, tmax);
+                        m = tmax;
+                    } else {
+                        float a0, a1, a2, a3, a4, a5, a6, a7;
+                        unpack2(acc[0], a0, a1);
+                        unpack2(acc[1], a2, a3);
+                        unpack2(acc[2], a4, a5);
+                        unpack2(acc[3], a6, a7);
+                        l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
                     }
                 }
-                l = l * scale + ((a0 + a1) + (a2 + a3));
-                if (MEASURE) w = w * scale + (w0 + w1);
-                m = mnew;
+            } else {
+                // measure passes also need the raw score (C_ij = |row|^2 + |col|^2 - S_ij);
+                // they run once per solve, so take the tile in two 64-column halves.
+                if (!mbar_wait(full + s, ph, p.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t ra[32], rb2[32];
+                    tmem_ld32(taddr + 64u * half, ra);
+                    tmem_ld32(taddr + 64u * half + 32u, rb2);
+                    tmem_ld_wait();
+                    if (half == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(sempty + grp);
+                    }
+                    const float4 *bq = reinterpret_cast<const float4 *>(sBias + s * kBlockCols + half * 64);
+                    const float4 *cq = reinterpret_cast<const float4 *>(sCN + s * kBlockCols + half * 64);
+                    float sv[64], z[64];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        sv[k] = __uint_as_float(ra[k]);
+                        sv[32 + k] = __uint_as_float(rb2[k]);
+                    }
+                    float t0 = -INFINITY, t1 = -INFINITY, t2 = -INFINITY, t3 = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < 64; k += 4) {
+                        const float4 bb = bq[k / 4];
+                        z[k + 0] = fmaf(sv[k + 0], c, bb.x);
+                        z[k + 1] = fmaf(sv[k + 1], c, bb.y);
+                        z[k + 2] = fmaf(sv[k + 2], c, bb.z);
+                        z[k + 3] = fmaf(sv[k + 3], c, bb.w);
+                        t0 = fmaxf(t0, z[k + 0]);
+                        t1 = fmaxf(t1, z[k + 1]);
+                        t2 = fmaxf(t2, z[k + 2]);
+                        t3 = fmaxf(t3, z[k + 3]);
+                    }
+                    const float mnew = fmaxf(m, fmaxf(fmaxf(t0, t1), fmaxf(t2, t3)));
+                    if (mnew != -INFINITY) {
+                        const float scale = ex2_approx(m - mnew);
+                        float a0 = 0.f, a1 = 0.f, w0 = 0.f, w1 = 0.f;
+#pragma unroll
+                        for (int k = 0; k < 64; k += 4) {
+                            const float4 cn = cq[k / 4];
+                            const float e0 = ex2_approx(z[k + 0] - mnew);
+                            const float e1 = ex2_approx(z[k + 1] - mnew);
+                            const float e2 = ex2_approx(z[k + 2] - mnew);
+                            const float e3 = ex2_approx(z[k + 3] - mnew);
+                            a0 += e0 + e2;
+                            a1 += e1 + e3;
+                            w0 = fmaf(e0, xn + cn.x - sv[k + 0], w0);
+                            w1 = fmaf(e1, xn + cn.y - sv[k + 1], w1);
+                            w0 = fmaf(e2, xn + cn.z - sv[k + 2], w0);
+                            w1 = fmaf(e3, xn + cn.w - sv[k + 3], w1);
+                        }
+                        l = l * scale + (a0 + a1);
+                        w = w * scale + (w0 + w1);
+                        m = mnew;
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty + s);
@@ -411,10 +506,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicOr(p.err, kDevErrTimeout);
             *abort_flag = 1;
         }
-        // Merge the two column halves of each row, then finish the row block.
-        if (h == 1) sMerge[rl] = make_float4(m, l, w, 0.f);
+        // Merge the two tile-parity groups' states of each row, then finish the row block.
+        if (grp == 1) sMerge[rl] = make_float4(m, l, w, 0.f);
         named_barrier(1, 256);
-        if (h == 0) {
+        if (grp == 0) {
             const float4 o = sMerge[rl];
             lse_merge(m, l, w, o.x, o.y, o.z);
             finish_rows<MEASURE>(p, rl, m, l, w, 2, sRed, flag);
