@@ -178,6 +178,28 @@ FS_API fs_status fs_solve_host(const fs_desc *desc, const void *X_host, const vo
                         float *g_host, int iters, fs_schedule schedule, double *err_row,
                         double *err_col, double *dual, double *primal, void *stream);
 
+/*
+ * One f-update that allocates nothing (no counterpart on the pages: an
+ * interface for callers that cannot allocate device memory when they need
+ * an update -- inside CUDA graph capture, in plug-ins whose host framework
+ * owns all device memory, or in latency-critical loops).
+ * Inputs: device X [n][d], Y [m][d] (fp32, row-major), b [m] (NULL = uniform
+ * 1/m), g [m]; output: device f [n], with
+ *   f_i = |x_i|^2 - eps LSE_j[(2 x_i.y_j + g_j - |y_j|^2)/eps + log b_j].
+ * Computed in plain fp32 on CUDA cores on the uncentred inputs, enqueued on
+ * `stream` (a cudaStream_t, NULL = legacy default); returns without waiting.
+ * Scratch (squared norms and the column bias) is a fixed 4 MiB device array
+ * inside the library, held by every GPU that loads it until the process
+ * exits, so: n_pad + m + m_pad <= 1048576 (n_pad, m_pad = n, m rounded up to
+ * 128) and d <= 256, else FS_ERR_INVALID_ARG; all calls on a device share the
+ * array, so calls that overlap on the GPU race -- order them on one stream.
+ * The first call on each device looks up the array's address and sets a
+ * kernel attribute: make it before any stream capture.  Errors: return
+ * codes, message in fs_last_error(NULL).
+ */
+FS_API fs_status fs_update_f_noalloc(int n, int m, int d, float eps, const float *X, const float *Y,
+                                     const float *b, const float *g, float *f, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

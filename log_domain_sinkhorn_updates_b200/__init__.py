@@ -10,7 +10,7 @@ be imported on machines without the built library.
 import importlib
 
 __all__ = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_err", "fs_ot_cost", "fs_sync",
-           "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches", "FsError", "Handle"]
+           "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches", "fs_update_f_noalloc", "FsError", "Handle"]
 
 
 def __getattr__(name):

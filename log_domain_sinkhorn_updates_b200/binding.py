@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_CUDA", 3: "FS_ER
                 4: "FS_ERR_NONFINITE", 5: "FS_ERR_TIMEOUT", 6: "FS_ERR_OOM"}
 
 EXPORTS = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_err", "fs_ot_cost",
-           "fs_sync", "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches"]
+           "fs_sync", "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches",
+           "fs_update_f_noalloc"]
 
 
 class FsDesc(ctypes.Structure):
@@ -75,6 +76,8 @@ def lib():
         L.fs_last_error.restype = ctypes.c_char_p
         L.fs_solve_host.argtypes = [ctypes.POINTER(FsDesc), vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int,
                                     dp, dp, dp, dp, vp]
+        L.fs_update_f_noalloc.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, vp, vp, vp, vp,
+                                          vp, vp]
         L.fs_kernel_launches.argtypes = []
         L.fs_kernel_launches.restype = ctypes.c_ulonglong
         for name in EXPORTS:
@@ -212,6 +215,17 @@ def fs_destroy(h: Handle):
 def fs_last_error(h: Handle = None) -> str:
     msg = lib().fs_last_error(h.ptr if h is not None else None)
     return msg.decode() if msg else ""
+
+
+def fs_update_f_noalloc(X, Y, b, g, f, eps, stream=None):
+    """One f-update through the allocation-free entry point: X [n, d], Y [m, d] float32 CUDA
+    tensors, b [m] or None (uniform), g [m], output f [n].  Asynchronous on the stream."""
+    if X.dim() != 2 or Y.dim() != 2 or X.shape[1] != Y.shape[1]:
+        raise ValueError("X [n, d] and Y [m, d] expected")
+    n, d = X.shape
+    m = Y.shape[0]
+    _check(lib().fs_update_f_noalloc(n, m, d, float(eps), _f32(X), _f32(Y), _f32(b), _f32(g), _f32(f),
+                                     _stream_ptr(stream)))
 
 
 def fs_kernel_launches() -> int:

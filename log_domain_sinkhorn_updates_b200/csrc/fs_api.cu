@@ -250,6 +250,8 @@ fs_status measure(fs_handle *h, const float *f, const float *g, bool fdir, int s
 
 }  // namespace
 
+void fs::set_thread_error(const char *msg) { g_last_error = msg; }
+
 extern "C" {
 
 unsigned long long fs_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }

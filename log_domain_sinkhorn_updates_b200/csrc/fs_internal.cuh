@@ -130,5 +130,7 @@ cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec
                           const void *map_rows, const void *map_cols, size_t smem_bytes,
                           cudaStream_t s);
 size_t tc_smem_bytes(int row_bytes, int stages, bool measure);
+// Record msg as this thread's handle-less error (what fs_last_error(NULL) returns).
+void set_thread_error(const char *msg);
 int tc_max_stages(int row_bytes, bool measure);
 }  // namespace fs
