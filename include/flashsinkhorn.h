@@ -54,13 +54,19 @@ typedef enum {
 
 typedef enum { FS_F32 = 0, FS_BF16 = 1 } fs_dtype; /* element type of X and Y */
 
-/* Operand precision of the score product X Y^T (accumulation is always fp32). */
+/* Operand precision of the score product X Y^T (accumulation is always fp32).
+ * The tensor-core modes need packed rows of at most 512 bytes: d <= 256 for
+ * BF16, d <= 128 for TF32 and 3XF16, d <= 64 for 3XTF32 (FS_ERR_UNSUPPORTED
+ * beyond). */
 typedef enum {
-    FS_PREC_AUTO = 0,     /* BF16 for bf16 inputs, 3XTF32 for fp32 inputs             */
+    FS_PREC_AUTO = 0,     /* BF16 for bf16 inputs; 3XF16 for fp32 inputs with d <= 128,
+                             else F32_SIMT (d <= 256)                                */
     FS_PREC_BF16 = 1,     /* one bf16 tensor-core pass (exact for bf16 inputs)        */
     FS_PREC_TF32 = 2,     /* one tf32 tensor-core pass                                */
     FS_PREC_3XTF32 = 3,   /* hi*hi + lo*hi + hi*lo tf32 passes (~fp32 accurate)       */
-    FS_PREC_F32_SIMT = 5  /* plain fp32 FMA on CUDA cores (validation path)           */
+    FS_PREC_3XF16 = 4,    /* the same three passes on fp16 hi/lo planes, power-of-two
+                             scaled per cloud (~fp32 accurate, half the MMAs)         */
+    FS_PREC_F32_SIMT = 5  /* plain fp32 FMA on CUDA cores (validation path, d <= 256) */
 } fs_precision;
 
 typedef enum {
@@ -90,6 +96,7 @@ typedef struct {
     int launches_update;    /* kernel launches of one fs_update_f / fs_update_g */
     int launches_solve_iter;/* kernel launches per fs_solve iteration           */
     size_t device_bytes;    /* device memory owned by the handle                */
+    int cta_pair;           /* 1: each MMA spans a pair of SMs (tcgen05 cta_group::2) */
 } fs_info;
 
 /*

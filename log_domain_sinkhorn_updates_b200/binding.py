@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libflashsinkhorn.so")
 
 FS_OK, FS_ERR_INVALID_ARG, FS_ERR_CUDA, FS_ERR_UNSUPPORTED, FS_ERR_NONFINITE, FS_ERR_TIMEOUT, FS_ERR_OOM = range(7)
 FS_F32, FS_BF16 = 0, 1
-PRECISIONS = {"auto": 0, "bf16": 1, "tf32": 2, "3xtf32": 3, "f32_simt": 5}
+PRECISIONS = {"auto": 0, "bf16": 1, "tf32": 2, "3xtf32": 3, "3xf16": 4, "f32_simt": 5}
 PRECISION_NAMES = {v: k for k, v in PRECISIONS.items()}
 SCHEDULES = {"alternating": 0, "symmetric": 1}
 STATUS_NAMES = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_CUDA", 3: "FS_ERR_UNSUPPORTED",
@@ -38,7 +38,7 @@ class FsInfo(ctypes.Structure):
                 ("swizzle_bytes", ctypes.c_int), ("stages", ctypes.c_int), ("block_rows", ctypes.c_int),
                 ("block_cols", ctypes.c_int), ("splits_f", ctypes.c_int), ("splits_g", ctypes.c_int),
                 ("launches_update", ctypes.c_int), ("launches_solve_iter", ctypes.c_int),
-                ("device_bytes", ctypes.c_size_t)]
+                ("device_bytes", ctypes.c_size_t), ("cta_pair", ctypes.c_int)]
 
     def as_dict(self):
         d = {k: getattr(self, k) for k, _ in self._fields_}

@@ -44,11 +44,14 @@ struct fs_handle {
     int *err = nullptr;
     std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
     int host_err[4] = {0, 0, 0, 0};
-    CUtensorMap mapX{}, mapY{};
+    CUtensorMap mapX_r{}, mapX_c{}, mapY_r{}, mapY_c{};  // row-side (128-row box) / column-side (256-row box)
     int splits_f = 1, tps_f = 1, splits_g = 1, tps_g = 1;
     int stages = 2, stages_meas = 2;
+    bool pair = false;  // run the passes on CTA pairs (one MMA over two SMs); FS_CTA_PAIR=1
     size_t smem = 0, smem_meas = 0;
     unsigned long long timeout_ns = 2000000000ull;
+    float sscale = 1.f;             // raw MMA score -> S_ij (3xF16 operand scaling)
+    float qscale = 1.f, kscale = 1.f;  // power-of-two operand scales (3xF16)
     std::string last_error;
 };
 
@@ -149,13 +152,15 @@ void plan_splits(int row_blocks, int col_tiles, int sms, int *splits, int *tps) 
     }
 }
 
-fs_status encode_map(fs_handle *h, CUtensorMap *map, void *base, int rows_total) {
+fs_status encode_map(fs_handle *h, CUtensorMap *map, void *base, int rows_total, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
-    const CUtensorMapDataType dt = h->elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapDataType dt = h->elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : (h->prec == FS_PREC_3XF16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     cuuint64_t gdim[2] = {(cuuint64_t)(h->row_bytes / h->elem), (cuuint64_t)rows_total};
     cuuint64_t gstride[1] = {(cuuint64_t)h->row_bytes};
-    cuuint32_t box[2] = {(cuuint32_t)(h->swz / h->elem), (cuuint32_t)kBlockRows};
+    cuuint32_t box[2] = {(cuuint32_t)(h->swz / h->elem), (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     const CUtensorMapSwizzle sw = h->swz == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : h->swz == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -182,7 +187,8 @@ fs::PassParams make_pass(const fs_handle *h, bool fdir, bool measure) {
     p.col_tiles = p.cols_pad / kBlockCols;
     p.stages = measure ? h->stages_meas : h->stages;
     p.eps = (double)D.eps;
-    p.scale2 = (float)(fs::kLog2ed / (double)D.eps);
+    p.scale2 = (float)(fs::kLog2ed / (double)D.eps * (double)h->sscale);
+    p.sscale = h->sscale;
     p.col_bias = fdir ? h->bias_col : h->bias_row;
     p.row_norm = fdir ? h->xn : h->yn;
     p.row_logw2 = fdir ? h->la2 : h->lb2;
@@ -199,8 +205,11 @@ fs::PassParams make_pass(const fs_handle *h, bool fdir, bool measure) {
 
 cudaError_t run_pass(fs_handle *h, const fs::PassParams &p, bool fdir, bool measure) {
     if (h->prec == FS_PREC_F32_SIMT) return fs::launch_lse_simt(p, h->desc.batch, measure, h->stream);
-    const CUtensorMap *mr = fdir ? &h->mapX : &h->mapY;
-    const CUtensorMap *mc = fdir ? &h->mapY : &h->mapX;
+    if (h->pair)  // 128-row boxes for both roles: each CTA of a pair loads half of a 256-column tile
+        return fs::launch_lse_tc2(p, h->desc.batch, measure, h->prec, fdir ? &h->mapX_r : &h->mapY_r,
+                                  fdir ? &h->mapY_r : &h->mapX_r, measure ? h->smem_meas : h->smem, h->stream);
+    const CUtensorMap *mr = fdir ? &h->mapX_r : &h->mapY_r;
+    const CUtensorMap *mc = fdir ? &h->mapY_c : &h->mapX_c;
     return fs::launch_lse_tc(p, h->desc.batch, measure, h->prec, mr, mc, measure ? h->smem_meas : h->smem,
                              h->stream);
 }
@@ -278,7 +287,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         return fail(nullptr, FS_ERR_INVALID_ARG, "eps must be finite and > 0");
     if (D.dtype != FS_F32 && D.dtype != FS_BF16) return fail(nullptr, FS_ERR_INVALID_ARG, "unknown dtype");
     if (D.prec != FS_PREC_AUTO && D.prec != FS_PREC_BF16 && D.prec != FS_PREC_TF32 && D.prec != FS_PREC_3XTF32 &&
-        D.prec != FS_PREC_F32_SIMT)
+        D.prec != FS_PREC_3XF16 && D.prec != FS_PREC_F32_SIMT)
         return fail(nullptr, FS_ERR_INVALID_ARG, "unknown precision");
     if ((long long)D.batch * (D.n + 127) > (1LL << 31) || (long long)D.batch * (D.m + 127) > (1LL << 31))
         return fail(nullptr, FS_ERR_UNSUPPORTED, "batch * rows exceeds 2^31");
@@ -310,7 +319,8 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
 
     // ---- precision and packed layout ----
     int prec = D.prec;
-    if (prec == FS_PREC_AUTO) prec = D.dtype == FS_BF16 ? FS_PREC_BF16 : FS_PREC_3XTF32;
+    if (prec == FS_PREC_AUTO)
+        prec = D.dtype == FS_BF16 ? FS_PREC_BF16 : (D.d <= 128 ? FS_PREC_3XF16 : FS_PREC_F32_SIMT);
     h->prec = prec;
     if (prec == FS_PREC_F32_SIMT) {
         if (D.d > 256) {
@@ -327,9 +337,9 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         h->pack_mode = fs::kPackPlain;
         h->row_elems = D.d;
     } else {
-        h->elem = prec == FS_PREC_BF16 ? 2 : 4;
-        h->planes = prec == FS_PREC_3XTF32 ? 2 : 1;
-        const int kstep = prec == FS_PREC_BF16 ? 16 : 8;  // elements per 32-byte MMA K slice
+        h->elem = (prec == FS_PREC_BF16 || prec == FS_PREC_3XF16) ? 2 : 4;
+        h->planes = (prec == FS_PREC_3XTF32 || prec == FS_PREC_3XF16) ? 2 : 1;
+        const int kstep = 32 / h->elem;  // elements per 32-byte MMA K slice
         h->d_p = round_up(D.d, kstep);
         h->plane_bytes = h->d_p * h->elem;
         const int used = h->planes * h->plane_bytes;
@@ -343,23 +353,38 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             h->row_bytes = round_up(used, 128);
             h->swz = 128;
         }
-        h->pack_mode = prec == FS_PREC_BF16 ? fs::kPackBf16 : (prec == FS_PREC_TF32 ? fs::kPackTf32 : fs::kPack3xTf32);
+        h->pack_mode = prec == FS_PREC_BF16    ? fs::kPackBf16
+                       : prec == FS_PREC_TF32  ? fs::kPackTf32
+                       : prec == FS_PREC_3XF16 ? fs::kPack3xF16
+                                               : fs::kPack3xTf32;
         h->row_elems = h->row_bytes / h->elem;
-        h->stages = fs::tc_max_stages(h->row_bytes, false);
-        h->stages_meas = fs::tc_max_stages(h->row_bytes, true);
-        if (h->stages < 2 || h->stages_meas < 2) {
+        if (const char *env = getenv("FS_CTA_PAIR")) h->pair = atoi(env) != 0;
+        if (h->row_bytes > 512) {  // four swizzle atoms: the kernels' per-tile descriptor table
             fail(nullptr, FS_ERR_UNSUPPORTED,
                  "d=%d needs %d-byte operand rows; the tensor-core pass supports rows up to 512 bytes "
-                 "(bf16 d<=256, tf32 d<=128, 3xTF32 d<=64)",
+                 "(bf16 d<=256, tf32 and 3xF16 d<=128, 3xTF32 d<=64)",
                  D.d, h->row_bytes);
             delete h;
             return FS_ERR_UNSUPPORTED;
         }
-        h->smem = fs::tc_smem_bytes(h->row_bytes, h->stages, false);
-        h->smem_meas = fs::tc_smem_bytes(h->row_bytes, h->stages_meas, true);
+        h->stages = h->pair ? fs::tc2_max_stages(h->row_bytes, false) : fs::tc_max_stages(h->row_bytes, false);
+        h->stages_meas = h->pair ? fs::tc2_max_stages(h->row_bytes, true) : fs::tc_max_stages(h->row_bytes, true);
+        if (h->stages < 2 || h->stages_meas < 2) {
+            fail(nullptr, FS_ERR_UNSUPPORTED,
+                 "d=%d needs %d-byte operand rows; the single-CTA tensor-core pass supports rows up to "
+                 "256 bytes (bf16 d<=128, tf32 and 3xF16 d<=64, 3xTF32 d<=32)",
+                 D.d, h->row_bytes);
+            delete h;
+            return FS_ERR_UNSUPPORTED;
+        }
+        h->smem = h->pair ? fs::tc2_smem_bytes(h->row_bytes, h->stages, false)
+                          : fs::tc_smem_bytes(h->row_bytes, h->stages, false);
+        h->smem_meas = h->pair ? fs::tc2_smem_bytes(h->row_bytes, h->stages_meas, true)
+                               : fs::tc_smem_bytes(h->row_bytes, h->stages_meas, true);
     }
-    h->n_pad = round_up(D.n, kBlockRows);
-    h->m_pad = round_up(D.m, kBlockRows);
+    // Both clouds serve as rows (128-row blocks) and as columns (256-column tiles).
+    h->n_pad = round_up(D.n, kBlockCols);
+    h->m_pad = round_up(D.m, kBlockCols);
     plan_splits(D.batch * (h->n_pad / kBlockRows), h->m_pad / kBlockCols, h->sms, &h->splits_f, &h->tps_f);
     plan_splits(D.batch * (h->m_pad / kBlockRows), h->n_pad / kBlockCols, h->sms, &h->splits_g, &h->tps_g);
 
@@ -384,7 +409,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     const size_t o_ctr = carve(B * max_rb * 4);
     const size_t o_stats = carve(B * max_rb * 4 * 8);
     const size_t o_red = carve(2 * B * 8 * 8);
-    const size_t o_wstat = carve(2 * B * 2 * 8);
+    const size_t o_wstat = carve(2 * B * 2 * 8 + 16);
     const size_t o_err = carve(16);
     h->bytes = off;
     {
@@ -428,9 +453,27 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             FS_LAUNCH(h, fs::launch_center(X, Y, bf16, D.batch, D.n, D.m, D.d, h->center, h->stream));
             t = h->center;
         }
-        FS_LAUNCH(h, fs::launch_pack(X, bf16, D.n, h->n_pad, D.d, D.batch, t, 1.f, h->pack_mode, h->d_p, h->row_elems,
+        if (h->pack_mode == fs::kPack3xF16) {
+            // Power-of-two scales putting each cloud's largest |value| (Y side
+            // counted with its factor 2) at most 2^14: exact, and far from the
+            // fp16 overflow; the MMA's raw score is divided back by their product.
+            float *mx = reinterpret_cast<float *>(h->wstat + 4 * B);
+            FS_LAUNCH(h, fs::launch_maxabs(X, bf16, D.n, D.d, D.batch, t, mx, h->stream));
+            FS_LAUNCH(h, fs::launch_maxabs(Y, bf16, D.m, D.d, D.batch, t, mx + 1, h->stream));
+            float hm[2] = {0.f, 0.f};
+            FS_CUDA(h, cudaMemcpyAsync(hm, mx, sizeof(hm), cudaMemcpyDeviceToHost, h->stream));
+            FS_CUDA(h, cudaStreamSynchronize(h->stream));
+            auto pow2_scale = [](float maxabs) {
+                if (!(maxabs > 0.f) || !std::isfinite(maxabs)) return 1.f;
+                return std::ldexp(1.f, 14 - (int)std::ceil(std::log2((double)maxabs)));
+            };
+            h->qscale = pow2_scale(hm[0]);
+            h->kscale = pow2_scale(2.f * hm[1]);
+            h->sscale = 1.f / (h->qscale * h->kscale);
+        }
+        FS_LAUNCH(h, fs::launch_pack(X, bf16, D.n, h->n_pad, D.d, D.batch, t, h->qscale, h->pack_mode, h->d_p, h->row_elems,
                                    h->packX, h->xn, h->err, h->stream));
-        FS_LAUNCH(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, 2.f, h->pack_mode, h->d_p, h->row_elems,
+        FS_LAUNCH(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, 2.f * h->kscale, h->pack_mode, h->d_p, h->row_elems,
                                    h->packY, h->yn, h->err, h->stream));
         FS_LAUNCH(h, fs::launch_weights(a, D.batch, D.n, h->n_pad, h->la2, h->wstat, h->stream));
         FS_LAUNCH(h, fs::launch_weights(b, D.batch, D.m, h->m_pad, h->lb2, h->wstat + 2 * B, h->stream));
@@ -450,9 +493,10 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         }
         if (h->host_err[0] & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in X or Y");
         if (prec != FS_PREC_F32_SIMT) {
-            fs_status s2 = encode_map(h, &h->mapX, h->packX, D.batch * h->n_pad);
-            if (s2 != FS_OK) return s2;
-            s2 = encode_map(h, &h->mapY, h->packY, D.batch * h->m_pad);
+            fs_status s2 = encode_map(h, &h->mapX_r, h->packX, D.batch * h->n_pad, kBlockRows);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, kBlockCols);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_r, h->packY, D.batch * h->m_pad, kBlockRows);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, kBlockCols);
             if (s2 != FS_OK) return s2;
         }
         return FS_OK;
@@ -574,6 +618,7 @@ fs_status fs_get_info(const fs_handle *h, fs_info *info) {
     info->launches_update = 2;
     info->launches_solve_iter = 2;
     info->device_bytes = h->bytes;
+    info->cta_pair = (h->prec != FS_PREC_F32_SIMT && h->pair) ? 1 : 0;
     return FS_OK;
 }
 

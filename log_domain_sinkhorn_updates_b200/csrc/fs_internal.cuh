@@ -20,7 +20,7 @@
 namespace fs {
 
 constexpr int kBlockRows = 128;   // rows of one CTA (one TMEM lane per row)
-constexpr int kBlockCols = 128;   // columns of one streamed tile
+constexpr int kBlockCols = 256;   // columns of one streamed tile (the MMA's N)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr double kLn2d = 0.69314718055994530942;
 constexpr double kLog2ed = 1.44269504088896340736;
@@ -42,7 +42,8 @@ struct PassParams {
     int tiles_per_split;       // column tiles handled by one split
     int col_tiles;             // total column tiles
     int stages;                // pipeline depth (tensor-core path)
-    float scale2;              // log2(e)/eps
+    float scale2;              // log2(e)/eps, times sscale
+    float sscale;              // factor from the MMA's raw score to S_ij (1 unless operands were scaled)
     double eps;
     const float *col_bias;     // [batch][cols_pad], base-2, -inf on padding
     const float *row_norm;     // [batch][rows_pad] |row - t|^2
@@ -130,6 +131,11 @@ cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec
                           const void *map_rows, const void *map_cols, size_t smem_bytes,
                           cudaStream_t s);
 size_t tc_smem_bytes(int row_bytes, int stages, bool measure);
+// The CTA-pair variant (one MMA over two SMs; rows_pad / 128 must be even).
+cudaError_t launch_lse_tc2(const PassParams &p, int batch, bool measure, int prec, const void *map_rows,
+                           const void *map_cols, size_t smem_bytes, cudaStream_t s);
+size_t tc2_smem_bytes(int row_bytes, int stages, bool measure);
+int tc2_max_stages(int row_bytes, bool measure);
 // Record msg as this thread's handle-less error (what fs_last_error(NULL) returns).
 void set_thread_error(const char *msg);
 int tc_max_stages(int row_bytes, bool measure);

@@ -2,6 +2,7 @@
 // with squared norms, log-weights, column/row biases, and the final
 // deterministic reduction of measure-pass statistics.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "fs_prep.cuh"
 
@@ -68,7 +69,7 @@ __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int bat
             float v = 0.f;
             int k = e;
             int plane = 0;
-            if (mode == kPack3xTf32) {
+            if (mode == kPack3xTf32 || mode == kPack3xF16) {
                 plane = e / d_p;
                 k = e % d_p;
                 if (plane > 1) k = d;  // padding beyond the two planes
@@ -88,6 +89,16 @@ __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int bat
             } else if (mode == kPackTf32) {
                 out = round_tf32(scale * v);
                 if (k < d) acc += (double)v * v;
+            } else if (mode == kPack3xF16) {
+                // scale is a power of two chosen so that |scale * v| <= 2^14: exact,
+                // and far inside the fp16 range.
+                const float sv = scale * v;
+                const __half hi = __float2half_rn(sv);
+                const __half lo = __float2half_rn(sv - __half2float(hi));
+                if (plane == 0 && k < d) acc += (double)v * v;
+                static_cast<__half *>(dst)[wr * row_elems + e] =
+                    plane == 0 ? hi : (plane == 1 ? lo : __float2half_rn(0.f));
+                continue;
             } else if (mode == kPack3xTf32) {
                 const float sv = scale * v;
                 const float hi = round_tf32(sv);
@@ -103,6 +114,28 @@ __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int bat
         if (bad) atomicOr(err, kDevErrNonfinite);
         if (lane == 0) norm[wr] = valid ? (float)acc : 0.f;
     }
+}
+
+// max |src - t| over every element of every problem (one block per problem,
+// fixed-order tree; the per-problem maxima are folded with atomicMax on the
+// float bits, which orders like the values for non-negative floats).
+template <typename T>
+__global__ void maxabs_kernel(const T *src, int rows, int d, const float *t, unsigned *out) {
+    __shared__ float sh[256];
+    const int bz = blockIdx.x;
+    float mx = 0.f;
+    for (size_t e = threadIdx.x; e < (size_t)rows * d; e += 256) {
+        const int k = (int)(e % d);
+        const float v = load_val(src, (size_t)bz * rows * d + e) - (t ? t[(size_t)bz * d + k] : 0.f);
+        mx = fmaxf(mx, fabsf(v));
+    }
+    sh[threadIdx.x] = mx;
+    __syncthreads();
+    for (int s = 128; s > 0; s >>= 1) {
+        if ((int)threadIdx.x < s) sh[threadIdx.x] = fmaxf(sh[threadIdx.x], sh[threadIdx.x + s]);
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) atomicMax(out, __float_as_uint(sh[0]));
 }
 
 // log2 of the weights (uniform when w == null), -inf on padding; per-problem
@@ -202,6 +235,18 @@ cudaError_t launch_pack(const void *src, bool bf16, int rows, int rows_pad, int 
     else
         pack_kernel<<<grid, 256, 0, s>>>(static_cast<const float *>(src), rows, rows_pad, d, batch, t, scale,
                                         mode, d_p, row_elems, dst, norm, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_maxabs(const void *src, bool bf16, int rows, int d, int batch, const float *t, float *out,
+                          cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    unsigned *o = reinterpret_cast<unsigned *>(out);
+    if (bf16)
+        maxabs_kernel<<<batch, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), rows, d, t, o);
+    else
+        maxabs_kernel<<<batch, 256, 0, s>>>(static_cast<const float *>(src), rows, d, t, o);
     return cudaGetLastError();
 }
 

@@ -10,12 +10,16 @@ constexpr int kPackBf16 = 0;    // one bf16 plane
 constexpr int kPackTf32 = 1;    // one fp32 plane rounded to tf32
 constexpr int kPack3xTf32 = 2;  // [hi | lo] fp32 planes, hi = tf32(v), lo = v - hi
 constexpr int kPackPlain = 3;   // plain fp32 rows of d values (SIMT path)
+constexpr int kPack3xF16 = 4;   // [hi | lo] fp16 planes of the scaled value, hi = f16(v), lo = f16(v - hi)
 
 cudaError_t launch_center(const void *X, const void *Y, bool bf16, int batch, int n, int m, int d, float *t,
                           cudaStream_t s);
 cudaError_t launch_pack(const void *src, bool bf16, int rows, int rows_pad, int d, int batch, const float *t,
                         float scale, int mode, int d_p, int row_elems, void *dst, float *norm, int *err,
                         cudaStream_t s);
+// out[0] = max over every problem of |src - t| (fp32), for the 3xF16 scaling.
+cudaError_t launch_maxabs(const void *src, bool bf16, int rows, int d, int batch, const float *t, float *out,
+                          cudaStream_t s);
 cudaError_t launch_weights(const float *w, int batch, int cnt, int cnt_pad, float *lw2, double *wstat,
                            cudaStream_t s);
 cudaError_t launch_fill(float *p, size_t count, float v, cudaStream_t s);

@@ -22,7 +22,15 @@ SMALL = {
     "highdim": dict(n=700, m=650),
     "batched": dict(batch=3, n=600, m=520),
 }
-PRECS = ["auto", "f32_simt"]
+# every mode that is meant to be ~fp32 accurate on the workload's inputs
+PRECS = {
+    "tiny": ["auto", "f32_simt", "3xtf32", "3xf16"],
+    "middim": ["auto", "f32_simt", "3xf16", "3xtf32"],
+    "cloud3d": ["auto", "f32_simt", "3xtf32", "3xf16"],
+    "highdim": ["auto", "f32_simt"],
+    "batched": ["auto", "f32_simt", "3xtf32", "3xf16"],
+}
+CASES = [(name, prec) for name in SMALL for prec in PRECS[name]]
 
 
 def _fs():
@@ -30,8 +38,7 @@ def _fs():
     return fs
 
 
-@pytest.mark.parametrize("prec", PRECS)
-@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("name,prec", CASES)
 def test_single_update_parity(cuda_device, name, prec):
     import torch
     fs = _fs()
@@ -56,8 +63,21 @@ def test_single_update_parity(cuda_device, name, prec):
         eg = np.abs(g[k] - go).max()
         assert ef <= tol[k], (name, prec, k, ef, tol[k])
         assert eg <= tol[k], (name, prec, k, eg, tol[k])
-        if prec == "auto":  # the chosen mode must leave 4x margin to the bar
-            assert max(ef, eg) <= tol[k] / 4, (name, k, ef, eg, tol[k])
+        # every mode here is ~fp32 accurate and must leave a 4x margin to the bar
+        assert max(ef, eg) <= tol[k] / 4, (name, prec, k, ef, eg, tol[k])
+
+
+def test_unsupported_row_width_is_reported(cuda_device):
+    """3xTF32 rows of d = 65 (640 bytes) exceed the 512-byte operand rows of the tensor-core pass."""
+    import torch
+    fs = _fs()
+    rng = np.random.default_rng(4)
+    X = torch.from_numpy(rng.standard_normal((300, 65)).astype(np.float32)).to(cuda_device)
+    Y = torch.from_numpy(rng.standard_normal((310, 65)).astype(np.float32)).to(cuda_device)
+    with pytest.raises(fs.FsError) as e:
+        fs.fs_create(X, Y, eps=0.1, prec="3xtf32")
+    assert e.value.status == 3
+    fs.fs_create(X, Y, eps=0.1)  # the default (3xF16, 320-byte rows) runs
 
 
 SOLVE = {
@@ -142,3 +162,29 @@ def test_measure_parity(cuda_device, name):
         assert abs(ec[k] - eo[1]) <= 1e-3 * eo[1] + tau, (name, k, ec[k], eo[1], tau)
         assert abs(dual[k] - co["dual"]) <= 1e-3 * abs(co["dual"]), (name, k)
         assert abs(primal[k] - co["primal"]) <= 1e-3 * abs(co["primal"]), (name, k)
+
+
+@pytest.mark.parametrize("name", ["middim", "highdim", "batched"])
+def test_cta_pair_kernel_parity(cuda_device, name, monkeypatch):
+    """The CTA-pair tensor-core pass (FS_CTA_PAIR=1, one MMA over two SMs) and the
+    single-CTA pass that runs by default, both against the oracle."""
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a, b = device_inputs(prob)
+    rng = np.random.default_rng(78)
+    g_in = torch.from_numpy(np.stack([smooth_potential(rng, prob.m, 0.5) for _ in range(prob.batch)])).to(cuda_device)
+    outs = {}
+    for pair in ("0", "1"):
+        monkeypatch.setenv("FS_CTA_PAIR", pair)
+        h = fs.fs_create(X, Y, a, b, eps=prob.eps)
+        assert fs.fs_get_info(h)["cta_pair"] == int(pair)
+        f = torch.empty(prob.batch, prob.n, device=cuda_device)
+        fs.fs_update_f(h, g_in, f)
+        fs.fs_sync(h)
+        outs[pair] = f.cpu().numpy()
+    tol = 1e-4 * max_cost(prob)
+    for k, (Xo, Yo, _, logb) in enumerate(oracle_arrays(prob)):
+        fo = oracle.update_f(Xo, Yo, logb, g_in[k].cpu().numpy().astype(np.float64), prob.eps)
+        for pair in ("0", "1"):
+            assert np.abs(outs[pair][k] - fo).max() <= tol[k] / 4, (name, pair, k)
