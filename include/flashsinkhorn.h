@@ -96,7 +96,9 @@ typedef struct {
     int launches_update;    /* kernel launches of one fs_update_f / fs_update_g */
     int launches_solve_iter;/* kernel launches per fs_solve iteration           */
     size_t device_bytes;    /* device memory owned by the handle                */
-    int cta_pair;           /* 1: each MMA spans a pair of SMs (tcgen05 cta_group::2) */
+    int cta_pair;           /* 1: each MMA spans a pair of SMs (tcgen05 cta_group::2); chosen for
+                               512-byte operand rows, or for every width when the environment
+                               variable FS_CTA_PAIR=1 (FS_CTA_PAIR=0 forbids it) */
 } fs_info;
 
 /*

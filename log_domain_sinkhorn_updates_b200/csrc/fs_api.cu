@@ -31,7 +31,12 @@ struct fs_handle {
     int device = 0, sms = 148;
     // packed operand layout
     int d_p = 0, planes = 1, elem = 4, row_bytes = 0, swz = 0, plane_bytes = 0, pack_mode = 0, row_elems = 0;
-    int n_pad = 0, m_pad = 0;
+    // Packed operand rows per problem (a multiple of 256: 128-row blocks, in
+    // pairs for the CTA-pair pass), and the per-problem stride of the per-point
+    // arrays (norms, log-weights, biases): 256 more, so that any column tile of
+    // width <= 256 starting below the valid count stays inside them.
+    int n_pad = 0, m_pad = 0, n_stride = 0, m_stride = 0;
+    int tile = kBlockCols;  // column tile width of the tensor-core pass in use
     // device memory (one allocation, carved)
     void *block = nullptr;
     size_t bytes = 0;
@@ -176,15 +181,20 @@ fs::PassParams make_pass(const fs_handle *h, bool fdir, bool measure) {
     const fs_desc &D = h->desc;
     p.rows = fdir ? D.n : D.m;
     p.rows_pad = fdir ? h->n_pad : h->m_pad;
+    p.rows_stride = fdir ? h->n_stride : h->m_stride;
     p.cols = fdir ? D.m : D.n;
-    p.cols_pad = fdir ? h->m_pad : h->n_pad;
+    p.cols_rows = fdir ? h->m_pad : h->n_pad;
+    p.cols_stride = fdir ? h->m_stride : h->n_stride;
     p.row_bytes = h->row_bytes;
     p.swz = h->swz;
     p.plane_bytes = h->plane_bytes;
     p.d = D.d;
     p.splits = fdir ? h->splits_f : h->splits_g;
     p.tiles_per_split = fdir ? h->tps_f : h->tps_g;
-    p.col_tiles = p.cols_pad / kBlockCols;
+    {
+        const int tile = (h->prec == FS_PREC_F32_SIMT || h->pair) ? kBlockCols : h->tile;
+        p.col_tiles = (p.cols + tile - 1) / tile;
+    }
     p.stages = measure ? h->stages_meas : h->stages;
     p.eps = (double)D.eps;
     p.scale2 = (float)(fs::kLog2ed / (double)D.eps * (double)h->sscale);
@@ -210,8 +220,8 @@ cudaError_t run_pass(fs_handle *h, const fs::PassParams &p, bool fdir, bool meas
                                   fdir ? &h->mapY_r : &h->mapX_r, measure ? h->smem_meas : h->smem, h->stream);
     const CUtensorMap *mr = fdir ? &h->mapX_r : &h->mapY_r;
     const CUtensorMap *mc = fdir ? &h->mapY_c : &h->mapX_c;
-    return fs::launch_lse_tc(p, h->desc.batch, measure, h->prec, mr, mc, measure ? h->smem_meas : h->smem,
-                             h->stream);
+    return fs::launch_lse_tc(p, h->desc.batch, measure, h->prec, h->tile, mr, mc,
+                             measure ? h->smem_meas : h->smem, h->stream);
 }
 
 // Bias of the pass that has `cnt`-side columns, from potential pot of that side.
@@ -219,8 +229,8 @@ cudaError_t run_bias(fs_handle *h, const float *pot, bool col_is_y) {
     const fs_desc &D = h->desc;
     const double scale2 = fs::kLog2ed / (double)D.eps;
     if (col_is_y)
-        return fs::launch_bias(pot, D.batch, D.m, h->m_pad, h->yn, h->lb2, scale2, h->bias_col, h->stream);
-    return fs::launch_bias(pot, D.batch, D.n, h->n_pad, h->xn, h->la2, scale2, h->bias_row, h->stream);
+        return fs::launch_bias(pot, D.batch, D.m, h->m_stride, h->yn, h->lb2, scale2, h->bias_col, h->stream);
+    return fs::launch_bias(pot, D.batch, D.n, h->n_stride, h->xn, h->la2, scale2, h->bias_row, h->stream);
 }
 
 fs_status update(fs_handle *h, const float *in, float *out, bool fdir, bool write_next_bias) {
@@ -252,7 +262,7 @@ fs_status measure(fs_handle *h, const float *f, const float *g, bool fdir, int s
     FS_LAUNCH(h, run_pass(h, p, fdir, true));
     const int row_blocks = p.rows_pad / kBlockRows;
     FS_LAUNCH(h, fs::launch_finalize(h->stats, D.batch, row_blocks, want_col_sum ? (fdir ? g : f) : nullptr,
-                                   fdir ? h->lb2 : h->la2, p.cols, p.cols_pad, h->red + (size_t)slot * D.batch * 8,
+                                   fdir ? h->lb2 : h->la2, p.cols, p.cols_stride, h->red + (size_t)slot * D.batch * 8,
                                    h->stream));
     return FS_OK;
 }
@@ -358,6 +368,10 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
                        : prec == FS_PREC_3XF16 ? fs::kPack3xF16
                                                : fs::kPack3xTf32;
         h->row_elems = h->row_bytes / h->elem;
+        // CTA pairs halve the shared memory each CTA spends on column tiles; they
+        // serve the rows too wide for the single-CTA ring (512-byte rows), and
+        // any width when FS_CTA_PAIR=1.
+        h->pair = fs::tc_max_stages(h->row_bytes, kBlockCols, true) == 0;
         if (const char *env = getenv("FS_CTA_PAIR")) h->pair = atoi(env) != 0;
         if (h->row_bytes > 512) {  // four swizzle atoms: the kernels' per-tile descriptor table
             fail(nullptr, FS_ERR_UNSUPPORTED,
@@ -367,26 +381,34 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             delete h;
             return FS_ERR_UNSUPPORTED;
         }
-        h->stages = h->pair ? fs::tc2_max_stages(h->row_bytes, false) : fs::tc_max_stages(h->row_bytes, false);
-        h->stages_meas = h->pair ? fs::tc2_max_stages(h->row_bytes, true) : fs::tc_max_stages(h->row_bytes, true);
+        // Column tile of the tensor-core passes: N of every MMA.
+        h->tile = kBlockCols;
+        h->stages = h->pair ? fs::tc2_max_stages(h->row_bytes, false) : fs::tc_max_stages(h->row_bytes, h->tile, false);
+        h->stages_meas =
+            h->pair ? fs::tc2_max_stages(h->row_bytes, true) : fs::tc_max_stages(h->row_bytes, h->tile, true);
         if (h->stages < 2 || h->stages_meas < 2) {
             fail(nullptr, FS_ERR_UNSUPPORTED,
-                 "d=%d needs %d-byte operand rows; the single-CTA tensor-core pass supports rows up to "
-                 "256 bytes (bf16 d<=128, tf32 and 3xF16 d<=64, 3xTF32 d<=32)",
+                 "d=%d needs %d-byte operand rows; no K ring of at least one tile plus one slot fits in "
+                 "shared memory",
                  D.d, h->row_bytes);
             delete h;
             return FS_ERR_UNSUPPORTED;
         }
         h->smem = h->pair ? fs::tc2_smem_bytes(h->row_bytes, h->stages, false)
-                          : fs::tc_smem_bytes(h->row_bytes, h->stages, false);
+                          : fs::tc_smem_bytes(h->row_bytes, h->tile, h->stages, false);
         h->smem_meas = h->pair ? fs::tc2_smem_bytes(h->row_bytes, h->stages_meas, true)
-                               : fs::tc_smem_bytes(h->row_bytes, h->stages_meas, true);
+                               : fs::tc_smem_bytes(h->row_bytes, h->tile, h->stages_meas, true);
     }
     // Both clouds serve as rows (128-row blocks) and as columns (256-column tiles).
-    h->n_pad = round_up(D.n, kBlockCols);
-    h->m_pad = round_up(D.m, kBlockCols);
-    plan_splits(D.batch * (h->n_pad / kBlockRows), h->m_pad / kBlockCols, h->sms, &h->splits_f, &h->tps_f);
-    plan_splits(D.batch * (h->m_pad / kBlockRows), h->n_pad / kBlockCols, h->sms, &h->splits_g, &h->tps_g);
+    h->n_pad = round_up(D.n, 256);
+    h->m_pad = round_up(D.m, 256);
+    h->n_stride = h->n_pad + 256;
+    h->m_stride = h->m_pad + 256;
+    {
+        const int tile = (prec == FS_PREC_F32_SIMT || h->pair) ? kBlockCols : h->tile;
+        plan_splits(D.batch * (h->n_pad / kBlockRows), (D.m + tile - 1) / tile, h->sms, &h->splits_f, &h->tps_f);
+        plan_splits(D.batch * (h->m_pad / kBlockRows), (D.n + tile - 1) / tile, h->sms, &h->splits_g, &h->tps_g);
+    }
 
     // ---- one device allocation, carved ----
     const size_t B = (size_t)D.batch;
@@ -401,9 +423,9 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     };
     const size_t o_packX = carve(B * h->n_pad * h->row_bytes);
     const size_t o_packY = carve(B * h->m_pad * h->row_bytes);
-    const size_t o_xn = carve(B * h->n_pad * 4), o_yn = carve(B * h->m_pad * 4);
-    const size_t o_la2 = carve(B * h->n_pad * 4), o_lb2 = carve(B * h->m_pad * 4);
-    const size_t o_brow = carve(B * h->n_pad * 4), o_bcol = carve(B * h->m_pad * 4);
+    const size_t o_xn = carve(B * h->n_stride * 4), o_yn = carve(B * h->m_stride * 4);
+    const size_t o_la2 = carve(B * h->n_stride * 4), o_lb2 = carve(B * h->m_stride * 4);
+    const size_t o_brow = carve(B * h->n_stride * 4), o_bcol = carve(B * h->m_stride * 4);
     const size_t o_center = carve(B * D.d * 4);
     const size_t o_part = carve(max_splits > 1 ? B * max_splits * max_pad * 16 : 16);
     const size_t o_ctr = carve(B * max_rb * 4);
@@ -471,14 +493,16 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             h->kscale = pow2_scale(2.f * hm[1]);
             h->sscale = 1.f / (h->qscale * h->kscale);
         }
-        FS_LAUNCH(h, fs::launch_pack(X, bf16, D.n, h->n_pad, D.d, D.batch, t, h->qscale, h->pack_mode, h->d_p, h->row_elems,
-                                   h->packX, h->xn, h->err, h->stream));
-        FS_LAUNCH(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, 2.f * h->kscale, h->pack_mode, h->d_p, h->row_elems,
-                                   h->packY, h->yn, h->err, h->stream));
-        FS_LAUNCH(h, fs::launch_weights(a, D.batch, D.n, h->n_pad, h->la2, h->wstat, h->stream));
-        FS_LAUNCH(h, fs::launch_weights(b, D.batch, D.m, h->m_pad, h->lb2, h->wstat + 2 * B, h->stream));
-        FS_LAUNCH(h, fs::launch_fill(h->bias_row, B * h->n_pad, -INFINITY, h->stream));
-        FS_LAUNCH(h, fs::launch_fill(h->bias_col, B * h->m_pad, -INFINITY, h->stream));
+        FS_CUDA(h, cudaMemsetAsync(h->xn, 0, B * h->n_stride * 4, h->stream));
+        FS_CUDA(h, cudaMemsetAsync(h->yn, 0, B * h->m_stride * 4, h->stream));
+        FS_LAUNCH(h, fs::launch_pack(X, bf16, D.n, h->n_pad, D.d, D.batch, t, h->qscale, h->pack_mode, h->d_p,
+                                     h->row_elems, h->packX, h->xn, h->n_stride, h->err, h->stream));
+        FS_LAUNCH(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, 2.f * h->kscale, h->pack_mode, h->d_p,
+                                     h->row_elems, h->packY, h->yn, h->m_stride, h->err, h->stream));
+        FS_LAUNCH(h, fs::launch_weights(a, D.batch, D.n, h->n_stride, h->la2, h->wstat, h->stream));
+        FS_LAUNCH(h, fs::launch_weights(b, D.batch, D.m, h->m_stride, h->lb2, h->wstat + 2 * B, h->stream));
+        FS_LAUNCH(h, fs::launch_fill(h->bias_row, B * h->n_stride, -INFINITY, h->stream));
+        FS_LAUNCH(h, fs::launch_fill(h->bias_col, B * h->m_stride, -INFINITY, h->stream));
         double *hw = h->host_red.data() + 2 * B * 8;
         FS_CUDA(h, cudaMemcpyAsync(hw, h->wstat, 4 * B * 8, cudaMemcpyDeviceToHost, h->stream));
         FS_CUDA(h, cudaMemcpyAsync(h->host_err, h->err, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
@@ -494,9 +518,9 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         if (h->host_err[0] & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in X or Y");
         if (prec != FS_PREC_F32_SIMT) {
             fs_status s2 = encode_map(h, &h->mapX_r, h->packX, D.batch * h->n_pad, kBlockRows);
-            if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, kBlockCols);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, h->tile);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_r, h->packY, D.batch * h->m_pad, kBlockRows);
-            if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, kBlockCols);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, h->tile);
             if (s2 != FS_OK) return s2;
         }
         return FS_OK;
@@ -612,7 +636,7 @@ fs_status fs_get_info(const fs_handle *h, fs_info *info) {
     info->swizzle_bytes = h->swz;
     info->stages = h->stages;
     info->block_rows = kBlockRows;
-    info->block_cols = kBlockCols;
+    info->block_cols = (h->prec == FS_PREC_F32_SIMT || h->pair) ? kBlockCols : h->tile;
     info->splits_f = h->splits_f;
     info->splits_g = h->splits_g;
     info->launches_update = 2;

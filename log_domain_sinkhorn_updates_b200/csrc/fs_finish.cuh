@@ -16,7 +16,7 @@ __device__ void finish_rows(const PassParams &p, int rl, float m, float l, float
     const int rb = blockIdx.x, split = blockIdx.y, bz = blockIdx.z;
     const int row_blocks = p.rows_pad / kBlockRows;
     const int row = rb * kBlockRows + rl;
-    const size_t prow = (size_t)bz * p.rows_pad + row;
+    const size_t prow = (size_t)bz * p.rows_stride + row;  // per-point arrays of the row side
 
     if (p.splits > 1) {
         // Publish this split's partial state, then let the last CTA of the row

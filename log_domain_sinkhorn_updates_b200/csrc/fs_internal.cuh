@@ -32,31 +32,33 @@ constexpr int kDevErrBadWeights = 4;
 
 // Parameters of one streamed LSE pass (row side R against column side C).
 struct PassParams {
-    int rows, rows_pad;        // valid and padded rows of the row side
-    int cols, cols_pad;        // valid and padded columns
+    int rows, rows_pad;        // valid rows of the row side; packed operand rows per problem
+    int rows_stride;           // per-problem stride of the row side's per-point arrays
+    int cols, cols_rows;       // valid columns; packed operand rows per problem of the column side
+    int cols_stride;           // per-problem stride of the column side's per-point arrays
     int row_bytes;             // bytes of a packed operand row (tensor-core paths)
     int swz;                   // swizzle span in bytes (32, 64 or 128)
     int plane_bytes;           // bytes of one operand plane (multiple of 32)
     int d;                     // feature dim of the plain fp32 layout (SIMT path)
     int splits;                // column splits (grid.y)
     int tiles_per_split;       // column tiles handled by one split
-    int col_tiles;             // total column tiles
+    int col_tiles;             // column tiles of the pass's tile width covering cols
     int stages;                // pipeline depth (tensor-core path)
     float scale2;              // log2(e)/eps, times sscale
     float sscale;              // factor from the MMA's raw score to S_ij (1 unless operands were scaled)
     double eps;
-    const float *col_bias;     // [batch][cols_pad], base-2, -inf on padding
-    const float *row_norm;     // [batch][rows_pad] |row - t|^2
-    const float *row_logw2;    // [batch][rows_pad] log2 of the row weights
-    const float *col_norm;     // [batch][cols_pad] (measure passes only)
+    const float *col_bias;     // [batch][cols_stride], base-2, -inf beyond cols
+    const float *row_norm;     // [batch][rows_stride] |row - t|^2
+    const float *row_logw2;    // [batch][rows_stride] log2 of the row weights
+    const float *col_norm;     // [batch][cols_stride] (measure passes only)
     const float *pot_in;       // [batch][rows] current row potential (measure passes)
     float *pot_out;            // [batch][rows] new row potential (update passes)
-    float *next_bias;          // [batch][rows_pad] base-2 bias for the opposite pass, or null
+    float *next_bias;          // [batch][rows_stride] base-2 bias for the opposite pass, or null
     float4 *part;              // [batch][splits][rows_pad] split partials (m, l, w, -)
     unsigned *counters;        // [batch][row_blocks] arrival counters (self-resetting)
     double *stats;             // [batch][row_blocks][4] measure partial sums
     const void *plain_rows;    // SIMT path: [batch][rows_pad][d] fp32
-    const void *plain_cols;    // SIMT path: [batch][cols_pad][d] fp32
+    const void *plain_cols;    // SIMT path: [batch][cols_rows][d] fp32
     unsigned long long timeout_ns;
     int *err;
 };
@@ -127,10 +129,12 @@ __device__ void finish_rows(const PassParams &p, int row_local, float m, float l
 // Launchers (defined in the .cu files); all return cudaGetLastError().
 namespace fs {
 cudaError_t launch_lse_simt(const PassParams &p, int batch, bool measure, cudaStream_t s);
-cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec,
+// Single-CTA pass; tile = column tile width (224 for rows <= 256 bytes, 192 for <= 512).
+cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int tile,
                           const void *map_rows, const void *map_cols, size_t smem_bytes,
                           cudaStream_t s);
-size_t tc_smem_bytes(int row_bytes, int stages, bool measure);
+size_t tc_smem_bytes(int row_bytes, int tile, int stages, bool measure);
+int tc_max_stages(int row_bytes, int tile, bool measure);
 // The CTA-pair variant (one MMA over two SMs; rows_pad / 128 must be even).
 cudaError_t launch_lse_tc2(const PassParams &p, int batch, bool measure, int prec, const void *map_rows,
                            const void *map_cols, size_t smem_bytes, cudaStream_t s);
@@ -138,5 +142,4 @@ size_t tc2_smem_bytes(int row_bytes, int stages, bool measure);
 int tc2_max_stages(int row_bytes, bool measure);
 // Record msg as this thread's handle-less error (what fs_last_error(NULL) returns).
 void set_thread_error(const char *msg);
-int tc_max_stages(int row_bytes, bool measure);
 }  // namespace fs

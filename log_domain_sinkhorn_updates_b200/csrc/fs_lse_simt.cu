@@ -27,16 +27,16 @@ __global__ void __launch_bounds__(kBlockRows) lse_simt_kernel(const PassParams p
     const int rl = threadIdx.x;
     const int rb = blockIdx.x, split = blockIdx.y, bz = blockIdx.z;
     const float *rows = static_cast<const float *>(p.plain_rows) + ((size_t)bz * p.rows_pad + (size_t)rb * kBlockRows) * d;
-    const float *cols = static_cast<const float *>(p.plain_cols) + (size_t)bz * p.cols_pad * d;
-    const float *bias = p.col_bias + (size_t)bz * p.cols_pad;
-    const float *cnorm = MEASURE ? p.col_norm + (size_t)bz * p.cols_pad : nullptr;
+    const float *cols = static_cast<const float *>(p.plain_cols) + (size_t)bz * p.cols_rows * d;
+    const float *bias = p.col_bias + (size_t)bz * p.cols_stride;
+    const float *cnorm = MEASURE ? p.col_norm + (size_t)bz * p.cols_stride : nullptr;
 
     for (int e = rl; e < kBlockRows * d; e += kBlockRows) srow[(e / d) * ld + (e % d)] = rows[e];
 
     const int c_begin = split * p.tiles_per_split * kBlockCols;
-    const int c_end = min(p.cols_pad, c_begin + p.tiles_per_split * kBlockCols);
+    const int c_end = min(p.cols_rows, c_begin + p.tiles_per_split * kBlockCols);
     const float c = p.scale2;
-    const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_pad + rb * kBlockRows + rl] : 0.f;
+    const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_stride + rb * kBlockRows + rl] : 0.f;
     float m = -INFINITY, l = 0.f, w = 0.f;
 
     for (int c0 = c_begin; c0 < c_end; c0 += kSimtCols) {

@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mbar_expect_tx(full + s, slot_bytes);
                     tma_load_2d(saddr(sK + (size_t)s * slot_bytes), &map_cols, saddr(full + s), a * box_inner,
-                                bz * p.cols_pad + col0);
+                                bz * p.cols_rows + col0);
                     slots_issued = i + 1;
                 }
                 if (!ok) break;
@@ -162,10 +162,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 mbar_expect_tx(bfull + j, bias_bytes * (MEASURE ? 2 : 1));
-                bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_pad + col0, bias_bytes,
+                bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_stride + col0, bias_bytes,
                           saddr(bfull + j));
                 if (MEASURE)
-                    bulk_load(saddr(sCN + j * kBlockCols), p.col_norm + (size_t)bz * p.cols_pad + col0, bias_bytes,
+                    bulk_load(saddr(sCN + j * kBlockCols), p.col_norm + (size_t)bz * p.cols_stride + col0, bias_bytes,
                               saddr(bfull + j));
                 bias_issued = t + 1;
             }
@@ -248,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int grp = (warp - 2) >> 2; // tile parity handled by this warp
         const int rl = q * 32 + lane;    // row within the block
         const float c = p.scale2;
-        const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_pad + rb * kBlockRows + rl] : 0.f;
+        const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_stride + rb * kBlockRows + rl] : 0.f;
         float m = -INFINITY, l = 0.f, w = 0.f;
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * kBlockCols);
         bool ok = true;
@@ -335,24 +335,26 @@ cudaError_t launch_variant(const PassParams &p, int batch, const void *map_rows,
 
 }  // namespace
 
-size_t tc_smem_bytes(int row_bytes, int slots, bool measure) {
+size_t tc_smem_bytes(int row_bytes, int tile, int slots, bool measure) {
+    (void)tile;  // always kBlockCols
     return (size_t)smem_layout(row_bytes, slots, measure).total + 1024;  // + alignment slack
 }
 
 // The deepest K ring that fits (at most 8 slots); 0 if not even one tile plus
 // one slot of look-ahead fits.
-int tc_max_stages(int row_bytes, bool measure) {
+int tc_max_stages(int row_bytes, int tile, bool measure) {
     const size_t limit = 227 * 1024;
     const int atoms = row_bytes / swizzle_of(row_bytes);
     int best = 0;
     for (int s = atoms + 1; s <= 8; ++s)
-        if (tc_smem_bytes(row_bytes, s, measure) <= limit) best = s;
+        if (tc_smem_bytes(row_bytes, tile, s, measure) <= limit) best = s;
     return best;
 }
 
-// prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16.
-cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, const void *map_rows,
+// prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16; tile must be kBlockCols.
+cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int tile, const void *map_rows,
                           const void *map_cols, size_t smem, cudaStream_t s) {
+    if (tile != kBlockCols) return cudaErrorInvalidValue;
     if (prec == 1)
         return measure ? launch_variant<0, 1, true>(p, batch, map_rows, map_cols, smem, s)
                        : launch_variant<0, 1, false>(p, batch, map_rows, map_cols, smem, s);

@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (rank == 0) mbar_expect_tx(full + s, 2u * slot_bytes);
                     tma_load_2d_pair(saddr(sK + (size_t)s * slot_bytes), &map_cols, cluster_addr(saddr(full + s), 0),
-                                     a * box_inner, bz * p.cols_pad + col0 + (int)rank * kHalfCols);
+                                     a * box_inner, bz * p.cols_rows + col0 + (int)rank * kHalfCols);
                     slots_issued = i + 1;
                 }
                 if (!ok) break;
@@ -161,10 +161,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 mbar_expect_tx(bfull + j, bias_bytes * (MEASURE ? 2 : 1));
-                bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_pad + col0, bias_bytes,
+                bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_stride + col0, bias_bytes,
                           saddr(bfull + j));
                 if (MEASURE)
-                    bulk_load(saddr(sCN + j * kBlockCols), p.col_norm + (size_t)bz * p.cols_pad + col0, bias_bytes,
+                    bulk_load(saddr(sCN + j * kBlockCols), p.col_norm + (size_t)bz * p.cols_stride + col0, bias_bytes,
                               saddr(bfull + j));
                 bias_issued = t + 1;
             }
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int grp = (warp - 2) >> 2;
         const int rl = q * 32 + lane;
         const float c = p.scale2;
-        const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_pad + rb * kBlockRows + rl] : 0.f;
+        const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_stride + rb * kBlockRows + rl] : 0.f;
         float m = -INFINITY, l = 0.f, w = 0.f;
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * kBlockCols);
         const uint32_t sempty0 = cluster_addr(saddr(sempty + grp), 0);

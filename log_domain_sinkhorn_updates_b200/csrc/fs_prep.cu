@@ -56,7 +56,7 @@ __device__ __forceinline__ float round_tf32(float x) {
 // layout of `mode`, norm = |v|^2 (double accumulation, fixed shuffle tree).
 template <typename T>
 __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int batch, const float *t, float scale,
-                            int mode, int d_p, int row_elems, void *dst, float *norm, int *err) {
+                            int mode, int d_p, int row_elems, void *dst, float *norm, int norm_stride, int *err) {
     const int lane = threadIdx.x & 31;
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
@@ -112,7 +112,7 @@ __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int bat
         }
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (bad) atomicOr(err, kDevErrNonfinite);
-        if (lane == 0) norm[wr] = valid ? (float)acc : 0.f;
+        if (lane == 0) norm[(size_t)bz * norm_stride + r] = valid ? (float)acc : 0.f;
     }
 }
 
@@ -225,16 +225,16 @@ cudaError_t launch_center(const void *X, const void *Y, bool bf16, int batch, in
 }
 
 cudaError_t launch_pack(const void *src, bool bf16, int rows, int rows_pad, int d, int batch, const float *t,
-                        float scale, int mode, int d_p, int row_elems, void *dst, float *norm, int *err,
-                        cudaStream_t s) {
+                        float scale, int mode, int d_p, int row_elems, void *dst, float *norm, int norm_stride,
+                        int *err, cudaStream_t s) {
     const size_t warps = (size_t)batch * rows_pad;
     const int grid = grid_for(warps * 32, 256);
     if (bf16)
         pack_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), rows, rows_pad, d, batch, t,
-                                        scale, mode, d_p, row_elems, dst, norm, err);
+                                        scale, mode, d_p, row_elems, dst, norm, norm_stride, err);
     else
         pack_kernel<<<grid, 256, 0, s>>>(static_cast<const float *>(src), rows, rows_pad, d, batch, t, scale,
-                                        mode, d_p, row_elems, dst, norm, err);
+                                        mode, d_p, row_elems, dst, norm, norm_stride, err);
     return cudaGetLastError();
 }
 

@@ -15,8 +15,8 @@ constexpr int kPack3xF16 = 4;   // [hi | lo] fp16 planes of the scaled value, hi
 cudaError_t launch_center(const void *X, const void *Y, bool bf16, int batch, int n, int m, int d, float *t,
                           cudaStream_t s);
 cudaError_t launch_pack(const void *src, bool bf16, int rows, int rows_pad, int d, int batch, const float *t,
-                        float scale, int mode, int d_p, int row_elems, void *dst, float *norm, int *err,
-                        cudaStream_t s);
+                        float scale, int mode, int d_p, int row_elems, void *dst, float *norm, int norm_stride,
+                        int *err, cudaStream_t s);
 // out[0] = max over every problem of |src - t| (fp32), for the 3xF16 scaling.
 cudaError_t launch_maxabs(const void *src, bool bf16, int rows, int d, int batch, const float *t, float *out,
                           cudaStream_t s);

@@ -90,6 +90,36 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
             : "memory");
     }
 }
+// D (TMEM) (+)= A (TMEM: one row per lane, K along 32-bit columns) x B^T (shared memory).
+template <int KIND>
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accum) {
+    if constexpr (KIND != 1) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+            "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
+            : "memory");
+    }
+}
+// 32 TMEM lanes (this warp's quadrant) x 32 consecutive 32-bit columns, from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
 // 32 TMEM lanes (this warp's quadrant) x 32 consecutive 32-bit columns.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
     asm volatile(
@@ -123,10 +153,10 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t addr, uint32_t swz) {
 // Instruction descriptor: fp32 accumulator, A/B format (kind::f16: 0 = fp16,
 // 1 = bf16; kind::tf32: 2), both K-major, M rows (128, or 256 for a CTA pair),
 // N = 256.
-template <int KIND, int M = kBlockRows>
+template <int KIND, int M = kBlockRows, int N = kBlockCols>
 __device__ __forceinline__ uint32_t make_idesc() {
     const uint32_t fmt = KIND == 0 ? 1u : (KIND == 1 ? 2u : 0u);
-    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(kBlockCols >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // ---- CTA pairs (cluster of two CTAs on two SMs sharing one MMA) -------------
@@ -206,12 +236,13 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t local_bar, uint16_t cta_
         : "memory");
 }
 
-// sum_k 2^(z_k - ref) over 128 columns, fp32 pairs.
-__device__ __forceinline__ float sum_exp2_128(const float (&z)[128], float ref) {
+// sum_k 2^(z_k - ref) over CNT columns, fp32 pairs.
+template <int CNT>
+__device__ __forceinline__ float sum_exp2(const float (&z)[CNT], float ref) {
     const uint64_t rn = pack2(-ref, -ref);
     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-    for (int k = 0; k < 128; k += 2) {
+    for (int k = 0; k < CNT; k += 2) {
         float d0, d1;
         unpack2(add2(pack2(z[k], z[k + 1]), rn), d0, d1);
         acc[(k / 2) & 3] = add2(acc[(k / 2) & 3], pack2(ex2_approx(d0), ex2_approx(d1)));
@@ -224,18 +255,18 @@ __device__ __forceinline__ float sum_exp2_128(const float (&z)[128], float ref) 
     return ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
 }
 
-// Fold 128 scores (raw fp32 bits from TMEM) into a row's online state (m, l):
+// Fold CNT scores (raw fp32 bits from TMEM) into a row's online state (m, l):
 // z = S * c + beta.  The first block of a row takes two passes (max, then
 // exponentials); later blocks take exponentials against the running max as
 // it stood, with the block max alongside, and redo the block only when the
 // max grew by more than 2^kLazy.
-__device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float *bias, float c, float &m,
-                                           float &l) {
+template <int CNT>
+__device__ __forceinline__ void consume(const uint32_t (&r)[CNT], const float *bias, float c, float &m, float &l) {
     const float4 *bq = reinterpret_cast<const float4 *>(bias);
     const uint64_t cc = pack2(c, c);
-    float z[128];
+    float z[CNT];
 #pragma unroll
-    for (int k = 0; k < 128; k += 4) {
+    for (int k = 0; k < CNT; k += 4) {
         const float4 bb = bq[k / 4];
         unpack2(fma2(pack2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), cc, pack2(bb.x, bb.y)), z[k],
                 z[k + 1]);
@@ -245,7 +276,7 @@ __device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float
     if (m == -INFINITY) {
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int k = 0; k < 128; k += 8) {
+        for (int k = 0; k < CNT; k += 8) {
             mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k], z[k + 1]);
             mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 2], z[k + 3]);
             mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 4], z[k + 5]);
@@ -253,7 +284,7 @@ __device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float
         }
         const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         if (tmax != -INFINITY) {
-            l = sum_exp2_128(z, tmax);
+            l = sum_exp2<CNT>(z, tmax);
             m = tmax;
         }
     } else {
@@ -261,7 +292,7 @@ __device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float
         const uint64_t mneg = pack2(-m, -m);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int k = 0; k < 128; k += 2) {
+        for (int k = 0; k < CNT; k += 2) {
             float d0, d1;
             unpack2(add2(pack2(z[k], z[k + 1]), mneg), d0, d1);
             acc[(k / 2) & 3] = add2(acc[(k / 2) & 3], pack2(ex2_approx(d0), ex2_approx(d1)));
@@ -269,7 +300,7 @@ __device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float
         }
         const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         if (tmax > m + kLazy) {
-            l = l * ex2_approx(m - tmax) + sum_exp2_128(z, tmax);
+            l = l * ex2_approx(m - tmax) + sum_exp2<CNT>(z, tmax);
             m = tmax;
         } else {
             float a0, a1, a2, a3, a4, a5, a6, a7;
@@ -280,6 +311,51 @@ __device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float
             l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
         }
     }
+}
+__device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float *bias, float c, float &m,
+                                           float &l) {
+    consume<128>(r, bias, c, m, l);
+}
+
+// Measure-mode fold over 32 columns: also accumulates w = sum 2^(z - m) C_ij
+// with C_ij = |row|^2 + |col|^2 - S_ij (S_ij = raw score * sscale).
+__device__ __forceinline__ void consume32_measure(const uint32_t (&r)[32], const float *bias, const float *cnorm,
+                                                  float c, float sscale, float xn, float &m, float &l, float &w) {
+    const float4 *bq = reinterpret_cast<const float4 *>(bias);
+    const float4 *cq = reinterpret_cast<const float4 *>(cnorm);
+    float z[32];
+    float t0 = -INFINITY, t1 = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+        const float4 bb = bq[k / 4];
+        z[k + 0] = fmaf(__uint_as_float(r[k + 0]), c, bb.x);
+        z[k + 1] = fmaf(__uint_as_float(r[k + 1]), c, bb.y);
+        z[k + 2] = fmaf(__uint_as_float(r[k + 2]), c, bb.z);
+        z[k + 3] = fmaf(__uint_as_float(r[k + 3]), c, bb.w);
+        t0 = fmaxf(t0, fmaxf(z[k + 0], z[k + 1]));
+        t1 = fmaxf(t1, fmaxf(z[k + 2], z[k + 3]));
+    }
+    const float mnew = fmaxf(m, fmaxf(t0, t1));
+    if (mnew == -INFINITY) return;
+    const float scale = ex2_approx(m - mnew);
+    float a0 = 0.f, a1 = 0.f, w0 = 0.f, w1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+        const float4 cn = cq[k / 4];
+        const float e0 = ex2_approx(z[k + 0] - mnew);
+        const float e1 = ex2_approx(z[k + 1] - mnew);
+        const float e2 = ex2_approx(z[k + 2] - mnew);
+        const float e3 = ex2_approx(z[k + 3] - mnew);
+        a0 += e0 + e2;
+        a1 += e1 + e3;
+        w0 = fmaf(e0, fmaf(-__uint_as_float(r[k + 0]), sscale, xn + cn.x), w0);
+        w1 = fmaf(e1, fmaf(-__uint_as_float(r[k + 1]), sscale, xn + cn.y), w1);
+        w0 = fmaf(e2, fmaf(-__uint_as_float(r[k + 2]), sscale, xn + cn.z), w0);
+        w1 = fmaf(e3, fmaf(-__uint_as_float(r[k + 3]), sscale, xn + cn.w), w1);
+    }
+    l = l * scale + (a0 + a1);
+    w = w * scale + (w0 + w1);
+    m = mnew;
 }
 
 // Measure-mode version over 64 columns: also accumulates w = sum 2^(z - m) C_ij
