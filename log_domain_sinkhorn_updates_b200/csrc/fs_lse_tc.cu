@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(empty + s, 1);  // the MMA commit of the tile that read the slot
+            mbar_init(empty + s, 1);  // the softmax group of the tile that read the slot
         }
         for (int j = 0; j < kBiasSlots; ++j) {
             mbar_init(bfull + j, 1);
@@ -226,7 +226,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
                     tc_mma<KIND>(dt, adesc0 + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
                 }
-                for (int a = 0; a < atoms; ++a) tc_commit(saddr(empty + ((t * atoms + a) % NS)));
+                // One commit per tile: it completes when the tile's MMAs have read
+                // their K slots and written S, and the softmax group that waits on
+                // it hands the slots back.  (A commit stalls the MMA pipe, so the
+                // chain carries no other.)
                 tc_commit(saddr(sfull + b));
             }
             if (!ok) {
@@ -260,6 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            if (q == 2 && lane == 0)  // the MMAs of tile t are complete: its K slots are free
+                for (int a = 0; a < atoms; ++a) mbar_arrive(empty + ((t * atoms + a) % NS));
             const float *bias = sBias + j * kBlockCols;
             if (!MEASURE) {
 #pragma unroll 1

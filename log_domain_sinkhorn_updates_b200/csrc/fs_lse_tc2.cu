@@ -227,7 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
                     tc_mma_pair<KIND>(dt, adesc0 + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
                 }
-                for (int a = 0; a < atoms; ++a) tc_commit_pair(saddr(empty + ((t * atoms + a) % NS)), (uint16_t)3);
+                // One commit per tile (a commit stalls the MMA pipe): the softmax
+                // groups of both CTAs hand the tile's K slots back when it lands.
                 tc_commit_pair(saddr(sfull + b), (uint16_t)3);
             }
             if (!ok) {
@@ -258,6 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            if (q == 2 && lane == 0)  // the pair's MMAs of tile t are complete: this CTA's K slots are free
+                for (int a = 0; a < atoms; ++a) mbar_arrive(empty + ((t * atoms + a) % NS));
             const float *bias = sBias + j * kBlockCols;
             if (!MEASURE) {
 #pragma unroll 1
