@@ -91,7 +91,9 @@ typedef struct {
     int row_bytes;          /* bytes of one packed operand row                  */
     int swizzle_bytes;      /* shared-memory swizzle span of the operand tiles  */
     int stages;             /* column-tile pipeline depth                       */
-    int block_rows, block_cols; /* tile shape of one CTA step                   */
+    int block_rows, block_cols; /* rows per CTA (128, or 256 when two row blocks share
+                                   every column tile; FS_ROW_BLOCKS=1 forces 128) x columns
+                                   per streamed tile                               */
     int splits_f, splits_g; /* column splits of the f- and g-direction passes   */
     int launches_update;    /* kernel launches of one fs_update_f / fs_update_g */
     int launches_solve_iter;/* kernel launches per fs_solve iteration           */

@@ -32,11 +32,11 @@ struct fs_handle {
     // packed operand layout
     int d_p = 0, planes = 1, elem = 4, row_bytes = 0, swz = 0, plane_bytes = 0, pack_mode = 0, row_elems = 0;
     // Packed operand rows per problem (a multiple of 256: 128-row blocks, in
-    // pairs for the CTA-pair pass), and the per-problem stride of the per-point
-    // arrays (norms, log-weights, biases): 256 more, so that any column tile of
-    // width <= 256 starting below the valid count stays inside them.
+    // pairs for the 256-row and CTA-pair passes), and the per-problem stride of
+    // the per-point arrays (norms, log-weights, biases): 256 more, so that a
+    // column tile starting below the valid count stays inside them.
     int n_pad = 0, m_pad = 0, n_stride = 0, m_stride = 0;
-    int tile = kBlockCols;  // column tile width of the tensor-core pass in use
+    int qt = 1;  // 128-row blocks per CTA of the single-CTA tensor-core pass
     // device memory (one allocation, carved)
     void *block = nullptr;
     size_t bytes = 0;
@@ -191,10 +191,7 @@ fs::PassParams make_pass(const fs_handle *h, bool fdir, bool measure) {
     p.d = D.d;
     p.splits = fdir ? h->splits_f : h->splits_g;
     p.tiles_per_split = fdir ? h->tps_f : h->tps_g;
-    {
-        const int tile = (h->prec == FS_PREC_F32_SIMT || h->pair) ? kBlockCols : h->tile;
-        p.col_tiles = (p.cols + tile - 1) / tile;
-    }
+    p.col_tiles = (p.cols + kBlockCols - 1) / kBlockCols;
     p.stages = measure ? h->stages_meas : h->stages;
     p.eps = (double)D.eps;
     p.scale2 = (float)(fs::kLog2ed / (double)D.eps * (double)h->sscale);
@@ -220,7 +217,7 @@ cudaError_t run_pass(fs_handle *h, const fs::PassParams &p, bool fdir, bool meas
                                   fdir ? &h->mapY_r : &h->mapX_r, measure ? h->smem_meas : h->smem, h->stream);
     const CUtensorMap *mr = fdir ? &h->mapX_r : &h->mapY_r;
     const CUtensorMap *mc = fdir ? &h->mapY_c : &h->mapX_c;
-    return fs::launch_lse_tc(p, h->desc.batch, measure, h->prec, h->tile, mr, mc,
+    return fs::launch_lse_tc(p, h->desc.batch, measure, h->prec, h->qt, mr, mc,
                              measure ? h->smem_meas : h->smem, h->stream);
 }
 
@@ -371,7 +368,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         // CTA pairs halve the shared memory each CTA spends on column tiles; they
         // serve the rows too wide for the single-CTA ring (512-byte rows), and
         // any width when FS_CTA_PAIR=1.
-        h->pair = fs::tc_max_stages(h->row_bytes, kBlockCols, true) == 0;
+        h->pair = fs::tc_max_stages(h->row_bytes, 1, true) == 0;
         if (const char *env = getenv("FS_CTA_PAIR")) h->pair = atoi(env) != 0;
         if (h->row_bytes > 512) {  // four swizzle atoms: the kernels' per-tile descriptor table
             fail(nullptr, FS_ERR_UNSUPPORTED,
@@ -381,11 +378,14 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             delete h;
             return FS_ERR_UNSUPPORTED;
         }
-        // Column tile of the tensor-core passes: N of every MMA.
-        h->tile = kBlockCols;
-        h->stages = h->pair ? fs::tc2_max_stages(h->row_bytes, false) : fs::tc_max_stages(h->row_bytes, h->tile, false);
+        // Two resident 128-row blocks per CTA when their Q tiles and a K ring of
+        // at least one tile plus one slot fit in shared memory: every K tile
+        // then serves 256 rows.  FS_ROW_BLOCKS=1 forces one.
+        h->qt = fs::tc_max_stages(h->row_bytes, 2, true) > 0 ? 2 : 1;
+        if (const char *env = getenv("FS_ROW_BLOCKS")) h->qt = atoi(env) == 1 ? 1 : h->qt;
+        h->stages = h->pair ? fs::tc2_max_stages(h->row_bytes, false) : fs::tc_max_stages(h->row_bytes, h->qt, false);
         h->stages_meas =
-            h->pair ? fs::tc2_max_stages(h->row_bytes, true) : fs::tc_max_stages(h->row_bytes, h->tile, true);
+            h->pair ? fs::tc2_max_stages(h->row_bytes, true) : fs::tc_max_stages(h->row_bytes, h->qt, true);
         if (h->stages < 2 || h->stages_meas < 2) {
             fail(nullptr, FS_ERR_UNSUPPORTED,
                  "d=%d needs %d-byte operand rows; no K ring of at least one tile plus one slot fits in "
@@ -395,9 +395,9 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             return FS_ERR_UNSUPPORTED;
         }
         h->smem = h->pair ? fs::tc2_smem_bytes(h->row_bytes, h->stages, false)
-                          : fs::tc_smem_bytes(h->row_bytes, h->tile, h->stages, false);
+                          : fs::tc_smem_bytes(h->row_bytes, h->qt, h->stages, false);
         h->smem_meas = h->pair ? fs::tc2_smem_bytes(h->row_bytes, h->stages_meas, true)
-                               : fs::tc_smem_bytes(h->row_bytes, h->tile, h->stages_meas, true);
+                               : fs::tc_smem_bytes(h->row_bytes, h->qt, h->stages_meas, true);
     }
     // Both clouds serve as rows (128-row blocks) and as columns (256-column tiles).
     h->n_pad = round_up(D.n, 256);
@@ -405,9 +405,11 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     h->n_stride = h->n_pad + 256;
     h->m_stride = h->m_pad + 256;
     {
-        const int tile = (prec == FS_PREC_F32_SIMT || h->pair) ? kBlockCols : h->tile;
-        plan_splits(D.batch * (h->n_pad / kBlockRows), (D.m + tile - 1) / tile, h->sms, &h->splits_f, &h->tps_f);
-        plan_splits(D.batch * (h->m_pad / kBlockRows), (D.n + tile - 1) / tile, h->sms, &h->splits_g, &h->tps_g);
+        // CTAs along the rows: one per 128-row block, or per 256 rows on the two-block pass.
+        const int rows_per_cta = (prec == FS_PREC_F32_SIMT || h->pair) ? kBlockRows : kBlockRows * h->qt;
+        const int tile = kBlockCols;
+        plan_splits(D.batch * (h->n_pad / rows_per_cta), (D.m + tile - 1) / tile, h->sms, &h->splits_f, &h->tps_f);
+        plan_splits(D.batch * (h->m_pad / rows_per_cta), (D.n + tile - 1) / tile, h->sms, &h->splits_g, &h->tps_g);
     }
 
     // ---- one device allocation, carved ----
@@ -518,9 +520,9 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         if (h->host_err[0] & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in X or Y");
         if (prec != FS_PREC_F32_SIMT) {
             fs_status s2 = encode_map(h, &h->mapX_r, h->packX, D.batch * h->n_pad, kBlockRows);
-            if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, h->tile);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, kBlockCols);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_r, h->packY, D.batch * h->m_pad, kBlockRows);
-            if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, h->tile);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, kBlockCols);
             if (s2 != FS_OK) return s2;
         }
         return FS_OK;
@@ -635,8 +637,8 @@ fs_status fs_get_info(const fs_handle *h, fs_info *info) {
     info->row_bytes = h->row_bytes;
     info->swizzle_bytes = h->swz;
     info->stages = h->stages;
-    info->block_rows = kBlockRows;
-    info->block_cols = (h->prec == FS_PREC_F32_SIMT || h->pair) ? kBlockCols : h->tile;
+    info->block_rows = (h->prec == FS_PREC_F32_SIMT || h->pair) ? kBlockRows : kBlockRows * h->qt;
+    info->block_cols = kBlockCols;
     info->splits_f = h->splits_f;
     info->splits_g = h->splits_g;
     info->launches_update = 2;

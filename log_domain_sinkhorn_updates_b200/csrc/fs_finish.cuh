@@ -10,10 +10,12 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// rb: the 128-row block this CTA's rows belong to; the CTA's 128 threads of
+// that block call this together (named barrier bar_id).
 template <bool MEASURE>
-__device__ void finish_rows(const PassParams &p, int rl, float m, float l, float w, int bar_id,
+__device__ void finish_rows(const PassParams &p, int rb, int rl, float m, float l, float w, int bar_id,
                             double *red, int *flag) {
-    const int rb = blockIdx.x, split = blockIdx.y, bz = blockIdx.z;
+    const int split = blockIdx.y, bz = blockIdx.z;
     const int row_blocks = p.rows_pad / kBlockRows;
     const int row = rb * kBlockRows + rl;
     const size_t prow = (size_t)bz * p.rows_stride + row;  // per-point arrays of the row side

@@ -129,12 +129,13 @@ __device__ void finish_rows(const PassParams &p, int row_local, float m, float l
 // Launchers (defined in the .cu files); all return cudaGetLastError().
 namespace fs {
 cudaError_t launch_lse_simt(const PassParams &p, int batch, bool measure, cudaStream_t s);
-// Single-CTA pass; tile = column tile width (224 for rows <= 256 bytes, 192 for <= 512).
-cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int tile,
+// Single-CTA pass; qt = 128-row blocks resident per CTA (1 or 2; rows_pad / 128
+// must be a multiple of qt).
+cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int qt,
                           const void *map_rows, const void *map_cols, size_t smem_bytes,
                           cudaStream_t s);
-size_t tc_smem_bytes(int row_bytes, int tile, int stages, bool measure);
-int tc_max_stages(int row_bytes, int tile, bool measure);
+size_t tc_smem_bytes(int row_bytes, int qt, int stages, bool measure);
+int tc_max_stages(int row_bytes, int qt, bool measure);
 // The CTA-pair variant (one MMA over two SMs; rows_pad / 128 must be even).
 cudaError_t launch_lse_tc2(const PassParams &p, int batch, bool measure, int prec, const void *map_rows,
                            const void *map_cols, size_t smem_bytes, cudaStream_t s);

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kBlockRows) lse_simt_kernel(const PassParams p
         if (MEASURE) w = w * scale + accw;
         m = mnew;
     }
-    finish_rows<MEASURE>(p, rl, m, l, w, 0, red, flag);
+    finish_rows<MEASURE>(p, blockIdx.x, rl, m, l, w, 0, red, flag);
 }
 
 size_t simt_smem_bytes(int d) {

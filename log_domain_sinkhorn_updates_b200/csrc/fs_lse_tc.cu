@@ -1,16 +1,22 @@
 // Streamed LSE pass on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// One CTA owns a block of 128 rows of the row side ("row-stationary
-// traversal", FlashSinkhorn Metodologia section 2): its packed operand tile
-// Q (128 x row_bytes) is loaded once by TMA and stays in shared memory, while
-// 256-column tiles K of the column side stream through a ring of TMA slots
-// (one slot = 256 rows x one swizzle atom of the row).  For every tile one
-// thread issues the tcgen05.mma chain S = Q K^T (M = 128, N = 256: at M = 128
-// the tensor core needs N = 256 for its full rate) into one of two TMEM
-// accumulators of 256 fp32 columns, so the MMA of one tile overlaps the
-// exponentials of the previous ones.  Eight "softmax" warps (two per TMEM lane
-// quadrant; one group of four takes the even tiles, the other the odd ones)
-// read S with tcgen05.ld, form
+// One CTA owns QT blocks of 128 rows of the row side ("row-stationary
+// traversal", FlashSinkhorn Metodologia section 2): their packed operand
+// tiles Q_0..Q_{QT-1} (128 x row_bytes each) are loaded once by TMA and stay in
+// shared memory, while 256-column tiles K of the column side stream through a
+// ring of TMA slots (one slot = 256 rows x one swizzle atom of the row).  Every
+// K tile is multiplied by each resident Q tile, so with QT = 2 a tile crosses
+// L2 -> SM, and is written into shared memory, once per 256 rows instead of
+// once per 128.
+//
+// The MMA issuer runs a sequence of jobs; job j computes S = Q K^T (M = 128,
+// N = 256, both operands in shared memory) into TMEM buffer j & 1 (two buffers
+// of 256 fp32 columns), so the MMA of one job overlaps the exponentials of the
+// previous ones.  With QT = 1, job j is tile j; with QT = 2, job j is tile j/2
+// times Q tile j % 2.  Eight "softmax" warps in two groups of four (one warp per
+// TMEM lane quadrant) take the jobs of their buffer: group g handles jobs
+// j = g mod 2, i.e. the even or odd tiles (QT = 1) or every tile of Q tile g
+// (QT = 2).  They read S with tcgen05.ld, form
 //   z_ij = S_ij * log2(e)/eps + beta_j
 // (beta_j arrives in a separate small ring of bias slices) and update a per-row
 // online maximum and sum of 2^(z - max) in registers (online LSE, section 2).
@@ -45,24 +51,24 @@ struct SmemLayout {
 
 __host__ __device__ inline int swizzle_of(int row_bytes) { return row_bytes <= 32 ? 32 : (row_bytes <= 64 ? 64 : 128); }
 
-// slots: K ring slots of kBlockCols rows x one swizzle atom each.
-__host__ __device__ inline SmemLayout smem_layout(int row_bytes, int slots, bool measure) {
+// slots: K ring slots of kBlockCols rows x one swizzle atom each; qt: resident Q tiles.
+__host__ __device__ inline SmemLayout smem_layout(int row_bytes, int slots, bool measure, int qt) {
     SmemLayout L;
     const uint32_t swz = (uint32_t)swizzle_of(row_bytes);
     L.q = 0;
-    L.k = (uint32_t)kBlockRows * row_bytes;
+    L.k = (uint32_t)(qt * kBlockRows) * row_bytes;
     L.bias = L.k + (uint32_t)slots * kBlockCols * swz;
     L.cnorm = L.bias + kBiasSlots * kBlockCols * 4;
     L.merge = L.cnorm + (measure ? kBiasSlots * kBlockCols * 4 : 0);
     L.red = L.merge + kBlockRows * 16;
-    L.koff = L.red + 4 * kBlockRows * 8;
+    L.koff = L.red + (uint32_t)qt * 4 * kBlockRows * 8;
     L.bars = L.koff + 3 * kMaxKsteps * 4;
     L.misc = L.bars + (2 * slots + 2 * kBiasSlots + 6) * 8;
-    L.total = L.misc + 16;
+    L.total = L.misc + 32;
     return L;
 }
 
-template <int KIND, int NPASS, bool MEASURE>
+template <int KIND, int NPASS, bool MEASURE, int QT>
 __global__ void __launch_bounds__(kThreads, 1)
     lse_tc_kernel(const __grid_constant__ CUtensorMap map_rows, const __grid_constant__ CUtensorMap map_cols,
                   const PassParams p) {
@@ -74,7 +80,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int atoms = p.row_bytes / p.swz;
     const uint32_t slot_bytes = (uint32_t)kBlockCols * swz;
     const int box_inner = p.swz / (KIND == 1 ? 4 : 2);
-    const SmemLayout L = smem_layout(p.row_bytes, NS, MEASURE);
+    const SmemLayout L = smem_layout(p.row_bytes, NS, MEASURE, QT);
 
     uint8_t *sQ = smem + L.q;
     uint8_t *sK = smem + L.k;
@@ -92,22 +98,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *sempty = sfull + 2;  // [2]
     uint64_t *drain = sempty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L.misc);
-    int *flag = reinterpret_cast<int *>(smem + L.misc + 4);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 8);
+    int *flag = reinterpret_cast<int *>(smem + L.misc + 4);  // [QT]
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rb = blockIdx.x, split = blockIdx.y, bz = blockIdx.z;
     const int tile_begin = split * p.tiles_per_split;
     const int ntiles = min(p.tiles_per_split, p.col_tiles - tile_begin);
+    const int njobs = ntiles * QT;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(empty + s, 1);  // the softmax group of the tile that read the slot
+            mbar_init(empty + s, 1);  // the softmax group of the tile's last job
         }
         for (int j = 0; j < kBiasSlots; ++j) {
             mbar_init(bfull + j, 1);
-            mbar_init(bempty + j, 4);  // the four warps of the tile's softmax group
+            mbar_init(bempty + j, 4 * QT);  // the warps of the softmax groups that read the tile
         }
         mbar_init(qfull, 1);
         for (int b = 0; b < 2; ++b) {
@@ -134,10 +141,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             bool ok = true;
             int slots_issued = 0, bias_issued = 0;
-            const int qrow = bz * p.rows_pad + rb * kBlockRows;
-            mbar_expect_tx(qfull, (uint32_t)kBlockRows * p.row_bytes);
-            for (int a = 0; a < atoms; ++a)
-                tma_load_2d(saddr(sQ) + a * kBlockRows * swz, &map_rows, saddr(qfull), a * box_inner, qrow);
+            const int qrow = bz * p.rows_pad + rb * (QT * kBlockRows);
+            mbar_expect_tx(qfull, (uint32_t)(QT * kBlockRows) * p.row_bytes);
+            for (int g = 0; g < QT; ++g)
+                for (int a = 0; a < atoms; ++a)
+                    tma_load_2d(saddr(sQ) + (g * atoms + a) * kBlockRows * swz, &map_rows, saddr(qfull),
+                                a * box_inner, qrow + g * kBlockRows);
             const uint32_t bias_bytes = kBlockCols * 4;
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int col0 = (tile_begin + t) * kBlockCols;
@@ -200,36 +209,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                 koff[2 * kMaxKsteps + i] = (bo % swz) >> 4;
             }
             const uint64_t adesc0 = make_sdesc(saddr(sQ), swz);
+            const uint32_t qstride = (uint32_t)(atoms * kBlockRows * swz) >> 4;  // one Q tile, in descriptor units
             bool ok = mbar_wait(qfull, 0, p.timeout_ns);
-            for (int t = 0; ok && t < ntiles; ++t) {
-                const int b = t & 1;
-                if (t >= 2 && !mbar_wait(sempty + b, ((uint32_t)(t >> 1) & 1u) ^ 1u, p.timeout_ns)) {
+            uint64_t bdesc[kMaxAtoms];
+            for (int jb = 0; ok && jb < njobs; ++jb) {
+                const int b = jb & 1;
+                const int t = QT == 2 ? (jb >> 1) : jb;
+                const int qt = QT == 2 ? b : 0;
+                if (jb >= 2 && !mbar_wait(sempty + b, ((uint32_t)(jb >> 1) & 1u) ^ 1u, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
-                uint64_t bdesc[kMaxAtoms];
+                if (qt == 0) {  // first job of tile t: wait for its K slots
 #pragma unroll
-                for (int a = 0; a < kMaxAtoms; ++a) {
-                    if (a < atoms) {
-                        const int i = t * atoms + a;
-                        if (!mbar_wait(full + (i % NS), (uint32_t)(i / NS) & 1u, p.timeout_ns)) ok = false;
-                        bdesc[a] = make_sdesc(saddr(sK + (size_t)(i % NS) * slot_bytes), swz);
-                    } else {
-                        bdesc[a] = 0ull;
+                    for (int a = 0; a < kMaxAtoms; ++a) {
+                        if (a < atoms) {
+                            const int i = t * atoms + a;
+                            if (!mbar_wait(full + (i % NS), (uint32_t)(i / NS) & 1u, p.timeout_ns)) ok = false;
+                            bdesc[a] = make_sdesc(saddr(sK + (size_t)(i % NS) * slot_bytes), swz);
+                        } else {
+                            bdesc[a] = 0ull;
+                        }
                     }
                 }
                 if (!ok || *abort_flag) break;
                 tc_fence_after();
                 const uint32_t dt = tmem_base + (uint32_t)(b * kBlockCols);
+                const uint64_t adesc = adesc0 + (uint64_t)(qt * qstride);
                 for (int i = 0; i < nk; ++i) {
                     const uint32_t ba = koff[kMaxKsteps + i];
                     const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
-                    tc_mma<KIND>(dt, adesc0 + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
+                    tc_mma<KIND>(dt, adesc + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
                 }
-                // One commit per tile: it completes when the tile's MMAs have read
-                // their K slots and written S, and the softmax group that waits on
-                // it hands the slots back.  (A commit stalls the MMA pipe, so the
-                // chain carries no other.)
+                // One commit per job: it completes when the job's MMAs have read
+                // their operands and written S.  The softmax group that waits on
+                // it hands the tile's K slots back after the tile's last job.  (A
+                // commit stalls the MMA pipe, so the chain carries no other.)
                 tc_commit(saddr(sfull + b));
             }
             if (!ok) {
@@ -250,20 +265,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;          // TMEM lane quadrant this warp may access
         const int grp = (warp - 2) >> 2; // tile parity handled by this warp
         const int rl = q * 32 + lane;    // row within the block
+        const int rblk = rb * QT + (QT == 2 ? grp : 0);  // this warp's 128-row block
         const float c = p.scale2;
-        const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_stride + rb * kBlockRows + rl] : 0.f;
+        const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_stride + rblk * kBlockRows + rl] : 0.f;
         float m = -INFINITY, l = 0.f, w = 0.f;
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * kBlockCols);
         bool ok = true;
-        for (int t = grp; t < ntiles; t += 2) {
+        for (int jb = grp; jb < njobs; jb += 2) {
+            const int t = QT == 2 ? (jb >> 1) : jb;
             const int j = t % kBiasSlots;
-            if (!mbar_wait(sfull + grp, (uint32_t)(t >> 1) & 1u, p.timeout_ns) ||
+            if (!mbar_wait(sfull + grp, (uint32_t)(jb >> 1) & 1u, p.timeout_ns) ||
                 !mbar_wait(bfull + j, (uint32_t)(t / kBiasSlots) & 1u, p.timeout_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            if (q == 2 && lane == 0)  // the MMAs of tile t are complete: its K slots are free
+            if (q == 2 && lane == 0 && (QT == 1 || grp == 1))  // tile t's last job is complete: its K slots are free
                 for (int a = 0; a < atoms; ++a) mbar_arrive(empty + ((t * atoms + a) % NS));
             const float *bias = sBias + j * kBlockCols;
             if (!MEASURE) {
@@ -307,13 +324,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             atomicOr(p.err, kDevErrTimeout);
             *abort_flag = 1;
         }
-        // Merge the two tile-parity groups' states of each row, then finish the row block.
-        if (grp == 1) sMerge[rl] = make_float4(m, l, w, 0.f);
-        named_barrier(1, 256);
-        if (grp == 0) {
-            const float4 o = sMerge[rl];
-            lse_merge(m, l, w, o.x, o.y, o.z);
-            finish_rows<MEASURE>(p, rl, m, l, w, 2, sRed, flag);
+        if (QT == 1) {
+            // Merge the two tile-parity groups' states of each row, then finish the row block.
+            if (grp == 1) sMerge[rl] = make_float4(m, l, w, 0.f);
+            named_barrier(1, 256);
+            if (grp == 0) {
+                const float4 o = sMerge[rl];
+                lse_merge(m, l, w, o.x, o.y, o.z);
+                finish_rows<MEASURE>(p, rblk, rl, m, l, w, 2, sRed, flag);
+            }
+        } else {
+            // Each group holds whole rows of its own row block.
+            finish_rows<MEASURE>(p, rblk, rl, m, l, w, 2 + grp, sRed + grp * 4 * kBlockRows, flag + grp);
         }
     }
 
@@ -326,51 +348,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int KIND, int NPASS, bool MEASURE>
+template <int KIND, int NPASS, bool MEASURE, int QT>
 cudaError_t launch_variant(const PassParams &p, int batch, const void *map_rows, const void *map_cols,
                            size_t smem, cudaStream_t s) {
-    auto kern = lse_tc_kernel<KIND, NPASS, MEASURE>;
+    auto kern = lse_tc_kernel<KIND, NPASS, MEASURE, QT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.rows_pad / kBlockRows, p.splits, batch);
+    dim3 grid(p.rows_pad / (QT * kBlockRows), p.splits, batch);
     kern<<<grid, kThreads, smem, s>>>(*static_cast<const CUtensorMap *>(map_rows),
                                       *static_cast<const CUtensorMap *>(map_cols), p);
     return cudaGetLastError();
 }
 
-}  // namespace
-
-size_t tc_smem_bytes(int row_bytes, int tile, int slots, bool measure) {
-    (void)tile;  // always kBlockCols
-    return (size_t)smem_layout(row_bytes, slots, measure).total + 1024;  // + alignment slack
+template <int KIND, int NPASS>
+cudaError_t launch_kind(const PassParams &p, int batch, bool measure, int qt, const void *map_rows,
+                        const void *map_cols, size_t smem, cudaStream_t s) {
+    if (qt == 2)
+        return measure ? launch_variant<KIND, NPASS, true, 2>(p, batch, map_rows, map_cols, smem, s)
+                       : launch_variant<KIND, NPASS, false, 2>(p, batch, map_rows, map_cols, smem, s);
+    return measure ? launch_variant<KIND, NPASS, true, 1>(p, batch, map_rows, map_cols, smem, s)
+                   : launch_variant<KIND, NPASS, false, 1>(p, batch, map_rows, map_cols, smem, s);
 }
 
-// The deepest K ring that fits (at most 8 slots); 0 if not even one tile plus
-// one slot of look-ahead fits.
-int tc_max_stages(int row_bytes, int tile, bool measure) {
+}  // namespace
+
+size_t tc_smem_bytes(int row_bytes, int qt, int slots, bool measure) {
+    return (size_t)smem_layout(row_bytes, slots, measure, qt).total + 1024;  // + alignment slack
+}
+
+// The deepest K ring that fits (at most 8 slots) with qt resident Q tiles; 0
+// if not even one tile plus one slot of look-ahead fits.
+int tc_max_stages(int row_bytes, int qt, bool measure) {
     const size_t limit = 227 * 1024;
     const int atoms = row_bytes / swizzle_of(row_bytes);
     int best = 0;
     for (int s = atoms + 1; s <= 8; ++s)
-        if (tc_smem_bytes(row_bytes, tile, s, measure) <= limit) best = s;
+        if (tc_smem_bytes(row_bytes, qt, s, measure) <= limit) best = s;
     return best;
 }
 
-// prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16; tile must be kBlockCols.
-cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int tile, const void *map_rows,
+// prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16; qt: 128-row blocks per CTA (1 or 2).
+cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int qt, const void *map_rows,
                           const void *map_cols, size_t smem, cudaStream_t s) {
-    if (tile != kBlockCols) return cudaErrorInvalidValue;
-    if (prec == 1)
-        return measure ? launch_variant<0, 1, true>(p, batch, map_rows, map_cols, smem, s)
-                       : launch_variant<0, 1, false>(p, batch, map_rows, map_cols, smem, s);
-    if (prec == 2)
-        return measure ? launch_variant<1, 1, true>(p, batch, map_rows, map_cols, smem, s)
-                       : launch_variant<1, 1, false>(p, batch, map_rows, map_cols, smem, s);
-    if (prec == 3)
-        return measure ? launch_variant<1, 3, true>(p, batch, map_rows, map_cols, smem, s)
-                       : launch_variant<1, 3, false>(p, batch, map_rows, map_cols, smem, s);
-    return measure ? launch_variant<2, 3, true>(p, batch, map_rows, map_cols, smem, s)
-                   : launch_variant<2, 3, false>(p, batch, map_rows, map_cols, smem, s);
+    if (qt != 1 && qt != 2) return cudaErrorInvalidValue;
+    if (prec == 1) return launch_kind<0, 1>(p, batch, measure, qt, map_rows, map_cols, smem, s);
+    if (prec == 2) return launch_kind<1, 1>(p, batch, measure, qt, map_rows, map_cols, smem, s);
+    if (prec == 3) return launch_kind<1, 3>(p, batch, measure, qt, map_rows, map_cols, smem, s);
+    return launch_kind<2, 3>(p, batch, measure, qt, map_rows, map_cols, smem, s);
 }
 
 }  // namespace fs

@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (grp == 0) {
             const float4 o = sMerge[rl];
             lse_merge(m, l, w, o.x, o.y, o.z);
-            finish_rows<MEASURE>(p, rl, m, l, w, 2, sRed, flag);
+            finish_rows<MEASURE>(p, blockIdx.x, rl, m, l, w, 2, sRed, flag);
         }
     }
 

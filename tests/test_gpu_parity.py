@@ -1,7 +1,7 @@
 """GPU parity against the CPU oracle, through the C ABI.
 
 Single updates: every workload recipe at sizes the oracle finishes in seconds,
-spanning several 128-row/128-column tiles with ragged tails; the bar is
+spanning several 128-row/256-column tiles with ragged tails; the bar is
 max |f_gpu - f_oracle| <= 1e-4 * max_ij C_ij (both sides see the same float32
 inputs, the oracle in double).  Full solves: marginal L1 error and dual cost
 after the recipe's iteration count within 1e-3 relative (plus the float32
@@ -188,3 +188,35 @@ def test_cta_pair_kernel_parity(cuda_device, name, monkeypatch):
         fo = oracle.update_f(Xo, Yo, logb, g_in[k].cpu().numpy().astype(np.float64), prob.eps)
         for pair in ("0", "1"):
             assert np.abs(outs[pair][k] - fo).max() <= tol[k] / 4, (name, pair, k)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_row_block_pairing_parity(cuda_device, name, monkeypatch):
+    """The single-CTA pass with two resident 128-row blocks per CTA (each K tile
+    serves 256 rows; the default where it fits) and with one (FS_ROW_BLOCKS=1),
+    both against the oracle, for the f- and the g-update."""
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a, b = device_inputs(prob)
+    rng = np.random.default_rng(79)
+    g_in = np.stack([smooth_potential(rng, prob.m, 0.5) for _ in range(prob.batch)])
+    f_in = np.stack([smooth_potential(rng, prob.n, 0.5) for _ in range(prob.batch)])
+    outs = {}
+    for mode in ("1", "2"):
+        monkeypatch.setenv("FS_ROW_BLOCKS", mode)
+        h = fs.fs_create(X, Y, a, b, eps=prob.eps)
+        assert fs.fs_get_info(h)["block_rows"] == 128 * int(mode)
+        f = torch.empty(prob.batch, prob.n, device=cuda_device)
+        g = torch.empty(prob.batch, prob.m, device=cuda_device)
+        fs.fs_update_f(h, torch.from_numpy(g_in).to(cuda_device), f)
+        fs.fs_update_g(h, torch.from_numpy(f_in).to(cuda_device), g)
+        fs.fs_sync(h)
+        outs[mode] = (f.cpu().numpy(), g.cpu().numpy())
+    tol = 1e-4 * max_cost(prob)
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fo = oracle.update_f(Xo, Yo, logb, g_in[k].astype(np.float64), prob.eps)
+        go = oracle.update_g(Xo, Yo, loga, f_in[k].astype(np.float64), prob.eps)
+        for mode in ("1", "2"):
+            assert np.abs(outs[mode][0][k] - fo).max() <= tol[k] / 4, (name, mode, k, "f")
+            assert np.abs(outs[mode][1][k] - go).max() <= tol[k] / 4, (name, mode, k, "g")
