@@ -13,6 +13,7 @@ namespace tc {
 // Largest growth (base 2) of a row's maximum that is absorbed without a
 // rescale: terms up to 2^kLazy stay in the running sum as they are.
 constexpr float kLazy = 12.f;
+constexpr float kLazySum = 4096.f;  // 2^kLazy: a block sum above it forces the rescale
 
 __device__ __forceinline__ uint32_t saddr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -257,9 +258,11 @@ __device__ __forceinline__ float sum_exp2(const float (&z)[CNT], float ref) {
 
 // Fold CNT scores (raw fp32 bits from TMEM) into a row's online state (m, l):
 // z = S * c + beta.  The first block of a row takes two passes (max, then
-// exponentials); later blocks take exponentials against the running max as
-// it stood, with the block max alongside, and redo the block only when the
-// max grew by more than 2^kLazy.
+// exponentials).  Later blocks take their exponentials against the running max
+// as it stood and add them up; only when that block sum exceeds 2^kLazy (which
+// every entry more than kLazy above the running max forces, and which an
+// overflow to inf or a NaN also fails) is the block's max taken and the block
+// redone against it.  The common case thus spends no instruction on the max.
 template <int CNT>
 __device__ __forceinline__ void consume(const uint32_t (&r)[CNT], const float *bias, float c, float &m, float &l) {
     const float4 *bq = reinterpret_cast<const float4 *>(bias);
@@ -273,22 +276,8 @@ __device__ __forceinline__ void consume(const uint32_t (&r)[CNT], const float *b
         unpack2(fma2(pack2(__uint_as_float(r[k + 2]), __uint_as_float(r[k + 3])), cc, pack2(bb.z, bb.w)), z[k + 2],
                 z[k + 3]);
     }
-    if (m == -INFINITY) {
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int k = 0; k < CNT; k += 8) {
-            mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k], z[k + 1]);
-            mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 2], z[k + 3]);
-            mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 4], z[k + 5]);
-            mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 6], z[k + 7]);
-        }
-        const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        if (tmax != -INFINITY) {
-            l = sum_exp2<CNT>(z, tmax);
-            m = tmax;
-        }
-    } else {
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    float s;
+    if (m != -INFINITY) {
         const uint64_t mneg = pack2(-m, -m);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -296,21 +285,31 @@ __device__ __forceinline__ void consume(const uint32_t (&r)[CNT], const float *b
             float d0, d1;
             unpack2(add2(pack2(z[k], z[k + 1]), mneg), d0, d1);
             acc[(k / 2) & 3] = add2(acc[(k / 2) & 3], pack2(ex2_approx(d0), ex2_approx(d1)));
-            mx[(k / 2) & 3] = max3(mx[(k / 2) & 3], z[k], z[k + 1]);
         }
-        const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-        if (tmax > m + kLazy) {
-            l = l * ex2_approx(m - tmax) + sum_exp2<CNT>(z, tmax);
-            m = tmax;
-        } else {
-            float a0, a1, a2, a3, a4, a5, a6, a7;
-            unpack2(acc[0], a0, a1);
-            unpack2(acc[1], a2, a3);
-            unpack2(acc[2], a4, a5);
-            unpack2(acc[3], a6, a7);
-            l += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+        float a0, a1, a2, a3, a4, a5, a6, a7;
+        unpack2(acc[0], a0, a1);
+        unpack2(acc[1], a2, a3);
+        unpack2(acc[2], a4, a5);
+        unpack2(acc[3], a6, a7);
+        s = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+        if (s <= kLazySum) {
+            l += s;
+            return;
         }
     }
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int k = 0; k < CNT; k += 8) {
+        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k], z[k + 1]);
+        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 2], z[k + 3]);
+        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 4], z[k + 5]);
+        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 6], z[k + 7]);
+    }
+    const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    if (tmax == -INFINITY) return;  // nothing but padding so far
+    const float mnew = fmaxf(m, tmax);
+    l = (m == -INFINITY ? 0.f : l * ex2_approx(m - mnew)) + sum_exp2<CNT>(z, mnew);
+    m = mnew;
 }
 __device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float *bias, float c, float &m,
                                            float &l) {
