@@ -1,4 +1,4 @@
-"""CPU oracle for log-domain Sinkhorn with squared-Euclidean cost.
+"""CPU oracle for log-domain Sinkhorn with squared-Euclidean or cosine cost.
 
 TEST INFRASTRUCTURE ONLY: only the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg may import this package.  It shares no code with
@@ -13,5 +13,5 @@ Two independent implementations live here:
 """
 from .core import (  # noqa: F401
     log_weights, update_f, update_g, update_f_rows, solve, marginals, marginal_error,
-    plan_stats, costs, minplus_bounds, num_threads, problem_arrays,
+    plan_stats, costs, minplus_bounds, num_threads, problem_arrays, COSTS,
 )

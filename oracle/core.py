@@ -6,6 +6,10 @@ Every function takes one problem's float64 arrays (X [n,d], Y [m,d], log
 weights, potentials) and follows "FlashSinkhorn: IO-aware EOT on GPU",
 Metodologia section 1 (the stabilised log-domain updates).  Batched
 workloads are handled by the caller, one problem at a time.
+
+``cost`` selects C: "sqeuclidean" (C = |x - y|^2, the page's cost) or
+"cosine" (C = 1 - cos(x, y), the cosine distance that the page's closing
+remarks name as the other cost the method covers after normalisation).
 """
 from __future__ import annotations
 
@@ -27,13 +31,13 @@ def _load():
         path = _build.build()
         lib = ctypes.CDLL(path)
         L, I, D = ctypes.c_long, ctypes.c_int, ctypes.c_double
-        lib.so_update_f.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, _dp]
-        lib.so_update_g.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, _dp]
-        lib.so_solve.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, I, _dp, _dp]
-        lib.so_marginals.argtypes = [L, L, I, _dp, _dp, _dp, _dp, _dp, _dp, D, _dp, _dp]
-        lib.so_plan_stats.argtypes = [L, L, I, _dp, _dp, _dp, _dp, _dp, _dp, D, _dp]
-        lib.so_minplus_bounds.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, _dp, _dp, _dp]
-        lib.so_update_f_rows.argtypes = [L, _lp, L, I, _dp, _dp, _dp, _dp, D, _dp]
+        lib.so_update_f.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, _dp, I]
+        lib.so_update_g.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, _dp, I]
+        lib.so_solve.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, I, _dp, _dp, I]
+        lib.so_marginals.argtypes = [L, L, I, _dp, _dp, _dp, _dp, _dp, _dp, D, _dp, _dp, I]
+        lib.so_plan_stats.argtypes = [L, L, I, _dp, _dp, _dp, _dp, _dp, _dp, D, _dp, I]
+        lib.so_minplus_bounds.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, _dp, _dp, _dp, I]
+        lib.so_update_f_rows.argtypes = [L, _lp, L, I, _dp, _dp, _dp, _dp, D, _dp, I]
         lib.so_num_threads.argtypes = []
         for name in ("so_update_f", "so_update_g", "so_solve", "so_plan_stats", "so_update_f_rows",
                      "so_num_threads"):
@@ -47,6 +51,20 @@ def _load():
 def _c(a):
     a = np.ascontiguousarray(a, dtype=np.float64)
     return a, a.ctypes.data_as(_dp)
+
+
+COSTS = {"sqeuclidean": 0, "cosine": 1}
+
+
+def _cost(cost, *clouds):
+    """The C code of ``cost``; the cosine distance is undefined for a zero vector."""
+    if cost not in COSTS:
+        raise ValueError(f"unknown cost {cost!r}")
+    if cost == "cosine":
+        for P in clouds:
+            if np.any(np.sum(np.asarray(P, dtype=np.float64) ** 2, axis=1) == 0.0):
+                raise ValueError("the cosine cost is undefined for a zero vector")
+    return COSTS[cost]
 
 
 def num_threads() -> int:
@@ -70,8 +88,9 @@ def problem_arrays(prob, k=0):
     return X, Y, loga, logb
 
 
-def update_f(X, Y, logb, g, eps):
+def update_f(X, Y, logb, g, eps, cost="sqeuclidean"):
     """f_i = -eps LSE_j[(g_j - C_ij)/eps + log b_j]  (the f-update of Proposition 1's setting)."""
+    ci = _cost(cost, X, Y)
     X, px = _c(X)
     Y, py = _c(Y)
     logb, pb = _c(logb)
@@ -79,13 +98,14 @@ def update_f(X, Y, logb, g, eps):
     n, d = X.shape
     m = Y.shape[0]
     f = np.empty(n)
-    if _load().so_update_f(n, m, d, px, py, pb, pg, float(eps), f.ctypes.data_as(_dp)):
+    if _load().so_update_f(n, m, d, px, py, pb, pg, float(eps), f.ctypes.data_as(_dp), ci):
         raise MemoryError("oracle update_f")
     return f
 
 
-def update_g(X, Y, loga, f, eps):
+def update_g(X, Y, loga, f, eps, cost="sqeuclidean"):
     """g_j = -eps LSE_i[(f_i - C_ij)/eps + log a_i]  (the transposed update)."""
+    ci = _cost(cost, X, Y)
     X, px = _c(X)
     Y, py = _c(Y)
     loga, pa = _c(loga)
@@ -93,13 +113,14 @@ def update_g(X, Y, loga, f, eps):
     n, d = X.shape
     m = Y.shape[0]
     g = np.empty(m)
-    if _load().so_update_g(n, m, d, px, py, pa, pf, float(eps), g.ctypes.data_as(_dp)):
+    if _load().so_update_g(n, m, d, px, py, pa, pf, float(eps), g.ctypes.data_as(_dp), ci):
         raise MemoryError("oracle update_g")
     return g
 
 
-def update_f_rows(rows, X, Y, logb, g, eps):
+def update_f_rows(rows, X, Y, logb, g, eps, cost="sqeuclidean"):
     """The f-update at selected rows only (for spot checks at full size)."""
+    ci = _cost(cost, np.asarray(X)[np.asarray(rows, dtype=np.int64)], Y)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
     X, px = _c(X)
     Y, py = _c(Y)
@@ -109,13 +130,14 @@ def update_f_rows(rows, X, Y, logb, g, eps):
     m = Y.shape[0]
     out = np.empty(rows.shape[0])
     if _load().so_update_f_rows(rows.shape[0], rows.ctypes.data_as(_lp), m, d, px, py, pb, pg,
-                                float(eps), out.ctypes.data_as(_dp)):
+                                float(eps), out.ctypes.data_as(_dp), ci):
         raise MemoryError("oracle update_f_rows")
     return out
 
 
-def solve(X, Y, loga, logb, eps, iters, g0=None):
+def solve(X, Y, loga, logb, eps, iters, g0=None, cost="sqeuclidean"):
     """Alternating Sinkhorn from g0 (default 0): iters x {f <- update_f(g); g <- update_g(f)}."""
+    ci = _cost(cost, X, Y)
     X, px = _c(X)
     Y, py = _c(Y)
     loga, pa = _c(loga)
@@ -125,13 +147,14 @@ def solve(X, Y, loga, logb, eps, iters, g0=None):
     f = np.zeros(n)
     g = np.zeros(m) if g0 is None else np.array(g0, dtype=np.float64)
     if _load().so_solve(n, m, d, px, py, pa, pb, float(eps), int(iters), f.ctypes.data_as(_dp),
-                        g.ctypes.data_as(_dp)):
+                        g.ctypes.data_as(_dp), ci):
         raise MemoryError("oracle solve")
     return f, g
 
 
-def marginals(X, Y, loga, logb, f, g, eps):
+def marginals(X, Y, loga, logb, f, g, eps, cost="sqeuclidean"):
     """(r, c): row and column sums of P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps)."""
+    ci = _cost(cost, X, Y)
     X, px = _c(X)
     Y, py = _c(Y)
     loga, pa = _c(loga)
@@ -143,18 +166,19 @@ def marginals(X, Y, loga, logb, f, g, eps):
     r = np.empty(n)
     c = np.empty(m)
     _load().so_marginals(n, m, d, px, py, pa, pb, pf, pg, float(eps), r.ctypes.data_as(_dp),
-                         c.ctypes.data_as(_dp))
+                         c.ctypes.data_as(_dp), ci)
     return r, c
 
 
-def marginal_error(X, Y, loga, logb, f, g, eps):
+def marginal_error(X, Y, loga, logb, f, g, eps, cost="sqeuclidean"):
     """(err_row, err_col) = (sum_i |r_i - a_i|, sum_j |c_j - b_j|)."""
-    r, c = marginals(X, Y, loga, logb, f, g, eps)
+    r, c = marginals(X, Y, loga, logb, f, g, eps, cost)
     return float(np.abs(r - np.exp(loga)).sum()), float(np.abs(c - np.exp(logb)).sum())
 
 
-def plan_stats(X, Y, loga, logb, f, g, eps):
+def plan_stats(X, Y, loga, logb, f, g, eps, cost="sqeuclidean"):
     """sum P, <P,C>, sum P log(P/(a b)), max C, min C -- one pass over all pairs."""
+    ci = _cost(cost, X, Y)
     X, px = _c(X)
     Y, py = _c(Y)
     loga, pa = _c(loga)
@@ -164,19 +188,19 @@ def plan_stats(X, Y, loga, logb, f, g, eps):
     n, d = X.shape
     m = Y.shape[0]
     out = np.empty(5)
-    if _load().so_plan_stats(n, m, d, px, py, pa, pb, pf, pg, float(eps), out.ctypes.data_as(_dp)):
+    if _load().so_plan_stats(n, m, d, px, py, pa, pb, pf, pg, float(eps), out.ctypes.data_as(_dp), ci):
         raise MemoryError("oracle plan_stats")
     return dict(sum_p=out[0], primal=out[1], p_log_ratio=out[2], max_cost=out[3], min_cost=out[4])
 
 
-def costs(X, Y, loga, logb, f, g, eps):
+def costs(X, Y, loga, logb, f, g, eps, cost="sqeuclidean"):
     """Dual and primal objectives of entropic OT at the pair (f, g).
 
     dual            D = <a,f> + <b,g> - eps (sum_ij P_ij - 1)
     primal          <P, C>                         (transport cost of the plan)
     entropic_primal <P, C> + eps KL(P | a (x) b),  KL(P|Q) = sum P log(P/Q) - sum P + 1
     """
-    s = plan_stats(X, Y, loga, logb, f, g, eps)
+    s = plan_stats(X, Y, loga, logb, f, g, eps, cost)
     a = np.exp(np.asarray(loga, dtype=np.float64))
     b = np.exp(np.asarray(logb, dtype=np.float64))
     dual = float(a @ f + b @ g - eps * (s["sum_p"] - 1.0))
@@ -185,11 +209,12 @@ def costs(X, Y, loga, logb, f, g, eps):
                 sum_p=float(s["sum_p"]), max_cost=float(s["max_cost"]), min_cost=float(s["min_cost"]))
 
 
-def minplus_bounds(X, Y, logb, g, eps):
+def minplus_bounds(X, Y, logb, g, eps, cost="sqeuclidean"):
     """Per row: (min_j (C_ij - g_j), min_j (C_ij - g_j - eps log b_j), max_j C_ij).
 
     The soft c-transform (the f-update) lies between the first two for every
     row (hard c-transform sandwich)."""
+    ci = _cost(cost, X, Y)
     X, px = _c(X)
     Y, py = _c(Y)
     logb, pb = _c(logb)
@@ -200,7 +225,7 @@ def minplus_bounds(X, Y, logb, g, eps):
     hi = np.empty(n)
     cm = np.empty(n)
     _load().so_minplus_bounds(n, m, d, px, py, pb, pg, float(eps), lo.ctypes.data_as(_dp),
-                              hi.ctypes.data_as(_dp), cm.ctypes.data_as(_dp))
+                              hi.ctypes.data_as(_dp), cm.ctypes.data_as(_dp), ci)
     return lo, hi, cm
 
 

@@ -12,9 +12,19 @@ import numpy as np
 from scipy.special import logsumexp
 
 
-def cost_matrix(X, Y):
-    """C_ij = |x_i - y_j|^2 from the differences (broadcast, n*m*d doubles)."""
-    diff = np.asarray(X, dtype=np.float64)[:, None, :] - np.asarray(Y, dtype=np.float64)[None, :, :]
+def cost_matrix(X, Y, cost="sqeuclidean"):
+    """C_ij = |x_i - y_j|^2 from the differences (broadcast, n*m*d doubles), or
+    for cost="cosine" C_ij = 1 - x_i.y_j / (|x_i| |y_j|) (matrix product of the
+    raw vectors, divided by the outer product of their norms)."""
+    X = np.asarray(X, dtype=np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+    if cost == "cosine":
+        nx = np.sqrt(np.sum(X * X, axis=1))
+        ny = np.sqrt(np.sum(Y * Y, axis=1))
+        return 1.0 - (X @ Y.T) / (nx[:, None] * ny[None, :])
+    if cost != "sqeuclidean":
+        raise ValueError(f"unknown cost {cost!r}")
+    diff = X[:, None, :] - Y[None, :, :]
     return np.einsum("ijk,ijk->ij", diff, diff)
 
 

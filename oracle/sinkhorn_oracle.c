@@ -1,5 +1,5 @@
 /*
- * CPU oracle for log-domain Sinkhorn with squared-Euclidean cost.
+ * CPU oracle for log-domain Sinkhorn with squared-Euclidean or cosine cost.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
  * call this file; only the tests, the smoke check and the benchmark's CPU
@@ -13,6 +13,12 @@
  *   C_ij = |x_i - y_j|^2                         (evaluated directly as a sum of
  *                                                 squared differences, never in
  *                                                 the dot-product form)
+ *   or, for the cosine cost (the other cost whose structure the method covers,
+ *   per the closing remarks of the same page, "cosine distance after
+ *   normalisation"),
+ *   C_ij = 1 - x_i.y_j / (|x_i| |y_j|)           (from the raw vectors, in
+ *                                                 double; undefined for a zero
+ *                                                 vector)
  *   f_i  = -eps * LSE_j [ (g_j - C_ij)/eps + log b_j ]          (f-update)
  *   g_j  = -eps * LSE_i [ (f_i - C_ij)/eps + log a_i ]          (g-update, the
  *                                                 transpose of the f-update)
@@ -46,6 +52,25 @@ static inline double sq_dist(const double *p, const double *q, int d)
     return s;
 }
 
+/* 1 - cos(p, q) over d coordinates, from the dot product and the two norms. */
+static inline double cos_dist(const double *p, const double *q, int d)
+{
+    double pq = 0.0, pp = 0.0, qq = 0.0;
+#pragma omp simd reduction(+ : pq, pp, qq)
+    for (int k = 0; k < d; ++k) {
+        pq += p[k] * q[k];
+        pp += p[k] * p[k];
+        qq += q[k] * q[k];
+    }
+    return 1.0 - pq / (sqrt(pp) * sqrt(qq));
+}
+
+/* The cost between two points: cost 0 = squared Euclidean, 1 = cosine. */
+static inline double cost_ij(int cost, const double *p, const double *q, int d)
+{
+    return cost == 1 ? cos_dist(p, q, d) : sq_dist(p, q, d);
+}
+
 /*
  * One entry of a log-domain update seen from point p against the cloud pts:
  *   out = -eps * LSE_j [ (pot_j - |p - pts_j|^2)/eps + logw_j ]
@@ -54,11 +79,11 @@ static inline double sq_dist(const double *p, const double *q, int d)
 SO_CLONES
 static double soft_c_transform(const double *p, const double *pts, long cnt, int d,
                                const double *logw, const double *pot, double eps,
-                               double *buf)
+                               double *buf, int cost)
 {
     double mx = -INFINITY;
     for (long j = 0; j < cnt; ++j) {
-        double v = (pot[j] - sq_dist(p, pts + (size_t)j * d, d)) / eps + logw[j];
+        double v = (pot[j] - cost_ij(cost, p, pts + (size_t)j * d, d)) / eps + logw[j];
         buf[j] = v;
         if (v > mx)
             mx = v;
@@ -71,9 +96,10 @@ static double soft_c_transform(const double *p, const double *pts, long cnt, int
     return -eps * (mx + log(s));
 }
 
-/* out_i = -eps * LSE_j [ (pot_j - |P_i - Q_j|^2)/eps + logw_j ], i < np_. */
+/* out_i = -eps * LSE_j [ (pot_j - C(P_i, Q_j))/eps + logw_j ], i < np_. */
 static int soft_transform_all(long np_, long nq, int d, const double *P, const double *Q,
-                              const double *logw, const double *pot, double eps, double *out)
+                              const double *logw, const double *pot, double eps, double *out,
+                              int cost)
 {
     int fail = 0;
 #pragma omp parallel
@@ -85,7 +111,7 @@ static int soft_transform_all(long np_, long nq, int d, const double *P, const d
         } else {
 #pragma omp for schedule(dynamic, 16)
             for (long i = 0; i < np_; ++i)
-                out[i] = soft_c_transform(P + (size_t)i * d, Q, nq, d, logw, pot, eps, buf);
+                out[i] = soft_c_transform(P + (size_t)i * d, Q, nq, d, logw, pot, eps, buf, cost);
             free(buf);
         }
     }
@@ -94,16 +120,16 @@ static int soft_transform_all(long np_, long nq, int d, const double *P, const d
 
 /* f-update: f_i = -eps LSE_j[(g_j - C_ij)/eps + log b_j]. */
 int so_update_f(long n, long m, int d, const double *X, const double *Y, const double *logb,
-                const double *g, double eps, double *f)
+                const double *g, double eps, double *f, int cost)
 {
-    return soft_transform_all(n, m, d, X, Y, logb, g, eps, f);
+    return soft_transform_all(n, m, d, X, Y, logb, g, eps, f, cost);
 }
 
 /* g-update: g_j = -eps LSE_i[(f_i - C_ij)/eps + log a_i]  (C_ij = C_ji^T). */
 int so_update_g(long n, long m, int d, const double *X, const double *Y, const double *loga,
-                const double *f, double eps, double *g)
+                const double *f, double eps, double *g, int cost)
 {
-    return soft_transform_all(m, n, d, Y, X, loga, f, eps, g);
+    return soft_transform_all(m, n, d, Y, X, loga, f, eps, g, cost);
 }
 
 /*
@@ -112,12 +138,12 @@ int so_update_g(long n, long m, int d, const double *X, const double *Y, const d
  * the first half-step overwrites it); both hold the final pair on exit.
  */
 int so_solve(long n, long m, int d, const double *X, const double *Y, const double *loga,
-             const double *logb, double eps, int iters, double *f, double *g)
+             const double *logb, double eps, int iters, double *f, double *g, int cost)
 {
     for (int t = 0; t < iters; ++t) {
-        if (so_update_f(n, m, d, X, Y, logb, g, eps, f))
+        if (so_update_f(n, m, d, X, Y, logb, g, eps, f, cost))
             return -1;
-        if (so_update_g(n, m, d, X, Y, loga, f, eps, g))
+        if (so_update_g(n, m, d, X, Y, loga, f, eps, g, cost))
             return -1;
     }
     return 0;
@@ -125,17 +151,18 @@ int so_solve(long n, long m, int d, const double *X, const double *Y, const doub
 
 /*
  * Row sums of the plan, straight from its definition:
- *   out_i = sum_j exp(logwp_i + logwq_j + (potp_i + potq_j - |P_i - Q_j|^2)/eps)
+ *   out_i = sum_j exp(logwp_i + logwq_j + (potp_i + potq_j - C(P_i, Q_j))/eps)
  * With (P,Q)=(X,Y) this is the row marginal r_i; with (Y,X) the column
  * marginal c_j.
  */
 SO_CLONES
 static double plan_row_sum(const double *p, const double *Q, long nq, int d, double logwp_i,
-                           const double *logwq, double potp_i, const double *potq, double eps)
+                           const double *logwq, double potp_i, const double *potq, double eps,
+                           int cost)
 {
     double s = 0.0;
     for (long j = 0; j < nq; ++j) {
-        double c = sq_dist(p, Q + (size_t)j * d, d);
+        double c = cost_ij(cost, p, Q + (size_t)j * d, d);
         s += exp(logwp_i + logwq[j] + (potp_i + potq[j] - c) / eps);
     }
     return s;
@@ -143,22 +170,22 @@ static double plan_row_sum(const double *p, const double *Q, long nq, int d, dou
 
 static void plan_sums(long np_, long nq, int d, const double *P, const double *Q,
                       const double *logwp, const double *logwq, const double *potp,
-                      const double *potq, double eps, double *out)
+                      const double *potq, double eps, double *out, int cost)
 {
 #pragma omp parallel for schedule(dynamic, 16)
     for (long i = 0; i < np_; ++i)
-        out[i] = plan_row_sum(P + (size_t)i * d, Q, nq, d, logwp[i], logwq, potp[i], potq, eps);
+        out[i] = plan_row_sum(P + (size_t)i * d, Q, nq, d, logwp[i], logwq, potp[i], potq, eps, cost);
 }
 
 /* r_i = sum_j P_ij and c_j = sum_i P_ij. */
 void so_marginals(long n, long m, int d, const double *X, const double *Y, const double *loga,
                   const double *logb, const double *f, const double *g, double eps, double *r,
-                  double *c)
+                  double *c, int cost)
 {
     if (r)
-        plan_sums(n, m, d, X, Y, loga, logb, f, g, eps, r);
+        plan_sums(n, m, d, X, Y, loga, logb, f, g, eps, r, cost);
     if (c)
-        plan_sums(m, n, d, Y, X, logb, loga, g, f, eps, c);
+        plan_sums(m, n, d, Y, X, logb, loga, g, f, eps, c, cost);
 }
 
 /*
@@ -172,11 +199,11 @@ void so_marginals(long n, long m, int d, const double *X, const double *Y, const
 SO_CLONES
 static void plan_row_stats(const double *p, const double *Q, long nq, int d, double loga_i,
                            const double *logb, double f_i, const double *g, double eps,
-                           double *acc)
+                           double *acc, int cost)
 {
     double sp = 0.0, spc = 0.0, spl = 0.0, cmax = -INFINITY, cmin = INFINITY;
     for (long j = 0; j < nq; ++j) {
-        double c = sq_dist(p, Q + (size_t)j * d, d);
+        double c = cost_ij(cost, p, Q + (size_t)j * d, d);
         double lr = (f_i + g[j] - c) / eps;
         double pij = exp(loga_i + logb[j] + lr);
         sp += pij;
@@ -196,14 +223,14 @@ static void plan_row_stats(const double *p, const double *Q, long nq, int d, dou
 
 int so_plan_stats(long n, long m, int d, const double *X, const double *Y, const double *loga,
                   const double *logb, const double *f, const double *g, double eps,
-                  double *out)
+                  double *out, int cost)
 {
     double *rows = (double *)malloc(sizeof(double) * 5 * (size_t)(n > 0 ? n : 1));
     if (!rows)
         return -1;
 #pragma omp parallel for schedule(dynamic, 16)
     for (long i = 0; i < n; ++i)
-        plan_row_stats(X + (size_t)i * d, Y, m, d, loga[i], logb, f[i], g, eps, rows + 5 * i);
+        plan_row_stats(X + (size_t)i * d, Y, m, d, loga[i], logb, f[i], g, eps, rows + 5 * i, cost);
     double sp = 0.0, spc = 0.0, spl = 0.0, cmax = -INFINITY, cmin = INFINITY;
     for (long i = 0; i < n; ++i) {
         sp += rows[5 * i + 0];
@@ -227,11 +254,11 @@ int so_plan_stats(long n, long m, int d, const double *X, const double *Y, const
  * (the two sides of the c-transform sandwich for the f-update). */
 SO_CLONES
 static void row_minplus(const double *p, const double *Q, long nq, int d, const double *logw,
-                        const double *pot, double eps, double *lo, double *hi, double *cmax)
+                        const double *pot, double eps, double *lo, double *hi, double *cmax, int cost)
 {
     double l = INFINITY, h = INFINITY, cm = -INFINITY;
     for (long j = 0; j < nq; ++j) {
-        double c = sq_dist(p, Q + (size_t)j * d, d);
+        double c = cost_ij(cost, p, Q + (size_t)j * d, d);
         double v = c - pot[j];
         if (v < l)
             l = v;
@@ -248,17 +275,17 @@ static void row_minplus(const double *p, const double *Q, long nq, int d, const 
 
 void so_minplus_bounds(long np_, long nq, int d, const double *P, const double *Q,
                        const double *logw, const double *pot, double eps, double *lo,
-                       double *hi, double *cmax_row)
+                       double *hi, double *cmax_row, int cost)
 {
 #pragma omp parallel for schedule(dynamic, 16)
     for (long i = 0; i < np_; ++i)
-        row_minplus(P + (size_t)i * d, Q, nq, d, logw, pot, eps, lo + i, hi + i, cmax_row + i);
+        row_minplus(P + (size_t)i * d, Q, nq, d, logw, pot, eps, lo + i, hi + i, cmax_row + i, cost);
 }
 
 /* Selected rows of the f-update (sampled parity at sizes where a full pass is too slow). */
 int so_update_f_rows(long nrows, const long *rows, long m, int d, const double *X,
                      const double *Y, const double *logb, const double *g, double eps,
-                     double *f_rows)
+                     double *f_rows, int cost)
 {
     int fail = 0;
 #pragma omp parallel
@@ -271,7 +298,7 @@ int so_update_f_rows(long nrows, const long *rows, long m, int d, const double *
 #pragma omp for schedule(dynamic, 1)
             for (long k = 0; k < nrows; ++k)
                 f_rows[k] =
-                    soft_c_transform(X + (size_t)rows[k] * d, Y, m, d, logb, g, eps, buf);
+                    soft_c_transform(X + (size_t)rows[k] * d, Y, m, d, logb, g, eps, buf, cost);
             free(buf);
         }
     }

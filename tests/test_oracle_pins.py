@@ -244,3 +244,74 @@ def test_planted_mistakes_fail_a_pin(mutant):
     # agreement with the oracle
     oracle_ok = np.allclose(f_bad, oracle.update_f(X, Y, logb, g, eps), rtol=1e-10, atol=1e-10)
     assert not marg_ok and not oracle_ok
+
+
+# ---- cosine cost ("cosine distance after normalisation", the second cost the
+# method covers per the closing remarks of "FlashSinkhorn: IO-aware EOT on GPU")
+
+def test_cosine_cost_matrix_matches_scipy_cdist():
+    X, Y, _, _ = _rand_problem(19, 21, 7, 31)
+    np.testing.assert_allclose(dense.cost_matrix(X, Y, "cosine"), cdist(X, Y, "cosine"), rtol=1e-12,
+                               atol=1e-13)
+
+
+@pytest.mark.parametrize("n,m,d", [(37, 53, 5), (1, 9, 3), (40, 40, 128)])
+def test_cosine_streaming_matches_dense(n, m, d):
+    X, Y, loga, logb = _rand_problem(n, m, d, 40 + n + m)
+    rng = np.random.default_rng(8)
+    g = 0.1 * rng.standard_normal(m)
+    f0 = 0.1 * rng.standard_normal(n)
+    eps = 0.05
+    C = dense.cost_matrix(X, Y, "cosine")
+    np.testing.assert_allclose(oracle.update_f(X, Y, logb, g, eps, cost="cosine"),
+                               dense.update_f(C, logb, g, eps), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(oracle.update_g(X, Y, loga, f0, eps, cost="cosine"),
+                               dense.update_g(C, loga, f0, eps), rtol=1e-12, atol=1e-12)
+    rows = np.array([0, n - 1])
+    np.testing.assert_allclose(oracle.update_f_rows(rows, X, Y, logb, g, eps, cost="cosine"),
+                               dense.update_f(C, logb, g, eps)[rows], rtol=1e-12, atol=1e-12)
+    fs, gs = oracle.solve(X, Y, loga, logb, eps, 20, cost="cosine")
+    fd, gd = dense.solve(C, loga, logb, eps, 20)
+    np.testing.assert_allclose(fs, fd, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(gs, gd, rtol=1e-10, atol=1e-10)
+    co = oracle.costs(X, Y, loga, logb, fs, gs, eps, cost="cosine")
+    cd = dense.costs(C, loga, logb, fd, gd, eps)
+    for key in ("dual", "primal", "entropic_primal", "sum_p"):
+        assert abs(co[key] - cd[key]) <= 1e-10 * max(1.0, abs(cd[key])), key
+    assert abs(co["max_cost"] - C.max()) <= 1e-14 and abs(co["min_cost"] - C.min()) <= 1e-14
+
+
+def test_cosine_on_the_sphere_is_half_the_squared_distance():
+    """For unit vectors |x - y|^2 = 2 (1 - cos): the cosine solve at eps equals half
+    the squared-Euclidean solve at 2 eps (f-update: -eps LSE[(g - C/2)/eps + log b]
+    = (1/2)(-2 eps LSE[(2g - C)/(2 eps) + log b]), so every iterate is halved)."""
+    X, Y, loga, logb = _rand_problem(30, 25, 4, 55)
+    X /= np.linalg.norm(X, axis=1, keepdims=True)
+    Y /= np.linalg.norm(Y, axis=1, keepdims=True)
+    eps = 0.07
+    fc, gc = oracle.solve(X, Y, loga, logb, eps, 15, cost="cosine")
+    fq, gq = oracle.solve(X, Y, loga, logb, 2 * eps, 15)
+    np.testing.assert_allclose(fc, 0.5 * fq, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(gc, 0.5 * gq, rtol=1e-11, atol=1e-12)
+
+
+def test_cosine_is_scale_invariant_and_marginal_exact():
+    X, Y, loga, logb = _rand_problem(24, 31, 6, 56)
+    rng = np.random.default_rng(57)
+    sx = rng.uniform(0.2, 5.0, (24, 1))
+    sy = rng.uniform(0.2, 5.0, (31, 1))
+    eps = 0.05
+    f1, g1 = oracle.solve(X, Y, loga, logb, eps, 10, cost="cosine")
+    f2, g2 = oracle.solve(X * sx, Y * sy, loga, logb, eps, 10, cost="cosine")
+    np.testing.assert_allclose(f1, f2, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(g1, g2, rtol=1e-11, atol=1e-12)
+    # after the closing g-update the column marginal is exact
+    _, c = oracle.marginals(X, Y, loga, logb, f1, g1, eps, cost="cosine")
+    np.testing.assert_allclose(c, np.exp(logb), rtol=1e-12)
+
+
+def test_cosine_rejects_zero_vectors():
+    X, Y, loga, logb = _rand_problem(5, 6, 3, 58)
+    X[2] = 0.0
+    with pytest.raises(ValueError):
+        oracle.update_f(X, Y, logb, np.zeros(6), 0.1, cost="cosine")
