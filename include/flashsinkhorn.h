@@ -74,12 +74,27 @@ typedef enum {
     FS_SCHED_SYMMETRIC = 1    /* f and g both from the previous pair (Jacobi)     */
 } fs_schedule;
 
+/*
+ * Ground cost C_ij ("FlashSinkhorn: IO-aware EOT on GPU": the squared
+ * Euclidean cost of Proposition 1, and the cosine distance after
+ * normalisation that the closing remarks name as the other cost the method
+ * covers).
+ *   FS_COST_SQEUCLIDEAN  C_ij = |x_i - y_j|^2
+ *   FS_COST_COSINE       C_ij = 1 - x_i.y_j / (|x_i| |y_j|); X and Y rows must
+ *                        be non-zero (FS_ERR_INVALID_ARG otherwise).  Rows are
+ *                        normalised in fp32 on the device; the default
+ *                        precision is then 3xF16 for d <= 128 whatever the
+ *                        input dtype (normalised bf16 rows are no longer bf16).
+ */
+typedef enum { FS_COST_SQEUCLIDEAN = 0, FS_COST_COSINE = 1 } fs_cost;
+
 typedef struct {
     int batch;          /* independent problems sharing n, m, d, eps            */
     int n, m, d;        /* points in X, in Y, and their dimension               */
     fs_dtype dtype;     /* element type of X and Y                              */
     fs_precision prec;  /* score-product precision                              */
     float eps;          /* entropic regularisation, absolute units of C         */
+    fs_cost cost;       /* ground cost (0 = squared Euclidean)                  */
 } fs_desc;
 
 typedef struct fs_handle fs_handle;

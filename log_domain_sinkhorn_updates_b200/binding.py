@@ -20,6 +20,7 @@ FS_F32, FS_BF16 = 0, 1
 PRECISIONS = {"auto": 0, "bf16": 1, "tf32": 2, "3xtf32": 3, "3xf16": 4, "f32_simt": 5}
 PRECISION_NAMES = {v: k for k, v in PRECISIONS.items()}
 SCHEDULES = {"alternating": 0, "symmetric": 1}
+COSTS = {"sqeuclidean": 0, "cosine": 1}
 STATUS_NAMES = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_CUDA", 3: "FS_ERR_UNSUPPORTED",
                 4: "FS_ERR_NONFINITE", 5: "FS_ERR_TIMEOUT", 6: "FS_ERR_OOM"}
 
@@ -30,7 +31,7 @@ EXPORTS = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_e
 
 class FsDesc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int), ("n", ctypes.c_int), ("m", ctypes.c_int), ("d", ctypes.c_int),
-                ("dtype", ctypes.c_int), ("prec", ctypes.c_int), ("eps", ctypes.c_float)]
+                ("dtype", ctypes.c_int), ("prec", ctypes.c_int), ("eps", ctypes.c_float), ("cost", ctypes.c_int)]
 
 
 class FsInfo(ctypes.Structure):
@@ -143,8 +144,9 @@ class Handle:
             pass
 
 
-def fs_create(X, Y, a=None, b=None, eps=0.1, prec="auto", stream=None) -> Handle:
-    """X [batch, n, d] / [n, d], Y likewise (CUDA float32 or bfloat16), a [batch, n], b [batch, m] or None."""
+def fs_create(X, Y, a=None, b=None, eps=0.1, prec="auto", stream=None, cost="sqeuclidean") -> Handle:
+    """X [batch, n, d] / [n, d], Y likewise (CUDA float32 or bfloat16), a [batch, n], b [batch, m] or None.
+    cost: "sqeuclidean" (C = |x - y|^2) or "cosine" (C = 1 - cos(x, y))."""
     import torch
     if X.dim() == 2:
         X, Y = X.unsqueeze(0), Y.unsqueeze(0)
@@ -159,7 +161,8 @@ def fs_create(X, Y, a=None, b=None, eps=0.1, prec="auto", stream=None) -> Handle
     m = Y.shape[1]
     if Y.shape[0] != B or Y.shape[2] != d:
         raise ValueError("X and Y shapes disagree")
-    desc = FsDesc(B, n, m, d, dtype, PRECISIONS[prec] if isinstance(prec, str) else int(prec), float(eps))
+    desc = FsDesc(B, n, m, d, dtype, PRECISIONS[prec] if isinstance(prec, str) else int(prec), float(eps),
+                  COSTS[cost])
     out = ctypes.c_void_p()
     st = lib().fs_create(ctypes.byref(desc), _ptr(X), _ptr(Y), _f32(a), _f32(b), _stream_ptr(stream),
                          ctypes.byref(out))
@@ -234,7 +237,7 @@ def fs_kernel_launches() -> int:
 
 
 def fs_solve_host(X, Y, a, b, g0, eps, iters, dtype="f32", prec="auto", schedule="alternating", stream=None,
-                  measure=True, out=None):
+                  measure=True, out=None, cost="sqeuclidean"):
     """End-to-end solve from host (numpy) arrays through ``fs_solve_host``.
 
     X, Y: [batch, n|m, d] float32 (or uint16 bfloat16 bits with dtype="bf16"),
@@ -247,7 +250,7 @@ def fs_solve_host(X, Y, a, b, g0, eps, iters, dtype="f32", prec="auto", schedule
         X, Y = X[None], Y[None]
     B, n, d = X.shape
     m = Y.shape[1]
-    desc = FsDesc(B, n, m, d, FS_BF16 if dtype == "bf16" else FS_F32, PRECISIONS[prec], float(eps))
+    desc = FsDesc(B, n, m, d, FS_BF16 if dtype == "bf16" else FS_F32, PRECISIONS[prec], float(eps), COSTS[cost])
     if out is None:
         f = np.empty((B, n), np.float32)
         g = np.array(g0, dtype=np.float32).reshape(B, m)

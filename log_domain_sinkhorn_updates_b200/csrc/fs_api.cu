@@ -293,6 +293,8 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     if (!(D.eps > 0.f) || !std::isfinite(D.eps))
         return fail(nullptr, FS_ERR_INVALID_ARG, "eps must be finite and > 0");
     if (D.dtype != FS_F32 && D.dtype != FS_BF16) return fail(nullptr, FS_ERR_INVALID_ARG, "unknown dtype");
+    if (D.cost != FS_COST_SQEUCLIDEAN && D.cost != FS_COST_COSINE)
+        return fail(nullptr, FS_ERR_INVALID_ARG, "unknown cost");
     if (D.prec != FS_PREC_AUTO && D.prec != FS_PREC_BF16 && D.prec != FS_PREC_TF32 && D.prec != FS_PREC_3XTF32 &&
         D.prec != FS_PREC_3XF16 && D.prec != FS_PREC_F32_SIMT)
         return fail(nullptr, FS_ERR_INVALID_ARG, "unknown precision");
@@ -326,8 +328,9 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
 
     // ---- precision and packed layout ----
     int prec = D.prec;
-    if (prec == FS_PREC_AUTO)
-        prec = D.dtype == FS_BF16 ? FS_PREC_BF16 : (D.d <= 128 ? FS_PREC_3XF16 : FS_PREC_F32_SIMT);
+    const bool cosine = D.cost == FS_COST_COSINE;
+    if (prec == FS_PREC_AUTO)  // normalised rows are fp32 values, whatever the input dtype
+        prec = (D.dtype == FS_BF16 && !cosine) ? FS_PREC_BF16 : (D.d <= 128 ? FS_PREC_3XF16 : FS_PREC_F32_SIMT);
     h->prec = prec;
     if (prec == FS_PREC_F32_SIMT) {
         if (D.d > 256) {
@@ -473,7 +476,8 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         FS_CUDA(h, cudaMemsetAsync(h->counters, 0, B * max_rb * 4, h->stream));
         FS_CUDA(h, cudaMemsetAsync(h->err, 0, 16, h->stream));
         const float *t = nullptr;
-        if (!bf16) {
+        const bool cosine = D.cost == FS_COST_COSINE;  // normalised rows; C is not translation-invariant
+        if (!bf16 && !cosine) {
             FS_LAUNCH(h, fs::launch_center(X, Y, bf16, D.batch, D.n, D.m, D.d, h->center, h->stream));
             t = h->center;
         }
@@ -481,12 +485,14 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             // Power-of-two scales putting each cloud's largest |value| (Y side
             // counted with its factor 2) at most 2^14: exact, and far from the
             // fp16 overflow; the MMA's raw score is divided back by their product.
-            float *mx = reinterpret_cast<float *>(h->wstat + 4 * B);
-            FS_LAUNCH(h, fs::launch_maxabs(X, bf16, D.n, D.d, D.batch, t, mx, h->stream));
-            FS_LAUNCH(h, fs::launch_maxabs(Y, bf16, D.m, D.d, D.batch, t, mx + 1, h->stream));
-            float hm[2] = {0.f, 0.f};
-            FS_CUDA(h, cudaMemcpyAsync(hm, mx, sizeof(hm), cudaMemcpyDeviceToHost, h->stream));
-            FS_CUDA(h, cudaStreamSynchronize(h->stream));
+            float hm[2] = {1.f, 0.5f};  // normalised rows: |value| <= 1 on both sides (Y counted x2 below)
+            if (!cosine) {
+                float *mx = reinterpret_cast<float *>(h->wstat + 4 * B);
+                FS_LAUNCH(h, fs::launch_maxabs(X, bf16, D.n, D.d, D.batch, t, mx, h->stream));
+                FS_LAUNCH(h, fs::launch_maxabs(Y, bf16, D.m, D.d, D.batch, t, mx + 1, h->stream));
+                FS_CUDA(h, cudaMemcpyAsync(hm, mx, sizeof(hm), cudaMemcpyDeviceToHost, h->stream));
+                FS_CUDA(h, cudaStreamSynchronize(h->stream));
+            }
             auto pow2_scale = [](float maxabs) {
                 if (!(maxabs > 0.f) || !std::isfinite(maxabs)) return 1.f;
                 return std::ldexp(1.f, 14 - (int)std::ceil(std::log2((double)maxabs)));
@@ -497,10 +503,12 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         }
         FS_CUDA(h, cudaMemsetAsync(h->xn, 0, B * h->n_stride * 4, h->stream));
         FS_CUDA(h, cudaMemsetAsync(h->yn, 0, B * h->m_stride * 4, h->stream));
+        // K = 2(Y - t) for the squared Euclidean cost, K = Y/|Y| for the cosine cost
         FS_LAUNCH(h, fs::launch_pack(X, bf16, D.n, h->n_pad, D.d, D.batch, t, h->qscale, h->pack_mode, h->d_p,
-                                     h->row_elems, h->packX, h->xn, h->n_stride, h->err, h->stream));
-        FS_LAUNCH(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, 2.f * h->kscale, h->pack_mode, h->d_p,
-                                     h->row_elems, h->packY, h->yn, h->m_stride, h->err, h->stream));
+                                     h->row_elems, h->packX, h->xn, h->n_stride, h->err, h->stream, cosine));
+        FS_LAUNCH(h, fs::launch_pack(Y, bf16, D.m, h->m_pad, D.d, D.batch, t, (cosine ? 1.f : 2.f) * h->kscale,
+                                     h->pack_mode, h->d_p, h->row_elems, h->packY, h->yn, h->m_stride, h->err,
+                                     h->stream, cosine));
         FS_LAUNCH(h, fs::launch_weights(a, D.batch, D.n, h->n_stride, h->la2, h->wstat, h->stream));
         FS_LAUNCH(h, fs::launch_weights(b, D.batch, D.m, h->m_stride, h->lb2, h->wstat + 2 * B, h->stream));
         FS_LAUNCH(h, fs::launch_fill(h->bias_row, B * h->n_stride, -INFINITY, h->stream));
@@ -518,6 +526,8 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
                             is_a ? "a" : "b", is_a ? k : k - B, s);
         }
         if (h->host_err[0] & fs::kDevErrNonfinite) return fail(h, FS_ERR_NONFINITE, "non-finite value in X or Y");
+        if (h->host_err[0] & fs::kDevErrZeroRow)
+            return fail(h, FS_ERR_INVALID_ARG, "the cosine cost is undefined for a zero row of X or Y");
         if (prec != FS_PREC_F32_SIMT) {
             fs_status s2 = encode_map(h, &h->mapX_r, h->packX, D.batch * h->n_pad, kBlockRows);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, kBlockCols);

@@ -29,6 +29,7 @@ constexpr double kLog2ed = 1.44269504088896340736;
 constexpr int kDevErrNonfinite = 1;
 constexpr int kDevErrTimeout = 2;
 constexpr int kDevErrBadWeights = 4;
+constexpr int kDevErrZeroRow = 8;  // a zero row under the cosine cost
 
 // Parameters of one streamed LSE pass (row side R against column side C).
 struct PassParams {

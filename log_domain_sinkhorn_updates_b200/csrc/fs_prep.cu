@@ -54,9 +54,11 @@ __device__ __forceinline__ float round_tf32(float x) {
 
 // One warp per padded row: v = src - t (fp32), packed = scale * v in the
 // layout of `mode`, norm = |v|^2 (double accumulation, fixed shuffle tree).
+// With `normalize`, v = src / |src| instead and norm = 1/2 (cosine cost).
 template <typename T>
 __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int batch, const float *t, float scale,
-                            int mode, int d_p, int row_elems, void *dst, float *norm, int norm_stride, int *err) {
+                            int mode, int d_p, int row_elems, void *dst, float *norm, int norm_stride, int *err,
+                            bool normalize) {
     const int lane = threadIdx.x & 31;
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
@@ -65,6 +67,21 @@ __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int bat
         const bool valid = r < rows;
         double acc = 0.0;
         bool bad = false;
+        float inv = 1.f;
+        if (normalize) {
+            double ss = 0.0;
+            if (valid)
+                for (int k = lane; k < d; k += 32) {
+                    const double x = load_val(src, ((size_t)bz * rows + r) * d + k);
+                    ss += x * x;
+                }
+            for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if (valid && !(ss > 0.0)) {
+                if (lane == 0) atomicOr(err, kDevErrZeroRow);
+            } else if (valid) {
+                inv = (float)(1.0 / sqrt(ss));
+            }
+        }
         for (int e = lane; e < row_elems; e += 32) {
             float v = 0.f;
             int k = e;
@@ -77,7 +94,7 @@ __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int bat
             if (valid && k < d) {
                 float x = load_val(src, ((size_t)bz * rows + r) * d + k);
                 if (!isfinite(x)) bad = true;
-                v = x - (t ? t[(size_t)bz * d + k] : 0.f);
+                v = normalize ? x * inv : x - (t ? t[(size_t)bz * d + k] : 0.f);
             }
             float out;
             if (mode == kPackBf16) {
@@ -112,7 +129,7 @@ __global__ void pack_kernel(const T *src, int rows, int rows_pad, int d, int bat
         }
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
         if (bad) atomicOr(err, kDevErrNonfinite);
-        if (lane == 0) norm[(size_t)bz * norm_stride + r] = valid ? (float)acc : 0.f;
+        if (lane == 0) norm[(size_t)bz * norm_stride + r] = valid ? (normalize ? 0.5f : (float)acc) : 0.f;
     }
 }
 
@@ -226,15 +243,15 @@ cudaError_t launch_center(const void *X, const void *Y, bool bf16, int batch, in
 
 cudaError_t launch_pack(const void *src, bool bf16, int rows, int rows_pad, int d, int batch, const float *t,
                         float scale, int mode, int d_p, int row_elems, void *dst, float *norm, int norm_stride,
-                        int *err, cudaStream_t s) {
+                        int *err, cudaStream_t s, bool normalize) {
     const size_t warps = (size_t)batch * rows_pad;
     const int grid = grid_for(warps * 32, 256);
     if (bf16)
         pack_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), rows, rows_pad, d, batch, t,
-                                        scale, mode, d_p, row_elems, dst, norm, norm_stride, err);
+                                        scale, mode, d_p, row_elems, dst, norm, norm_stride, err, normalize);
     else
         pack_kernel<<<grid, 256, 0, s>>>(static_cast<const float *>(src), rows, rows_pad, d, batch, t, scale,
-                                        mode, d_p, row_elems, dst, norm, norm_stride, err);
+                                        mode, d_p, row_elems, dst, norm, norm_stride, err, normalize);
     return cudaGetLastError();
 }
 

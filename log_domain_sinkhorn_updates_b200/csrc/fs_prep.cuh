@@ -14,9 +14,13 @@ constexpr int kPack3xF16 = 4;   // [hi | lo] fp16 planes of the scaled value, hi
 
 cudaError_t launch_center(const void *X, const void *Y, bool bf16, int batch, int n, int m, int d, float *t,
                           cudaStream_t s);
+// normalize: divide each row by its Euclidean norm first (cosine cost; t must
+// be null) and store 1/2 as its squared norm: with the column side packed at
+// scale 1 instead of 2, |q|^2 + |k|^2 - q.k = 1/2 + 1/2 - cos = 1 - cos.
+// A zero row raises kDevErrZeroRow.
 cudaError_t launch_pack(const void *src, bool bf16, int rows, int rows_pad, int d, int batch, const float *t,
                         float scale, int mode, int d_p, int row_elems, void *dst, float *norm, int norm_stride,
-                        int *err, cudaStream_t s);
+                        int *err, cudaStream_t s, bool normalize = false);
 // out[0] = max over every problem of |src - t| (fp32), for the 3xF16 scaling.
 cudaError_t launch_maxabs(const void *src, bool bf16, int rows, int d, int batch, const float *t, float *out,
                           cudaStream_t s);

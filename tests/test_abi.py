@@ -48,7 +48,7 @@ def test_invalid_arguments_rejected_on_host(L):
     dummy = ctypes.c_void_p(16)
     for desc in [FsDesc(1, 0, 5, 3, 0, 0, 0.1), FsDesc(1, 5, 5, 0, 0, 0, 0.1), FsDesc(0, 5, 5, 3, 0, 0, 0.1),
                  FsDesc(1, 5, 5, 3, 0, 0, 0.0), FsDesc(1, 5, 5, 3, 0, 0, float("nan")),
-                 FsDesc(1, 5, 5, 3, 7, 0, 0.1), FsDesc(1, 5, 5, 3, 0, 9, 0.1)]:
+                 FsDesc(1, 5, 5, 3, 7, 0, 0.1), FsDesc(1, 5, 5, 3, 0, 9, 0.1), FsDesc(1, 5, 5, 3, 0, 0, 0.1, 7)]:
         st = L.fs_create(ctypes.byref(desc), dummy, dummy, None, None, None, ctypes.byref(out))
         assert st == FS_ERR_INVALID_ARG
         assert out.value is None
