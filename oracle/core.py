@@ -38,9 +38,10 @@ def _load():
         lib.so_plan_stats.argtypes = [L, L, I, _dp, _dp, _dp, _dp, _dp, _dp, D, _dp, I]
         lib.so_minplus_bounds.argtypes = [L, L, I, _dp, _dp, _dp, _dp, D, _dp, _dp, _dp, I]
         lib.so_update_f_rows.argtypes = [L, _lp, L, I, _dp, _dp, _dp, _dp, D, _dp, I]
+        lib.so_transport_apply.argtypes = [L, L, I, _dp, _dp, _dp, _dp, _dp, _dp, D, I, _dp, _dp, _dp, I]
         lib.so_num_threads.argtypes = []
         for name in ("so_update_f", "so_update_g", "so_solve", "so_plan_stats", "so_update_f_rows",
-                     "so_num_threads"):
+                     "so_transport_apply", "so_num_threads"):
             getattr(lib, name).restype = ctypes.c_int
         lib.so_marginals.restype = None
         lib.so_minplus_bounds.restype = None
@@ -230,3 +231,43 @@ def minplus_bounds(X, Y, logb, g, eps, cost="sqeuclidean"):
 
 
 os.environ.setdefault("OMP_WAIT_POLICY", "PASSIVE")
+
+
+def transport_apply(X, Y, loga, logb, f, g, eps, V, cost="sqeuclidean"):
+    """(out, r): out_i = sum_j P_ij V_j and r_i = sum_j P_ij for P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps)
+    ("FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 3: applying the plan without forming it)."""
+    ci = _cost(cost, X, Y)
+    X, px = _c(X)
+    Y, py = _c(Y)
+    loga, pa = _c(loga)
+    logb, pb = _c(logb)
+    f, pf = _c(f)
+    g, pg = _c(g)
+    V = np.asarray(V, dtype=np.float64)
+    V = V.reshape(V.shape[0], -1)
+    V, pv = _c(V)
+    n, d = X.shape
+    m = Y.shape[0]
+    if V.shape[0] != m:
+        raise ValueError("V must have one row per column point")
+    dv = V.shape[1]
+    out = np.empty((n, dv))
+    r = np.empty(n)
+    _load().so_transport_apply(n, m, d, px, py, pa, pb, pf, pg, float(eps), dv, pv, out.ctypes.data_as(_dp),
+                               r.ctypes.data_as(_dp), ci)
+    return out, r
+
+
+def barycentric_projection(X, Y, loga, logb, f, g, eps, cost="sqeuclidean"):
+    """T(x_i) = sum_j P_ij y_j / sum_j P_ij (the plan's barycentric map)."""
+    out, r = transport_apply(X, Y, loga, logb, f, g, eps, Y, cost)
+    return out / r[:, None]
+
+
+def grad_x(X, Y, loga, logb, f, g, eps):
+    """Gradient of the entropic OT cost with respect to the positions X at the
+    potentials (f, g), squared-Euclidean cost: sum_j P_ij dC_ij/dx_i =
+    2 (r_i x_i - sum_j P_ij y_j).  At optimal potentials this is the gradient of
+    the optimal value (envelope theorem)."""
+    out, r = transport_apply(X, Y, loga, logb, f, g, eps, Y)
+    return 2.0 * (r[:, None] * np.asarray(X, dtype=np.float64) - out)

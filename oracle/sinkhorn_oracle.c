@@ -305,6 +305,37 @@ int so_update_f_rows(long nrows, const long *rows, long m, int d, const double *
     return fail ? -1 : 0;
 }
 
+/*
+ * Transport application ("FlashSinkhorn: IO-aware EOT on GPU", Metodologia
+ * section 3: barycentric projection and gradient as weighted averages under
+ * the plan), straight from the plan's definition:
+ *   out_i = sum_j P_ij V_j   (V: [m][dv]),   r_i = sum_j P_ij,
+ *   P_ij  = a_i b_j exp((f_i + g_j - C_ij)/eps).
+ * Each row is summed in column order.
+ */
+int so_transport_apply(long n, long m, int d, const double *X, const double *Y, const double *loga,
+                       const double *logb, const double *f, const double *g, double eps, int dv,
+                       const double *V, double *out, double *r, int cost)
+{
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long i = 0; i < n; ++i) {
+        double *o = out + (size_t)i * dv;
+        for (int c = 0; c < dv; ++c)
+            o[c] = 0.0;
+        double s = 0.0;
+        for (long j = 0; j < m; ++j) {
+            double cij = cost_ij(cost, X + (size_t)i * d, Y + (size_t)j * d, d);
+            double p = exp(loga[i] + logb[j] + (f[i] + g[j] - cij) / eps);
+            s += p;
+            const double *v = V + (size_t)j * dv;
+            for (int c = 0; c < dv; ++c)
+                o[c] += p * v[c];
+        }
+        r[i] = s;
+    }
+    return 0;
+}
+
 int so_num_threads(void)
 {
     int t = 1;

@@ -315,3 +315,65 @@ def test_cosine_rejects_zero_vectors():
     X[2] = 0.0
     with pytest.raises(ValueError):
         oracle.update_f(X, Y, logb, np.zeros(6), 0.1, cost="cosine")
+
+
+# ---- transport application (Metodologia section 3 of "FlashSinkhorn: IO-aware
+# EOT on GPU": barycentric projection and gradient as plan-weighted averages)
+
+@pytest.mark.parametrize("cost", ["sqeuclidean", "cosine"])
+def test_transport_apply_matches_dense_plan(cost):
+    X, Y, loga, logb = _rand_problem(23, 31, 4, 70)
+    rng = np.random.default_rng(71)
+    f = 0.2 * rng.standard_normal(23)
+    g = 0.2 * rng.standard_normal(31)
+    V = rng.standard_normal((31, 5))
+    eps = 0.3
+    out, r = oracle.transport_apply(X, Y, loga, logb, f, g, eps, V, cost=cost)
+    P = dense.plan(dense.cost_matrix(X, Y, cost), loga, logb, f, g, eps)
+    np.testing.assert_allclose(out, P @ V, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(r, P.sum(axis=1), rtol=1e-12)
+    # V = 1 gives the row marginal
+    ones, _ = oracle.transport_apply(X, Y, loga, logb, f, g, eps, np.ones((31, 1)), cost=cost)
+    np.testing.assert_allclose(ones[:, 0], oracle.marginals(X, Y, loga, logb, f, g, eps, cost=cost)[0], rtol=1e-12)
+
+
+def test_grad_x_matches_finite_differences_of_the_optimal_value():
+    """At optimal potentials the entropic OT value (the dual) has gradient
+    sum_j P_ij dC_ij/dx_i with respect to x_i (envelope theorem)."""
+    rng = np.random.default_rng(72)
+    n, m, d, eps = 6, 5, 2, 0.5
+    X = rng.standard_normal((n, d))
+    Y = rng.standard_normal((m, d))
+    a = rng.uniform(0.5, 1.5, n)
+    b = rng.uniform(0.5, 1.5, m)
+    loga, logb = np.log(a / a.sum()), np.log(b / b.sum())
+
+    def value(Xv):
+        f, g = oracle.solve(Xv, Y, loga, logb, eps, 400)
+        return oracle.costs(Xv, Y, loga, logb, f, g, eps)["dual"], f, g
+
+    _, f, g = value(X)
+    G = oracle.grad_x(X, Y, loga, logb, f, g, eps)
+    h = 1e-5
+    for i in range(n):
+        for k in range(d):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[i, k] += h
+            Xm[i, k] -= h
+            fd = (value(Xp)[0] - value(Xm)[0]) / (2 * h)
+            assert abs(G[i, k] - fd) <= 1e-8, (i, k, G[i, k], fd)
+
+
+def test_barycentric_projection_tends_to_the_optimal_assignment():
+    """Uniform weights, n = m: as eps -> 0 the plan tends to an optimal permutation
+    (here unique), so the barycentric map sends x_i to its assigned y (Hungarian
+    algorithm, scipy's linear_sum_assignment)."""
+    from scipy.optimize import linear_sum_assignment
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((8, 2))
+    Y = rng.standard_normal((8, 2)) + 0.2
+    loga = logb = np.full(8, -np.log(8))
+    f, g = oracle.solve(X, Y, loga, logb, 0.02, 3000)
+    T = oracle.barycentric_projection(X, Y, loga, logb, f, g, 0.02)
+    _, cols = linear_sum_assignment(dense.cost_matrix(X, Y))
+    assert np.abs(T - Y[cols]).max() < 1e-2
