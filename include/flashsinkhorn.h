@@ -182,6 +182,33 @@ FS_API fs_status fs_get_info(const fs_handle *h, fs_info *info);
  * already enqueued that uses the handle completes first.  NULL is accepted. */
 FS_API fs_status fs_destroy(fs_handle *h);
 
+/*
+ * Transport application ("FlashSinkhorn: IO-aware EOT on GPU", Metodologia
+ * section 3: the barycentric projection and the gradient as plan-weighted
+ * averages, computed without forming the plan).  At device potentials (f, g),
+ * with P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps) of each problem k:
+ *   out[k][i][c] = sum_j P_ij V[k][j][c]      (V: device fp32 [batch][m][dv])
+ *   r[k][i]      = sum_j P_ij                 (device [batch][n]; may be NULL)
+ * out: device fp32 [batch][n][dv].  Scores come from the handle's packed
+ * operands (its precision); the exponent is formed in double and the sums in
+ * fp32.  Asynchronous.  Errors: FS_ERR_INVALID_ARG (null pointer, dv < 1).
+ */
+FS_API fs_status fs_transport_apply(fs_handle *h, const float *f, const float *g, const float *V, int dv,
+                                    float *out, float *r);
+
+/* Barycentric map T(x_i) = sum_j P_ij y_j / sum_j P_ij: Y is the caller's
+ * device [batch][m][d] cloud in the handle's dtype (the handle keeps only its
+ * packed form); out: device fp32 [batch][n][d].  Asynchronous. */
+FS_API fs_status fs_barycentric_map(fs_handle *h, const float *f, const float *g, const void *Y, float *out);
+
+/* Gradient of the entropic OT cost with respect to the positions X at (f, g),
+ * squared Euclidean cost: grad_i = sum_j P_ij 2 (x_i - y_j) = 2 (r_i x_i -
+ * sum_j P_ij y_j) (at optimal potentials, the gradient of the optimal value).
+ * X, Y: the caller's device clouds in the handle's dtype; grad: device fp32
+ * [batch][n][d].  FS_ERR_UNSUPPORTED for the cosine cost.  Asynchronous. */
+FS_API fs_status fs_grad_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
+                           float *grad);
+
 /* Number of CUDA kernels this library has launched in this process so far
  * (all handles, all threads).  Host-side counter; never synchronises. */
 FS_API unsigned long long fs_kernel_launches(void);

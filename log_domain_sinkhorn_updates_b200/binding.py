@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_CUDA", 3: "FS_ER
 
 EXPORTS = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_err", "fs_ot_cost",
            "fs_sync", "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches",
-           "fs_update_f_noalloc"]
+           "fs_update_f_noalloc", "fs_transport_apply", "fs_barycentric_map", "fs_grad_x"]
 
 
 class FsDesc(ctypes.Structure):
@@ -79,6 +79,9 @@ def lib():
                                     dp, dp, dp, dp, vp]
         L.fs_update_f_noalloc.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, vp, vp, vp, vp,
                                           vp, vp]
+        L.fs_transport_apply.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp]
+        L.fs_barycentric_map.argtypes = [vp, vp, vp, vp, vp]
+        L.fs_grad_x.argtypes = [vp, vp, vp, vp, vp, vp]
         L.fs_kernel_launches.argtypes = []
         L.fs_kernel_launches.restype = ctypes.c_ulonglong
         for name in EXPORTS:
@@ -268,3 +271,22 @@ def fs_solve_host(X, Y, a, b, g0, eps, iters, dtype="f32", prec="auto", schedule
                              None if stream is None else ctypes.c_void_p(stream.cuda_stream))
     _check(st)
     return (f, g, *res)
+
+
+def fs_transport_apply(h: Handle, f, g, V, out, r=None):
+    """out[k, i, :] = sum_j P_ij V[k, j, :] (V float32 [batch, m, dv]); r[k, i] = sum_j P_ij if given."""
+    import torch
+    if V.dtype != torch.float32 or out.dtype != torch.float32:
+        raise ValueError("V and out must be float32")
+    dv = V.shape[-1]
+    _check(lib().fs_transport_apply(h.ptr, _f32(f), _f32(g), _ptr(V), int(dv), _ptr(out), _f32(r)), h.ptr)
+
+
+def fs_barycentric_map(h: Handle, f, g, Y, out):
+    """out[k, i, :] = sum_j P_ij y_j / sum_j P_ij (Y in the handle's dtype, [batch, m, d])."""
+    _check(lib().fs_barycentric_map(h.ptr, _f32(f), _f32(g), _ptr(Y), _f32(out)), h.ptr)
+
+
+def fs_grad_x(h: Handle, f, g, X, Y, grad):
+    """grad[k, i, :] = 2 (r_i x_i - sum_j P_ij y_j) (squared Euclidean cost)."""
+    _check(lib().fs_grad_x(h.ptr, _f32(f), _f32(g), _ptr(X), _ptr(Y), _f32(grad)), h.ptr)

@@ -43,6 +43,7 @@ struct fs_handle {
     void *packX = nullptr, *packY = nullptr;
     float *xn = nullptr, *yn = nullptr, *la2 = nullptr, *lb2 = nullptr;
     float *bias_row = nullptr, *bias_col = nullptr, *center = nullptr;
+    float *rsum = nullptr;  // row sums of a transport application [batch][n_pad]
     float4 *part = nullptr;
     unsigned *counters = nullptr;
     double *stats = nullptr, *red = nullptr, *wstat = nullptr;
@@ -268,7 +269,69 @@ fs_status measure(fs_handle *h, const float *f, const float *g, bool fdir, int s
 
 void fs::set_thread_error(const char *msg) { g_last_error = msg; }
 
+namespace {
+fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, bool v_bf16, int dv, float *out,
+                float *r, bool divide) {
+    const fs_desc &D = h->desc;
+    FS_CUDA(h, cudaSetDevice(h->device));
+    FS_LAUNCH(h, run_bias(h, g, true));  // column bias beta_j from g, as for an f-update
+    fs::ApplyParams p{};
+    p.rows = D.n;
+    p.rows_pad = h->n_pad;
+    p.rows_stride = h->n_stride;
+    p.cols = D.m;
+    p.cols_rows = h->m_pad;
+    p.cols_stride = h->m_stride;
+    p.d = D.d;
+    p.d_p = h->d_p;
+    p.row_elems = h->row_elems;
+    p.pack_mode = h->pack_mode;
+    p.dv = dv;
+    p.q_unscale = 1.f / h->qscale;
+    p.k_unscale = 1.f / h->kscale;
+    p.scale = fs::kLog2ed / (double)D.eps;
+    p.packQ = h->packX;
+    p.packK = h->packY;
+    p.row_norm = h->xn;
+    p.row_logw2 = h->la2;
+    p.pot_row = f;
+    p.col_bias = h->bias_col;
+    p.V = V;
+    p.v_bf16 = v_bf16 ? 1 : 0;
+    p.out = out;
+    p.rsum = r;
+    p.divide = divide ? 1 : 0;
+    FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
+    return FS_OK;
+}
+}  // namespace
+
 extern "C" {
+
+// ---- transport application ("FlashSinkhorn: IO-aware EOT on GPU", Metodologia
+// section 3: barycentric projection and gradient as plan-weighted averages) ----
+fs_status fs_transport_apply(fs_handle *h, const float *f, const float *g, const float *V, int dv, float *out,
+                             float *r) {
+    if (!h || !f || !g || !V || !out || dv < 1) return fail(h, FS_ERR_INVALID_ARG, "bad argument");
+    return apply(h, f, g, V, false, dv, out, r, false);
+}
+
+fs_status fs_barycentric_map(fs_handle *h, const float *f, const float *g, const void *Y, float *out) {
+    if (!h || !f || !g || !Y || !out) return fail(h, FS_ERR_INVALID_ARG, "null argument");
+    return apply(h, f, g, Y, h->desc.dtype == FS_BF16, h->desc.d, out, nullptr, true);
+}
+
+fs_status fs_grad_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y, float *grad) {
+    if (!h || !f || !g || !X || !Y || !grad) return fail(h, FS_ERR_INVALID_ARG, "null argument");
+    if (h->desc.cost != FS_COST_SQEUCLIDEAN)
+        return fail(h, FS_ERR_UNSUPPORTED, "fs_grad_x is defined for the squared Euclidean cost");
+    const fs_desc &D = h->desc;
+    const bool bf16 = D.dtype == FS_BF16;
+    fs_status st = apply(h, f, g, Y, bf16, D.d, grad, h->rsum, false);  // grad <- P Y, rsum <- P 1
+    if (st != FS_OK) return st;
+    FS_LAUNCH(h, fs::launch_grad_combine(X, bf16, h->rsum, grad, D.batch, D.n, D.d, grad, h->stream));
+    return FS_OK;
+}
 
 unsigned long long fs_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -432,6 +495,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     const size_t o_la2 = carve(B * h->n_stride * 4), o_lb2 = carve(B * h->m_stride * 4);
     const size_t o_brow = carve(B * h->n_stride * 4), o_bcol = carve(B * h->m_stride * 4);
     const size_t o_center = carve(B * D.d * 4);
+    const size_t o_rsum = carve(B * h->n_pad * 4);
     const size_t o_part = carve(max_splits > 1 ? B * max_splits * max_pad * 16 : 16);
     const size_t o_ctr = carve(B * max_rb * 4);
     const size_t o_stats = carve(B * max_rb * 4 * 8);
@@ -460,6 +524,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     h->la2 = reinterpret_cast<float *>(base + o_la2);
     h->lb2 = reinterpret_cast<float *>(base + o_lb2);
     h->bias_row = reinterpret_cast<float *>(base + o_brow);
+    h->rsum = reinterpret_cast<float *>(base + o_rsum);
     h->bias_col = reinterpret_cast<float *>(base + o_bcol);
     h->center = reinterpret_cast<float *>(base + o_center);
     h->part = reinterpret_cast<float4 *>(base + o_part);

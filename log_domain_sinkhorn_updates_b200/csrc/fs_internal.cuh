@@ -127,8 +127,26 @@ __device__ void finish_rows(const PassParams &p, int row_local, float m, float l
 
 }  // namespace fs
 
-// Launchers (defined in the .cu files); all return cudaGetLastError().
 namespace fs {
+// Parameters of a transport application (P V with P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps)
+// at given potentials), in the orientation of the f-direction pass.
+struct ApplyParams {
+    int rows, rows_pad, rows_stride;  // row side (X): valid, padded, per-point stride
+    int cols, cols_rows, cols_stride; // column side (Y)
+    int d, d_p, row_elems, pack_mode, dv;
+    float q_unscale, k_unscale;       // packed value x this = the operand's true value
+    double scale;                     // log2(e)/eps
+    const void *packQ, *packK;        // packed operand rows ([batch][rows_pad|cols_rows][row_elems])
+    const float *row_norm, *row_logw2, *pot_row;  // |x_i|^2 term, log2 a_i, f
+    const float *col_bias;            // ((g_j - |y_j|^2)/eps + ln b_j) log2 e, -inf padding
+    const void *V;                    // [batch][cols][dv], fp32 or bf16 (v_bf16)
+    int v_bf16;
+    float *out;                       // [batch][rows][dv]
+    float *rsum;                      // [batch][rows] or null
+    int divide;                       // 1: out = P V / r (barycentric map)
+};
+
+// Launchers (defined in the .cu files); all return cudaGetLastError().
 cudaError_t launch_lse_simt(const PassParams &p, int batch, bool measure, cudaStream_t s);
 // Single-CTA pass; qt = 128-row blocks resident per CTA (1 or 2; rows_pad / 128
 // must be a multiple of qt).
@@ -137,6 +155,11 @@ cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec
                           cudaStream_t s);
 size_t tc_smem_bytes(int row_bytes, int qt, int stages, bool measure);
 int tc_max_stages(int row_bytes, int qt, bool measure);
+// Transport application on CUDA cores (fp32): out = P V (or P V / r), rsum = P 1.
+cudaError_t launch_apply_simt(const ApplyParams &p, int batch, cudaStream_t s);
+// grad[bz][i][k] = 2 (r_i x_ik - pv[bz][i][k]) from the caller's X (fp32 or bf16).
+cudaError_t launch_grad_combine(const void *X, bool bf16, const float *r, const float *pv, int batch, int rows,
+                                int d, float *grad, cudaStream_t s);
 // The CTA-pair variant (one MMA over two SMs; rows_pad / 128 must be even).
 cudaError_t launch_lse_tc2(const PassParams &p, int batch, bool measure, int prec, const void *map_rows,
                            const void *map_cols, size_t smem_bytes, cudaStream_t s);

@@ -1,0 +1,149 @@
+"""Transport application (out_i = sum_j P_ij V_j, the barycentric map and the
+position gradient; "FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 3)
+through the C ABI, against the oracle at the same float32 potentials.
+
+Tolerance, derived from the arithmetic of the GPU path.  log2 P_ij =
+alpha_i + beta_j + S_ij log2(e)/eps is formed in double from float32 terms:
+- alpha_i and beta_j are each rounded to fp32;
+- the score S_ij is an fp32 dot product of operands that are exact or split to
+  about 2^-22.
+So the exponent is off by at most 2^-23 M_i with
+M_i = |alpha_i| + max_j (|beta_j| + (2d + 2) |S_ij| log2(e)/eps).
+exp2f adds 2^-21, and the fp32 sum over m terms adds m 2^-24.  Hence
+
+  |out_gpu - out_oracle|_i <= (ln2 2^-23 M_i + 2^-21 + m 2^-24) sum_j P_ij |V_j|.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import device_inputs, make_problem, oracle_arrays
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": dict(),
+    "middim": dict(n=1000, m=900),
+    "cloud3d": dict(n=1500, m=1100),
+    "highdim": dict(n=700, m=650),
+    "batched": dict(batch=3, n=600, m=520),
+}
+LOG2E = 1.0 / np.log(2.0)
+
+
+def _fs():
+    import log_domain_sinkhorn_updates_b200 as fs
+    return fs
+
+
+def _potentials(prob, cost, iters=8):
+    """A few oracle iterations from g = 0, rounded to float32 (the same bytes on both sides)."""
+    fs_, gs_ = [], []
+    for Xo, Yo, loga, logb in oracle_arrays(prob):
+        f, g = oracle.solve(Xo, Yo, loga, logb, prob.eps, iters, cost=cost)
+        fs_.append(f.astype(np.float32))
+        gs_.append(g.astype(np.float32))
+    return np.stack(fs_), np.stack(gs_)
+
+
+def _rel_bound(Xo, Yo, loga, logb, f, g, eps, cost):
+    d = Xo.shape[1]
+    if cost == "cosine":
+        xs = Xo / np.linalg.norm(Xo, axis=1, keepdims=True)
+        ys = Yo / np.linalg.norm(Yo, axis=1, keepdims=True)
+        xn = np.full(len(Xo), 0.5)
+        yn = np.full(len(Yo), 0.5)
+        nx, ny = np.ones(len(Xo)), np.ones(len(Yo))
+    else:
+        t = 0.5 * (Xo.mean(axis=0) + Yo.mean(axis=0))
+        xs, ys = Xo - t, Yo - t
+        xn, yn = (xs ** 2).sum(1), (ys ** 2).sum(1)
+        nx, ny = 2 * np.sqrt(xn), np.sqrt(yn)
+    alpha = loga * LOG2E + (f - xn) * LOG2E / eps
+    beta = logb * LOG2E + (g - yn) * LOG2E / eps
+    M = np.abs(alpha) + np.max(np.abs(beta)[None, :] + (2 * d + 2) * nx[:, None] * ny[None, :] * LOG2E / eps, axis=1)
+    return np.log(2.0) * 2.0 ** -23 * M + 2.0 ** -21 + len(Yo) * 2.0 ** -24
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("dv", [1, 5, 33, 70])
+def test_transport_apply_parity(cuda_device, name, dv):
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    f32, g32 = _potentials(prob, "sqeuclidean")
+    rng = np.random.default_rng(100 + dv)
+    V = rng.standard_normal((prob.batch, prob.m, dv)).astype(np.float32)
+    out = torch.empty(prob.batch, prob.n, dv, device=cuda_device)
+    r = torch.empty(prob.batch, prob.n, device=cuda_device)
+    fs.fs_transport_apply(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device),
+                          torch.from_numpy(V).to(cuda_device), out, r)
+    fs.fs_sync(h)
+    out, r = out.cpu().numpy(), r.cpu().numpy()
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
+        oo, ro = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, V[k].astype(np.float64))
+        absw, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(V[k]).astype(np.float64))
+        rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean")
+        err = np.abs(out[k] - oo) / (rel[:, None] * absw)
+        rerr = np.abs(r[k] - ro) / (rel * ro)
+        print(f"{name}[{k}] dv={dv} worst err / bound = {err.max():.3f}, row sums {rerr.max():.3f}")
+        assert err.max() <= 1.0 and rerr.max() <= 1.0
+
+
+@pytest.mark.parametrize("name", ["tiny", "middim", "highdim"])
+def test_barycentric_map_and_grad_parity(cuda_device, name):
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    f32, g32 = _potentials(prob, "sqeuclidean", iters=30)
+    fd, gd = torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device)
+    T = torch.empty(prob.batch, prob.n, prob.d, device=cuda_device)
+    G = torch.empty(prob.batch, prob.n, prob.d, device=cuda_device)
+    fs.fs_barycentric_map(h, fd, gd, Y, T)
+    fs.fs_grad_x(h, fd, gd, X, Y, G)
+    fs.fs_sync(h)
+    T, G = T.cpu().numpy(), G.cpu().numpy()
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
+        To = oracle.barycentric_projection(Xo, Yo, loga, logb, fk, gk, prob.eps)
+        Go = oracle.grad_x(Xo, Yo, loga, logb, fk, gk, prob.eps)
+        py, r = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(Yo))
+        rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean")[:, None]
+        # T = (P Y)/r: both factors carry rel; G = 2 (r x - P Y)
+        tb = 2 * rel * py / r[:, None] + 1e-6 * np.abs(To)
+        gb = 2 * rel * (r[:, None] * np.abs(Xo) + py) + 2.0 ** -22 * np.abs(Go)
+        et, eg = (np.abs(T[k] - To) / tb).max(), (np.abs(G[k] - Go) / gb).max()
+        print(f"{name}[{k}] barycentric err/bound {et:.3f}  grad err/bound {eg:.3f}")
+        assert et <= 1.0 and eg <= 1.0
+
+
+def test_transport_apply_cosine_parity(cuda_device):
+    import torch
+    fs = _fs()
+    prob = make_problem("middim", n=1000, m=900)
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps, cost="cosine")
+    f32, g32 = _potentials(prob, "cosine")
+    rng = np.random.default_rng(7)
+    V = rng.standard_normal((1, prob.m, 9)).astype(np.float32)
+    out = torch.empty(1, prob.n, 9, device=cuda_device)
+    fs.fs_transport_apply(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device),
+                          torch.from_numpy(V).to(cuda_device), out)
+    fs.fs_sync(h)
+    Xo, Yo, loga, logb = oracle.problem_arrays(prob, 0)
+    fk, gk = f32[0].astype(np.float64), g32[0].astype(np.float64)
+    oo, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, V[0].astype(np.float64), cost="cosine")
+    absw, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(V[0]).astype(np.float64),
+                                     cost="cosine")
+    rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "cosine")
+    err = (np.abs(out.cpu().numpy()[0] - oo) / (rel[:, None] * absw)).max()
+    print(f"cosine transport err / bound {err:.3f}")
+    assert err <= 1.0
+    with pytest.raises(fs.FsError):
+        fs.fs_grad_x(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device), X, Y,
+                     torch.empty(1, prob.n, prob.d, device=cuda_device))
