@@ -51,6 +51,7 @@ struct fs_handle {
     std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
     int host_err[4] = {0, 0, 0, 0};
     CUtensorMap mapX_r{}, mapX_c{}, mapY_r{}, mapY_c{};  // row-side (128-row box) / column-side (256-row box)
+    CUtensorMap mapY_64{};  // column side in 64-row boxes (tensor-core transport application)
     int splits_f = 1, tps_f = 1, splits_g = 1, tps_g = 1;
     int stages = 2, stages_meas = 2;
     bool pair = false;  // run the passes on CTA pairs (one MMA over two SMs); FS_CTA_PAIR=1
@@ -301,7 +302,58 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     p.out = out;
     p.rsum = r;
     p.divide = divide ? 1 : 0;
-    FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
+    // Tensor cores where the operand rows fit the single-CTA layout (up to 256
+    // bytes) and dv <= 256; the CUDA-core kernel otherwise or with FS_APPLY_SIMT=1.
+    const int dv_pad = (dv + 15) / 16 * 16;
+    const int vpl = v_bf16 ? 1 : 2;
+    int kslots = 0, vslots = 0;
+    const char *force_simt = getenv("FS_APPLY_SIMT");
+    const size_t smem = (h->prec != FS_PREC_F32_SIMT && !h->pair && h->row_bytes <= 256 && dv <= 256 &&
+                         !(force_simt && atoi(force_simt) != 0))
+                            ? fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &vslots)
+                            : 0;
+    if (smem == 0) {
+        FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
+        return FS_OK;
+    }
+    p.row_bytes = h->row_bytes;
+    p.swz = h->swz;
+    p.plane_bytes = h->plane_bytes;
+    p.dv_pad = dv_pad;
+    p.kslots = kslots;
+    p.vslots = vslots;
+    p.sscale = h->sscale;
+    p.timeout_ns = h->timeout_ns;
+    p.err = h->err;
+    // V~: V transposed, bf16 planes [batch][vpl][dv_pad][m_pad], from the pool for this call
+    const size_t vt_bytes = (size_t)D.batch * vpl * dv_pad * h->m_pad * 2;
+    cudaMemPool_t pool;
+    void *vt = nullptr;
+    FS_CUDA(h, device_pool(h->device, &pool));
+    FS_CUDA(h, cudaMallocFromPoolAsync(&vt, vt_bytes, pool, h->stream));
+    cudaError_t e = fs::launch_vt_pack(V, v_bf16, D.batch, D.m, dv, h->m_pad, dv_pad, vpl, vt, h->stream);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    CUtensorMap map_v{};
+    fs_status st = FS_OK;
+    if (e == cudaSuccess) {
+        auto fn = encode_fn();
+        cuuint64_t gdim[2] = {(cuuint64_t)h->m_pad, (cuuint64_t)D.batch * vpl * dv_pad};
+        cuuint64_t gstride[1] = {(cuuint64_t)h->m_pad * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)dv_pad};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r2 = fn ? fn(&map_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vt, gdim, gstride, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
+                         : CUDA_ERROR_NOT_SUPPORTED;
+        if (r2 != CUDA_SUCCESS) st = fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed for V (%d)", (int)r2);
+    }
+    if (e == cudaSuccess && st == FS_OK) {
+        e = fs::launch_apply_tc(p, D.batch, h->prec, vpl, &h->mapX_r, &h->mapY_64, &map_v, smem, h->stream);
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+    cudaFreeAsync(vt, h->stream);
+    if (st != FS_OK) return st;
+    FS_CUDA(h, e);
     return FS_OK;
 }
 }  // namespace
@@ -598,6 +650,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, kBlockCols);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_r, h->packY, D.batch * h->m_pad, kBlockRows);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, kBlockCols);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_64, h->packY, D.batch * h->m_pad, 64);
             if (s2 != FS_OK) return s2;
         }
         return FS_OK;

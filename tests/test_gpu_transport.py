@@ -12,6 +12,11 @@ M_i = |alpha_i| + max_j (|beta_j| + (2d + 2) |S_ij| log2(e)/eps).
 exp2f adds 2^-21, and the fp32 sum over m terms adds m 2^-24.  Hence
 
   |out_gpu - out_oracle|_i <= (ln2 2^-23 M_i + 2^-21 + m 2^-24) sum_j P_ij |V_j|.
+
+The tensor-core path also splits P/a_i and V into bf16 hi + lo pairs, which
+carry 2^-16 each and drop a term of 2^-16 relative size, so its bound adds
+2^-14.  Every test runs both paths: the tensor-core default and the CUDA-core
+validation kernel (FS_APPLY_SIMT=1).
 """
 import numpy as np
 import pytest
@@ -65,10 +70,16 @@ def _rel_bound(Xo, Yo, loga, logb, f, g, eps, cost):
     return np.log(2.0) * 2.0 ** -23 * M + 2.0 ** -21 + len(Yo) * 2.0 ** -24
 
 
+PATHS = {"tc": "0", "simt": "1"}
+SPLIT = {"tc": 2.0 ** -14, "simt": 0.0}
+
+
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", list(SMALL))
-@pytest.mark.parametrize("dv", [1, 5, 33, 70])
-def test_transport_apply_parity(cuda_device, name, dv):
+@pytest.mark.parametrize("dv", [1, 5, 33, 70, 256])
+def test_transport_apply_parity(cuda_device, name, dv, path, monkeypatch):
     import torch
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
     fs = _fs()
     prob = make_problem(name, **SMALL[name])
     X, Y, a_d, b_d = device_inputs(prob)
@@ -86,16 +97,18 @@ def test_transport_apply_parity(cuda_device, name, dv):
         fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
         oo, ro = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, V[k].astype(np.float64))
         absw, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(V[k]).astype(np.float64))
-        rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean")
+        rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean") + SPLIT[path]
         err = np.abs(out[k] - oo) / (rel[:, None] * absw)
         rerr = np.abs(r[k] - ro) / (rel * ro)
-        print(f"{name}[{k}] dv={dv} worst err / bound = {err.max():.3f}, row sums {rerr.max():.3f}")
+        print(f"{path} {name}[{k}] dv={dv} worst err / bound = {err.max():.3f}, row sums {rerr.max():.3f}")
         assert err.max() <= 1.0 and rerr.max() <= 1.0
 
 
-@pytest.mark.parametrize("name", ["tiny", "middim", "highdim"])
-def test_barycentric_map_and_grad_parity(cuda_device, name):
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("name", ["tiny", "middim", "highdim", "batched"])
+def test_barycentric_map_and_grad_parity(cuda_device, name, path, monkeypatch):
     import torch
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
     fs = _fs()
     prob = make_problem(name, **SMALL[name])
     X, Y, a_d, b_d = device_inputs(prob)
@@ -113,17 +126,19 @@ def test_barycentric_map_and_grad_parity(cuda_device, name):
         To = oracle.barycentric_projection(Xo, Yo, loga, logb, fk, gk, prob.eps)
         Go = oracle.grad_x(Xo, Yo, loga, logb, fk, gk, prob.eps)
         py, r = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(Yo))
-        rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean")[:, None]
+        rel = (_rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean") + SPLIT[path])[:, None]
         # T = (P Y)/r: both factors carry rel; G = 2 (r x - P Y)
         tb = 2 * rel * py / r[:, None] + 1e-6 * np.abs(To)
         gb = 2 * rel * (r[:, None] * np.abs(Xo) + py) + 2.0 ** -22 * np.abs(Go)
         et, eg = (np.abs(T[k] - To) / tb).max(), (np.abs(G[k] - Go) / gb).max()
-        print(f"{name}[{k}] barycentric err/bound {et:.3f}  grad err/bound {eg:.3f}")
+        print(f"{path} {name}[{k}] barycentric err/bound {et:.3f}  grad err/bound {eg:.3f}")
         assert et <= 1.0 and eg <= 1.0
 
 
-def test_transport_apply_cosine_parity(cuda_device):
+@pytest.mark.parametrize("path", list(PATHS))
+def test_transport_apply_cosine_parity(cuda_device, path, monkeypatch):
     import torch
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
     fs = _fs()
     prob = make_problem("middim", n=1000, m=900)
     X, Y, a_d, b_d = device_inputs(prob)
@@ -140,7 +155,7 @@ def test_transport_apply_cosine_parity(cuda_device):
     oo, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, V[0].astype(np.float64), cost="cosine")
     absw, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(V[0]).astype(np.float64),
                                      cost="cosine")
-    rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "cosine")
+    rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "cosine") + SPLIT[path]
     err = (np.abs(out.cpu().numpy()[0] - oo) / (rel[:, None] * absw)).max()
     print(f"cosine transport err / bound {err:.3f}")
     assert err <= 1.0
