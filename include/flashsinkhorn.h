@@ -209,6 +209,23 @@ FS_API fs_status fs_barycentric_map(fs_handle *h, const float *f, const float *g
 FS_API fs_status fs_grad_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
                            float *grad);
 
+/* The transposed application: out[k][j][c] = sum_i P_ij U[k][i][c] (U: device
+ * fp32 [batch][n][du]), c[k][j] = sum_i P_ij (device [batch][m]; may be NULL);
+ * out: device fp32 [batch][m][du].  Same arithmetic as fs_transport_apply.
+ * Asynchronous. */
+FS_API fs_status fs_transport_apply_t(fs_handle *h, const float *f, const float *g, const float *U, int du,
+                                      float *out, float *c);
+
+/* Gradient of the entropic OT cost with respect to the positions Y at (f, g),
+ * squared Euclidean cost: grad_j = sum_i P_ij 2 (y_j - x_i) = 2 (c_j y_j -
+ * sum_i P_ij x_i).  With fs_grad_x and the potentials themselves (the
+ * gradients with respect to the weights a and b, up to the constant fixed by
+ * sum a = sum b = 1) this is the backward pass of the EOT loss.  X, Y: the
+ * caller's device clouds in the handle's dtype; grad: device fp32
+ * [batch][m][d].  FS_ERR_UNSUPPORTED for the cosine cost.  Asynchronous. */
+FS_API fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
+                           float *grad);
+
 /* Number of CUDA kernels this library has launched in this process so far
  * (all handles, all threads).  Host-side counter; never synchronises. */
 FS_API unsigned long long fs_kernel_launches(void);

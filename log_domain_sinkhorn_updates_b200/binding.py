@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_CUDA", 3: "FS_ER
 
 EXPORTS = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_err", "fs_ot_cost",
            "fs_sync", "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches",
-           "fs_update_f_noalloc", "fs_transport_apply", "fs_barycentric_map", "fs_grad_x"]
+           "fs_update_f_noalloc", "fs_transport_apply", "fs_barycentric_map", "fs_grad_x",
+           "fs_transport_apply_t", "fs_grad_y"]
 
 
 class FsDesc(ctypes.Structure):
@@ -82,6 +83,8 @@ def lib():
         L.fs_transport_apply.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp]
         L.fs_barycentric_map.argtypes = [vp, vp, vp, vp, vp]
         L.fs_grad_x.argtypes = [vp, vp, vp, vp, vp, vp]
+        L.fs_transport_apply_t.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp]
+        L.fs_grad_y.argtypes = [vp, vp, vp, vp, vp, vp]
         L.fs_kernel_launches.argtypes = []
         L.fs_kernel_launches.restype = ctypes.c_ulonglong
         for name in EXPORTS:
@@ -290,3 +293,17 @@ def fs_barycentric_map(h: Handle, f, g, Y, out):
 def fs_grad_x(h: Handle, f, g, X, Y, grad):
     """grad[k, i, :] = 2 (r_i x_i - sum_j P_ij y_j) (squared Euclidean cost)."""
     _check(lib().fs_grad_x(h.ptr, _f32(f), _f32(g), _ptr(X), _ptr(Y), _f32(grad)), h.ptr)
+
+
+def fs_transport_apply_t(h: Handle, f, g, U, out, c=None):
+    """out[k, j, :] = sum_i P_ij U[k, i, :] (U float32 [batch, n, du]); c[k, j] = sum_i P_ij if given."""
+    import torch
+    if U.dtype != torch.float32 or out.dtype != torch.float32:
+        raise ValueError("U and out must be float32")
+    _check(lib().fs_transport_apply_t(h.ptr, _f32(f), _f32(g), _ptr(U), int(U.shape[-1]), _ptr(out), _f32(c)),
+           h.ptr)
+
+
+def fs_grad_y(h: Handle, f, g, X, Y, grad):
+    """grad[k, j, :] = 2 (c_j y_j - sum_i P_ij x_i) (squared Euclidean cost)."""
+    _check(lib().fs_grad_y(h.ptr, _f32(f), _f32(g), _ptr(X), _ptr(Y), _f32(grad)), h.ptr)

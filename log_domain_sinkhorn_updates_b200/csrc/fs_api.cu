@@ -43,7 +43,7 @@ struct fs_handle {
     void *packX = nullptr, *packY = nullptr;
     float *xn = nullptr, *yn = nullptr, *la2 = nullptr, *lb2 = nullptr;
     float *bias_row = nullptr, *bias_col = nullptr, *center = nullptr;
-    float *rsum = nullptr;  // row sums of a transport application [batch][n_pad]
+    float *rsum = nullptr;  // row sums of a transport application [batch][max(n_pad, m_pad)]
     float4 *part = nullptr;
     unsigned *counters = nullptr;
     double *stats = nullptr, *red = nullptr, *wstat = nullptr;
@@ -51,7 +51,7 @@ struct fs_handle {
     std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
     int host_err[4] = {0, 0, 0, 0};
     CUtensorMap mapX_r{}, mapX_c{}, mapY_r{}, mapY_c{};  // row-side (128-row box) / column-side (256-row box)
-    CUtensorMap mapY_64{};  // column side in 64-row boxes (tensor-core transport application)
+    CUtensorMap mapX_64{}, mapY_64{};  // 64-row boxes (tensor-core transport application)
     int splits_f = 1, tps_f = 1, splits_g = 1, tps_g = 1;
     int stages = 2, stages_meas = 2;
     bool pair = false;  // run the passes on CTA pairs (one MMA over two SMs); FS_CTA_PAIR=1
@@ -271,32 +271,36 @@ fs_status measure(fs_handle *h, const float *f, const float *g, bool fdir, int s
 void fs::set_thread_error(const char *msg) { g_last_error = msg; }
 
 namespace {
+// fdir: out_i = sum_j P_ij V_j over the X side's rows (V indexed by Y's points);
+// otherwise the transposed application out_j = sum_i P_ij V_i over Y's rows.
 fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, bool v_bf16, int dv, float *out,
-                float *r, bool divide) {
+                float *r, bool divide, bool fdir = true) {
     const fs_desc &D = h->desc;
     FS_CUDA(h, cudaSetDevice(h->device));
-    FS_LAUNCH(h, run_bias(h, g, true));  // column bias beta_j from g, as for an f-update
+    FS_LAUNCH(h, run_bias(h, fdir ? g : f, fdir));  // the column bias of the pass in this direction
     fs::ApplyParams p{};
-    p.rows = D.n;
-    p.rows_pad = h->n_pad;
-    p.rows_stride = h->n_stride;
-    p.cols = D.m;
-    p.cols_rows = h->m_pad;
-    p.cols_stride = h->m_stride;
+    p.rows = fdir ? D.n : D.m;
+    p.rows_pad = fdir ? h->n_pad : h->m_pad;
+    p.rows_stride = fdir ? h->n_stride : h->m_stride;
+    p.cols = fdir ? D.m : D.n;
+    p.cols_rows = fdir ? h->m_pad : h->n_pad;
+    p.cols_stride = fdir ? h->m_stride : h->n_stride;
     p.d = D.d;
     p.d_p = h->d_p;
     p.row_elems = h->row_elems;
     p.pack_mode = h->pack_mode;
     p.dv = dv;
-    p.q_unscale = 1.f / h->qscale;
-    p.k_unscale = 1.f / h->kscale;
+    // packed X holds qscale (x - t), packed Y kscale * 2 (y - t) (or the
+    // normalised rows): unscaled, their dot product is S_ij either way round
+    p.q_unscale = 1.f / (fdir ? h->qscale : h->kscale);
+    p.k_unscale = 1.f / (fdir ? h->kscale : h->qscale);
     p.scale = fs::kLog2ed / (double)D.eps;
-    p.packQ = h->packX;
-    p.packK = h->packY;
-    p.row_norm = h->xn;
-    p.row_logw2 = h->la2;
-    p.pot_row = f;
-    p.col_bias = h->bias_col;
+    p.packQ = fdir ? h->packX : h->packY;
+    p.packK = fdir ? h->packY : h->packX;
+    p.row_norm = fdir ? h->xn : h->yn;
+    p.row_logw2 = fdir ? h->la2 : h->lb2;
+    p.pot_row = fdir ? f : g;
+    p.col_bias = fdir ? h->bias_col : h->bias_row;
     p.V = V;
     p.v_bf16 = v_bf16 ? 1 : 0;
     p.out = out;
@@ -326,19 +330,19 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     p.timeout_ns = h->timeout_ns;
     p.err = h->err;
     // V~: V transposed, bf16 planes [batch][vpl][dv_pad][m_pad], from the pool for this call
-    const size_t vt_bytes = (size_t)D.batch * vpl * dv_pad * h->m_pad * 2;
+    const size_t vt_bytes = (size_t)D.batch * vpl * dv_pad * p.cols_rows * 2;
     cudaMemPool_t pool;
     void *vt = nullptr;
     FS_CUDA(h, device_pool(h->device, &pool));
     FS_CUDA(h, cudaMallocFromPoolAsync(&vt, vt_bytes, pool, h->stream));
-    cudaError_t e = fs::launch_vt_pack(V, v_bf16, D.batch, D.m, dv, h->m_pad, dv_pad, vpl, vt, h->stream);
+    cudaError_t e = fs::launch_vt_pack(V, v_bf16, D.batch, p.cols, dv, p.cols_rows, dv_pad, vpl, vt, h->stream);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     CUtensorMap map_v{};
     fs_status st = FS_OK;
     if (e == cudaSuccess) {
         auto fn = encode_fn();
-        cuuint64_t gdim[2] = {(cuuint64_t)h->m_pad, (cuuint64_t)D.batch * vpl * dv_pad};
-        cuuint64_t gstride[1] = {(cuuint64_t)h->m_pad * 2};
+        cuuint64_t gdim[2] = {(cuuint64_t)p.cols_rows, (cuuint64_t)D.batch * vpl * dv_pad};
+        cuuint64_t gstride[1] = {(cuuint64_t)p.cols_rows * 2};
         cuuint32_t box[2] = {64, (cuuint32_t)dv_pad};
         cuuint32_t estr[2] = {1, 1};
         CUresult r2 = fn ? fn(&map_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vt, gdim, gstride, box, estr,
@@ -348,7 +352,8 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
         if (r2 != CUDA_SUCCESS) st = fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed for V (%d)", (int)r2);
     }
     if (e == cudaSuccess && st == FS_OK) {
-        e = fs::launch_apply_tc(p, D.batch, h->prec, vpl, &h->mapX_r, &h->mapY_64, &map_v, smem, h->stream);
+        e = fs::launch_apply_tc(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r,
+                                fdir ? &h->mapY_64 : &h->mapX_64, &map_v, smem, h->stream);
         g_launches.fetch_add(1, std::memory_order_relaxed);
     }
     cudaFreeAsync(vt, h->stream);
@@ -382,6 +387,24 @@ fs_status fs_grad_x(fs_handle *h, const float *f, const float *g, const void *X,
     fs_status st = apply(h, f, g, Y, bf16, D.d, grad, h->rsum, false);  // grad <- P Y, rsum <- P 1
     if (st != FS_OK) return st;
     FS_LAUNCH(h, fs::launch_grad_combine(X, bf16, h->rsum, grad, D.batch, D.n, D.d, grad, h->stream));
+    return FS_OK;
+}
+
+fs_status fs_transport_apply_t(fs_handle *h, const float *f, const float *g, const float *U, int du, float *out,
+                               float *c) {
+    if (!h || !f || !g || !U || !out || du < 1) return fail(h, FS_ERR_INVALID_ARG, "bad argument");
+    return apply(h, f, g, U, false, du, out, c, false, false);
+}
+
+fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const void *X, const void *Y, float *grad) {
+    if (!h || !f || !g || !X || !Y || !grad) return fail(h, FS_ERR_INVALID_ARG, "null argument");
+    if (h->desc.cost != FS_COST_SQEUCLIDEAN)
+        return fail(h, FS_ERR_UNSUPPORTED, "fs_grad_y is defined for the squared Euclidean cost");
+    const fs_desc &D = h->desc;
+    const bool bf16 = D.dtype == FS_BF16;
+    fs_status st = apply(h, f, g, X, bf16, D.d, grad, h->rsum, false, false);  // grad <- P^T X, rsum <- P^T 1
+    if (st != FS_OK) return st;
+    FS_LAUNCH(h, fs::launch_grad_combine(Y, bf16, h->rsum, grad, D.batch, D.m, D.d, grad, h->stream));
     return FS_OK;
 }
 
@@ -547,7 +570,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     const size_t o_la2 = carve(B * h->n_stride * 4), o_lb2 = carve(B * h->m_stride * 4);
     const size_t o_brow = carve(B * h->n_stride * 4), o_bcol = carve(B * h->m_stride * 4);
     const size_t o_center = carve(B * D.d * 4);
-    const size_t o_rsum = carve(B * h->n_pad * 4);
+    const size_t o_rsum = carve(B * max_pad * 4);
     const size_t o_part = carve(max_splits > 1 ? B * max_splits * max_pad * 16 : 16);
     const size_t o_ctr = carve(B * max_rb * 4);
     const size_t o_stats = carve(B * max_rb * 4 * 8);
@@ -651,6 +674,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_r, h->packY, D.batch * h->m_pad, kBlockRows);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, kBlockCols);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_64, h->packY, D.batch * h->m_pad, 64);
+            if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_64, h->packX, D.batch * h->n_pad, 64);
             if (s2 != FS_OK) return s2;
         }
         return FS_OK;

@@ -14,5 +14,5 @@ Two independent implementations live here:
 from .core import (  # noqa: F401
     log_weights, update_f, update_g, update_f_rows, solve, marginals, marginal_error,
     plan_stats, costs, minplus_bounds, num_threads, problem_arrays, COSTS, transport_apply,
-    barycentric_projection, grad_x,
+    barycentric_projection, grad_x, grad_y,
 )

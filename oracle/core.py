@@ -271,3 +271,10 @@ def grad_x(X, Y, loga, logb, f, g, eps):
     the optimal value (envelope theorem)."""
     out, r = transport_apply(X, Y, loga, logb, f, g, eps, Y)
     return 2.0 * (r[:, None] * np.asarray(X, dtype=np.float64) - out)
+
+
+def grad_y(X, Y, loga, logb, f, g, eps):
+    """Gradient of the entropic OT cost with respect to the positions Y at (f, g),
+    squared-Euclidean cost: 2 (c_j y_j - sum_i P_ij x_i) -- grad_x with the roles
+    of the two clouds (and weights, potentials) exchanged, C being symmetric."""
+    return grad_x(Y, X, logb, loga, g, f, eps)

@@ -162,3 +162,41 @@ def test_transport_apply_cosine_parity(cuda_device, path, monkeypatch):
     with pytest.raises(fs.FsError):
         fs.fs_grad_x(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device), X, Y,
                      torch.empty(1, prob.n, prob.d, device=cuda_device))
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("name", ["tiny", "cloud3d", "highdim", "batched"])
+def test_transposed_apply_and_grad_y_parity(cuda_device, name, path, monkeypatch):
+    """out_j = sum_i P_ij U_i and the gradient with respect to Y (the backward pass's
+    second half) against the oracle, whose transposed forms exchange the two
+    clouds' roles (C is symmetric)."""
+    import torch
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    f32, g32 = _potentials(prob, "sqeuclidean", iters=20)
+    fd, gd = torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device)
+    rng = np.random.default_rng(123)
+    U = rng.standard_normal((prob.batch, prob.n, 7)).astype(np.float32)
+    out = torch.empty(prob.batch, prob.m, 7, device=cuda_device)
+    c = torch.empty(prob.batch, prob.m, device=cuda_device)
+    G = torch.empty(prob.batch, prob.m, prob.d, device=cuda_device)
+    fs.fs_transport_apply_t(h, fd, gd, torch.from_numpy(U).to(cuda_device), out, c)
+    fs.fs_grad_y(h, fd, gd, X, Y, G)
+    fs.fs_sync(h)
+    out, c, G = out.cpu().numpy(), c.cpu().numpy(), G.cpu().numpy()
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
+        oo, co = oracle.transport_apply(Yo, Xo, logb, loga, gk, fk, prob.eps, U[k].astype(np.float64))
+        absw, _ = oracle.transport_apply(Yo, Xo, logb, loga, gk, fk, prob.eps, np.abs(U[k]).astype(np.float64))
+        px, _ = oracle.transport_apply(Yo, Xo, logb, loga, gk, fk, prob.eps, np.abs(Xo))
+        Go = oracle.grad_y(Xo, Yo, loga, logb, fk, gk, prob.eps)
+        rel = _rel_bound(Yo, Xo, logb, loga, gk, fk, prob.eps, "sqeuclidean") + SPLIT[path]
+        e1 = (np.abs(out[k] - oo) / (rel[:, None] * absw)).max()
+        e2 = (np.abs(c[k] - co) / (rel * co)).max()
+        gb = 2 * rel[:, None] * (co[:, None] * np.abs(Yo) + px) + 2.0 ** -22 * np.abs(Go)
+        e3 = (np.abs(G[k] - Go) / gb).max()
+        print(f"{path} {name}[{k}] transposed err/bound {e1:.3f} col sums {e2:.3f} grad_y {e3:.3f}")
+        assert e1 <= 1.0 and e2 <= 1.0 and e3 <= 1.0

@@ -377,3 +377,28 @@ def test_barycentric_projection_tends_to_the_optimal_assignment():
     T = oracle.barycentric_projection(X, Y, loga, logb, f, g, 0.02)
     _, cols = linear_sum_assignment(dense.cost_matrix(X, Y))
     assert np.abs(T - Y[cols]).max() < 1e-2
+
+
+def test_grad_y_matches_finite_differences_of_the_optimal_value():
+    rng = np.random.default_rng(73)
+    n, m, d, eps = 5, 6, 2, 0.4
+    X = rng.standard_normal((n, d))
+    Y = rng.standard_normal((m, d)) + 0.3
+    a = rng.uniform(0.5, 1.5, n)
+    b = rng.uniform(0.5, 1.5, m)
+    loga, logb = np.log(a / a.sum()), np.log(b / b.sum())
+
+    def value(Yv):
+        f, g = oracle.solve(X, Yv, loga, logb, eps, 500)
+        return oracle.costs(X, Yv, loga, logb, f, g, eps)["dual"], f, g
+
+    _, f, g = value(Y)
+    G = oracle.grad_y(X, Y, loga, logb, f, g, eps)
+    h = 1e-5
+    for j in range(m):
+        for k in range(d):
+            Yp, Ym = Y.copy(), Y.copy()
+            Yp[j, k] += h
+            Ym[j, k] -= h
+            fd = (value(Yp)[0] - value(Ym)[0]) / (2 * h)
+            assert abs(G[j, k] - fd) <= 1e-8, (j, k, G[j, k], fd)
