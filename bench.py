@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline sample duration")
+    ap.add_argument("--op", choices=["solve", "transport"], default="solve",
+                    help="solve: the Sinkhorn solve (the headline); transport: the barycentric map at the "
+                         "converged potentials (transport application, tensor-core kernel)")
     return ap.parse_args()
 
 
@@ -222,10 +225,102 @@ def load_peaks():
 # ----------------------------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------------------------
+def run_transport(args):
+    """Barycentric map sum_j P_ij y_j / sum_j P_ij at the workload's converged potentials: one
+    application per step, timed with CUDA events; roofline against the tensor pipe."""
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    import log_domain_sinkhorn_updates_b200 as fs
+    prob = make_problem(args.workload, n=args.n, m=args.m, batch=args.batch)
+    B, n, m, d = prob.batch, prob.n, prob.m, prob.d
+    if prob.dtype == "bf16":
+        X = torch.from_numpy(prob.X_dev.view(np.int16)).view(torch.bfloat16).to(dev)
+        Y = torch.from_numpy(prob.Y_dev.view(np.int16)).view(torch.bfloat16).to(dev)
+    else:
+        X, Y = torch.from_numpy(prob.X_dev).to(dev), torch.from_numpy(prob.Y_dev).to(dev)
+    a = None if prob.a_dev is None else torch.from_numpy(prob.a_dev).to(dev)
+    b = None if prob.b_dev is None else torch.from_numpy(prob.b_dev).to(dev)
+    h = fs.fs_create(X, Y, a, b, eps=prob.eps)
+    f = torch.zeros(B, n, device=dev)
+    g = torch.zeros(B, m, device=dev)
+    fs.fs_solve(h, f, g, args.iters or prob.iters)
+    out = torch.empty(B, n, d, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        fs.fs_barycentric_map(h, f, g, Y, out)
+    fs.fs_sync(h)
+    sampler = ClockSampler(gpu_identifier(torch, dev))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    launches0 = fs.fs_kernel_launches()
+    tot = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fs.fs_barycentric_map(h, f, g, Y, out)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        tot += e0.elapsed_time(e1)
+    fs.fs_sync(h)
+    launches = fs.fs_kernel_launches() - launches0
+    clocks = sampler.stop()
+    tt = torch.tensor([tot], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    tot = tt.item()
+    info = fs.fs_get_info(h)
+    entries = B * n * m
+    app_s = tot / 1e3 / args.steps
+    # S = Q K^T in the handle's precision, then P~ (hi + lo) times V~ (one bf16 plane for bf16 Y, two else)
+    npass_s = 3 if info["prec"] in ("3xtf32", "3xf16") else 1
+    npass_o = 2 if prob.dtype == "bf16" else 3
+    flops = 2.0 * entries * (d * npass_s + d * npass_o)
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    line = {
+        "metric": "transport application (barycentric map) cost-entries/s at the converged potentials",
+        "value": world * entries / app_s, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if info["prec"] == "bf16" else "f32", "data": "synthetic",
+        "config": workload_config(prob, args.iters or prob.iters, {
+            "op": "fs_barycentric_map", "dv": d, "precision": info["prec"], "parallelism": f"replicas x{world}",
+            "step": f"fs_barycentric_map at the potentials of fs_solve({args.iters or prob.iters}) (solve untimed)",
+            "half_iters_per_step": 0}),
+        "roofline": {"bound": "tensor", "achieved": flops / app_s / 1e12, "peak": peak, "unit": "TFLOP/s",
+                     "frac": flops / app_s / 1e12 / peak, "traffic": None, "peak_source": peak_src,
+                     "kernel": "apply_tc_kernel (S = Q K^T, then O += P~ V~)",
+                     "flops_per_launch": flops},
+        "cpu_baseline": None, "e2e": None, "clocks": clocks, "gpu_launches": int(launches),
+    }
+    fs.fs_destroy(h)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "transport":
+        return run_transport(args)
 
     import torch
     import torch.distributed as dist
