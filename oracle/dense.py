@@ -101,3 +101,38 @@ def two_by_two_plan(C, a1, b1, eps):
     assert len(p) >= 1, (roots, lo, hi)
     p = p[0]
     return np.array([[p, a1 - p], [b1 - p, 1.0 - a1 - b1 + p]])
+
+
+def hvp_x(X, Y, loga, logb, f, g, eps, V):
+    """Hessian-vector product of the entropic OT cost with respect to the positions X
+    (squared Euclidean cost) at optimal potentials (f, g), in direction V [n, d].
+
+    The gradient is G_i = 2 sum_j P_ij (x_i - y_j).  Moving X along V changes P
+    directly through C (dC_ij = 2 (x_i - y_j).v_i) and through the potentials,
+    whose response (df, dg) keeps both marginals fixed:
+        r_i df_i + (P dg)_i   = sum_j P_ij dC_ij
+        (P^T df)_j + c_j dg_j = sum_i P_ij dC_ij
+    (a singular system: (k, -k) is free and does not change the result).  Then
+        dG_i = 2 r_i v_i + (2/eps) sum_j P_ij (df_i + dg_j - dC_ij)(x_i - y_j).
+    Everything here is dense (tiny inputs only): P materialised, the linear
+    system solved by least squares.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    P = plan(cost_matrix(X, Y), np.asarray(loga, float), np.asarray(logb, float), np.asarray(f, float),
+             np.asarray(g, float), eps)
+    n, m = P.shape
+    D = X[:, None, :] - Y[None, :, :]                 # x_i - y_j
+    dC = 2.0 * np.einsum("ijk,ik->ij", D, V)          # 2 (x_i - y_j).v_i
+    r, c = P.sum(axis=1), P.sum(axis=0)
+    A = np.zeros((n + m, n + m))
+    A[:n, :n] = np.diag(r)
+    A[:n, n:] = P
+    A[n:, :n] = P.T
+    A[n:, n:] = np.diag(c)
+    rhs = np.concatenate([(P * dC).sum(axis=1), (P * dC).sum(axis=0)])
+    sol = np.linalg.lstsq(A, rhs, rcond=None)[0]
+    df, dg = sol[:n], sol[n:]
+    W = P * (df[:, None] + dg[None, :] - dC)
+    return 2.0 * r[:, None] * V + (2.0 / eps) * np.einsum("ij,ijk->ik", W, D)

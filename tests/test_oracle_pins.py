@@ -402,3 +402,42 @@ def test_grad_y_matches_finite_differences_of_the_optimal_value():
             Ym[j, k] -= h
             fd = (value(Yp)[0] - value(Ym)[0]) / (2 * h)
             assert abs(G[j, k] - fd) <= 1e-8, (j, k, G[j, k], fd)
+
+
+# ---- streaming HVP (Metodologia section 3: Hessian-vector products of the EOT
+# loss as sequences of transport-vector and transport-matrix products)
+
+def test_hvp_x_matches_finite_differences_of_the_gradient():
+    """dense.hvp_x against central differences of the gradient at re-converged
+    potentials: (G(X + hV) - G(X - hV)) / 2h."""
+    rng = np.random.default_rng(74)
+    n, m, d, eps = 7, 6, 3, 0.6
+    X = rng.standard_normal((n, d))
+    Y = rng.standard_normal((m, d)) + 0.2
+    a = rng.uniform(0.5, 1.5, n)
+    b = rng.uniform(0.5, 1.5, m)
+    loga, logb = np.log(a / a.sum()), np.log(b / b.sum())
+    V = rng.standard_normal((n, d))
+
+    def grad(Xv):
+        f, g = oracle.solve(Xv, Y, loga, logb, eps, 800)
+        return oracle.grad_x(Xv, Y, loga, logb, f, g, eps), f, g
+
+    _, f, g = grad(X)
+    H = dense.hvp_x(X, Y, loga, logb, f, g, eps, V)
+    h = 1e-5
+    fd = (grad(X + h * V)[0] - grad(X - h * V)[0]) / (2 * h)
+    np.testing.assert_allclose(H, fd, rtol=1e-6, atol=1e-8)
+
+
+def test_hvp_x_is_symmetric():
+    """<W, H V> = <V, H W>: the Hessian is symmetric."""
+    rng = np.random.default_rng(75)
+    n, m, d, eps = 6, 8, 2, 0.5
+    X = rng.standard_normal((n, d))
+    Y = rng.standard_normal((m, d))
+    loga, logb = np.full(n, -np.log(n)), np.full(m, -np.log(m))
+    f, g = oracle.solve(X, Y, loga, logb, eps, 800)
+    V, W = rng.standard_normal((n, d)), rng.standard_normal((n, d))
+    assert abs(np.sum(W * dense.hvp_x(X, Y, loga, logb, f, g, eps, V)) -
+               np.sum(V * dense.hvp_x(X, Y, loga, logb, f, g, eps, W))) <= 1e-10
