@@ -226,6 +226,24 @@ FS_API fs_status fs_transport_apply_t(fs_handle *h, const float *f, const float 
 FS_API fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
                            float *grad);
 
+/*
+ * Hessian-vector product of the entropic OT cost with respect to the positions
+ * X, squared Euclidean cost, at optimal device potentials (f, g), in the
+ * direction V (device fp32 [n][d]); out: device fp32 [n][d].  Streaming
+ * ("FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 3): a sequence of
+ * transport-vector and transport-matrix products, O((n + m) d) memory.  The
+ * potentials' response solves
+ *   [diag(c) - P^T diag(1/r) P] dg = w - P^T (u / r)
+ * by conjugate gradients (each step one transport-vector product each way),
+ * stopped after max_cg_iters steps or when the residual falls below
+ * cg_rtol times its start; *cg_iters_done (may be NULL) receives the steps.
+ * One problem only (batch = 1).  X, Y: the caller's device clouds in the
+ * handle's dtype.  Synchronises the stream once per CG step.
+ * Errors: FS_ERR_INVALID_ARG, FS_ERR_UNSUPPORTED (cosine cost, batch > 1).
+ */
+FS_API fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
+                          const float *V, float *out, int max_cg_iters, double cg_rtol, int *cg_iters_done);
+
 /* Number of CUDA kernels this library has launched in this process so far
  * (all handles, all threads).  Host-side counter; never synchronises. */
 FS_API unsigned long long fs_kernel_launches(void);

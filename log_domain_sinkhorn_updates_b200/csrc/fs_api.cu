@@ -408,6 +408,118 @@ fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const void *X,
     return FS_OK;
 }
 
+fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y, const float *V,
+                   float *out, int max_cg_iters, double cg_rtol, int *cg_iters_done) {
+    if (!h || !f || !g || !X || !Y || !V || !out || max_cg_iters < 1 || !(cg_rtol > 0.0))
+        return fail(h, FS_ERR_INVALID_ARG, "bad argument");
+    const fs_desc &D = h->desc;
+    if (D.cost != FS_COST_SQEUCLIDEAN)
+        return fail(h, FS_ERR_UNSUPPORTED, "fs_hvp_x is defined for the squared Euclidean cost");
+    if (D.batch != 1) return fail(h, FS_ERR_UNSUPPORTED, "fs_hvp_x takes one problem (batch = 1)");
+    FS_CUDA(h, cudaSetDevice(h->device));
+    const size_t n = (size_t)D.n, m = (size_t)D.m, d = (size_t)D.d;
+    const bool bf16 = D.dtype == FS_BF16;
+    const int nq = d >= 256 ? 1 : (int)(256 / d);  // columns of y folded into one transport-matrix product
+    // scratch, O((n + m) d), from the pool for this call
+    size_t off = 0;
+    auto carve = [&](size_t count) {
+        size_t o = off;
+        off += (count * 4 + 255) / 256 * 256;
+        return o;
+    };
+    const size_t oPY = carve(n * d), o_r = carve(n), o_c = carve(m), oW1 = carve(n * (d + 1)), oT = carve(m * (d + 1));
+    const size_t o_u = carve(n), o_w = carve(m), o_tn = carve(n), o_tm = carve(m), o_z = carve(m), o_x = carve(m);
+    const size_t o_res = carve(m), o_p = carve(m), o_Ap = carve(m), o_Pdg = carve(n), o_df = carve(n);
+    const size_t o_dgY = carve(m * d), oQ1 = carve(n * d), oMV = carve(n * d), o_ones = carve(n);
+    const size_t oVc = carve(m * nq * d), oOc = carve(n * nq * d);
+    const size_t o_part = carve(2 * 4096), o_sc = carve(2 * 8);
+    cudaMemPool_t pool;
+    uint8_t *blk = nullptr;
+    FS_CUDA(h, device_pool(h->device, &pool));
+    FS_CUDA(h, cudaMallocFromPoolAsync((void **)&blk, off, pool, h->stream));
+    auto F = [&](size_t o) { return reinterpret_cast<float *>(blk + o); };
+    double *part = reinterpret_cast<double *>(blk + o_part);
+    double *sc = reinterpret_cast<double *>(blk + o_sc);  // [0] rr, [1] p.Ap, [2] rr_new, [3] sum, [4] z.z
+    float *PY = F(oPY), *r = F(o_r), *c = F(o_c), *W1 = F(oW1), *Tm = F(oT), *u = F(o_u), *w = F(o_w);
+    float *tn = F(o_tn), *tm = F(o_tm), *z = F(o_z), *x = F(o_x), *res = F(o_res), *p = F(o_p), *Ap = F(o_Ap);
+    float *Pdg = F(o_Pdg), *df = F(o_df), *dgY = F(o_dgY), *Q1 = F(oQ1), *MV = F(oMV), *ones = F(o_ones);
+    float *Vc = F(oVc), *Oc = F(oOc);
+    cudaStream_t s = h->stream;
+    fs_status st = FS_OK;
+    int it = 0;
+    auto run = [&]() -> fs_status {
+        // transport products that do not depend on the CG solution
+        fs_status s2 = apply(h, f, g, Y, bf16, (int)d, PY, r, false, true);  // P Y, r = P 1
+        if (s2 != FS_OK) return s2;
+        FS_LAUNCH(h, fs::launch_fill(ones, n, 1.f, s));
+        s2 = apply(h, f, g, ones, false, 1, tm, c, false, false);  // c = P^T 1
+        if (s2 != FS_OK) return s2;
+        FS_LAUNCH(h, fs::hvp_prep(X, bf16, V, PY, r, (int)n, (int)d, u, W1, s));
+        s2 = apply(h, f, g, W1, false, (int)d + 1, Tm, nullptr, false, false);  // P^T [V | x.v]
+        if (s2 != FS_OK) return s2;
+        FS_LAUNCH(h, fs::hvp_w(Y, bf16, Tm, (int)m, (int)d, w, s));
+        FS_LAUNCH(h, fs::hvp_vec(n, u, r, 1.f, nullptr, 0.f, true, tn, s));  // u / r
+        s2 = apply(h, f, g, tn, false, 1, tm, nullptr, false, false);        // P^T (u / r)
+        if (s2 != FS_OK) return s2;
+        FS_LAUNCH(h, fs::hvp_vec(m, w, nullptr, 1.f, tm, -1.f, false, z, s));  // z = w - P^T (u / r)
+        FS_LAUNCH(h, fs::hvp_dot(m, z, nullptr, part, sc + 3, s));
+        FS_LAUNCH(h, fs::hvp_center(m, sc + 3, z, s));
+        // CG on [diag(c) - P^T diag(1/r) P] dg = z, iterates kept orthogonal to 1
+        FS_CUDA(h, cudaMemsetAsync(x, 0, m * 4, s));
+        FS_CUDA(h, cudaMemcpyAsync(res, z, m * 4, cudaMemcpyDeviceToDevice, s));
+        FS_CUDA(h, cudaMemcpyAsync(p, z, m * 4, cudaMemcpyDeviceToDevice, s));
+        FS_LAUNCH(h, fs::hvp_dot(m, z, z, part, sc + 0, s));
+        FS_LAUNCH(h, fs::hvp_dot(m, z, z, part, sc + 4, s));
+        double host[5];
+        FS_CUDA(h, cudaMemcpyAsync(host, sc, 5 * 8, cudaMemcpyDeviceToHost, s));
+        FS_CUDA(h, cudaStreamSynchronize(s));
+        const double zz = host[4];
+        double rr = host[0];
+        while (it < max_cg_iters && rr > cg_rtol * cg_rtol * zz && zz > 0.0) {
+            s2 = apply(h, f, g, p, false, 1, tn, nullptr, false, true);  // P p
+            if (s2 != FS_OK) return s2;
+            FS_LAUNCH(h, fs::hvp_vec(n, tn, r, 1.f, nullptr, 0.f, true, tn, s));  // / r
+            s2 = apply(h, f, g, tn, false, 1, tm, nullptr, false, false);       // P^T (P p / r)
+            if (s2 != FS_OK) return s2;
+            FS_LAUNCH(h, fs::hvp_vec(m, p, c, 1.f, tm, -1.f, false, Ap, s));  // c o p - ...
+            FS_LAUNCH(h, fs::hvp_dot(m, Ap, nullptr, part, sc + 3, s));
+            FS_LAUNCH(h, fs::hvp_center(m, sc + 3, Ap, s));
+            FS_LAUNCH(h, fs::hvp_dot(m, p, Ap, part, sc + 1, s));
+            FS_LAUNCH(h, fs::hvp_cg_step(m, sc + 0, sc + 1, p, Ap, x, res, s));
+            FS_LAUNCH(h, fs::hvp_dot(m, res, res, part, sc + 2, s));
+            FS_LAUNCH(h, fs::hvp_cg_dir(m, sc + 2, sc + 0, res, p, s));
+            FS_CUDA(h, cudaMemcpyAsync(sc + 0, sc + 2, 8, cudaMemcpyDeviceToDevice, s));
+            FS_CUDA(h, cudaMemcpyAsync(&rr, sc + 2, 8, cudaMemcpyDeviceToHost, s));
+            FS_CUDA(h, cudaStreamSynchronize(s));
+            ++it;
+        }
+        // df = (u - P dg) / r
+        s2 = apply(h, f, g, x, false, 1, Pdg, nullptr, false, true);
+        if (s2 != FS_OK) return s2;
+        FS_LAUNCH(h, fs::hvp_vec(n, u, nullptr, 1.f, Pdg, -1.f, false, df, s));
+        FS_LAUNCH(h, fs::hvp_vec(n, df, r, 1.f, nullptr, 0.f, true, df, s));
+        // P (dg o Y)
+        FS_LAUNCH(h, fs::hvp_dgy(Y, bf16, x, (int)m, (int)d, dgY, s));
+        s2 = apply(h, f, g, dgY, false, (int)d, Q1, nullptr, false, true);
+        if (s2 != FS_OK) return s2;
+        // sum_j P_ij (y_j.v_i) y_j, nq columns of y at a time
+        FS_CUDA(h, cudaMemsetAsync(MV, 0, n * d * 4, s));
+        for (int k0 = 0; k0 < (int)d; k0 += nq) {
+            const int q = (int)d - k0 < nq ? (int)d - k0 : nq;
+            FS_LAUNCH(h, fs::hvp_ychunk(Y, bf16, (int)m, (int)d, k0, q, Vc, s));
+            s2 = apply(h, f, g, Vc, false, q * (int)d, Oc, nullptr, false, true);
+            if (s2 != FS_OK) return s2;
+            FS_LAUNCH(h, fs::hvp_mv_acc(V, Oc, (int)n, (int)d, k0, q, MV, s));
+        }
+        FS_LAUNCH(h, fs::hvp_final(X, bf16, V, PY, r, df, Pdg, Q1, MV, (int)n, (int)d, D.eps, out, s));
+        return FS_OK;
+    };
+    st = run();
+    cudaFreeAsync(blk, s);
+    if (cg_iters_done) *cg_iters_done = it;
+    return st;
+}
+
 unsigned long long fs_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char *fs_last_error(const fs_handle *h) { return h ? h->last_error.c_str() : g_last_error.c_str(); }

@@ -1,0 +1,245 @@
+// Element-wise and reduction kernels of the streaming Hessian-vector product
+// of the entropic OT cost with respect to X (squared Euclidean cost;
+// "FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 3: the HVP as a
+// sequence of transport-vector and transport-matrix products).  The transport
+// products themselves are the transport-application kernels; these kernels
+// combine their outputs, all O((n + m) d).
+//
+// With P at optimal potentials, r = P 1, c = P^T 1, a direction V [n][d] and
+// dC_ij = 2 (x_i - y_j).v_i:
+//   u_i = sum_j P_ij dC_ij = 2 (r_i x_i - (P Y)_i).v_i
+//   w_j = sum_i P_ij dC_ij = 2 ((P^T (x.v))_j - y_j.(P^T V)_j)
+//   [diag(c) - P^T diag(1/r) P] dg = w - P^T (u / r),   df = (u - P dg) / r
+//   (H V)_i = 2 r_i v_i + (2/eps) [ df_i (r_i x_i - (P Y)_i) + (P dg)_i x_i - (P (dg o Y))_i
+//             - 2 ( (x_i.v_i)(r_i x_i - (P Y)_i) - x_i ((P Y)_i.v_i) + sum_j P_ij (y_j.v_i) y_j ) ]
+#include <cuda_bf16.h>
+
+#include "fs_internal.cuh"
+
+namespace fs {
+namespace {
+
+template <typename T>
+__device__ __forceinline__ float ldv(const T *p, size_t i);
+template <>
+__device__ __forceinline__ float ldv<float>(const float *p, size_t i) {
+    return p[i];
+}
+template <>
+__device__ __forceinline__ float ldv<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+
+__host__ __device__ inline int blocks_for(size_t n) {
+    const size_t b = (n + 255) / 256;
+    return (int)(b < 4096 ? (b > 0 ? b : 1) : 4096);
+}
+
+#define GRID_LOOP(i, n) for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < (n); i += (size_t)gridDim.x * blockDim.x)
+
+// u_i = 2 (r_i x_i - PY_i).v_i;  W1_i = [v_i | x_i.v_i]  ([n][d+1])
+template <typename T>
+__global__ void prep_kernel(const T *X, const float *V, const float *PY, const float *r, int n, int d, float *u,
+                            float *W1) {
+    GRID_LOOP(i, (size_t)n) {
+        float su = 0.f, sxv = 0.f;
+        for (int k = 0; k < d; ++k) {
+            const float x = ldv(X, i * d + k), v = V[i * d + k];
+            su = fmaf(r[i] * x - PY[i * d + k], v, su);
+            sxv = fmaf(x, v, sxv);
+            W1[i * (d + 1) + k] = v;
+        }
+        W1[i * (d + 1) + d] = sxv;
+        u[i] = 2.f * su;
+    }
+}
+
+// w_j = 2 (T_j[d] - y_j . T_j[0:d]),  T = P^T W1  ([m][d+1])
+template <typename T>
+__global__ void w_kernel(const T *Y, const float *Tm, int m, int d, float *w) {
+    GRID_LOOP(j, (size_t)m) {
+        float s = 0.f;
+        for (int k = 0; k < d; ++k) s = fmaf(ldv(Y, j * d + k), Tm[j * (d + 1) + k], s);
+        w[j] = 2.f * (Tm[j * (d + 1) + d] - s);
+    }
+}
+
+// out = alpha * x o a + beta * y  (a or y may be null: treated as 1 / 0); or out = x / a when div
+__global__ void vec_kernel(size_t n, const float *x, const float *a, float alpha, const float *y, float beta,
+                           bool div, float *out) {
+    GRID_LOOP(i, n) {
+        const float av = a ? a[i] : 1.f;
+        const float t = div ? x[i] / av : alpha * x[i] * av;
+        out[i] = t + (y ? beta * y[i] : 0.f);
+    }
+}
+
+// Deterministic dot product: fixed-order block trees, then one block over the partials.
+__global__ void dot_partial_kernel(size_t n, const float *x, const float *y, double *part) {
+    __shared__ double sh[256];
+    double s = 0.0;
+    GRID_LOOP(i, n) s += (double)x[i] * (double)(y ? y[i] : 1.f);
+    sh[threadIdx.x] = s;
+    __syncthreads();
+    for (int k = 128; k > 0; k >>= 1) {
+        if ((int)threadIdx.x < k) sh[threadIdx.x] += sh[threadIdx.x + k];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) part[blockIdx.x] = sh[0];
+}
+__global__ void dot_final_kernel(int nb, const double *part, double *out) {
+    __shared__ double sh[256];
+    double s = 0.0;
+    for (int i = threadIdx.x; i < nb; i += 256) s += part[i];
+    sh[threadIdx.x] = s;
+    __syncthreads();
+    for (int k = 128; k > 0; k >>= 1) {
+        if ((int)threadIdx.x < k) sh[threadIdx.x] += sh[threadIdx.x + k];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) *out = sh[0];
+}
+
+// x -= s / n (s: a device double), keeping CG iterates orthogonal to the constant vector
+__global__ void center_vec_kernel(size_t n, const double *s, float *x) {
+    const float mean = (float)(*s / (double)n);
+    GRID_LOOP(i, n) x[i] -= mean;
+}
+
+// CG update on the device, from device scalars rr (r.r) and pap (p.Ap):
+//   alpha = rr / pap;  x += alpha p;  res -= alpha Ap
+__global__ void cg_step_kernel(size_t n, const double *rr, const double *pap, const float *p, const float *Ap,
+                               float *x, float *res) {
+    const float alpha = (float)(*rr / *pap);
+    GRID_LOOP(i, n) {
+        x[i] = fmaf(alpha, p[i], x[i]);
+        res[i] = fmaf(-alpha, Ap[i], res[i]);
+    }
+}
+// p = res + (rr_new / rr) p
+__global__ void cg_dir_kernel(size_t n, const double *rr_new, const double *rr, const float *res, float *p) {
+    const float beta = (float)(*rr_new / *rr);
+    GRID_LOOP(i, n) p[i] = fmaf(beta, p[i], res[i]);
+}
+
+// out_jk = dg_j y_jk
+template <typename T>
+__global__ void dgy_kernel(const T *Y, const float *dg, int m, int d, float *out) {
+    GRID_LOOP(i, (size_t)m * d) out[i] = dg[i / d] * ldv(Y, i);
+}
+
+// Vc_j[q d + k] = y_j[k0 + q] y_jk for q < nq  ([m][nq d])
+template <typename T>
+__global__ void ychunk_kernel(const T *Y, int m, int d, int k0, int nq, float *Vc) {
+    GRID_LOOP(i, (size_t)m * nq * d) {
+        const size_t j = i / ((size_t)nq * d);
+        const int q = (int)((i / d) % nq), k = (int)(i % d);
+        Vc[i] = ldv(Y, j * d + k0 + q) * ldv(Y, j * d + k);
+    }
+}
+
+// MV_ik += sum_q v_i[k0 + q] Oc_i[q d + k]
+__global__ void mv_acc_kernel(const float *V, const float *Oc, int n, int d, int k0, int nq, float *MV) {
+    GRID_LOOP(i, (size_t)n * d) {
+        const size_t row = i / d;
+        const int k = (int)(i % d);
+        float s = MV[i];
+        for (int q = 0; q < nq; ++q) s = fmaf(V[row * d + k0 + q], Oc[(row * nq + q) * d + k], s);
+        MV[i] = s;
+    }
+}
+
+template <typename T>
+__global__ void final_kernel(const T *X, const float *V, const float *PY, const float *r, const float *df,
+                             const float *Pdg, const float *Q1, const float *MV, int n, int d, float eps, float *out) {
+    GRID_LOOP(i, (size_t)n) {
+        float xv = 0.f, pyv = 0.f;
+        for (int k = 0; k < d; ++k) {
+            const float v = V[i * d + k];
+            xv = fmaf(ldv(X, i * d + k), v, xv);
+            pyv = fmaf(PY[i * d + k], v, pyv);
+        }
+        for (int k = 0; k < d; ++k) {
+            const float x = ldv(X, i * d + k);
+            const float gk = r[i] * x - PY[i * d + k];  // sum_j P_ij (x_i - y_j), component k
+            const float inner = df[i] * gk + Pdg[i] * x - Q1[i * d + k] -
+                                2.f * (xv * gk - x * pyv + MV[i * d + k]);
+            out[i * d + k] = 2.f * r[i] * V[i * d + k] + (2.f / eps) * inner;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t hvp_prep(const void *X, bool bf16, const float *V, const float *PY, const float *r, int n, int d,
+                     float *u, float *W1, cudaStream_t s) {
+    if (bf16)
+        prep_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(X), V, PY, r, n, d, u, W1);
+    else
+        prep_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const float *>(X), V, PY, r, n, d, u, W1);
+    return cudaGetLastError();
+}
+cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float *w, cudaStream_t s) {
+    if (bf16)
+        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), Tm, m, d, w);
+    else
+        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const float *>(Y), Tm, m, d, w);
+    return cudaGetLastError();
+}
+cudaError_t hvp_vec(size_t n, const float *x, const float *a, float alpha, const float *y, float beta, bool div,
+                    float *out, cudaStream_t s) {
+    vec_kernel<<<blocks_for(n), 256, 0, s>>>(n, x, a, alpha, y, beta, div, out);
+    return cudaGetLastError();
+}
+// *out = x.y (y null: sum of x); part holds at least 4096 doubles.
+cudaError_t hvp_dot(size_t n, const float *x, const float *y, double *part, double *out, cudaStream_t s) {
+    const int nb = blocks_for(n);
+    dot_partial_kernel<<<nb, 256, 0, s>>>(n, x, y, part);
+    dot_final_kernel<<<1, 256, 0, s>>>(nb, part, out);
+    return cudaGetLastError();
+}
+cudaError_t hvp_center(size_t n, const double *sum, float *x, cudaStream_t s) {
+    center_vec_kernel<<<blocks_for(n), 256, 0, s>>>(n, sum, x);
+    return cudaGetLastError();
+}
+cudaError_t hvp_cg_step(size_t n, const double *rr, const double *pap, const float *p, const float *Ap, float *x,
+                        float *res, cudaStream_t s) {
+    cg_step_kernel<<<blocks_for(n), 256, 0, s>>>(n, rr, pap, p, Ap, x, res);
+    return cudaGetLastError();
+}
+cudaError_t hvp_cg_dir(size_t n, const double *rr_new, const double *rr, const float *res, float *p, cudaStream_t s) {
+    cg_dir_kernel<<<blocks_for(n), 256, 0, s>>>(n, rr_new, rr, res, p);
+    return cudaGetLastError();
+}
+cudaError_t hvp_dgy(const void *Y, bool bf16, const float *dg, int m, int d, float *out, cudaStream_t s) {
+    if (bf16)
+        dgy_kernel<<<blocks_for((size_t)m * d), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), dg, m, d, out);
+    else
+        dgy_kernel<<<blocks_for((size_t)m * d), 256, 0, s>>>(static_cast<const float *>(Y), dg, m, d, out);
+    return cudaGetLastError();
+}
+cudaError_t hvp_ychunk(const void *Y, bool bf16, int m, int d, int k0, int nq, float *Vc, cudaStream_t s) {
+    if (bf16)
+        ychunk_kernel<<<blocks_for((size_t)m * nq * d), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), m, d, k0,
+                                                                     nq, Vc);
+    else
+        ychunk_kernel<<<blocks_for((size_t)m * nq * d), 256, 0, s>>>(static_cast<const float *>(Y), m, d, k0, nq, Vc);
+    return cudaGetLastError();
+}
+cudaError_t hvp_mv_acc(const float *V, const float *Oc, int n, int d, int k0, int nq, float *MV, cudaStream_t s) {
+    mv_acc_kernel<<<blocks_for((size_t)n * d), 256, 0, s>>>(V, Oc, n, d, k0, nq, MV);
+    return cudaGetLastError();
+}
+cudaError_t hvp_final(const void *X, bool bf16, const float *V, const float *PY, const float *r, const float *df,
+                      const float *Pdg, const float *Q1, const float *MV, int n, int d, float eps, float *out,
+                      cudaStream_t s) {
+    if (bf16)
+        final_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(X), V, PY, r, df, Pdg, Q1, MV,
+                                                   n, d, eps, out);
+    else
+        final_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const float *>(X), V, PY, r, df, Pdg, Q1, MV, n, d,
+                                                   eps, out);
+    return cudaGetLastError();
+}
+
+}  // namespace fs

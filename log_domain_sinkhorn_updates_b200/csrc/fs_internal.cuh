@@ -170,6 +170,23 @@ cudaError_t launch_vt_pack(const void *V, bool bf16, int batch, int m, int dv, i
                            void *out, cudaStream_t s);
 cudaError_t launch_apply_tc(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
                             const void *map_v, size_t smem, cudaStream_t s);
+// Element-wise pieces of the streaming Hessian-vector product (fs_hvp.cu).
+cudaError_t hvp_prep(const void *X, bool bf16, const float *V, const float *PY, const float *r, int n, int d,
+                     float *u, float *W1, cudaStream_t s);
+cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float *w, cudaStream_t s);
+cudaError_t hvp_vec(size_t n, const float *x, const float *a, float alpha, const float *y, float beta, bool div,
+                    float *out, cudaStream_t s);
+cudaError_t hvp_dot(size_t n, const float *x, const float *y, double *part, double *out, cudaStream_t s);
+cudaError_t hvp_center(size_t n, const double *sum, float *x, cudaStream_t s);
+cudaError_t hvp_cg_step(size_t n, const double *rr, const double *pap, const float *p, const float *Ap, float *x,
+                        float *res, cudaStream_t s);
+cudaError_t hvp_cg_dir(size_t n, const double *rr_new, const double *rr, const float *res, float *p, cudaStream_t s);
+cudaError_t hvp_dgy(const void *Y, bool bf16, const float *dg, int m, int d, float *out, cudaStream_t s);
+cudaError_t hvp_ychunk(const void *Y, bool bf16, int m, int d, int k0, int nq, float *Vc, cudaStream_t s);
+cudaError_t hvp_mv_acc(const float *V, const float *Oc, int n, int d, int k0, int nq, float *MV, cudaStream_t s);
+cudaError_t hvp_final(const void *X, bool bf16, const float *V, const float *PY, const float *r, const float *df,
+                      const float *Pdg, const float *Q1, const float *MV, int n, int d, float eps, float *out,
+                      cudaStream_t s);
 // grad[bz][i][k] = 2 (r_i x_ik - pv[bz][i][k]) from the caller's X (fp32 or bf16).
 cudaError_t launch_grad_combine(const void *X, bool bf16, const float *r, const float *pv, int batch, int rows,
                                 int d, float *grad, cudaStream_t s);
