@@ -105,6 +105,23 @@ def cpu_baseline(prob, seconds):
                        f"workload, {dt:.1f} s on {threads} threads")}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of per-rank timings over all ranks of the default process group
+    (identity on one process): every multi-GPU number is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_throughput(world, steps, units_per_step, total_ms):
+    """Whole-job throughput of `world` independent replicas: every rank processes
+    units_per_step per step, timed as the slowest rank's total over `steps` steps."""
+    return world * steps * units_per_step / (total_ms / 1e3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -278,10 +295,7 @@ def run_transport(args):
     fs.fs_sync(h)
     launches = fs.fs_kernel_launches() - launches0
     clocks = sampler.stop()
-    tt = torch.tensor([tot], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-    tot = tt.item()
+    tot = max_over_ranks([tot], dev)[0]
     info = fs.fs_get_info(h)
     entries = B * n * m
     app_s = tot / 1e3 / args.steps
@@ -293,7 +307,7 @@ def run_transport(args):
     peak = float(peaks.get("bf16_tflops", 1590.0))
     line = {
         "metric": "transport application (barycentric map) cost-entries/s at the converged potentials",
-        "value": world * entries / app_s, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "value": replica_throughput(world, args.steps, entries, tot), "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": tot / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if info["prec"] == "bf16" else "f32", "data": "synthetic",
         "config": workload_config(prob, args.iters or prob.iters, {
@@ -399,14 +413,11 @@ def main():
 
     step_ms = sum(e[0].elapsed_time(e[3]) for e in evs)
     solve_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    t = torch.tensor([step_ms, solve_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, solve_ms = t.tolist()
+    step_ms, solve_ms = max_over_ranks([step_ms, solve_ms], dev)
 
     entries_per_half = B * n * m
     half_per_step = 2 * iters
-    value = world * args.steps * half_per_step * entries_per_half / (step_ms / 1e3)
+    value = replica_throughput(world, args.steps, half_per_step * entries_per_half, step_ms)
 
     # ---- roofline of the dominant kernel (the streamed LSE pass) ----
     peaks, peak_src = load_peaks()
@@ -461,15 +472,12 @@ def main():
             e1.record(stream)
             torch.cuda.synchronize(dev)
             tot += e0.elapsed_time(e1)
-        tt = torch.tensor([tot], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        tot = tt.item()
+        tot = max_over_ranks([tot], dev)[0]
         h2d = Xh.numel() * Xh.element_size() + Yh.numel() * Yh.element_size() + g0.numel() * 4
         h2d += 0 if ap is None else ap.numel() * 4
         h2d += 0 if bp is None else bp.numel() * 4
         d2h = (fo.numel() + go.numel()) * 4 + 4 * B * 8
-        e2e = {"value": world * args.steps * half_per_step * entries_per_half / (tot / 1e3), "unit": UNIT,
+        e2e = {"value": replica_throughput(world, args.steps, half_per_step * entries_per_half, tot), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": tot / args.steps,
                "api": "fs_solve_host (C ABI, pinned host buffers)"}
 

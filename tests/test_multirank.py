@@ -1,0 +1,68 @@
+"""The multi-GPU path of the benchmark on CPU: world_size-2 gloo ranks.
+
+The benchmark spec is one GPU per problem; several GPUs run independent replicas
+(no data-path collective), so the only cross-rank steps are the barrier and the
+max-over-ranks timing reduction.  Those are exercised here with gloo, together
+with the reference arm's rank-0-only behaviour.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    local = [10.0 + 5.0 * rank, 3.0 - rank]  # per-rank step and solve times (ms)
+    dist.barrier()
+    step_ms, solve_ms = bench.max_over_ranks(local)
+    value = bench.replica_throughput(world, 4, 1000, step_ms)
+    out.put((rank, step_ms, solve_ms, value))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_replica_throughput_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, step_ms, solve_ms, value in res:
+        assert step_ms == 15.0 and solve_ms == 3.0  # the slowest rank's, on every rank
+        assert value == pytest.approx(2 * 4 * 1000 / 0.015)  # all ranks' units / slowest time
+
+
+def test_single_process_reduction_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
+    assert bench.replica_throughput(1, 2, 50, 100.0) == pytest.approx(1000.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2"],
+                       env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == ""
