@@ -124,3 +124,52 @@ def test_full_size_solve_against_stored_oracle(cuda_device, name):
         assert abs(primal[k] - gp["primal"]) <= 1e-3 * abs(gp["primal"]), (name, k, primal[k], gp["primal"])
         assert abs(e_gpu - e_o) <= 1e-2 * e_o + floor, (name, k, e_gpu, e_o, floor)
         assert pot_err <= 1e-3 * gp["max_cost"], (name, k, pot_err, gp["max_cost"])
+
+
+@pytest.mark.parametrize("name", ["highdim", "middim", "cloud3d"])
+def test_full_size_transport_sampled(cuda_device, name):
+    """The barycentric map on the full workload (the configuration `bench.py --op
+    transport` times), checked at sampled rows that the oracle computes one by one
+    from the plan's definition.
+
+    Potentials: a seeded smooth g, and f = the oracle's f-update of g.  The f-update
+    makes every row sum r_i equal a_i, as at a solution.  Arbitrary potentials at
+    these eps would put whole plan rows below the fp32 range; a solution never
+    does.  On highdim the full oracle pass would take minutes, and its costs are
+    small enough against eps that a seeded smooth f stays in range."""
+    import torch
+    fs = _fs()
+    prob = make_problem(name)
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    rng = np.random.default_rng(777)
+    g_in = smooth_potential(rng, prob.m, 0.05)[None]
+    if name == "highdim":
+        f_in = smooth_potential(rng, prob.n, 0.05)[None]
+    else:
+        Xo, Yo, _, logb = oracle.problem_arrays(prob, 0)
+        f_in = oracle.update_f(Xo, Yo, logb, g_in[0].astype(np.float64), prob.eps).astype(np.float32)[None]
+    fd, gd = torch.from_numpy(f_in).to(cuda_device), torch.from_numpy(g_in).to(cuda_device)
+    T = torch.empty(1, prob.n, prob.d, device=cuda_device)
+    fs.fs_barycentric_map(h, fd, gd, Y, T)
+    fs.fs_sync(h)
+    T = T.cpu().numpy()[0]
+    Xo, Yo, loga, logb = oracle.problem_arrays(prob, 0)
+    rows = np.unique(np.concatenate([[0, prob.n - 1], rng.choice(prob.n, 64, replace=False)]))
+    fk, gk = f_in[0].astype(np.float64), g_in[0].astype(np.float64)
+    out, r = oracle.transport_apply(Xo[rows], Yo, loga[rows], logb, fk[rows], gk, prob.eps, Yo)
+    absw, _ = oracle.transport_apply(Xo[rows], Yo, loga[rows], logb, fk[rows], gk, prob.eps, np.abs(Yo))
+    To = out / r[:, None]
+    # relative error bound of the plan entries (see tests/test_gpu_transport.py), 2^-14 for the
+    # tensor-core splits; T = (P Y)/r carries it twice
+    xs_t = 0.5 * (Xo.mean(0) + Yo.mean(0))
+    xs, ys = Xo[rows] - xs_t, Yo - xs_t
+    LOG2E = 1.0 / np.log(2.0)
+    alpha = loga[rows] * LOG2E + (fk[rows] - (xs ** 2).sum(1)) * LOG2E / prob.eps
+    beta = logb * LOG2E + (gk - (ys ** 2).sum(1)) * LOG2E / prob.eps
+    M = np.abs(alpha) + np.abs(beta).max() + (2 * prob.d + 2) * 2 * np.sqrt((xs ** 2).sum(1)) * \
+        np.sqrt((ys ** 2).sum(1)).max() * LOG2E / prob.eps
+    rel = np.log(2.0) * 2.0 ** -23 * M + 2.0 ** -21 + prob.m * 2.0 ** -24 + 2.0 ** -14
+    err = (np.abs(T[rows] - To) / (2 * rel[:, None] * absw / r[:, None] + 1e-6 * np.abs(To))).max()
+    print(f"{name} full-size barycentric map, sampled rows: worst err / bound = {err:.3f}")
+    assert err <= 1.0

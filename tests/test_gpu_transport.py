@@ -200,3 +200,39 @@ def test_transposed_apply_and_grad_y_parity(cuda_device, name, path, monkeypatch
         e3 = (np.abs(G[k] - Go) / gb).max()
         print(f"{path} {name}[{k}] transposed err/bound {e1:.3f} col sums {e2:.3f} grad_y {e3:.3f}")
         assert e1 <= 1.0 and e2 <= 1.0 and e3 <= 1.0
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("n,m,d", [(1, 1, 3), (1, 300, 5), (300, 1, 5), (129, 65, 2), (257, 200, 33)])
+def test_transport_apply_edge_shapes(cuda_device, n, m, d, path, monkeypatch):
+    """Single points, one-column plans and ragged row/column counts around the
+    128-row blocks and 64-column tiles."""
+    import torch
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
+    fs = _fs()
+    rng = np.random.default_rng(n * 1000 + m + d)
+    Xo = rng.standard_normal((n, d))
+    Yo = rng.standard_normal((m, d)) + 0.3
+    X = torch.from_numpy(Xo.astype(np.float32)).to(cuda_device)
+    Y = torch.from_numpy(Yo.astype(np.float32)).to(cuda_device)
+    eps = 0.2
+    h = fs.fs_create(X, Y, eps=eps)
+    Xd, Yd = X.double().cpu().numpy(), Y.double().cpu().numpy()
+    loga, logb = np.full(n, -np.log(n)), np.full(m, -np.log(m))
+    f, g = oracle.solve(Xd, Yd, loga, logb, eps, 10)
+    f32, g32 = f.astype(np.float32), g.astype(np.float32)
+    V = rng.standard_normal((m, 3)).astype(np.float32)
+    out = torch.empty(1, n, 3, device=cuda_device)
+    r = torch.empty(1, n, device=cuda_device)
+    fs.fs_transport_apply(h, torch.from_numpy(f32[None]).to(cuda_device), torch.from_numpy(g32[None]).to(cuda_device),
+                          torch.from_numpy(V[None]).to(cuda_device), out, r)
+    fs.fs_sync(h)
+    oo, ro = oracle.transport_apply(Xd, Yd, loga, logb, f32.astype(np.float64), g32.astype(np.float64), eps,
+                                    V.astype(np.float64))
+    absw, _ = oracle.transport_apply(Xd, Yd, loga, logb, f32.astype(np.float64), g32.astype(np.float64), eps,
+                                     np.abs(V).astype(np.float64))
+    rel = _rel_bound(Xd, Yd, loga, logb, f32.astype(np.float64), g32.astype(np.float64), eps, "sqeuclidean") + \
+        SPLIT[path]
+    err = (np.abs(out.cpu().numpy()[0] - oo) / (rel[:, None] * absw)).max()
+    rerr = (np.abs(r.cpu().numpy()[0] - ro) / (rel * ro)).max()
+    assert err <= 1.0 and rerr <= 1.0, (err, rerr)
