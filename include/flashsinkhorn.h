@@ -244,6 +244,12 @@ FS_API fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const v
 FS_API fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
                           const float *V, float *out, int max_cg_iters, double cg_rtol, int *cg_iters_done);
 
+/* Failure-path self test: launches on the handle's stream a kernel whose one
+ * bounded wait (the same wait every pass uses) can never complete, and waits
+ * for it.  Returns FS_ERR_TIMEOUT after about timeout_ms; the handle and the
+ * CUDA context stay usable.  FS_ERR_INVALID_ARG for timeout_ms < 1. */
+FS_API fs_status fs_selftest_wait(fs_handle *h, int timeout_ms);
+
 /* Number of CUDA kernels this library has launched in this process so far
  * (all handles, all threads).  Host-side counter; never synchronises. */
 FS_API unsigned long long fs_kernel_launches(void);

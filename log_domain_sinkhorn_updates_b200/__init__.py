@@ -12,6 +12,7 @@ import importlib
 __all__ = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_err", "fs_ot_cost", "fs_sync",
            "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches", "fs_update_f_noalloc",
            "fs_transport_apply", "fs_barycentric_map", "fs_grad_x", "fs_transport_apply_t", "fs_grad_y", "fs_hvp_x",
+           "fs_selftest_wait",
            "FsError", "Handle"]
 
 

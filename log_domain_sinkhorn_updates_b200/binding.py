@@ -27,7 +27,7 @@ STATUS_NAMES = {0: "FS_OK", 1: "FS_ERR_INVALID_ARG", 2: "FS_ERR_CUDA", 3: "FS_ER
 EXPORTS = ["fs_create", "fs_update_f", "fs_update_g", "fs_solve", "fs_marginal_err", "fs_ot_cost",
            "fs_sync", "fs_get_info", "fs_destroy", "fs_last_error", "fs_solve_host", "fs_kernel_launches",
            "fs_update_f_noalloc", "fs_transport_apply", "fs_barycentric_map", "fs_grad_x",
-           "fs_transport_apply_t", "fs_grad_y", "fs_hvp_x"]
+           "fs_transport_apply_t", "fs_grad_y", "fs_hvp_x", "fs_selftest_wait"]
 
 
 class FsDesc(ctypes.Structure):
@@ -86,6 +86,7 @@ def lib():
         L.fs_transport_apply_t.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp]
         L.fs_grad_y.argtypes = [vp, vp, vp, vp, vp, vp]
         L.fs_hvp_x.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_double, vp]
+        L.fs_selftest_wait.argtypes = [vp, ctypes.c_int]
         L.fs_kernel_launches.argtypes = []
         L.fs_kernel_launches.restype = ctypes.c_ulonglong
         for name in EXPORTS:
@@ -317,3 +318,8 @@ def fs_hvp_x(h: Handle, f, g, X, Y, V, out, max_cg_iters=200, cg_rtol=1e-6) -> i
     _check(lib().fs_hvp_x(h.ptr, _f32(f), _f32(g), _ptr(X), _ptr(Y), _f32(V), _f32(out), int(max_cg_iters),
                           float(cg_rtol), ctypes.byref(it)), h.ptr)
     return it.value
+
+
+def fs_selftest_wait(h: Handle, timeout_ms=50) -> int:
+    """Run the failure-path self test; returns the library status (FS_ERR_TIMEOUT = 5 expected)."""
+    return int(lib().fs_selftest_wait(h.ptr, int(timeout_ms)))

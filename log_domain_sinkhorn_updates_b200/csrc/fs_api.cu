@@ -520,6 +520,13 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     return st;
 }
 
+fs_status fs_selftest_wait(fs_handle *h, int timeout_ms) {
+    if (!h || timeout_ms < 1) return fail(h, FS_ERR_INVALID_ARG, "bad argument");
+    FS_CUDA(h, cudaSetDevice(h->device));
+    FS_LAUNCH(h, fs::launch_wait_probe((unsigned long long)timeout_ms * 1000000ull, h->err, h->stream));
+    return check_flags(h);
+}
+
 unsigned long long fs_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char *fs_last_error(const fs_handle *h) { return h ? h->last_error.c_str() : g_last_error.c_str(); }
@@ -572,8 +579,10 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         }
     }
     if (const char *env = getenv("FS_WAIT_TIMEOUT_MS")) {
+        // at least 100 ms: the same limit bounds the waits with which a timed-out
+        // kernel drains its own copies and MMAs before freeing shared memory and TMEM
         const long long ms = atoll(env);
-        if (ms > 0) h->timeout_ns = (unsigned long long)ms * 1000000ull;
+        if (ms > 0) h->timeout_ns = (unsigned long long)(ms < 100 ? 100 : ms) * 1000000ull;
     }
 
     // ---- precision and packed layout ----

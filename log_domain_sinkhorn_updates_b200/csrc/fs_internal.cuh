@@ -170,6 +170,9 @@ cudaError_t launch_vt_pack(const void *V, bool bf16, int batch, int m, int dv, i
                            void *out, cudaStream_t s);
 cudaError_t launch_apply_tc(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
                             const void *map_v, size_t smem, cudaStream_t s);
+// A kernel whose one bounded mbarrier wait nothing ever completes: after
+// timeout_ns it raises kDevErrTimeout and returns (fs_tc_common usage check).
+cudaError_t launch_wait_probe(unsigned long long timeout_ns, int *err, cudaStream_t s);
 // Element-wise pieces of the streaming Hessian-vector product (fs_hvp.cu).
 cudaError_t hvp_prep(const void *X, bool bf16, const float *V, const float *PY, const float *r, int n, int d,
                      float *u, float *W1, cudaStream_t s);

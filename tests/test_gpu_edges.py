@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 
 import oracle
-from helpers import device_inputs, make_problem
+from helpers import device_inputs, make_problem, max_cost, oracle_arrays
 
 pytestmark = pytest.mark.gpu
 
@@ -188,3 +188,25 @@ def test_input_validation(cuda_device):
     h = fs.fs_create(Xd, Yd, a, None, eps=0.1)  # valid weights pass
     info = fs.fs_get_info(h)
     assert info["device_bytes"] < 100 * (50 + 60) * 4 * 64 + (1 << 20)
+
+
+def test_bounded_wait_times_out_and_the_context_stays_usable(cuda_device):
+    """A kernel waits on an mbarrier that nothing completes: the bounded wait ends,
+    the status is FS_ERR_TIMEOUT, and the same handle then runs a correct update."""
+    import time
+    import torch
+    import log_domain_sinkhorn_updates_b200 as fs
+    prob = make_problem("tiny")
+    X, Y, a, b = device_inputs(prob)
+    h = fs.fs_create(X, Y, a, b, eps=prob.eps)
+    t0 = time.perf_counter()
+    st = fs.fs_selftest_wait(h, 50)
+    dt = time.perf_counter() - t0
+    assert st == 5 and dt >= 0.045, (st, dt)
+    g_in = torch.zeros(1, prob.m, device=cuda_device)
+    f = torch.empty(1, prob.n, device=cuda_device)
+    fs.fs_update_f(h, g_in, f)
+    fs.fs_sync(h)
+    Xo, Yo, _, logb = oracle_arrays(prob)[0]
+    fo = oracle.update_f(Xo, Yo, logb, np.zeros(prob.m), prob.eps)
+    assert np.abs(f.cpu().numpy()[0] - fo).max() <= 1e-4 * max_cost(prob)[0] / 4
