@@ -489,25 +489,6 @@ cudaError_t launch_vt_pack(const void *V, bool bf16, int batch, int m, int dv, i
     return cudaGetLastError();
 }
 
-namespace {
-// One mbarrier that nothing arrives at, waited on with the same bounded wait as
-// every pass: the failure path (error bit, clean return) without a fault.
-__global__ void wait_probe_kernel(unsigned long long timeout_ns, int *err) {
-    __shared__ uint64_t bar;
-    if (threadIdx.x == 0) {
-        mbar_init(&bar, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncthreads();
-    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, timeout_ns)) atomicOr(err, kDevErrTimeout);
-}
-}  // namespace
-
-cudaError_t launch_wait_probe(unsigned long long timeout_ns, int *err, cudaStream_t s) {
-    wait_probe_kernel<<<1, 32, 0, s>>>(timeout_ns, err);
-    return cudaGetLastError();
-}
-
 // prec: 1 = bf16, 2 = tf32, 3 = 3xTF32, 4 = 3xF16 (the S product); vpl: planes of V~.
 cudaError_t launch_apply_tc(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
                             const void *map_v, size_t smem, cudaStream_t s) {
