@@ -10,10 +10,11 @@
 namespace fs {
 namespace tc {
 
-// Largest growth (base 2) of a row's maximum that is absorbed without a
-// rescale: terms up to 2^kLazy stay in the running sum as they are.
-constexpr float kLazy = 12.f;
-constexpr float kLazySum = 4096.f;  // 2^kLazy: a block sum above it forces the rescale
+// Lazy rescaling of a row's running maximum: a block whose exponentials, taken
+// against the running max, sum to more than 2^12 forces the rescale; smaller
+// sums (every entry at most 12 above the running max) join the running sum as
+// they are.
+constexpr float kLazySum = 4096.f;
 
 __device__ __forceinline__ uint32_t saddr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -90,36 +91,6 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
             "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
             : "memory");
     }
-}
-// D (TMEM) (+)= A (TMEM: one row per lane, K along 32-bit columns) x B^T (shared memory).
-template <int KIND>
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accum) {
-    if constexpr (KIND != 1) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-            "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
-            : "memory");
-    } else {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-            "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
-            : "memory");
-    }
-}
-// 32 TMEM lanes (this warp's quadrant) x 32 consecutive 32-bit columns, from registers.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
 }
 // 32 TMEM lanes (this warp's quadrant) x 32 consecutive 32-bit columns.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r) {
@@ -259,8 +230,8 @@ __device__ __forceinline__ float sum_exp2(const float (&z)[CNT], float ref) {
 // Fold CNT scores (raw fp32 bits from TMEM) into a row's online state (m, l):
 // z = S * c + beta.  The first block of a row takes two passes (max, then
 // exponentials).  Later blocks take their exponentials against the running max
-// as it stood and add them up; only when that block sum exceeds 2^kLazy (which
-// every entry more than kLazy above the running max forces, and which an
+// as it stood and add them up; only when that block sum exceeds 2^12 (which
+// every entry more than 12 above the running max forces, and which an
 // overflow to inf or a NaN also fails) is the block's max taken and the block
 // redone against it.  The common case thus spends no instruction on the max.
 template <int CNT>
@@ -316,49 +287,9 @@ __device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float
     consume<128>(r, bias, c, m, l);
 }
 
-// Measure-mode fold over 32 columns: also accumulates w = sum 2^(z - m) C_ij
-// with C_ij = |row|^2 + |col|^2 - S_ij (S_ij = raw score * sscale).
-__device__ __forceinline__ void consume32_measure(const uint32_t (&r)[32], const float *bias, const float *cnorm,
-                                                  float c, float sscale, float xn, float &m, float &l, float &w) {
-    const float4 *bq = reinterpret_cast<const float4 *>(bias);
-    const float4 *cq = reinterpret_cast<const float4 *>(cnorm);
-    float z[32];
-    float t0 = -INFINITY, t1 = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < 32; k += 4) {
-        const float4 bb = bq[k / 4];
-        z[k + 0] = fmaf(__uint_as_float(r[k + 0]), c, bb.x);
-        z[k + 1] = fmaf(__uint_as_float(r[k + 1]), c, bb.y);
-        z[k + 2] = fmaf(__uint_as_float(r[k + 2]), c, bb.z);
-        z[k + 3] = fmaf(__uint_as_float(r[k + 3]), c, bb.w);
-        t0 = fmaxf(t0, fmaxf(z[k + 0], z[k + 1]));
-        t1 = fmaxf(t1, fmaxf(z[k + 2], z[k + 3]));
-    }
-    const float mnew = fmaxf(m, fmaxf(t0, t1));
-    if (mnew == -INFINITY) return;
-    const float scale = ex2_approx(m - mnew);
-    float a0 = 0.f, a1 = 0.f, w0 = 0.f, w1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 32; k += 4) {
-        const float4 cn = cq[k / 4];
-        const float e0 = ex2_approx(z[k + 0] - mnew);
-        const float e1 = ex2_approx(z[k + 1] - mnew);
-        const float e2 = ex2_approx(z[k + 2] - mnew);
-        const float e3 = ex2_approx(z[k + 3] - mnew);
-        a0 += e0 + e2;
-        a1 += e1 + e3;
-        w0 = fmaf(e0, fmaf(-__uint_as_float(r[k + 0]), sscale, xn + cn.x), w0);
-        w1 = fmaf(e1, fmaf(-__uint_as_float(r[k + 1]), sscale, xn + cn.y), w1);
-        w0 = fmaf(e2, fmaf(-__uint_as_float(r[k + 2]), sscale, xn + cn.z), w0);
-        w1 = fmaf(e3, fmaf(-__uint_as_float(r[k + 3]), sscale, xn + cn.w), w1);
-    }
-    l = l * scale + (a0 + a1);
-    w = w * scale + (w0 + w1);
-    m = mnew;
-}
-
-// Measure-mode version over 64 columns: also accumulates w = sum 2^(z - m) C_ij
-// with C_ij = |row|^2 + |col|^2 - S_ij.
+// Measure-mode fold over 64 columns (two 32-column TMEM loads): besides (m, l)
+// it accumulates w = sum_j 2^(z_j - m) C_ij with C_ij = |row|^2 + |col|^2 - S_ij
+// (S_ij = raw score * sscale), the plan-weighted cost of the row.
 __device__ __forceinline__ void consume64_measure(const uint32_t *ra, const uint32_t *rb, const float *bias,
                                                   const float *cnorm, float c, float sscale, float xn, float &m,
                                                   float &l, float &w) {
