@@ -11,7 +11,9 @@
 // units (-inf on padding columns).  The f-update is then
 //   f_i = |x_i - t|^2 - eps ln2 LSE2_i.
 // The g-update is the same pass with the two sides exchanged (the product is
-// symmetric in q and k: S_ji^T = <k_j, q_i>).
+// symmetric in q and k: S_ji^T = <k_j, q_i>).  For the cosine cost the rows
+// are normalised instead of centred, k = y^ (no factor 2) and every norm term
+// is 1/2, so the same pass computes C_ij = 1 - x^_i.y^_j.
 #pragma once
 
 #include <cstdint>
@@ -43,7 +45,7 @@ struct PassParams {
     int d;                     // feature dim of the plain fp32 layout (SIMT path)
     int splits;                // column splits (grid.y)
     int tiles_per_split;       // column tiles handled by one split
-    int col_tiles;             // column tiles of the pass's tile width covering cols
+    int col_tiles;             // 256-column tiles covering cols
     int stages;                // pipeline depth (tensor-core path)
     float scale2;              // log2(e)/eps, times sscale
     float sscale;              // factor from the MMA's raw score to S_ij (1 unless operands were scaled)

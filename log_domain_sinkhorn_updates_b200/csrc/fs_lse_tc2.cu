@@ -6,15 +6,16 @@
 // M = 256, N = 256).  Each CTA keeps its own 128 rows of Q and loads only half
 // (128 rows) of every 256-column K tile; the pair's first CTA issues the MMA,
 // which reads A and B from both CTAs' shared memory and writes each CTA's
-// 128 x 256 block of S into that CTA's TMEM.  So every K tile crosses the
-// L2 -> SM fabric once per 256 rows instead of once per 128: that halves the
-// pass's dominant data movement (K re-reads), which otherwise limits it below
-// the exp2 throughput.
+// 128 x 256 block of S into that CTA's TMEM.  Each CTA spends only half the
+// shared memory per K tile, which is what lets the rows of 512 bytes (3xTF32 at
+// d = 64, TF32 and 3xF16 at d = 128) that no single-CTA ring can hold run on
+// the tensor cores; FS_CTA_PAIR=1 selects it for every width.
 //
 // Synchronisation of the pair: both CTAs' TMA loads of a slot count on the
-// first CTA's `full` barrier; the MMA's completion is committed to the `empty`
-// and `sfull` barriers of both CTAs at once (multicast commit); both CTAs'
-// softmax groups release a TMEM buffer on the first CTA's `sempty` barrier.
+// first CTA's `full` barrier; the MMA's completion is committed to the `sfull`
+// barriers of both CTAs at once (multicast commit), and each CTA's softmax
+// groups then hand that CTA's K slots back; both CTAs' softmax groups release
+// a TMEM buffer on the first CTA's `sempty` barrier.
 // All waits are bounded as in the single-CTA kernel; both CTAs always reach
 // the final cluster barrier, so neither leaves while the other may still read
 // its shared memory or TMEM.
