@@ -51,7 +51,6 @@ struct fs_handle {
     std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
     int host_err[4] = {0, 0, 0, 0};
     CUtensorMap mapX_r{}, mapX_c{}, mapY_r{}, mapY_c{};  // row-side (128-row box) / column-side (256-row box)
-    CUtensorMap mapX_64{}, mapY_64{};  // 64-row boxes (tensor-core transport application)
     int splits_f = 1, tps_f = 1, splits_g = 1, tps_g = 1;
     int stages = 2, stages_meas = 2;
     bool pair = false;  // run the passes on CTA pairs (one MMA over two SMs); FS_CTA_PAIR=1
@@ -310,11 +309,11 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     // bytes) and dv <= 256; the CUDA-core kernel otherwise or with FS_APPLY_SIMT=1.
     const int dv_pad = (dv + 15) / 16 * 16;
     const int vpl = v_bf16 ? 1 : 2;
-    int kslots = 0, vslots = 0;
+    int kslots = 0, stages = 0;
     const char *force_simt = getenv("FS_APPLY_SIMT");
     const size_t smem = (h->prec != FS_PREC_F32_SIMT && !h->pair && h->row_bytes <= 256 && dv <= 256 &&
                          !(force_simt && atoi(force_simt) != 0))
-                            ? fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &vslots)
+                            ? fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages)
                             : 0;
     if (smem == 0) {
         FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
@@ -325,7 +324,7 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     p.plane_bytes = h->plane_bytes;
     p.dv_pad = dv_pad;
     p.kslots = kslots;
-    p.vslots = vslots;
+    p.stages = stages;
     p.sscale = h->sscale;
     p.timeout_ns = h->timeout_ns;
     p.err = h->err;
@@ -353,7 +352,7 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     }
     if (e == cudaSuccess && st == FS_OK) {
         e = fs::launch_apply_tc(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r,
-                                fdir ? &h->mapY_64 : &h->mapX_64, &map_v, smem, h->stream);
+                                fdir ? &h->mapY_r : &h->mapX_r, &map_v, smem, h->stream);
         g_launches.fetch_add(1, std::memory_order_relaxed);
     }
     cudaFreeAsync(vt, h->stream);
@@ -794,8 +793,6 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, kBlockCols);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_r, h->packY, D.batch * h->m_pad, kBlockRows);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, kBlockCols);
-            if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_64, h->packY, D.batch * h->m_pad, 64);
-            if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_64, h->packX, D.batch * h->n_pad, 64);
             if (s2 != FS_OK) return s2;
         }
         return FS_OK;

@@ -4,27 +4,32 @@
 // section 3: plan-weighted averages over the same streamed tiles, an
 // attention-style "P V" product).
 //
-// One CTA owns 128 rows.  Column tiles of 64 points stream through:
-//   1. S = Q K^T (M = 128, N = 64, the handle's operand precision) into one of
-//      two TMEM buffers;
-//   2. a softmax group forms p~_ij = P_ij / a_i = 2^(alpha'_i + beta_j + S_ij c)
-//      with alpha'_i = (f_i - |x_i|^2) log2(e)/eps and the pass's column bias
+// One CTA owns 128 rows.  Column tiles of 128 points stream through:
+//   1. S = Q K^T (M = 128, N = 128, the handle's operand precision) into one
+//      of two TMEM buffers;
+//   2. the tile's softmax group reads S in two halves of 64 columns.  For each
+//      half it forms p~_ij = P_ij / a_i = 2^(alpha'_i + beta_j + S_ij c) with
+//      alpha'_i = (f_i - |x_i|^2) log2(e)/eps and the pass's column bias
 //      beta_j, adds it to the row sum, splits it into bf16 hi + lo and writes
-//      both planes into shared memory in the 128-byte-swizzled K-major layout
-//      of an MMA operand;
+//      both planes into a shared-memory stage in the 128-byte-swizzled K-major
+//      layout of an MMA operand;
 //   3. O += P~ V~ (M = 128, N = dv rounded up to 16, K = 64) accumulates in
-//      TMEM; V~ is V transposed and packed in bf16 (one plane for bf16 inputs,
-//      hi + lo planes otherwise), so the product is hi.hi + lo.hi (+ hi.lo).
+//      TMEM, one product per half; V~ is V transposed and packed in bf16 (one
+//      plane for bf16 inputs, hi + lo planes otherwise), so the product is
+//      hi.hi + lo.hi (+ hi.lo).
+// A stage holds one half's P~ planes and its V~ planes; it is refilled once
+// the P~ V~ product that read it has completed (one tcgen05.commit frees both).
 // The reference a_i makes every p~ at most about 1 near a solution, so no
 // running maximum or rescaling is needed; bf16 keeps fp32's range, so small
 // entries do not underflow.  At the end out_i = a_i O_i (or O_i / sum_j p~_ij
 // for the barycentric map) and r_i = a_i sum_j p~_ij.
 //
 // Warp roles as in the streamed LSE pass: warp 0 TMA producer, warp 1 TMEM
-// allocator and MMA issuer (the S product of tile t, then the P V product of
-// tile t - 1), warps 2..9 two softmax groups taking the even and the odd
-// tiles.  Every wait is bounded; on expiry the kernel raises kDevErrTimeout,
-// stops, drains its own copies and MMAs, frees TMEM and returns.
+// allocator and MMA issuer (the S product of tile t, then the two P V
+// products of tile t - 1), warps 2..9 two softmax groups taking the even and
+// the odd tiles.  Every wait is bounded; on expiry the kernel raises
+// kDevErrTimeout, stops, drains its own copies and MMAs, frees TMEM and
+// returns.
 #include <cuda_bf16.h>
 
 #include "fs_tc_common.cuh"
@@ -35,29 +40,32 @@ namespace {
 using namespace tc;
 
 constexpr int kAThreads = 320;
-constexpr int kTN = 64;           // columns per tile (N of the S product, K of the P V product)
+constexpr int kTS = 128;          // columns per tile (N of the S product)
+constexpr int kTH = 64;           // columns per half (K of one P V product)
 constexpr int kAMaxKsteps = 64;
-constexpr int kABias = 4;         // bias-slice ring
+constexpr int kABias = 4;         // bias-slice ring (tiles)
 constexpr uint32_t kPBytes = kBlockRows * 128;  // one bf16 plane of P~: 128 rows x 64 values
 
 struct ALayout {
-    uint32_t q, k, v, p, bias, koff, rs, bars, misc, total;
+    uint32_t q, k, st, stage, bias, koff, rs, bars, misc, total;
 };
 
 __host__ __device__ inline int aswz(int row_bytes) { return row_bytes <= 32 ? 32 : (row_bytes <= 64 ? 64 : 128); }
 
-__host__ __device__ inline ALayout a_layout(int row_bytes, int kslots, int dv_pad, int vslots) {
+// Stage = [P~ hi | P~ lo | V~ plane 0 (| V~ plane 1)]; every part is a
+// multiple of 1024 bytes, so each starts on a swizzle-atom boundary.
+__host__ __device__ inline ALayout a_layout(int row_bytes, int kslots, int dv_pad, int vpl, int stages) {
     ALayout L;
     const uint32_t swz = (uint32_t)aswz(row_bytes);
     L.q = 0;
     L.k = L.q + (uint32_t)kBlockRows * row_bytes;
-    L.v = L.k + (uint32_t)kslots * kTN * swz;
-    L.p = L.v + (uint32_t)vslots * dv_pad * 128;
-    L.bias = L.p + 4 * kPBytes;  // [group][hi|lo]
-    L.koff = L.bias + kABias * kTN * 4;
+    L.st = L.k + (uint32_t)kslots * kTS * swz;
+    L.stage = 2 * kPBytes + (uint32_t)vpl * dv_pad * 128;
+    L.bias = L.st + (uint32_t)stages * L.stage;
+    L.koff = L.bias + kABias * kTS * 4;
     L.rs = L.koff + 3 * kAMaxKsteps * 4;
     L.bars = L.rs + kBlockRows * 4;
-    L.misc = L.bars + (2 * kslots + 2 * vslots + 2 * kABias + 10) * 8;
+    L.misc = L.bars + (2 * kslots + 2 * kABias + 3 * stages + 6) * 8;
     L.total = L.misc + 16;
     return L;
 }
@@ -68,40 +76,38 @@ __global__ void __launch_bounds__(kAThreads, 1)
                     const __grid_constant__ CUtensorMap map_v, const ApplyParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
-    const int KS = p.kslots, VS = p.vslots;
+    const int KS = p.kslots, NS = p.stages;
     const uint32_t swz = (uint32_t)p.swz;
     const int atoms = p.row_bytes / p.swz;
     const int box_inner = p.swz / (KIND == 1 ? 4 : 2);
-    const uint32_t kslot_bytes = (uint32_t)kTN * swz;
-    const uint32_t vslot_bytes = (uint32_t)p.dv_pad * 128u;
-    const ALayout L = a_layout(p.row_bytes, KS, p.dv_pad, VS);
+    const uint32_t kslot_bytes = (uint32_t)kTS * swz;
+    const uint32_t vplane_bytes = (uint32_t)p.dv_pad * 128u;
+    const ALayout L = a_layout(p.row_bytes, KS, p.dv_pad, VPL, NS);
 
     uint8_t *sQ = smem + L.q;
     uint8_t *sK = smem + L.k;
-    uint8_t *sV = smem + L.v;
-    uint8_t *sP = smem + L.p;
+    uint8_t *sSt = smem + L.st;
     float *sBias = reinterpret_cast<float *>(smem + L.bias);
     uint32_t *koff = reinterpret_cast<uint32_t *>(smem + L.koff);
     float *sRs = reinterpret_cast<float *>(smem + L.rs);
     uint64_t *kfull = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *kempty = kfull + KS;
-    uint64_t *vfull = kempty + KS;
-    uint64_t *vempty = vfull + VS;
-    uint64_t *bfull = vempty + VS;
+    uint64_t *bfull = kempty + KS;
     uint64_t *bempty = bfull + kABias;
-    uint64_t *qfull = bempty + kABias;
+    uint64_t *pfull = bempty + kABias;  // [NS] P~ of the stage written
+    uint64_t *vfull = pfull + NS;       // [NS] V~ of the stage loaded
+    uint64_t *stfree = vfull + NS;      // [NS] the P V product that read the stage is complete
+    uint64_t *qfull = stfree + NS;
     uint64_t *sfull = qfull + 1;   // [2]
     uint64_t *sempty = sfull + 2;  // [2]
-    uint64_t *pfull = sempty + 2;  // [2]
-    uint64_t *pempty = pfull + 2;  // [2]
-    uint64_t *ofull = pempty + 2;
+    uint64_t *ofull = sempty + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + L.misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rb = blockIdx.x, bz = blockIdx.z;
-    const int ntiles = (p.cols + kTN - 1) / kTN;
-    // S buffers in columns [0, 128), the O accumulator from column 256 (it
+    const int ntiles = (p.cols + kTS - 1) / kTS;
+    // S buffers in columns [0, 256), the O accumulator from column 256 (it
     // never straddles the middle of the allocation).
     const uint32_t tmem_cols = 512u;
 
@@ -110,20 +116,19 @@ __global__ void __launch_bounds__(kAThreads, 1)
             mbar_init(kfull + s, 1);
             mbar_init(kempty + s, 1);
         }
-        for (int s = 0; s < VS; ++s) {
-            mbar_init(vfull + s, 1);
-            mbar_init(vempty + s, 1);
-        }
         for (int j = 0; j < kABias; ++j) {
             mbar_init(bfull + j, 1);
             mbar_init(bempty + j, 4);
+        }
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(pfull + s, 4);
+            mbar_init(vfull + s, 1);
+            mbar_init(stfree + s, 1);
         }
         mbar_init(qfull, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(sfull + b, 1);
             mbar_init(sempty + b, 4);
-            mbar_init(pfull + b, 4);
-            mbar_init(pempty + b, 1);
         }
         mbar_init(ofull, 1);
         *abort_flag = 0;
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
                 tma_load_2d(saddr(sQ) + a * kBlockRows * swz, &map_q, saddr(qfull), a * box_inner,
                             bz * p.rows_pad + rb * kBlockRows);
             for (int t = 0; ok && t < ntiles; ++t) {
-                const int col0 = t * kTN;
+                const int col0 = t * kTS;
                 if (*abort_flag) break;
                 for (int a = 0; a < atoms && ok; ++a) {
                     const int i = t * atoms + a, s = i % KS;
@@ -165,27 +170,29 @@ __global__ void __launch_bounds__(kAThreads, 1)
                     k_issued = i + 1;
                 }
                 if (!ok) break;
-                // the bias slice before the V~ planes: the group that frees the V~
-                // slots this tile's planes wait for needs this tile's bias first
+                // the bias slice before the V~ planes: the group that frees the
+                // stages this tile's planes wait for needs this tile's bias first
                 const int j = t % kABias;
                 if (t >= kABias && !mbar_wait(bempty + j, ((uint32_t)(t / kABias) & 1u) ^ 1u, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
-                mbar_expect_tx(bfull + j, kTN * 4);
-                bulk_load(saddr(sBias + j * kTN), p.col_bias + (size_t)bz * p.cols_stride + col0, kTN * 4,
+                mbar_expect_tx(bfull + j, kTS * 4);
+                bulk_load(saddr(sBias + j * kTS), p.col_bias + (size_t)bz * p.cols_stride + col0, kTS * 4,
                           saddr(bfull + j));
                 b_issued = t + 1;
-                for (int pl = 0; pl < VPL && ok; ++pl) {
-                    const int i = t * VPL + pl, s = i % VS;
-                    if (i >= VS && !mbar_wait(vempty + s, ((uint32_t)(i / VS) & 1u) ^ 1u, p.timeout_ns)) {
+                for (int half = 0; half < 2; ++half) {
+                    const int hh = 2 * t + half, s = hh % NS;
+                    if (hh >= NS && !mbar_wait(stfree + s, ((uint32_t)(hh / NS) & 1u) ^ 1u, p.timeout_ns)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(vfull + s, vslot_bytes);
-                    tma_load_2d(saddr(sV + (size_t)s * vslot_bytes), &map_v, saddr(vfull + s), col0,
-                                (bz * VPL + pl) * p.dv_pad);
-                    v_issued = i + 1;
+                    uint8_t *sv = sSt + (size_t)s * L.stage + 2 * kPBytes;
+                    mbar_expect_tx(vfull + s, (uint32_t)VPL * vplane_bytes);
+                    for (int pl = 0; pl < VPL; ++pl)
+                        tma_load_2d(saddr(sv + pl * vplane_bytes), &map_v, saddr(vfull + s), col0 + half * kTH,
+                                    (bz * VPL + pl) * p.dv_pad);
+                    v_issued = hh + 1;
                 }
             }
             if (!ok) {
@@ -195,8 +202,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
             mbar_wait(qfull, 0, p.timeout_ns);
             for (int i = max(0, k_issued - KS); i < k_issued; ++i)
                 mbar_wait(kfull + (i % KS), (uint32_t)(i / KS) & 1u, p.timeout_ns);
-            for (int i = max(0, v_issued - VS); i < v_issued; ++i)
-                mbar_wait(vfull + (i % VS), (uint32_t)(i / VS) & 1u, p.timeout_ns);
+            for (int i = max(0, v_issued - NS); i < v_issued; ++i)
+                mbar_wait(vfull + (i % NS), (uint32_t)(i / NS) & 1u, p.timeout_ns);
             for (int t = max(0, b_issued - kABias); t < b_issued; ++t)
                 mbar_wait(bfull + (t % kABias), (uint32_t)(t / kABias) & 1u, p.timeout_ns);
         }
@@ -204,7 +211,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            const uint32_t idesc_s = make_idesc<KIND, kBlockRows, kTN>();
+            const uint32_t idesc_s = make_idesc<KIND, kBlockRows, kTS>();
             // P~ V~: bf16 x bf16 -> fp32, M = 128, N = dv_pad
             const uint32_t idesc_o = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.dv_pad >> 3) << 17) |
                                      ((uint32_t)(kBlockRows >> 4) << 24);
@@ -241,7 +248,7 @@ __global__ void __launch_bounds__(kAThreads, 1)
                     }
                     if (!ok || *abort_flag) break;
                     tc_fence_after();
-                    const uint32_t dt = tmem_base + (uint32_t)(b * kTN);
+                    const uint32_t dt = tmem_base + (uint32_t)(b * kTS);
                     for (int i = 0; i < nk; ++i) {
                         const uint32_t ba = koff[kAMaxKsteps + i];
                         const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
@@ -249,31 +256,33 @@ __global__ void __launch_bounds__(kAThreads, 1)
                     }
                     tc_commit(saddr(sfull + b));
                 }
-                if (t >= 1) {  // O += P~(u) V~(u), u = t - 1
-                    const int u = t - 1, bb = u & 1;
-                    if (!mbar_wait(pfull + bb, (uint32_t)(u >> 1) & 1u, p.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    uint64_t vdesc[VPL];
+                if (t >= 1) {  // O += P~ V~ over the two halves of tile t - 1
+                    for (int half = 0; ok && half < 2; ++half) {
+                        const int hh = 2 * (t - 1) + half, s = hh % NS;
+                        const uint32_t ph = (uint32_t)(hh / NS) & 1u;
+                        if (!mbar_wait(pfull + s, ph, p.timeout_ns) || !mbar_wait(vfull + s, ph, p.timeout_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        if (*abort_flag) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t st = saddr(sSt + (size_t)s * L.stage);
+                        const uint64_t phi = make_sdesc(st, 128u);
+                        const uint64_t plo = make_sdesc(st + kPBytes, 128u);
+                        const uint64_t v0 = make_sdesc(st + 2 * kPBytes, 128u);
+                        const uint64_t v1 = make_sdesc(st + 2 * kPBytes + (VPL - 1) * vplane_bytes, 128u);
 #pragma unroll
-                    for (int pl = 0; pl < VPL; ++pl) {
-                        const int i = u * VPL + pl;
-                        if (!mbar_wait(vfull + (i % VS), (uint32_t)(i / VS) & 1u, p.timeout_ns)) ok = false;
-                        vdesc[pl] = make_sdesc(saddr(sV + (size_t)(i % VS) * vslot_bytes), 128u);
+                        for (int ks = 0; ks < kTH / 16; ++ks) {  // 16 values = 32 bytes per K step
+                            const uint32_t acc0 = (hh > 0 || ks > 0) ? 1u : 0u;
+                            tc_mma<0>(tmem_o, phi + 2u * ks, v0 + 2u * ks, idesc_o, acc0);
+                            tc_mma<0>(tmem_o, plo + 2u * ks, v0 + 2u * ks, idesc_o, 1u);
+                            if (VPL == 2) tc_mma<0>(tmem_o, phi + 2u * ks, v1 + 2u * ks, idesc_o, 1u);
+                        }
+                        tc_commit(saddr(stfree + s));
                     }
-                    if (!ok || *abort_flag) break;
-                    tc_fence_after();
-                    const uint64_t phi = make_sdesc(saddr(sP + (2 * bb + 0) * kPBytes), 128u);
-                    const uint64_t plo = make_sdesc(saddr(sP + (2 * bb + 1) * kPBytes), 128u);
-#pragma unroll
-                    for (int ks = 0; ks < kTN / 16; ++ks) {  // 16 values = 32 bytes per K step
-                        const uint32_t acc0 = (u > 0 || ks > 0) ? 1u : 0u;
-                        tc_mma<0>(tmem_o, phi + 2u * ks, vdesc[0] + 2u * ks, idesc_o, acc0);
-                        tc_mma<0>(tmem_o, plo + 2u * ks, vdesc[0] + 2u * ks, idesc_o, 1u);
-                        if (VPL == 2) tc_mma<0>(tmem_o, phi + 2u * ks, vdesc[VPL - 1] + 2u * ks, idesc_o, 1u);
-                    }
-                    tc_commit(saddr(pempty + bb));
                 }
             }
             if (!ok) {
@@ -298,11 +307,11 @@ __global__ void __launch_bounds__(kAThreads, 1)
         const float c = (float)(p.scale * (double)p.sscale);
         const uint64_t cc = pack2(c, c), aa = pack2(alpha, alpha);
         const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
-        uint8_t *prow_hi = sP + (2 * grp + 0) * kPBytes + (rl >> 3) * 1024 + (rl & 7) * 128;
-        uint8_t *prow_lo = sP + (2 * grp + 1) * kPBytes + (rl >> 3) * 1024 + (rl & 7) * 128;
+        // this thread's row in a P~ plane (8-row swizzle atoms of 1024 bytes)
+        const uint32_t prow_off = (uint32_t)((rl >> 3) * 1024 + (rl & 7) * 128);
         float rs = 0.f;
         bool ok = true;
-        for (int t = grp; t < ntiles; t += 2) {
+        for (int t = grp; ok && t < ntiles; t += 2) {
             const int j = t % kABias;
             if (!mbar_wait(sfull + grp, (uint32_t)(t >> 1) & 1u, p.timeout_ns) ||
                 !mbar_wait(bfull + j, (uint32_t)(t / kABias) & 1u, p.timeout_ns)) {
@@ -312,68 +321,73 @@ __global__ void __launch_bounds__(kAThreads, 1)
             tc_fence_after();
             if (q == 2 && lane == 0)  // S(t) is complete: tile t's K slots are free
                 for (int a = 0; a < atoms; ++a) mbar_arrive(kempty + ((t * atoms + a) % KS));
-            uint32_t r[kTN];
-            tmem_ld32(lane_base + (uint32_t)(grp * kTN), &r[0]);
-            tmem_ld32(lane_base + (uint32_t)(grp * kTN + 32), &r[32]);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(sempty + grp);
-            const float4 *bq = reinterpret_cast<const float4 *>(sBias + j * kTN);
-            uint32_t hi[kTN / 2], lo[kTN / 2];
-            uint64_t acc2 = 0ull;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint32_t r[kTH];
+                tmem_ld32(lane_base + (uint32_t)(grp * kTS + half * kTH), &r[0]);
+                tmem_ld32(lane_base + (uint32_t)(grp * kTS + half * kTH + 32), &r[32]);
+                tmem_ld_wait();
+                if (half == 1) {  // both halves read: the S buffer is free
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(sempty + grp);
+                }
+                const float4 *bq = reinterpret_cast<const float4 *>(sBias + j * kTS + half * kTH);
+                uint32_t hi[kTH / 2], lo[kTH / 2];
+                uint64_t acc2 = 0ull;
 #pragma unroll
-            for (int k = 0; k < kTN; k += 4) {
-                const float4 bb = bq[k / 4];
-                float e0, e1, e2, e3;
-                unpack2(add2(fma2(pack2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), cc, pack2(bb.x, bb.y)), aa),
-                        e0, e1);
-                unpack2(add2(fma2(pack2(__uint_as_float(r[k + 2]), __uint_as_float(r[k + 3])), cc, pack2(bb.z, bb.w)),
-                             aa),
-                        e2, e3);
-                e0 = ex2_approx(e0);
-                e1 = ex2_approx(e1);
-                e2 = ex2_approx(e2);
-                e3 = ex2_approx(e3);
-                acc2 = add2(acc2, add2(pack2(e0, e1), pack2(e2, e3)));
-                const __nv_bfloat162 h01 = __floats2bfloat162_rn(e0, e1);
-                const __nv_bfloat162 h23 = __floats2bfloat162_rn(e2, e3);
-                const float2 f01 = __bfloat1622float2(h01);
-                const float2 f23 = __bfloat1622float2(h23);
-                const __nv_bfloat162 l01 = __floats2bfloat162_rn(e0 - f01.x, e1 - f01.y);
-                const __nv_bfloat162 l23 = __floats2bfloat162_rn(e2 - f23.x, e3 - f23.y);
-                hi[k / 2] = *reinterpret_cast<const uint32_t *>(&h01);
-                hi[k / 2 + 1] = *reinterpret_cast<const uint32_t *>(&h23);
-                lo[k / 2] = *reinterpret_cast<const uint32_t *>(&l01);
-                lo[k / 2 + 1] = *reinterpret_cast<const uint32_t *>(&l23);
-            }
-            float s0, s1;
-            unpack2(acc2, s0, s1);
-            rs += s0 + s1;
-            // this group's P~ buffer is free once the P V product of tile t - 2 is complete
-            if (t >= 2) {
-                if (!mbar_wait(pempty + grp, ((uint32_t)(t >> 1) & 1u) ^ 1u, p.timeout_ns)) {
+                for (int k = 0; k < kTH; k += 4) {
+                    const float4 bb = bq[k / 4];
+                    float e0, e1, e2, e3;
+                    unpack2(add2(fma2(pack2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), cc, pack2(bb.x, bb.y)),
+                                 aa),
+                            e0, e1);
+                    unpack2(add2(fma2(pack2(__uint_as_float(r[k + 2]), __uint_as_float(r[k + 3])), cc,
+                                      pack2(bb.z, bb.w)),
+                                 aa),
+                            e2, e3);
+                    e0 = ex2_approx(e0);
+                    e1 = ex2_approx(e1);
+                    e2 = ex2_approx(e2);
+                    e3 = ex2_approx(e3);
+                    acc2 = add2(acc2, add2(pack2(e0, e1), pack2(e2, e3)));
+                    const __nv_bfloat162 h01 = __floats2bfloat162_rn(e0, e1);
+                    const __nv_bfloat162 h23 = __floats2bfloat162_rn(e2, e3);
+                    const float2 f01 = __bfloat1622float2(h01);
+                    const float2 f23 = __bfloat1622float2(h23);
+                    const __nv_bfloat162 l01 = __floats2bfloat162_rn(e0 - f01.x, e1 - f01.y);
+                    const __nv_bfloat162 l23 = __floats2bfloat162_rn(e2 - f23.x, e3 - f23.y);
+                    hi[k / 2] = *reinterpret_cast<const uint32_t *>(&h01);
+                    hi[k / 2 + 1] = *reinterpret_cast<const uint32_t *>(&h23);
+                    lo[k / 2] = *reinterpret_cast<const uint32_t *>(&l01);
+                    lo[k / 2 + 1] = *reinterpret_cast<const uint32_t *>(&l23);
+                }
+                float s0, s1;
+                unpack2(acc2, s0, s1);
+                rs += s0 + s1;
+                // the stage is free once the P V product that last read it is complete
+                const int hh = 2 * t + half, s = hh % NS;
+                if (hh >= NS && !mbar_wait(stfree + s, ((uint32_t)(hh / NS) & 1u) ^ 1u, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
-                if (q == 2 && lane == 0)  // and so are tile t - 2's V~ slots
-                    for (int pl = 0; pl < VPL; ++pl) mbar_arrive(vempty + (((t - 2) * VPL + pl) % VS));
-            }
-            // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+                uint8_t *prow_hi = sSt + (size_t)s * L.stage + prow_off;
+                uint8_t *prow_lo = prow_hi + kPBytes;
+                // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint32_t off = (uint32_t)((ch ^ (rl & 7)) << 4);
-                *reinterpret_cast<uint4 *>(prow_hi + off) =
-                    make_uint4(hi[4 * ch], hi[4 * ch + 1], hi[4 * ch + 2], hi[4 * ch + 3]);
-                *reinterpret_cast<uint4 *>(prow_lo + off) =
-                    make_uint4(lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint32_t off = (uint32_t)((ch ^ (rl & 7)) << 4);
+                    *reinterpret_cast<uint4 *>(prow_hi + off) =
+                        make_uint4(hi[4 * ch], hi[4 * ch + 1], hi[4 * ch + 2], hi[4 * ch + 3]);
+                    *reinterpret_cast<uint4 *>(prow_lo + off) =
+                        make_uint4(lo[4 * ch], lo[4 * ch + 1], lo[4 * ch + 2], lo[4 * ch + 3]);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pfull + s);
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(pfull + grp);
-                mbar_arrive(bempty + j);
-            }
+            if (!ok) break;
+            if (lane == 0) mbar_arrive(bempty + j);
             if (*abort_flag) break;
         }
         if (!ok) {
@@ -460,20 +474,22 @@ cudaError_t launch_kind(const ApplyParams &p, int batch, int vpl, const void *mq
 
 }  // namespace
 
-// Shared memory of the tensor-core transport application and its ring depths;
-// 0 if it does not fit.  At least two tiles of K and of V~ in flight.
-size_t apply_tc_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *vslots) {
+// Shared memory of the tensor-core transport application, its K-ring depth
+// (slots of one operand atom of a 128-column tile) and its stage count (one
+// 64-column half of P~ and V~ each); 0 if it does not fit.  At least two
+// stages; two tiles of K where they fit, one otherwise.
+size_t apply_tc_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages) {
     const size_t limit = 227 * 1024;
     const int atoms = row_bytes / aswz(row_bytes);
-    for (int kt = 4; kt >= 2; --kt)
-        for (int vt = 3; vt >= 2; --vt) {
-            const size_t bytes = (size_t)a_layout(row_bytes, kt * atoms, dv_pad, vt * vpl).total + 1024;
-            if (bytes <= limit) {
-                *kslots = kt * atoms;
-                *vslots = vt * vpl;
-                return bytes < 120 * 1024 ? 120 * 1024 : bytes;  // one CTA per SM (TMEM)
-            }
+    const int plans[3][2] = {{2, 3}, {2, 2}, {1, 2}};  // {K tiles, stages}, best first
+    for (const auto &pl : plans) {
+        const size_t bytes = (size_t)a_layout(row_bytes, pl[0] * atoms, dv_pad, vpl, pl[1]).total + 1024;
+        if (bytes <= limit) {
+            *kslots = pl[0] * atoms;
+            *stages = pl[1];
+            return bytes < 120 * 1024 ? 120 * 1024 : bytes;  // one CTA per SM (TMEM)
         }
+    }
     return 0;
 }
 

@@ -147,7 +147,7 @@ struct ApplyParams {
     float *rsum;                      // [batch][rows] or null
     int divide;                       // 1: out = P V / r (barycentric map)
     // tensor-core path only
-    int row_bytes, swz, plane_bytes, dv_pad, kslots, vslots;
+    int row_bytes, swz, plane_bytes, dv_pad, kslots, stages;
     float sscale;                     // raw MMA score -> S_ij (3xF16 operand scaling)
     unsigned long long timeout_ns;
     int *err;
@@ -164,10 +164,11 @@ size_t tc_smem_bytes(int row_bytes, int qt, int stages, bool measure);
 int tc_max_stages(int row_bytes, int qt, bool measure);
 // Transport application on CUDA cores (fp32): out = P V (or P V / r), rsum = P 1.
 cudaError_t launch_apply_simt(const ApplyParams &p, int batch, cudaStream_t s);
-// Tensor-core transport application (fs_apply_tc.cu): shared memory and ring
-// depths for operand rows of row_bytes, dv_pad output columns and vpl planes
-// of V~ (0 if it does not fit); V~ packing; the launch (prec as the LSE pass).
-size_t apply_tc_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *vslots);
+// Tensor-core transport application (fs_apply_tc.cu): shared memory, K-ring
+// depth and P~/V~ stage count for operand rows of row_bytes, dv_pad output
+// columns and vpl planes of V~ (0 if it does not fit); V~ packing; the launch
+// (prec as the LSE pass).
+size_t apply_tc_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages);
 cudaError_t launch_vt_pack(const void *V, bool bf16, int batch, int m, int dv, int m_pad, int dv_pad, int vpl,
                            void *out, cudaStream_t s);
 cudaError_t launch_apply_tc(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
