@@ -35,6 +35,7 @@ METRIC = "Sinkhorn cost-entries/s (n·m per half-iter) at n=m=65536,d=128; % of 
 UNIT = "cost-entries/s"
 MUFU_EX2_PER_CLK_PER_SM = 16  # special-function-unit exp2 results per clock per SM
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "lse_tc_highdim_ncu.md")
+PROFILE_TRAFFIC_APPLY = os.path.join(ROOT, "profiles", "apply_tc_highdim_ncu.md")
 
 
 def parse_args():
@@ -211,17 +212,17 @@ def gpu_identifier(torch, dev):
         return None
 
 
-def profile_traffic():
+def profile_traffic(profile=PROFILE_TRAFFIC, source="fs_lse_tc.cu"):
     """Per-launch DRAM bytes of the dominant kernel from the committed ncu summary, if the kernel
     source has not changed since the capture (else None)."""
     import hashlib
     try:
-        txt = open(PROFILE_TRAFFIC).read()
+        txt = open(profile).read()
     except OSError:
         return None
     fields = dict(line.split(":", 1) for line in txt.splitlines() if line.startswith(("dram_bytes_per_launch:",
                                                                                        "kernel_source_sha256:")))
-    src = os.path.join(ROOT, "log_domain_sinkhorn_updates_b200", "csrc", "fs_lse_tc.cu")
+    src = os.path.join(ROOT, "log_domain_sinkhorn_updates_b200", "csrc", source)
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
     if fields.get("kernel_source_sha256", "").strip() != sha:
         return None
@@ -315,7 +316,11 @@ def run_transport(args):
             "step": f"fs_barycentric_map at the potentials of fs_solve({args.iters or prob.iters}) (solve untimed)",
             "half_iters_per_step": 0}),
         "roofline": {"bound": "tensor", "achieved": flops / app_s / 1e12, "peak": peak, "unit": "TFLOP/s",
-                     "frac": flops / app_s / 1e12 / peak, "traffic": None, "peak_source": peak_src,
+                     "frac": flops / app_s / 1e12 / peak,
+                     # the committed capture is of the full highdim workload
+                     "traffic": profile_traffic(PROFILE_TRAFFIC_APPLY, "fs_apply_tc.cu")
+                     if (args.workload, args.n, args.m, args.batch) == ("highdim", None, None, None) else None,
+                     "peak_source": peak_src,
                      "kernel": "apply_tc_kernel (S = Q K^T, then O += P~ V~)",
                      "flops_per_launch": flops},
         "cpu_baseline": None, "e2e": None, "clocks": clocks, "gpu_launches": int(launches),

@@ -476,12 +476,14 @@ cudaError_t launch_kind(const ApplyParams &p, int batch, int vpl, const void *mq
 
 // Shared memory of the tensor-core transport application, its K-ring depth
 // (slots of one operand atom of a 128-column tile) and its stage count (one
-// 64-column half of P~ and V~ each); 0 if it does not fit.  At least two
-// stages; two tiles of K where they fit, one otherwise.
+// 64-column half of P~ and V~ each); 0 if it does not fit.  A third stage
+// pays more than a second K tile: with two stages, writing P~ of a half waits
+// for the P V product of the half two back, which is issued only after the
+// S product this group has just read.
 size_t apply_tc_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages) {
     const size_t limit = 227 * 1024;
     const int atoms = row_bytes / aswz(row_bytes);
-    const int plans[3][2] = {{2, 3}, {2, 2}, {1, 2}};  // {K tiles, stages}, best first
+    const int plans[4][2] = {{2, 3}, {1, 3}, {2, 2}, {1, 2}};  // {K tiles, stages}, best first
     for (const auto &pl : plans) {
         const size_t bytes = (size_t)a_layout(row_bytes, pl[0] * atoms, dv_pad, vpl, pl[1]).total + 1024;
         if (bytes <= limit) {
