@@ -116,6 +116,10 @@ typedef struct {
     int cta_pair;           /* 1: each MMA spans a pair of SMs (tcgen05 cta_group::2); chosen for
                                512-byte operand rows, or for every width when the environment
                                variable FS_CTA_PAIR=1 (FS_CTA_PAIR=0 forbids it) */
+    int last_apply_path;    /* kernel of the handle's last transport application (fs_transport_apply
+                               and the calls built on it): 1 tensor cores, 2 CUDA cores (rows over
+                               256 bytes, dv over 256 or a plan that does not fit, the f32_simt
+                               precision, CTA pairs, or FS_APPLY_SIMT=1), 0 none yet */
 } fs_info;
 
 /*

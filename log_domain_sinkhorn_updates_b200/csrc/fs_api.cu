@@ -54,6 +54,7 @@ struct fs_handle {
     int splits_f = 1, tps_f = 1, splits_g = 1, tps_g = 1;
     int stages = 2, stages_meas = 2;
     bool pair = false;  // run the passes on CTA pairs (one MMA over two SMs); FS_CTA_PAIR=1
+    int last_apply = 0;  // kernel of the last transport application: 1 tensor cores, 2 CUDA cores
     size_t smem = 0, smem_meas = 0;
     unsigned long long timeout_ns = 2000000000ull;
     float sscale = 1.f;             // raw MMA score -> S_ij (3xF16 operand scaling)
@@ -316,9 +317,11 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
                             ? fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages)
                             : 0;
     if (smem == 0) {
+        h->last_apply = 2;
         FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
         return FS_OK;
     }
+    h->last_apply = 1;
     p.row_bytes = h->row_bytes;
     p.swz = h->swz;
     p.plane_bytes = h->plane_bytes;
@@ -915,6 +918,7 @@ fs_status fs_get_info(const fs_handle *h, fs_info *info) {
     info->launches_solve_iter = 2;
     info->device_bytes = h->bytes;
     info->cta_pair = (h->prec != FS_PREC_F32_SIMT && h->pair) ? 1 : 0;
+    info->last_apply_path = h->last_apply;
     return FS_OK;
 }
 

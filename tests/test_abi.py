@@ -77,3 +77,24 @@ def test_host_solve_rejects_bad_sizes(L):
     with pytest.raises(binding.FsError):
         binding.fs_solve_host(np.zeros((1, 0, 3), np.float32), np.zeros((1, 4, 3), np.float32), None, None,
                               np.zeros((1, 4), np.float32), 0.1, 3)
+
+
+def _struct_fields(name):
+    """Field names, in order, of the typedef struct `name` in include/flashsinkhorn.h."""
+    txt = open(os.path.join(ROOT, "include", "flashsinkhorn.h")).read()
+    body = re.search(r"typedef struct \{([^{}]*)\}\s*" + name + r"\s*;", txt).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if decl:
+            fields += [v.strip().lstrip("*") for v in decl.split(None, 1)[1].split(",")]
+    return fields
+
+
+@pytest.mark.parametrize("cname,pyname", [("fs_desc", "FsDesc"), ("fs_info", "FsInfo")])
+def test_ctypes_structs_match_header(cname, pyname):
+    """The binding's ctypes mirrors of the C structs list the header's fields in the
+    header's order (a missing or moved field would shift every later one)."""
+    from log_domain_sinkhorn_updates_b200 import binding
+    assert [f for f, _ in getattr(binding, pyname)._fields_] == _struct_fields(cname)

@@ -74,6 +74,21 @@ PATHS = {"tc": "0", "simt": "1"}
 SPLIT = {"tc": 2.0 ** -14, "simt": 0.0}
 
 
+def _assert_path(fs, h, path, dv):
+    """The kernel that ran, as the handle reports it: the CUDA-core one when it is
+    forced; the tensor-core one otherwise whenever dv <= 128, where every operand
+    width of these workloads fits its shared-memory plan; either one at larger dv,
+    where fp32 V takes two bf16 planes and the plan need not fit."""
+    ran = fs.fs_get_info(h)["last_apply_path"]
+    if path == "simt":
+        assert ran == "simt", ran
+    elif dv <= 128:
+        assert ran == "tc", ran
+    else:
+        assert ran in ("tc", "simt"), ran
+    return ran
+
+
 @pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", list(SMALL))
 @pytest.mark.parametrize("dv", [1, 5, 33, 70, 256])
@@ -92,6 +107,7 @@ def test_transport_apply_parity(cuda_device, name, dv, path, monkeypatch):
     fs.fs_transport_apply(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device),
                           torch.from_numpy(V).to(cuda_device), out, r)
     fs.fs_sync(h)
+    ran = _assert_path(fs, h, path, dv)
     out, r = out.cpu().numpy(), r.cpu().numpy()
     for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
         fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
@@ -100,7 +116,7 @@ def test_transport_apply_parity(cuda_device, name, dv, path, monkeypatch):
         rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean") + SPLIT[path]
         err = np.abs(out[k] - oo) / (rel[:, None] * absw)
         rerr = np.abs(r[k] - ro) / (rel * ro)
-        print(f"{path} {name}[{k}] dv={dv} worst err / bound = {err.max():.3f}, row sums {rerr.max():.3f}")
+        print(f"{path} ({ran}) {name}[{k}] dv={dv} worst err / bound = {err.max():.3f}, row sums {rerr.max():.3f}")
         assert err.max() <= 1.0 and rerr.max() <= 1.0
 
 
@@ -203,10 +219,12 @@ def test_transposed_apply_and_grad_y_parity(cuda_device, name, path, monkeypatch
 
 
 @pytest.mark.parametrize("path", list(PATHS))
-@pytest.mark.parametrize("n,m,d", [(1, 1, 3), (1, 300, 5), (300, 1, 5), (129, 65, 2), (257, 200, 33)])
+@pytest.mark.parametrize("n,m,d", [(1, 1, 3), (1, 300, 5), (300, 1, 5), (129, 65, 2), (257, 200, 33), (2, 129, 4),
+                                   (130, 385, 7)])
 def test_transport_apply_edge_shapes(cuda_device, n, m, d, path, monkeypatch):
     """Single points, one-column plans and ragged row/column counts around the
-    128-row blocks and 64-column tiles."""
+    128-row blocks, the 128-column tiles and their 64-column halves (one valid
+    column in the last tile, whole halves of padding)."""
     import torch
     monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
     fs = _fs()
@@ -227,6 +245,7 @@ def test_transport_apply_edge_shapes(cuda_device, n, m, d, path, monkeypatch):
     fs.fs_transport_apply(h, torch.from_numpy(f32[None]).to(cuda_device), torch.from_numpy(g32[None]).to(cuda_device),
                           torch.from_numpy(V[None]).to(cuda_device), out, r)
     fs.fs_sync(h)
+    _assert_path(fs, h, path, 3)
     oo, ro = oracle.transport_apply(Xd, Yd, loga, logb, f32.astype(np.float64), g32.astype(np.float64), eps,
                                     V.astype(np.float64))
     absw, _ = oracle.transport_apply(Xd, Yd, loga, logb, f32.astype(np.float64), g32.astype(np.float64), eps,
