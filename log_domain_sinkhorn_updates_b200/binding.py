@@ -40,12 +40,14 @@ class FsInfo(ctypes.Structure):
                 ("swizzle_bytes", ctypes.c_int), ("stages", ctypes.c_int), ("block_rows", ctypes.c_int),
                 ("block_cols", ctypes.c_int), ("splits_f", ctypes.c_int), ("splits_g", ctypes.c_int),
                 ("launches_update", ctypes.c_int), ("launches_solve_iter", ctypes.c_int),
-                ("device_bytes", ctypes.c_size_t), ("cta_pair", ctypes.c_int), ("last_apply_path", ctypes.c_int)]
+                ("device_bytes", ctypes.c_size_t), ("cta_pair", ctypes.c_int), ("last_apply_path", ctypes.c_int),
+                ("last_solve_graph", ctypes.c_int)]
 
     def as_dict(self):
         d = {k: getattr(self, k) for k, _ in self._fields_}
         d["prec"] = PRECISION_NAMES.get(d["prec"], d["prec"])
         d["last_apply_path"] = {0: None, 1: "tc", 2: "simt"}.get(d["last_apply_path"], d["last_apply_path"])
+        d["last_solve_graph"] = {0: None, 1: "graph", 2: "direct"}.get(d["last_solve_graph"], d["last_solve_graph"])
         return d
 
 

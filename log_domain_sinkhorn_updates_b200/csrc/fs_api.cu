@@ -55,6 +55,14 @@ struct fs_handle {
     int stages = 2, stages_meas = 2;
     bool pair = false;  // run the passes on CTA pairs (one MMA over two SMs); FS_CTA_PAIR=1
     int last_apply = 0;  // kernel of the last transport application: 1 tensor cores, 2 CUDA cores
+    // fs_solve's CUDA graph: captured on a private stream for one (f, g, iters,
+    // schedule), replayed there between two events on the caller's stream
+    cudaStream_t gstream = nullptr;
+    cudaEvent_t gev_in = nullptr, gev_out = nullptr;
+    cudaGraphExec_t gexec = nullptr;
+    const float *gkey_f = nullptr, *gkey_g = nullptr;
+    int gkey_iters = 0, gkey_sched = -1, gkernels = 0;
+    int last_solve_graph = 0;  // 1: the last fs_solve replayed its graph; 2: it launched directly
     size_t smem = 0, smem_meas = 0;
     unsigned long long timeout_ns = 2000000000ull;
     float sscale = 1.f;             // raw MMA score -> S_ij (3xF16 operand scaling)
@@ -66,6 +74,10 @@ namespace {
 
 thread_local std::string g_last_error;
 std::atomic<unsigned long long> g_launches{0};  // kernels this library has launched
+// While this thread captures a graph, launches are counted here instead (they
+// run when the graph is replayed, and are counted then).
+thread_local bool t_capturing = false;
+thread_local int t_captured = 0;
 
 fs_status fail(fs_handle *h, fs_status st, const char *fmt, ...) {
     char buf[512];
@@ -89,10 +101,13 @@ fs_status fail(fs_handle *h, fs_status st, const char *fmt, ...) {
     } while (0)
 
 // FS_CUDA for a call that launches one kernel: also counts the launch.
-#define FS_LAUNCH(h, call)                 \
-    do {                                   \
-        FS_CUDA(h, call);                  \
-        g_launches.fetch_add(1, std::memory_order_relaxed); \
+#define FS_LAUNCH(h, call)                                        \
+    do {                                                          \
+        FS_CUDA(h, call);                                         \
+        if (t_capturing)                                          \
+            ++t_captured;                                         \
+        else                                                      \
+            g_launches.fetch_add(1, std::memory_order_relaxed);   \
     } while (0)
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -363,6 +378,81 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     FS_CUDA(h, e);
     return FS_OK;
 }
+// The launches of fs_solve, in order, on h->stream.
+fs_status enqueue_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule schedule) {
+    if (schedule == FS_SCHED_ALTERNATING) {
+        // One bias launch from the initial g; afterwards every pass's fused
+        // epilogue writes the bias the next pass reads.
+        FS_LAUNCH(h, run_bias(h, g, true));
+        for (int it = 0; it < iters; ++it) {
+            fs::PassParams pf = make_pass(h, true, false);
+            pf.pot_out = f;
+            pf.next_bias = h->bias_row;
+            FS_LAUNCH(h, run_pass(h, pf, true, false));
+            fs::PassParams pg = make_pass(h, false, false);
+            pg.pot_out = g;
+            pg.next_bias = h->bias_col;
+            FS_LAUNCH(h, run_pass(h, pg, false, false));
+        }
+    } else {
+        for (int it = 0; it < iters; ++it) {
+            FS_LAUNCH(h, run_bias(h, g, true));
+            FS_LAUNCH(h, run_bias(h, f, false));
+            fs::PassParams pf = make_pass(h, true, false);
+            pf.pot_out = f;
+            FS_LAUNCH(h, run_pass(h, pf, true, false));
+            fs::PassParams pg = make_pass(h, false, false);
+            pg.pot_out = g;
+            FS_LAUNCH(h, run_pass(h, pg, false, false));
+        }
+    }
+    return FS_OK;
+}
+
+// Capture enqueue_solve into h->gexec on the handle's private stream.  Returns
+// false (with no error left pending and the stream usable) if the capture or
+// the instantiation fails; the caller then launches directly.
+bool capture_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule schedule) {
+    if (h->gexec) {
+        cudaGraphExecDestroy(h->gexec);
+        h->gexec = nullptr;
+    }
+    if (!h->gstream) {
+        if (cudaStreamCreateWithFlags(&h->gstream, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h->gev_in, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h->gev_out, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            return false;
+        }
+    }
+    if (cudaStreamBeginCapture(h->gstream, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    cudaStream_t user = h->stream;
+    h->stream = h->gstream;
+    t_capturing = true;
+    t_captured = 0;
+    const fs_status st = enqueue_solve(h, f, g, iters, schedule);
+    t_capturing = false;
+    h->stream = user;
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ec = cudaStreamEndCapture(h->gstream, &graph);  // always ends the capture
+    bool ok = st == FS_OK && ec == cudaSuccess && graph != nullptr &&
+              cudaGraphInstantiate(&h->gexec, graph, 0) == cudaSuccess;
+    if (graph) cudaGraphDestroy(graph);
+    if (!ok) {
+        cudaGetLastError();
+        h->gexec = nullptr;
+        return false;
+    }
+    h->gkey_f = f;
+    h->gkey_g = g;
+    h->gkey_iters = iters;
+    h->gkey_sched = (int)schedule;
+    h->gkernels = t_captured;
+    return true;
+}
 }  // namespace
 
 extern "C" {
@@ -536,6 +626,11 @@ const char *fs_last_error(const fs_handle *h) { return h ? h->last_error.c_str()
 fs_status fs_destroy(fs_handle *h) {
     if (!h) return FS_OK;
     cudaSetDevice(h->device);
+    // an in-flight replay completes first; these release on completion
+    if (h->gexec) cudaGraphExecDestroy(h->gexec);
+    if (h->gev_in) cudaEventDestroy(h->gev_in);
+    if (h->gev_out) cudaEventDestroy(h->gev_out);
+    if (h->gstream) cudaStreamDestroy(h->gstream);
     if (h->block) cudaFreeAsync(h->block, h->stream);  // stream-ordered: no device-wide sync
     delete h;
     return FS_OK;
@@ -828,33 +923,27 @@ fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule sche
         return fail(h, FS_ERR_INVALID_ARG, "unknown schedule");
     if (iters == 0) return FS_OK;
     FS_CUDA(h, cudaSetDevice(h->device));
-    if (schedule == FS_SCHED_ALTERNATING) {
-        // One bias launch from the initial g; afterwards every pass's fused
-        // epilogue writes the bias the next pass reads.
-        FS_LAUNCH(h, run_bias(h, g, true));
-        for (int it = 0; it < iters; ++it) {
-            fs::PassParams pf = make_pass(h, true, false);
-            pf.pot_out = f;
-            pf.next_bias = h->bias_row;
-            FS_LAUNCH(h, run_pass(h, pf, true, false));
-            fs::PassParams pg = make_pass(h, false, false);
-            pg.pot_out = g;
-            pg.next_bias = h->bias_col;
-            FS_LAUNCH(h, run_pass(h, pg, false, false));
-        }
-    } else {
-        for (int it = 0; it < iters; ++it) {
-            FS_LAUNCH(h, run_bias(h, g, true));
-            FS_LAUNCH(h, run_bias(h, f, false));
-            fs::PassParams pf = make_pass(h, true, false);
-            pf.pot_out = f;
-            FS_LAUNCH(h, run_pass(h, pf, true, false));
-            fs::PassParams pg = make_pass(h, false, false);
-            pg.pot_out = g;
-            FS_LAUNCH(h, run_pass(h, pg, false, false));
-        }
+    // The whole loop as one CUDA graph where launch latency is a visible part
+    // of a pass: batch * n * m up to 2^26 entries (FS_SOLVE_GRAPH=1 forces the
+    // graph at every size, FS_SOLVE_GRAPH=0 forbids it).  It is kept for the
+    // next call with the same buffers, count and schedule.
+    const char *env = getenv("FS_SOLVE_GRAPH");
+    const fs_desc &D = h->desc;
+    const bool want_graph = env && *env ? atoi(env) != 0 : (double)D.batch * D.n * D.m <= 67108864.0;
+    const bool have = h->gexec && h->gkey_f == f && h->gkey_g == g && h->gkey_iters == iters &&
+                      h->gkey_sched == (int)schedule;
+    if (want_graph && (have || capture_solve(h, f, g, iters, schedule))) {
+        FS_CUDA(h, cudaEventRecord(h->gev_in, h->stream));
+        FS_CUDA(h, cudaStreamWaitEvent(h->gstream, h->gev_in, 0));
+        FS_CUDA(h, cudaGraphLaunch(h->gexec, h->gstream));
+        FS_CUDA(h, cudaEventRecord(h->gev_out, h->gstream));
+        FS_CUDA(h, cudaStreamWaitEvent(h->stream, h->gev_out, 0));
+        g_launches.fetch_add((unsigned long long)h->gkernels, std::memory_order_relaxed);
+        h->last_solve_graph = 1;
+        return FS_OK;
     }
-    return FS_OK;
+    h->last_solve_graph = 2;
+    return enqueue_solve(h, f, g, iters, schedule);
 }
 
 fs_status fs_marginal_err(fs_handle *h, const float *f, const float *g, double *err_row, double *err_col) {
@@ -919,6 +1008,7 @@ fs_status fs_get_info(const fs_handle *h, fs_info *info) {
     info->device_bytes = h->bytes;
     info->cta_pair = (h->prec != FS_PREC_F32_SIMT && h->pair) ? 1 : 0;
     info->last_apply_path = h->last_apply;
+    info->last_solve_graph = h->last_solve_graph;
     return FS_OK;
 }
 
