@@ -511,7 +511,14 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     FS_CUDA(h, cudaSetDevice(h->device));
     const size_t n = (size_t)D.n, m = (size_t)D.m, d = (size_t)D.d;
     const bool bf16 = D.dtype == FS_BF16;
-    const int nq = d >= 256 ? 1 : (int)(256 / d);  // columns of y folded into one transport-matrix product
+    // Columns of y folded into one transport-matrix product (width nq d, fp32):
+    // as many as keep the width within 256 and, where the handle's operands
+    // suit the tensor-core application, within its shared-memory plan.
+    int nq = d >= 256 ? 1 : (int)(256 / d);
+    if (h->prec != FS_PREC_F32_SIMT && !h->pair && h->row_bytes <= 256) {
+        int ks = 0, stg = 0;
+        while (nq > 1 && fs::apply_tc_plan(h->row_bytes, (nq * (int)d + 15) / 16 * 16, 2, &ks, &stg) == 0) --nq;
+    }
     // scratch, O((n + m) d), from the pool for this call
     size_t off = 0;
     auto carve = [&](size_t count) {
