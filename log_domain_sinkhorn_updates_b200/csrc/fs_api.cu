@@ -934,9 +934,17 @@ fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule sche
     // of a pass: batch * n * m up to 2^26 entries (FS_SOLVE_GRAPH=1 forces the
     // graph at every size, FS_SOLVE_GRAPH=0 forbids it).  It is kept for the
     // next call with the same buffers, count and schedule.
+    // When the caller is itself capturing the handle's stream, the launches go
+    // straight into the caller's graph.
     const char *env = getenv("FS_SOLVE_GRAPH");
     const fs_desc &D = h->desc;
-    const bool want_graph = env && *env ? atoi(env) != 0 : (double)D.batch * D.n * D.m <= 67108864.0;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(h->stream, &cap) != cudaSuccess) {  // unknown: launch directly
+        cudaGetLastError();
+        cap = cudaStreamCaptureStatusActive;
+    }
+    const bool want_graph = cap == cudaStreamCaptureStatusNone &&
+                            (env && *env ? atoi(env) != 0 : (double)D.batch * D.n * D.m <= 67108864.0);
     const bool have = h->gexec && h->gkey_f == f && h->gkey_g == g && h->gkey_iters == iters &&
                       h->gkey_sched == (int)schedule;
     if (want_graph && (have || capture_solve(h, f, g, iters, schedule))) {

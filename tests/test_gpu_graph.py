@@ -93,3 +93,34 @@ def test_default_uses_the_graph_only_for_small_problems(cuda_device, monkeypatch
         fs.fs_sync(h)
         assert fs.fs_get_info(h)["last_solve_graph"] == want, (name, kw)
         fs.fs_destroy(h)
+
+
+def test_solve_inside_a_caller_graph(cuda_device, monkeypatch):
+    """A caller that captures the handle's stream gets fs_solve's kernels in its own
+    graph (no private graph is captured inside that capture); replaying the caller's
+    graph gives the bits of direct launches."""
+    import torch
+    fs = _fs()
+    monkeypatch.delenv("FS_SOLVE_GRAPH", raising=False)
+    prob = make_problem("tiny")
+    X, Y, a, b = device_inputs(prob)
+    s = torch.cuda.Stream()
+    h = fs.fs_create(X, Y, a, b, eps=prob.eps, stream=s)
+    f = torch.zeros(1, prob.n, device=cuda_device)
+    g = torch.zeros(1, prob.m, device=cuda_device)
+    torch.cuda.synchronize()
+    caller = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(caller, stream=s):
+        fs.fs_solve(h, f, g, 3)
+    assert fs.fs_get_info(h)["last_solve_graph"] == "direct"
+    caller.replay()
+    torch.cuda.synchronize()
+    monkeypatch.setenv("FS_SOLVE_GRAPH", "0")
+    f2 = torch.zeros(1, prob.n, device=cuda_device)
+    g2 = torch.zeros(1, prob.m, device=cuda_device)
+    fs.fs_solve(h, f2, g2, 3)
+    fs.fs_sync(h)
+    assert np.array_equal(f.cpu().numpy(), f2.cpu().numpy())
+    assert np.array_equal(g.cpu().numpy(), g2.cpu().numpy())
+    del caller
+    fs.fs_destroy(h)
