@@ -1,6 +1,6 @@
 """The multi-GPU path of the benchmark on CPU: world_size-2 gloo ranks.
 
-The benchmark spec is one GPU per problem; several GPUs run independent replicas
+Each problem runs on one GPU; several GPUs run independent replicas
 (no data-path collective), so the only cross-rank steps are the barrier and the
 max-over-ranks timing reduction.  Those are exercised here with gloo, together
 with the reference arm's rank-0-only behaviour.
