@@ -141,7 +141,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(prob, iters, {"step": f"oracle f-update of {rows} rows (bounded sample)"}),
+        "config": workload_config(prob, iters, {"step": f"oracle f-update of {rows} rows (bounded sample)",
+                                                "half_iters_per_step": round(rows / prob.n, 6),
+                                                "l2": "not applicable: host CPU oracle"}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{rows} rows x {prob.m} columns per step, d={prob.d}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
