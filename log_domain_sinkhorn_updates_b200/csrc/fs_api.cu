@@ -430,12 +430,14 @@ bool capture_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule sche
         return false;
     }
     cudaStream_t user = h->stream;
+    const std::string saved_error = h->last_error;  // a failed capture is not the caller's error
     h->stream = h->gstream;
     t_capturing = true;
     t_captured = 0;
     const fs_status st = enqueue_solve(h, f, g, iters, schedule);
     t_capturing = false;
     h->stream = user;
+    h->last_error = saved_error;
     cudaGraph_t graph = nullptr;
     const cudaError_t ec = cudaStreamEndCapture(h->gstream, &graph);  // always ends the capture
     bool ok = st == FS_OK && ec == cudaSuccess && graph != nullptr &&
