@@ -98,3 +98,39 @@ def test_ctypes_structs_match_header(cname, pyname):
     header's order (a missing or moved field would shift every later one)."""
     from log_domain_sinkhorn_updates_b200 import binding
     assert [f for f, _ in getattr(binding, pyname)._fields_] == _struct_fields(cname)
+
+
+def test_every_entry_point_rejects_a_null_handle_on_host(L):
+    """Every call that takes a handle answers FS_ERR_INVALID_ARG for a null handle (or
+    null required pointers) before any device work; the allocation-free update checks
+    its sizes and limits on the host too."""
+    from log_domain_sinkhorn_updates_b200.binding import FS_ERR_INVALID_ARG, FsInfo
+    p = ctypes.c_void_p(16)
+    d = ctypes.c_double()
+    info = FsInfo()
+    i = ctypes.c_int()
+    calls = {
+        "fs_update_g": (None, p, p),
+        "fs_marginal_err": (None, p, p, ctypes.byref(d), ctypes.byref(d)),
+        "fs_ot_cost": (None, p, p, ctypes.byref(d), ctypes.byref(d)),
+        "fs_sync": (None,),
+        "fs_get_info": (None, ctypes.byref(info)),
+        "fs_transport_apply": (None, p, p, p, 3, p, p),
+        "fs_transport_apply_t": (None, p, p, p, 3, p, p),
+        "fs_barycentric_map": (None, p, p, p, p),
+        "fs_grad_x": (None, p, p, p, p, p),
+        "fs_grad_y": (None, p, p, p, p, p),
+        "fs_selftest_wait": (None, 50),
+    }
+    for name, args in calls.items():
+        assert getattr(L, name)(*args) == FS_ERR_INVALID_ARG, name
+    # a private ctypes view of the library, so these argtypes leave the binding's alone
+    from log_domain_sinkhorn_updates_b200 import binding
+    L2 = ctypes.CDLL(binding.LIB_PATH)
+    L2.fs_hvp_x.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int, ctypes.c_double, ctypes.c_void_p]
+    assert L2.fs_hvp_x(None, p, p, p, p, p, p, 10, 1e-6, ctypes.byref(i)) == FS_ERR_INVALID_ARG
+    L2.fs_update_f_noalloc.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float] + \
+        [ctypes.c_void_p] * 6
+    for n, m, dd, eps in [(0, 5, 3, 0.1), (5, 5, 0, 0.1), (5, 5, 3, 0.0), (5, 5, 257, 0.1), (1 << 20, 5, 3, 0.1)]:
+        assert L2.fs_update_f_noalloc(n, m, dd, eps, p, p, None, p, p, None) == FS_ERR_INVALID_ARG, (n, m, dd, eps)
+    assert L2.fs_update_f_noalloc(5, 5, 3, 0.1, None, p, None, p, p, None) == FS_ERR_INVALID_ARG
