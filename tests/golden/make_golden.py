@@ -8,7 +8,7 @@ Every number is a plain double-precision oracle result (see
 "FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 1, for the updates).
 
 Usage:  python tests/golden/make_golden.py [workload ...]
-Long: the 65536 x 65536, d=128 solve takes hours on an 8-core host.
+Long: the 65536 x 65536, d=128 solve took 5 hours on 6 host threads.
 """
 import json
 import os
