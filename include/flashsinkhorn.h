@@ -155,13 +155,14 @@ FS_API fs_status fs_update_g(fs_handle *h, const float *f, float *g);
  * read (the first half-step overwrites it), so only g is an initial value.
  * SYMMETRIC: (f, g) <- (update_f(g), update_g(f)) from the previous pair;
  * both are initial values.  iters = 0 is a no-op.  Asynchronous.
- * For small problems (batch * n * m up to 2^26), where launch latency is a
- * visible part of a pass, the loop is captured once as a CUDA graph on a
+ * For small problems (batch * n * m up to 2^26, iters up to 1024), where launch
+ * latency is a visible part of a pass, the loop is captured once as a CUDA graph on a
  * stream private to the handle and replayed there, ordered after the work
  * already on the handle's stream and before what follows it (events on both
  * streams).  The graph is kept for the next call with the same f, g, iters
  * and schedule.  FS_SOLVE_GRAPH=1 in the environment uses the graph at every
- * size, FS_SOLVE_GRAPH=0 never.  Results are identical either way.
+ * problem size (still up to 1024 iterations), FS_SOLVE_GRAPH=0 never.  Results
+ * are identical either way.
  */
 FS_API fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule schedule);
 

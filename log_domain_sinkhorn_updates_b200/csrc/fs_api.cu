@@ -945,7 +945,9 @@ fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule sche
         cudaGetLastError();
         cap = cudaStreamCaptureStatusActive;
     }
-    const bool want_graph = cap == cudaStreamCaptureStatusNone &&
+    // A loop of more than 1024 iterations launches directly: its graph would take
+    // seconds to capture and hold millions of nodes.
+    const bool want_graph = cap == cudaStreamCaptureStatusNone && iters <= 1024 &&
                             (env && *env ? atoi(env) != 0 : (double)D.batch * D.n * D.m <= 67108864.0);
     const bool have = h->gexec && h->gkey_f == f && h->gkey_g == g && h->gkey_iters == iters &&
                       h->gkey_sched == (int)schedule;
