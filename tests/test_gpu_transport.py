@@ -255,3 +255,39 @@ def test_transport_apply_edge_shapes(cuda_device, n, m, d, path, monkeypatch):
     err = (np.abs(out.cpu().numpy()[0] - oo) / (rel[:, None] * absw)).max()
     rerr = (np.abs(r.cpu().numpy()[0] - ro) / (rel * ro)).max()
     assert err <= 1.0 and rerr <= 1.0, (err, rerr)
+
+
+@pytest.mark.parametrize("name,prec", [("tiny", "3xtf32"), ("cloud3d", "3xtf32"), ("batched", "3xtf32")])
+def test_transport_apply_tf32_kind(cuda_device, name, prec):
+    """The tensor-core application with the S product on the tf32 tensor-core kind
+    (3xTF32 split operands; the default for these fp32 workloads is 3xF16 on the
+    f16 kind), 64- and 128-byte swizzled rows.  The split leaves a score error of
+    about 2^-21 relative per product, 2 d 2^-21 max|q| max|k| in all, which adds
+    to the exponent of every plan entry on top of the bound used above."""
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps, prec=prec)
+    f32, g32 = _potentials(prob, "sqeuclidean")
+    rng = np.random.default_rng(7)
+    V = rng.standard_normal((prob.batch, prob.m, 5)).astype(np.float32)
+    out = torch.empty(prob.batch, prob.n, 5, device=cuda_device)
+    fs.fs_transport_apply(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device),
+                          torch.from_numpy(V).to(cuda_device), out, None)
+    fs.fs_sync(h)
+    assert fs.fs_get_info(h)["last_apply_path"] == "tc"
+    out = out.cpu().numpy()
+    u = 2.0 ** -21
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
+        oo, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, V[k].astype(np.float64))
+        absw, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(V[k]).astype(np.float64))
+        t = 0.5 * (Xo.mean(axis=0) + Yo.mean(axis=0))
+        xs, ys = Xo - t, Yo - t
+        # score error of the operand rounding, in the exponent (natural log units)
+        ds = 2 * prob.d * u * np.abs(xs).max() * np.abs(ys).max() * 2 / prob.eps
+        rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean") + SPLIT["tc"] + 2 * ds
+        err = (np.abs(out[k] - oo) / (rel[:, None] * absw)).max()
+        print(f"{prec} {name}[{k}] worst err / bound = {err:.3f}")
+        assert err <= 1.0
