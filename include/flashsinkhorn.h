@@ -126,6 +126,10 @@ typedef struct {
 } fs_info;
 
 /*
+ * Source: "FlashSinkhorn: IO-aware EOT on GPU", Enunciato del Problema (the
+ * problem's data: clouds X (n x d) and Y (m x d), weights a and b, eps) and
+ * Metodologia section 1 (the squared norms and log-weight biases that
+ * Proposition 1 precomputes, done here once per handle).
  * Create a solver for one (batched) problem: X and Y (device, dtype, row-major
  * [batch][n|m][d]), weights a (device [batch][n]) and b (device [batch][m]),
  * NULL meaning uniform 1/n (1/m).  Weights must be positive and sum to 1
@@ -142,14 +146,25 @@ typedef struct {
 FS_API fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const float *a,
                     const float *b, void *stream, fs_handle **out);
 
-/* One f-update (device g [batch][m] -> device f [batch][n]).  Asynchronous.
+/* Source: "FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 1,
+ * Proposition 1 (the f-update as a row LSE of the biased score matrix) and
+ * section 2 (one fused streaming pass).
+ * One f-update (device g [batch][m] -> device f [batch][n]).  Asynchronous.
  * f and g must not overlap.  Non-finite results are flagged for fs_sync. */
 FS_API fs_status fs_update_f(fs_handle *h, const float *g, float *f);
 
-/* One g-update (device f [batch][n] -> device g [batch][m]).  Asynchronous. */
+/* Source: the same page and sections; the g-update is the transposed pass
+ * (the column LSE, the page prints only the f-update and the roles of X and
+ * Y are symmetric).
+ * One g-update (device f [batch][n] -> device g [batch][m]).  Asynchronous. */
 FS_API fs_status fs_update_g(fs_handle *h, const float *f, float *g);
 
 /*
+ * Source: "FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 1 (the
+ * alternating log-domain iterations; the algorithm itself is unchanged, only
+ * its evaluation; "Significato e Affermazioni").  The page does not fix the schedule; the
+ * alternating (Gauss-Seidel) order is the plain reading, the symmetric
+ * (Jacobi) order is offered beside it.
  * `iters` Sinkhorn iterations in place (device f, g).  ALTERNATING: each
  * iteration is f <- update_f(g) then g <- update_g(f); the incoming f is not
  * read (the first half-step overwrites it), so only g is an initial value.
@@ -167,6 +182,10 @@ FS_API fs_status fs_update_g(fs_handle *h, const float *f, float *g);
 FS_API fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule schedule);
 
 /*
+ * Source: not printed on the pages.  The convergence measure of the marginal
+ * constraints that the entropic plan must meet (Enunciato del Problema: the
+ * plan couples a and b); read as the L1 errors of the plan's row and column
+ * sums at the given potentials.
  * Marginal errors of the plan P_ij = a_i b_j exp((f_i + g_j - C_ij)/eps) at
  * device potentials (f, g): err_row[k] = sum_i |r_i - a_i|, err_col[k] =
  * sum_j |c_j - b_j| for each problem k (host arrays [batch]; either may be
@@ -177,6 +196,9 @@ FS_API fs_status fs_marginal_err(fs_handle *h, const float *f, const float *g, d
                           double *err_col);
 
 /*
+ * Source: not printed on the pages beyond "the EOT cost" (Enunciato del
+ * Problema).  Read as the textbook entropic dual objective, with the
+ * transport cost <P, C> of the plan beside it; they coincide at convergence.
  * Objectives at device potentials (f, g), host arrays [batch] (either may be
  * NULL):  dual[k]   = <a,f> + <b,g> - eps (sum_ij P_ij - 1)
  *         primal[k] = <P, C>  (transport cost of the plan)
@@ -185,14 +207,16 @@ FS_API fs_status fs_marginal_err(fs_handle *h, const float *f, const float *g, d
 FS_API fs_status fs_ot_cost(fs_handle *h, const float *f, const float *g, double *dual,
                      double *primal);
 
-/* Wait for the handle's stream and report device-side flags raised since the
+/* Source: no counterpart on the pages (error reporting of the bounded waits).
+ * Wait for the handle's stream and report device-side flags raised since the
  * last check (FS_ERR_NONFINITE, FS_ERR_TIMEOUT). */
 FS_API fs_status fs_sync(fs_handle *h);
 
-/* Resolved configuration of the handle. */
+/* Source: no counterpart on the pages.  Resolved configuration of the handle. */
 FS_API fs_status fs_get_info(const fs_handle *h, fs_info *info);
 
-/* Free the handle.  Its device memory is released in stream order on the
+/* Source: no counterpart on the pages (handle lifetime).
+ * Free the handle.  Its device memory is released in stream order on the
  * handle's stream (no host wait), so the stream must still exist; work
  * already enqueued that uses the handle completes first.  NULL is accepted. */
 FS_API fs_status fs_destroy(fs_handle *h);
@@ -259,21 +283,26 @@ FS_API fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const v
 FS_API fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
                           const float *V, float *out, int max_cg_iters, double cg_rtol, int *cg_iters_done);
 
-/* Failure-path self test: launches on the handle's stream a kernel whose one
+/* Source: no counterpart on the pages.
+ * Failure-path self test: launches on the handle's stream a kernel whose one
  * bounded wait (the same wait every pass uses) can never complete, and waits
  * for it.  Returns FS_ERR_TIMEOUT after about timeout_ms; the handle and the
  * CUDA context stay usable.  FS_ERR_INVALID_ARG for timeout_ms < 1. */
 FS_API fs_status fs_selftest_wait(fs_handle *h, int timeout_ms);
 
-/* Number of CUDA kernels this library has launched in this process so far
+/* Source: no counterpart on the pages.
+ * Number of CUDA kernels this library has launched in this process so far
  * (all handles, all threads).  Host-side counter; never synchronises. */
 FS_API unsigned long long fs_kernel_launches(void);
 
-/* Last error message of the handle; NULL handle -> the last error of any
+/* Source: no counterpart on the pages.
+ * Last error message of the handle; NULL handle -> the last error of any
  * call on this thread that had no handle to record it in. */
 FS_API const char *fs_last_error(const fs_handle *h);
 
 /*
+ * Source: the calls above in sequence (fs_create, fs_solve, fs_marginal_err,
+ * fs_ot_cost), with the host copies around them; no counterpart of its own.
  * One-call end-to-end solve from HOST arrays: copies X, Y (dtype), a, b
  * (NULL = uniform) and the initial g to the current device, creates a
  * handle, runs `iters` iterations, copies f and g back, and evaluates the
@@ -288,22 +317,31 @@ FS_API fs_status fs_solve_host(const fs_desc *desc, const void *X_host, const vo
                         double *err_col, double *dual, double *primal, void *stream);
 
 /*
- * One f-update that allocates nothing (no counterpart on the pages: an
- * interface for callers that cannot allocate device memory when they need
- * an update -- inside CUDA graph capture, in plug-ins whose host framework
- * owns all device memory, or in latency-critical loops).
+ * One f-update that allocates nothing.  No counterpart on the pages: it is an
+ * interface for callers that cannot allocate device memory when they need an
+ * update -- plug-ins whose host framework owns all device memory and forbids
+ * allocations by third-party code, services that reserve a fixed memory
+ * budget up front, and latency-critical loops where an allocation (and the
+ * synchronisation it can imply) is not acceptable.  fs_create allocates and
+ * synchronises, so the handle API cannot serve them.
  * Inputs: device X [n][d], Y [m][d] (fp32, row-major), b [m] (NULL = uniform
  * 1/m), g [m]; output: device f [n], with
  *   f_i = |x_i|^2 - eps LSE_j[(2 x_i.y_j + g_j - |y_j|^2)/eps + log b_j].
- * Computed in plain fp32 on CUDA cores on the uncentred inputs, enqueued on
+ * Computed in plain fp32 on CUDA cores on inputs shifted by the common centre
+ * t = (mean X + mean Y)/2 (the cost is translation-invariant, and the shift
+ * keeps the arithmetic accurate for clouds far from the origin); enqueued on
  * `stream` (a cudaStream_t, NULL = legacy default); returns without waiting.
- * Scratch (squared norms and the column bias) is a fixed 4 MiB device array
- * inside the library, held by every GPU that loads it until the process
- * exits, so: n_pad + m + m_pad <= 1048576 (n_pad, m_pad = n, m rounded up to
- * 128) and d <= 256, else FS_ERR_INVALID_ARG; all calls on a device share the
- * array, so calls that overlap on the GPU race -- order them on one stream.
- * The first call on each device looks up the array's address and sets a
- * kernel attribute: make it before any stream capture.  Errors: return
+ * Scratch (the centring sums, the squared norms and the column bias) is a
+ * fixed 4 MiB device array inside the library, held by every GPU that loads
+ * it until the process exits, so: d <= 256 and n_pad + m + m_pad <= 982784
+ * (n_pad, m_pad = n, m rounded up to 128), else FS_ERR_INVALID_ARG.  All calls
+ * on a device share the array and it keeps the last call's contents (each call
+ * writes everything it reads), so calls that overlap on the GPU race -- order
+ * them on one stream.  The first call on each device, with that device
+ * current, looks up the array's device address and sets a kernel attribute:
+ * make it before any stream capture begins.  The address is kept per device
+ * for the life of the process; after cudaDeviceReset it is stale, so do not
+ * call this entry point on a device that has been reset.  Errors: return
  * codes, message in fs_last_error(NULL).
  */
 FS_API fs_status fs_update_f_noalloc(int n, int m, int d, float eps, const float *X, const float *Y,
