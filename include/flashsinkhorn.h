@@ -123,6 +123,10 @@ typedef struct {
     int last_solve_graph;   /* how the handle's last fs_solve ran: 1 as a replay of its CUDA graph,
                                2 as direct launches (a large problem, FS_SOLVE_GRAPH=0, or a
                                failed capture), 0 none yet */
+    int last_measure_fused; /* 1: the handle's last fs_marginal_err / fs_ot_cost reused the statistics
+                               the last alternating fs_solve reduced in its final pass (f and g were
+                               that solve's output, unchanged bit for bit); 0: it streamed its own
+                               measure passes */
 } fs_info;
 
 /*

@@ -48,6 +48,19 @@ struct fs_handle {
     unsigned *counters = nullptr;
     double *stats = nullptr, *red = nullptr, *wstat = nullptr;
     int *err = nullptr;
+    // The solve's tail: the last alternating fs_solve leaves the column-marginal
+    // statistics of its final g-pass in tail_stats and copies of its output
+    // potentials in snap_f / snap_g.  fs_marginal_err and fs_ot_cost reuse them
+    // (and one f-direction measure pass between them) while f and g still equal
+    // the copies bit for bit.
+    double *tail_stats = nullptr;
+    float *snap_f = nullptr, *snap_g = nullptr;
+    int *cmp = nullptr;
+    bool tail_ok = false;
+    const float *tail_f = nullptr, *tail_g = nullptr;
+    bool meas_ok = false;            // meas_cache holds the f-direction measure at the snapshot
+    std::vector<double> meas_cache;  // [batch][8] as in h->red
+    int last_measure_fused = 0;
     std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
     int host_err[4] = {0, 0, 0, 0};
     CUtensorMap mapX_r{}, mapX_c{}, mapY_r{}, mapY_c{};  // row-side (128-row box) / column-side (256-row box)
@@ -286,6 +299,26 @@ fs_status measure(fs_handle *h, const float *f, const float *g, bool fdir, int s
 void fs::set_thread_error(const char *msg) { g_last_error = msg; }
 
 namespace {
+// Whether (f, g) are still the last alternating solve's output, bit for bit
+// (the caller may have written them since): *same receives the answer.
+// Synchronises the stream.
+fs_status tail_matches(fs_handle *h, const float *f, const float *g, bool *same) {
+    *same = false;
+    if (!h->tail_ok || f != h->tail_f || g != h->tail_g) return FS_OK;
+    const fs_desc &D = h->desc;
+    int host = 1;
+    FS_CUDA(h, cudaMemsetAsync(h->cmp, 0, sizeof(int), h->stream));
+    FS_LAUNCH(h, fs::launch_differs(f, h->snap_f, (size_t)D.batch * D.n, h->cmp, h->stream));
+    FS_LAUNCH(h, fs::launch_differs(g, h->snap_g, (size_t)D.batch * D.m, h->cmp, h->stream));
+    FS_CUDA(h, cudaMemcpyAsync(&host, h->cmp, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
+    FS_CUDA(h, cudaStreamSynchronize(h->stream));
+    *same = host == 0;
+    return FS_OK;
+}
+}  // namespace
+void fs::count_launches(unsigned count) { g_launches.fetch_add(count, std::memory_order_relaxed); }
+
+namespace {
 // fdir: out_i = sum_j P_ij V_j over the X side's rows (V indexed by Y's points);
 // otherwise the transposed application out_j = sum_i P_ij V_i over Y's rows.
 fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, bool v_bf16, int dv, float *out,
@@ -392,7 +425,14 @@ fs_status enqueue_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule
             fs::PassParams pg = make_pass(h, false, false);
             pg.pot_out = g;
             pg.next_bias = h->bias_col;
+            // the final g-pass also reduces the column marginal of the pair it leaves
+            if (it == iters - 1) pg.tail_stats = h->tail_stats;
             FS_LAUNCH(h, run_pass(h, pg, false, false));
+        }
+        if (iters > 0) {
+            const fs_desc &D = h->desc;
+            FS_CUDA(h, cudaMemcpyAsync(h->snap_f, f, (size_t)D.batch * D.n * 4, cudaMemcpyDeviceToDevice, h->stream));
+            FS_CUDA(h, cudaMemcpyAsync(h->snap_g, g, (size_t)D.batch * D.m * 4, cudaMemcpyDeviceToDevice, h->stream));
         }
     } else {
         for (int it = 0; it < iters; ++it) {
@@ -804,6 +844,9 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     const size_t o_red = carve(2 * B * 8 * 8);
     const size_t o_wstat = carve(2 * B * 2 * 8 + 16);
     const size_t o_err = carve(16);
+    const size_t o_tail = carve(B * max_rb * 4 * 8);
+    const size_t o_snapf = carve(B * D.n * 4), o_snapg = carve(B * D.m * 4);
+    const size_t o_cmp = carve(16);
     h->bytes = off;
     {
         cudaMemPool_t pool = nullptr;
@@ -835,6 +878,10 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     h->red = reinterpret_cast<double *>(base + o_red);
     h->wstat = reinterpret_cast<double *>(base + o_wstat);
     h->err = reinterpret_cast<int *>(base + o_err);
+    h->tail_stats = reinterpret_cast<double *>(base + o_tail);
+    h->snap_f = reinterpret_cast<float *>(base + o_snapf);
+    h->snap_g = reinterpret_cast<float *>(base + o_snapg);
+    h->cmp = reinterpret_cast<int *>(base + o_cmp);
 
     // ---- set-up kernels ----
     fs_status st = FS_OK;
@@ -931,6 +978,8 @@ fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule sche
     if (schedule != FS_SCHED_ALTERNATING && schedule != FS_SCHED_SYMMETRIC)
         return fail(h, FS_ERR_INVALID_ARG, "unknown schedule");
     if (iters == 0) return FS_OK;
+    h->tail_ok = false;
+    h->meas_ok = false;
     FS_CUDA(h, cudaSetDevice(h->device));
     // The whole loop as one CUDA graph where launch latency is a visible part
     // of a pass: batch * n * m up to 2^26 entries (FS_SOLVE_GRAPH=1 forces the
@@ -959,31 +1008,56 @@ fs_status fs_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule sche
         FS_CUDA(h, cudaStreamWaitEvent(h->stream, h->gev_out, 0));
         g_launches.fetch_add((unsigned long long)h->gkernels, std::memory_order_relaxed);
         h->last_solve_graph = 1;
-        return FS_OK;
+    } else {
+        h->last_solve_graph = 2;
+        const fs_status st = enqueue_solve(h, f, g, iters, schedule);
+        if (st != FS_OK) {
+            h->tail_ok = false;
+            return st;
+        }
     }
-    h->last_solve_graph = 2;
-    return enqueue_solve(h, f, g, iters, schedule);
+    h->tail_ok = schedule == FS_SCHED_ALTERNATING;
+    h->tail_f = f;
+    h->tail_g = g;
+    h->meas_ok = false;
+    return FS_OK;
 }
 
 fs_status fs_marginal_err(fs_handle *h, const float *f, const float *g, double *err_row, double *err_col) {
     if (!h || !f || !g) return fail(h, FS_ERR_INVALID_ARG, "null argument");
     FS_CUDA(h, cudaSetDevice(h->device));
     const size_t B = (size_t)h->desc.batch;
-    if (err_row) {
-        fs_status s = measure(h, f, g, true, 0, false);
+    bool fused = false;
+    fs_status s = tail_matches(h, f, g, &fused);
+    if (s != FS_OK) return s;
+    // fs_ot_cost may have measured this very pair since the solve
+    const bool row_cached = err_row && fused && h->meas_ok;
+    if (err_row && !row_cached) {
+        // with the column sums too, so that fs_ot_cost at the same pair can reuse it
+        s = measure(h, f, g, true, 0, true);
         if (s != FS_OK) return s;
     }
     if (err_col) {
-        fs_status s = measure(h, f, g, false, 1, false);
-        if (s != FS_OK) return s;
+        if (fused)  // the solve's final g-pass reduced the column marginal already
+            FS_LAUNCH(h, fs::launch_finalize(h->tail_stats, h->desc.batch, h->m_pad / kBlockRows, nullptr, h->lb2,
+                                           h->desc.m, h->m_stride, h->red + B * 8, h->stream));
+        else {
+            s = measure(h, f, g, false, 1, false);
+            if (s != FS_OK) return s;
+        }
     }
     FS_CUDA(h, cudaMemcpyAsync(h->host_red.data(), h->red, 2 * B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
-    fs_status s = check_flags(h);
+    s = check_flags(h);
     if (s != FS_OK) return s;
     for (size_t k = 0; k < B; ++k) {
-        if (err_row) err_row[k] = h->host_red[k * 8 + 0];
+        if (err_row) err_row[k] = row_cached ? h->meas_cache[k * 8 + 0] : h->host_red[k * 8 + 0];
         if (err_col) err_col[k] = h->host_red[(B + k) * 8 + 0];
     }
+    if (fused && err_row && !row_cached) {
+        h->meas_cache.assign(h->host_red.begin(), h->host_red.begin() + B * 8);
+        h->meas_ok = true;
+    }
+    h->last_measure_fused = fused ? 1 : 0;
     return FS_OK;
 }
 
@@ -991,17 +1065,31 @@ fs_status fs_ot_cost(fs_handle *h, const float *f, const float *g, double *dual,
     if (!h || !f || !g) return fail(h, FS_ERR_INVALID_ARG, "null argument");
     FS_CUDA(h, cudaSetDevice(h->device));
     const size_t B = (size_t)h->desc.batch;
-    fs_status s = measure(h, f, g, true, 0, true);
+    bool fused = false;
+    fs_status s = tail_matches(h, f, g, &fused);
     if (s != FS_OK) return s;
-    FS_CUDA(h, cudaMemcpyAsync(h->host_red.data(), h->red, B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
-    s = check_flags(h);
-    if (s != FS_OK) return s;
+    const double *res = nullptr;
+    if (fused && h->meas_ok) {  // fs_marginal_err measured this very pair since the solve
+        res = h->meas_cache.data();
+    } else {
+        s = measure(h, f, g, true, 0, true);
+        if (s != FS_OK) return s;
+        FS_CUDA(h, cudaMemcpyAsync(h->host_red.data(), h->red, B * 8 * 8, cudaMemcpyDeviceToHost, h->stream));
+        s = check_flags(h);
+        if (s != FS_OK) return s;
+        res = h->host_red.data();
+        if (fused) {
+            h->meas_cache.assign(res, res + B * 8);
+            h->meas_ok = true;
+        }
+    }
     const double eps = (double)h->desc.eps;
     for (size_t k = 0; k < B; ++k) {
-        const double *r = h->host_red.data() + k * 8;  // [|r-a|, sum r, sum r*meanC, <a,f>, <b,g>]
+        const double *r = res + k * 8;  // [|r-a|, sum r, sum r*meanC, <a,f>, <b,g>]
         if (dual) dual[k] = r[3] + r[4] - eps * (r[1] - 1.0);
         if (primal) primal[k] = r[2];
     }
+    h->last_measure_fused = fused ? 1 : 0;
     return FS_OK;
 }
 
@@ -1028,6 +1116,7 @@ fs_status fs_get_info(const fs_handle *h, fs_info *info) {
     info->cta_pair = (h->prec != FS_PREC_F32_SIMT && h->pair) ? 1 : 0;
     info->last_apply_path = h->last_apply;
     info->last_solve_graph = h->last_solve_graph;
+    info->last_measure_fused = h->last_measure_fused;
     return FS_OK;
 }
 

@@ -51,6 +51,7 @@ __device__ void finish_rows(const PassParams &p, int rb, int rl, float m, float 
     const bool valid = row < p.rows;
     const double lse2 = (l > 0.f) ? (double)m + log2((double)l) : -INFINITY;
 
+    double c0 = 0.0, c1 = 0.0, c2 = 0.0, c3 = 0.0;
     if (!MEASURE) {
         if (valid) {
             const double pot = (double)p.row_norm[prow] - p.eps * kLn2d * lse2;
@@ -63,16 +64,23 @@ __device__ void finish_rows(const PassParams &p, int rb, int rl, float m, float 
             if (p.next_bias)
                 p.next_bias[prow] =
                     (float)__fma_rn((double)pot32 - (double)p.row_norm[prow], kLog2ed / p.eps, (double)p.row_logw2[prow]);
+            if (p.tail_stats) {
+                // The plan's row sum at the stored potential: the exact update is
+                // pot, the stored value pot32, so r_i = a_i exp((pot32 - pot)/eps)
+                // (what a measure pass at the same potentials computes).
+                const double a = exp2((double)p.row_logw2[prow]);
+                const double r = a * exp2(((double)pot32 - pot) * (kLog2ed / p.eps));
+                c0 = fabs(r - a);
+                c1 = r;
+                c3 = a * (double)pot32;
+            }
         }
-        return;
-    }
-
-    // Measure mode: with the current row potential pot_in, the plan's row sum is
-    //   r_i = a_i exp((pot_i - pot~_i)/eps),  pot~_i = |row|^2 - eps ln2 LSE2_i,
-    // i.e. log2 r_i = log2 a_i + (pot_i - |row|^2) log2(e)/eps + LSE2_i, and
-    // sum_j P_ij C_ij = r_i * (w_i / l_i).
-    double c0 = 0.0, c1 = 0.0, c2 = 0.0, c3 = 0.0;
-    if (valid) {
+        if (!p.tail_stats) return;  // uniform over the kernel: a launch parameter
+    } else if (valid) {
+        // Measure mode: with the current row potential pot_in, the plan's row sum is
+        //   r_i = a_i exp((pot_i - pot~_i)/eps),  pot~_i = |row|^2 - eps ln2 LSE2_i,
+        // i.e. log2 r_i = log2 a_i + (pot_i - |row|^2) log2(e)/eps + LSE2_i, and
+        // sum_j P_ij C_ij = r_i * (w_i / l_i).
         const double lw2 = (double)p.row_logw2[prow];
         const double pot = (double)p.pot_in[(size_t)bz * p.rows + row];
         const double a = exp2(lw2);
@@ -84,6 +92,7 @@ __device__ void finish_rows(const PassParams &p, int rb, int rl, float m, float 
         c3 = a * pot;
         if (!isfinite(r) || !isfinite(mc)) atomicOr(p.err, kDevErrNonfinite);
     }
+
     red[0 * kBlockRows + rl] = c0;
     red[1 * kBlockRows + rl] = c1;
     red[2 * kBlockRows + rl] = c2;
@@ -96,7 +105,8 @@ __device__ void finish_rows(const PassParams &p, int rb, int rl, float m, float 
         }
         named_barrier(bar_id, kBlockRows);
     }
-    if (rl < 4) p.stats[((size_t)bz * row_blocks + rb) * 4 + rl] = red[rl * kBlockRows];
+    double *out = MEASURE ? p.stats : p.tail_stats;
+    if (rl < 4) out[((size_t)bz * row_blocks + rb) * 4 + rl] = red[rl * kBlockRows];
 }
 
 }  // namespace fs

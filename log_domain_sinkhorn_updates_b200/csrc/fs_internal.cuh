@@ -60,6 +60,8 @@ struct PassParams {
     float4 *part;              // [batch][splits][rows_pad] split partials (m, l, w, -)
     unsigned *counters;        // [batch][row_blocks] arrival counters (self-resetting)
     double *stats;             // [batch][row_blocks][4] measure partial sums
+    double *tail_stats;        // update passes, or null: [batch][row_blocks][4] marginal statistics of the
+                               // potential this pass writes (the plan's row sums at that potential)
     const void *plain_rows;    // SIMT path: [batch][rows_pad][d] fp32
     const void *plain_cols;    // SIMT path: [batch][cols_rows][d] fp32
     unsigned long long timeout_ns;
@@ -203,4 +205,6 @@ size_t tc2_smem_bytes(int row_bytes, int stages, bool measure);
 int tc2_max_stages(int row_bytes, bool measure);
 // Record msg as this thread's handle-less error (what fs_last_error(NULL) returns).
 void set_thread_error(const char *msg);
+// Add `count` kernels launched outside fs_api.cu to what fs_kernel_launches reports.
+void count_launches(unsigned count);
 }  // namespace fs

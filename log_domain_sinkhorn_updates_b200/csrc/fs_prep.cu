@@ -221,6 +221,16 @@ __global__ void finalize_kernel(const double *stats, int row_blocks, const float
     if (threadIdx.x == 0) out[(size_t)bz * 8 + 4] = acc;
 }
 
+// flag |= 1 where a and b differ in any bit (a potential and its snapshot).
+__global__ void differs_kernel(const float *a, const float *b, size_t count, int *flag) {
+    const uint32_t *ua = reinterpret_cast<const uint32_t *>(a);
+    const uint32_t *ub = reinterpret_cast<const uint32_t *>(b);
+    int any = 0;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x)
+        any |= ua[i] != ub[i];
+    if (__syncthreads_or(any) && threadIdx.x == 0) atomicOr(flag, 1);
+}
+
 int grid_for(size_t work, int per_block) {
     size_t g = (work + per_block - 1) / per_block;
     if (g > 148 * 32) g = 148 * 32;
@@ -282,6 +292,11 @@ cudaError_t launch_bias(const float *pot, int batch, int cnt, int cnt_pad, const
                         double scale2, float *out, cudaStream_t s) {
     bias_kernel<<<grid_for((size_t)batch * cnt_pad, 256), 256, 0, s>>>(pot, cnt, cnt_pad, batch, norm, lw2, scale2,
                                                                       out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_differs(const float *a, const float *b, size_t count, int *flag, cudaStream_t s) {
+    differs_kernel<<<grid_for(count, 256), 256, 0, s>>>(a, b, count, flag);
     return cudaGetLastError();
 }
 

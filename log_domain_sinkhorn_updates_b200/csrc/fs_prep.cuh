@@ -29,6 +29,8 @@ cudaError_t launch_weights(const float *w, int batch, int cnt, int cnt_pad, floa
 cudaError_t launch_fill(float *p, size_t count, float v, cudaStream_t s);
 cudaError_t launch_bias(const float *pot, int batch, int cnt, int cnt_pad, const float *norm, const float *lw2,
                         double scale2, float *out, cudaStream_t s);
+// *flag |= 1 if the count floats at a and b differ in any bit.
+cudaError_t launch_differs(const float *a, const float *b, size_t count, int *flag, cudaStream_t s);
 cudaError_t launch_finalize(const double *stats, int batch, int row_blocks, const float *col_pot,
                             const float *col_lw2, int cols, int cols_pad, double *out, cudaStream_t s);
 

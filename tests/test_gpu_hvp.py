@@ -3,12 +3,20 @@
 the dense oracle (explicit plan, exact linear solve), at potentials the oracle
 converged and rounded to float32 (the same bytes on both sides).
 
-Bound: each transport product carries the relative error of the transport
-application (about 2^-14 on the tensor-core path, its bf16 splits), the
-conjugate-gradient solve stops at a relative residual of 1e-7, and the final
-combination subtracts terms of size (2/eps) max|x| |P Y| from each other.  The
-test takes |H_gpu - H_oracle| <= 2^-8 max|H_oracle| + 2^-12 (2/eps) S, with
-S = max_i sum_j P_ij |x_i - y_j|^2 |v_i| the size of the largest of those terms.
+Bound, per row i:  |H_gpu,i - H_oracle,i| <= 2^-14 (2/eps) S_i + 2^-10 max|H|,
+with S_i = sum_j P_ij |x_i - y_j|^2 max_k |v_ik| the size of the largest term the
+final combination subtracts (all of them are plan-weighted averages of
+(2/eps) |x_i - y_j|^2 |v_i|-sized quantities).
+* 2^-14 is the relative error of one transport product on the tensor-core
+  path (its bf16 hi/lo splits; the CUDA-core path is more accurate), measured
+  against the absolute size of what it sums.
+* 2^-10 max|H| bounds what the conjugate-gradient solve of the potentials'
+  response adds: it stops at a relative residual of 1e-7, but every operator
+  application carries the 2^-14 product error, which the solve amplifies by the
+  conditioning of the reduced system (at most 16 here).
+The cases include the recipes' own dimensions, d = 64 (3xF16 operands) and
+d = 128 (bf16 operands), where the transport-matrix product runs in column
+blocks on the tensor cores.
 """
 import numpy as np
 import pytest
@@ -24,6 +32,10 @@ CASES = {
     "cloud3d": dict(n=320, m=300),
     "middim": dict(n=260, m=240, d=16),
     "highdim": dict(n=256, m=240, d=16),
+    # the recipes' own dimensions: d = 64 (3xF16 operands, two columns of y per
+    # transport-matrix product) and d = 128 (bf16 operands, one column per product)
+    "middim-d64": dict(n=512, m=480),
+    "highdim-d128": dict(n=512, m=480),
 }
 
 
@@ -34,7 +46,7 @@ def test_hvp_x_parity(cuda_device, name, path, monkeypatch):
     monkeypatch.setenv("FS_APPLY_SIMT", "1" if path == "simt" else "0")
     import log_domain_sinkhorn_updates_b200 as fs
     from helpers import device_inputs
-    prob = make_problem(name, **CASES[name])
+    prob = make_problem(name.split("-")[0], **CASES[name])
     X, Y, a_d, b_d = device_inputs(prob)
     Xo, Yo, loga, logb = oracle.problem_arrays(prob, 0)
     f, g = oracle.solve(Xo, Yo, loga, logb, prob.eps, 400)
@@ -46,12 +58,18 @@ def test_hvp_x_parity(cuda_device, name, path, monkeypatch):
     its = fs.fs_hvp_x(h, torch.from_numpy(f32[None]).to(cuda_device), torch.from_numpy(g32[None]).to(cuda_device),
                       X, Y, torch.from_numpy(V[None]).to(cuda_device), out, max_cg_iters=500, cg_rtol=1e-7)
     fs.fs_sync(h)
+    if path == "tc":
+        assert fs.fs_get_info(h)["last_apply_path"] == "tc"
     H = out.cpu().numpy()[0]
     Ho = dense.hvp_x(Xo, Yo, loga, logb, f32.astype(np.float64), g32.astype(np.float64), prob.eps,
                      V.astype(np.float64))
     P = dense.plan(dense.cost_matrix(Xo, Yo), loga, logb, f32.astype(np.float64), g32.astype(np.float64), prob.eps)
     S = (P * dense.cost_matrix(Xo, Yo)).sum(axis=1) * np.abs(V).max(axis=1)
-    bound = 2.0 ** -8 * np.abs(Ho).max() + 2.0 ** -12 * (2.0 / prob.eps) * S.max()
+    bound = 2.0 ** -14 * (2.0 / prob.eps) * S + 2.0 ** -10 * np.abs(Ho).max()
     err = np.abs(H - Ho).max()
-    print(f"{path} {name}: cg steps {its}, max|dH| = {err:.3e}, bound {bound:.3e}, max|H| = {np.abs(Ho).max():.3e}")
-    assert err <= bound
+    rowerr = np.abs(H - Ho).max(axis=1)
+    print(f"{path} {name}: cg steps {its}, max|dH| = {err:.3e}, worst row err / bound {(rowerr / bound).max():.3f}, "
+          f"max|H| = {np.abs(Ho).max():.3e}, "
+          f"max_i |dH_i| / ((2/eps) S_i) = {(rowerr / ((2.0 / prob.eps) * S)).max():.3e}, "
+          f"max|dH| / max|H| = {err / np.abs(Ho).max():.3e}")
+    assert np.all(rowerr <= bound), (rowerr / bound).max()
