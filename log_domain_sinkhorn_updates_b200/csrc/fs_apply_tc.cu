@@ -70,7 +70,9 @@ __host__ __device__ inline ALayout a_layout(int row_bytes, int kslots, int dv_pa
     return L;
 }
 
-template <int KIND, int NPASS, int VPL>
+// PKS > 0: the K-step count of an operand plane, fixed at compile time (the S
+// product is issued with immediate descriptor offsets); PKS = 0: any width.
+template <int KIND, int NPASS, int VPL, int PKS>
 __global__ void __launch_bounds__(kAThreads, 1)
     apply_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const ApplyParams p) {
@@ -249,10 +251,16 @@ __global__ void __launch_bounds__(kAThreads, 1)
                     if (!ok || *abort_flag) break;
                     tc_fence_after();
                     const uint32_t dt = tmem_base + (uint32_t)(b * kTS);
-                    for (int i = 0; i < nk; ++i) {
-                        const uint32_t ba = koff[kAMaxKsteps + i];
-                        const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
-                        tc_mma<KIND>(dt, adesc0 + koff[i], bd + koff[2 * kAMaxKsteps + i], idesc_s, i > 0 ? 1u : 0u);
+                    if constexpr (PKS > 0) {
+                        issue_s_tile<KIND, NPASS, PKS, kBlockRows>(dt, adesc0, bdesc, idesc_s);
+                    } else {
+                        for (int i = 0; i < nk; ++i) {
+                            const uint32_t ba = koff[kAMaxKsteps + i];
+                            const uint64_t bd =
+                                ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
+                            tc_mma<KIND>(dt, adesc0 + koff[i], bd + koff[2 * kAMaxKsteps + i], idesc_s,
+                                         i > 0 ? 1u : 0u);
+                        }
                     }
                     tc_commit(saddr(sfull + b));
                 }
@@ -274,13 +282,20 @@ __global__ void __launch_bounds__(kAThreads, 1)
                         const uint64_t plo = make_sdesc(st + kPBytes, 128u);
                         const uint64_t v0 = make_sdesc(st + 2 * kPBytes, 128u);
                         const uint64_t v1 = make_sdesc(st + 2 * kPBytes + (VPL - 1) * vplane_bytes, 128u);
+                        // 16 values = 32 bytes per K step; every offset and accumulate
+                        // flag an immediate (the kernel's first product starts O afresh)
+                        auto pv = [&](const uint32_t first) {
 #pragma unroll
-                        for (int ks = 0; ks < kTH / 16; ++ks) {  // 16 values = 32 bytes per K step
-                            const uint32_t acc0 = (hh > 0 || ks > 0) ? 1u : 0u;
-                            tc_mma<0>(tmem_o, phi + 2u * ks, v0 + 2u * ks, idesc_o, acc0);
-                            tc_mma<0>(tmem_o, plo + 2u * ks, v0 + 2u * ks, idesc_o, 1u);
-                            if (VPL == 2) tc_mma<0>(tmem_o, phi + 2u * ks, v1 + 2u * ks, idesc_o, 1u);
-                        }
+                            for (int ks = 0; ks < kTH / 16; ++ks) {
+                                tc_mma<0>(tmem_o, phi + 2u * ks, v0 + 2u * ks, idesc_o, ks == 0 ? first : 1u);
+                                tc_mma<0>(tmem_o, plo + 2u * ks, v0 + 2u * ks, idesc_o, 1u);
+                                if (VPL == 2) tc_mma<0>(tmem_o, phi + 2u * ks, v1 + 2u * ks, idesc_o, 1u);
+                            }
+                        };
+                        if (hh == 0)
+                            pv(0u);
+                        else
+                            pv(1u);
                         tc_commit(saddr(stfree + s));
                     }
                 }
@@ -452,24 +467,45 @@ __global__ void vt_pack_kernel(const T *V, int m, int dv, int m_pad, int dv_pad,
     }
 }
 
+template <int KIND, int NPASS, int VPL, int KS>
+cudaError_t launch_one(const ApplyParams &p, int batch, const void *mq, const void *mk, const void *mv, size_t smem,
+                       cudaStream_t s) {
+    dim3 grid(p.rows_pad / kBlockRows, 1, batch);
+    auto kern = apply_tc_kernel<KIND, NPASS, VPL, KS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kAThreads, smem, s>>>(*static_cast<const CUtensorMap *>(mq), *static_cast<const CUtensorMap *>(mk),
+                                       *static_cast<const CUtensorMap *>(mv), p);
+    return cudaGetLastError();
+}
+
+template <int KIND, int NPASS, int KS>
+cudaError_t launch_ks(const ApplyParams &p, int batch, int vpl, const void *mq, const void *mk, const void *mv,
+                      size_t smem, cudaStream_t s) {
+    return vpl == 1 ? launch_one<KIND, NPASS, 1, KS>(p, batch, mq, mk, mv, smem, s)
+                    : launch_one<KIND, NPASS, 2, KS>(p, batch, mq, mk, mv, smem, s);
+}
+
+// The usual plane widths (d = 16, 32, 64 and, one-plane modes, 128 values)
+// take the S product with compile-time offsets; others the table.
+// The compile-time row geometry matches the pass's packed rows.
+template <int NPASS, int KS, typename Params>
+bool fits(const Params &p) {
+    return p.row_bytes == RowGeom<NPASS, KS>::kRowBytes && p.swz == RowGeom<NPASS, KS>::kSwz;
+}
+
 template <int KIND, int NPASS>
 cudaError_t launch_kind(const ApplyParams &p, int batch, int vpl, const void *mq, const void *mk, const void *mv,
                         size_t smem, cudaStream_t s) {
-    dim3 grid(p.rows_pad / kBlockRows, 1, batch);
-    if (vpl == 1) {
-        auto kern = apply_tc_kernel<KIND, NPASS, 1>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kAThreads, smem, s>>>(*static_cast<const CUtensorMap *>(mq), *static_cast<const CUtensorMap *>(mk),
-                                           *static_cast<const CUtensorMap *>(mv), p);
-    } else {
-        auto kern = apply_tc_kernel<KIND, NPASS, 2>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kAThreads, smem, s>>>(*static_cast<const CUtensorMap *>(mq), *static_cast<const CUtensorMap *>(mk),
-                                           *static_cast<const CUtensorMap *>(mv), p);
+    const int ks = p.plane_bytes / 32;
+    if (ks * 32 == p.plane_bytes) {
+        if (ks == 1 && fits<NPASS, 1>(p)) return launch_ks<KIND, NPASS, 1>(p, batch, vpl, mq, mk, mv, smem, s);
+        if (ks == 2 && fits<NPASS, 2>(p)) return launch_ks<KIND, NPASS, 2>(p, batch, vpl, mq, mk, mv, smem, s);
+        if (ks == 4 && fits<NPASS, 4>(p)) return launch_ks<KIND, NPASS, 4>(p, batch, vpl, mq, mk, mv, smem, s);
+        if constexpr (NPASS == 1)
+            if (ks == 8 && fits<NPASS, 8>(p)) return launch_ks<KIND, NPASS, 8>(p, batch, vpl, mq, mk, mv, smem, s);
     }
-    return cudaGetLastError();
+    return launch_ks<KIND, NPASS, 0>(p, batch, vpl, mq, mk, mv, smem, s);
 }
 
 }  // namespace

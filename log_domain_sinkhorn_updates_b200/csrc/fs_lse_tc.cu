@@ -68,7 +68,10 @@ __host__ __device__ inline SmemLayout smem_layout(int row_bytes, int slots, bool
     return L;
 }
 
-template <int KIND, int NPASS, bool MEASURE, int QT>
+// KS > 0: the plane's K-step count, fixed at compile time (the MMAs of a job
+// are issued with immediate descriptor offsets); KS = 0: any width, offsets
+// from a table in shared memory.
+template <int KIND, int NPASS, bool MEASURE, int QT, int KS>
 __global__ void __launch_bounds__(kThreads, 1)
     lse_tc_kernel(const __grid_constant__ CUtensorMap map_rows, const __grid_constant__ CUtensorMap map_cols,
                   const PassParams p) {
@@ -236,10 +239,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t dt = tmem_base + (uint32_t)(b * kBlockCols);
                 const uint64_t adesc = adesc0 + (uint64_t)(qt * qstride);
-                for (int i = 0; i < nk; ++i) {
-                    const uint32_t ba = koff[kMaxKsteps + i];
-                    const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
-                    tc_mma<KIND>(dt, adesc + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
+                if constexpr (KS > 0) {
+                    issue_s_tile<KIND, NPASS, KS, kBlockRows>(dt, adesc, bdesc, idesc);
+                } else {
+                    for (int i = 0; i < nk; ++i) {
+                        const uint32_t ba = koff[kMaxKsteps + i];
+                        const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
+                        tc_mma<KIND>(dt, adesc + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
+                    }
                 }
                 // One commit per job: it completes when the job's MMAs have read
                 // their operands and written S.  The softmax group that waits on
@@ -348,10 +355,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int KIND, int NPASS, bool MEASURE, int QT>
+template <int KIND, int NPASS, bool MEASURE, int QT, int KS>
 cudaError_t launch_variant(const PassParams &p, int batch, const void *map_rows, const void *map_cols,
                            size_t smem, cudaStream_t s) {
-    auto kern = lse_tc_kernel<KIND, NPASS, MEASURE, QT>;
+    auto kern = lse_tc_kernel<KIND, NPASS, MEASURE, QT, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.rows_pad / (QT * kBlockRows), p.splits, batch);
@@ -360,14 +367,37 @@ cudaError_t launch_variant(const PassParams &p, int batch, const void *map_rows,
     return cudaGetLastError();
 }
 
+template <int KIND, int NPASS, int KS>
+cudaError_t launch_update(const PassParams &p, int batch, int qt, const void *map_rows, const void *map_cols,
+                          size_t smem, cudaStream_t s) {
+    return qt == 2 ? launch_variant<KIND, NPASS, false, 2, KS>(p, batch, map_rows, map_cols, smem, s)
+                   : launch_variant<KIND, NPASS, false, 1, KS>(p, batch, map_rows, map_cols, smem, s);
+}
+
+// The compile-time row geometry matches the pass's packed rows.
+template <int NPASS, int KS, typename Params>
+bool fits(const Params &p) {
+    return p.row_bytes == RowGeom<NPASS, KS>::kRowBytes && p.swz == RowGeom<NPASS, KS>::kSwz;
+}
+
 template <int KIND, int NPASS>
 cudaError_t launch_kind(const PassParams &p, int batch, bool measure, int qt, const void *map_rows,
                         const void *map_cols, size_t smem, cudaStream_t s) {
-    if (qt == 2)
-        return measure ? launch_variant<KIND, NPASS, true, 2>(p, batch, map_rows, map_cols, smem, s)
-                       : launch_variant<KIND, NPASS, false, 2>(p, batch, map_rows, map_cols, smem, s);
-    return measure ? launch_variant<KIND, NPASS, true, 1>(p, batch, map_rows, map_cols, smem, s)
-                   : launch_variant<KIND, NPASS, false, 1>(p, batch, map_rows, map_cols, smem, s);
+    if (!measure) {
+        // The update passes of the usual widths issue their MMAs from compile-time
+        // offsets (d = 16, 32, 64 and, for one-plane modes, 128 values per plane).
+        const int ks = p.plane_bytes / 32;
+        if (ks * 32 == p.plane_bytes) {
+            if (ks == 1 && fits<NPASS, 1>(p)) return launch_update<KIND, NPASS, 1>(p, batch, qt, map_rows, map_cols, smem, s);
+            if (ks == 2 && fits<NPASS, 2>(p)) return launch_update<KIND, NPASS, 2>(p, batch, qt, map_rows, map_cols, smem, s);
+            if (ks == 4 && fits<NPASS, 4>(p)) return launch_update<KIND, NPASS, 4>(p, batch, qt, map_rows, map_cols, smem, s);
+            if constexpr (NPASS == 1)
+                if (ks == 8 && fits<NPASS, 8>(p)) return launch_update<KIND, NPASS, 8>(p, batch, qt, map_rows, map_cols, smem, s);
+        }
+        return launch_update<KIND, NPASS, 0>(p, batch, qt, map_rows, map_cols, smem, s);
+    }
+    return qt == 2 ? launch_variant<KIND, NPASS, true, 2, 0>(p, batch, map_rows, map_cols, smem, s)
+                   : launch_variant<KIND, NPASS, true, 1, 0>(p, batch, map_rows, map_cols, smem, s);
 }
 
 }  // namespace

@@ -56,7 +56,9 @@ __host__ __device__ inline SmemLayout2 smem_layout2(int row_bytes, int slots, bo
     return L;
 }
 
-template <int KIND, int NPASS, bool MEASURE>
+// KS > 0: the K-step count of an operand plane, fixed at compile time
+// (immediate descriptor offsets); KS = 0: any width, offsets from a table.
+template <int KIND, int NPASS, bool MEASURE, int KS>
 __global__ void __launch_bounds__(kThreads, 1)
     lse_tc2_kernel(const __grid_constant__ CUtensorMap map_rows, const __grid_constant__ CUtensorMap map_cols,
                    const PassParams p) {
@@ -223,10 +225,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok || *abort_flag) break;
                 tc_fence_after();
                 const uint32_t dt = tmem_base + (uint32_t)(b * kBlockCols);
-                for (int i = 0; i < nk; ++i) {
-                    const uint32_t ba = koff[kMaxKsteps + i];
-                    const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
-                    tc_mma_pair<KIND>(dt, adesc0 + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
+                if constexpr (KS > 0) {
+                    issue_s_tile<KIND, NPASS, KS, kBlockRows, true>(dt, adesc0, bdesc, idesc);
+                } else {
+                    for (int i = 0; i < nk; ++i) {
+                        const uint32_t ba = koff[kMaxKsteps + i];
+                        const uint64_t bd = ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
+                        tc_mma_pair<KIND>(dt, adesc0 + koff[i], bd + koff[2 * kMaxKsteps + i], idesc,
+                                          i > 0 ? 1u : 0u);
+                    }
                 }
                 // One commit per tile (a commit stalls the MMA pipe): the softmax
                 // groups of both CTAs hand the tile's K slots back when it lands.
@@ -323,10 +330,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int KIND, int NPASS, bool MEASURE>
+template <int KIND, int NPASS, bool MEASURE, int KS>
 cudaError_t launch_variant2(const PassParams &p, int batch, const void *map_rows, const void *map_cols,
                             size_t smem, cudaStream_t s) {
-    auto kern = lse_tc2_kernel<KIND, NPASS, MEASURE>;
+    auto kern = lse_tc2_kernel<KIND, NPASS, MEASURE, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -345,6 +352,19 @@ cudaError_t launch_variant2(const PassParams &p, int batch, const void *map_rows
                            *static_cast<const CUtensorMap *>(map_cols), p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// The 512-byte rows this kernel exists for (one plane of 256 values, or hi/lo
+// planes of 128) take the update passes with compile-time offsets.
+template <int KIND, int NPASS>
+cudaError_t launch_kind2(const PassParams &p, int batch, bool measure, const void *map_rows, const void *map_cols,
+                         size_t smem, cudaStream_t s) {
+    if (measure) return launch_variant2<KIND, NPASS, true, 0>(p, batch, map_rows, map_cols, smem, s);
+    constexpr int kWideKs = NPASS == 1 ? 16 : 8;
+    if (p.plane_bytes == 32 * kWideKs && p.row_bytes == RowGeom<NPASS, kWideKs>::kRowBytes &&
+        p.swz == RowGeom<NPASS, kWideKs>::kSwz)
+        return launch_variant2<KIND, NPASS, false, kWideKs>(p, batch, map_rows, map_cols, smem, s);
+    return launch_variant2<KIND, NPASS, false, 0>(p, batch, map_rows, map_cols, smem, s);
 }
 
 }  // namespace
@@ -367,17 +387,10 @@ int tc2_max_stages(int row_bytes, bool measure) {
 // prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16.  rows_pad / 128 must be even.
 cudaError_t launch_lse_tc2(const PassParams &p, int batch, bool measure, int prec, const void *map_rows,
                            const void *map_cols, size_t smem, cudaStream_t s) {
-    if (prec == 1)
-        return measure ? launch_variant2<0, 1, true>(p, batch, map_rows, map_cols, smem, s)
-                       : launch_variant2<0, 1, false>(p, batch, map_rows, map_cols, smem, s);
-    if (prec == 2)
-        return measure ? launch_variant2<1, 1, true>(p, batch, map_rows, map_cols, smem, s)
-                       : launch_variant2<1, 1, false>(p, batch, map_rows, map_cols, smem, s);
-    if (prec == 3)
-        return measure ? launch_variant2<1, 3, true>(p, batch, map_rows, map_cols, smem, s)
-                       : launch_variant2<1, 3, false>(p, batch, map_rows, map_cols, smem, s);
-    return measure ? launch_variant2<2, 3, true>(p, batch, map_rows, map_cols, smem, s)
-                   : launch_variant2<2, 3, false>(p, batch, map_rows, map_cols, smem, s);
+    if (prec == 1) return launch_kind2<0, 1>(p, batch, measure, map_rows, map_cols, smem, s);
+    if (prec == 2) return launch_kind2<1, 1>(p, batch, measure, map_rows, map_cols, smem, s);
+    if (prec == 3) return launch_kind2<1, 3>(p, batch, measure, map_rows, map_cols, smem, s);
+    return launch_kind2<2, 3>(p, batch, measure, map_rows, map_cols, smem, s);
 }
 
 }  // namespace fs

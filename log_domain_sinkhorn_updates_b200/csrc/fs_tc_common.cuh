@@ -208,6 +208,48 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t local_bar, uint16_t cta_
         : "memory");
 }
 
+// Geometry of a packed operand row whose plane holds KS K-steps of 32 bytes
+// and which carries one plane (NPASS = 1) or hi and lo planes (NPASS = 3),
+// known at compile time; the host packs rows by the same rule.
+template <int NPASS, int KS>
+struct RowGeom {
+    static constexpr int kPlane = 32 * KS;
+    static constexpr int kUsed = (NPASS == 3 ? 2 : 1) * kPlane;
+    static constexpr int kRowBytes = kUsed <= 32 ? 32 : (kUsed <= 64 ? 64 : (kUsed + 127) / 128 * 128);
+    static constexpr int kSwz = kRowBytes <= 32 ? 32 : (kRowBytes <= 64 ? 64 : 128);
+    static constexpr int kAtoms = kRowBytes / kSwz;
+};
+
+// The MMAs of one S tile, D (+)= A x B^T over the row's K-steps (and, for
+// NPASS = 3, the products (hi, hi), (lo, hi), (hi, lo) of the split planes).
+// A: AROWS-row tile of K-major swizzle atoms at adesc; B: one ring slot per
+// atom, bdesc[atom].  Every descriptor is a per-tile base plus an immediate:
+// an issue loop whose offsets are run-time values (a table in shared memory, or
+// arithmetic on a loop counter) spends far longer per instruction than the
+// tensor pipe needs for the MMA itself.
+// PAIR: one tcgen05.mma.cta_group::2 per K-step over a CTA pair (same
+// shared-memory offsets in both CTAs).  The wrapper is defined below.
+template <int KIND>
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accum);
+template <int KIND, int NPASS, int KS, int AROWS, bool PAIR = false>
+__device__ __forceinline__ void issue_s_tile(uint32_t d_tmem, uint64_t adesc, const uint64_t (&bdesc)[4],
+                                             uint32_t idesc) {
+    using G = RowGeom<NPASS, KS>;
+#pragma unroll
+    for (int i = 0; i < NPASS * KS; ++i) {
+        const int pass = i / KS, k = i % KS;
+        const int ao = (pass == 1 ? G::kPlane : 0) + 32 * k;
+        const int bo = (pass == 2 ? G::kPlane : 0) + 32 * k;
+        const uint64_t ad = adesc + (uint64_t)(((ao / G::kSwz) * (AROWS * G::kSwz) + ao % G::kSwz) >> 4);
+        const uint64_t bd = bdesc[bo / G::kSwz] + (uint64_t)((bo % G::kSwz) >> 4);
+        if constexpr (PAIR)
+            tc_mma_pair<KIND>(d_tmem, ad, bd, idesc, i > 0 ? 1u : 0u);
+        else
+            tc_mma<KIND>(d_tmem, ad, bd, idesc, i > 0 ? 1u : 0u);
+    }
+}
+
 // sum_k 2^(z_k - ref) over CNT columns, fp32 pairs.
 template <int CNT>
 __device__ __forceinline__ float sum_exp2(const float (&z)[CNT], float ref) {
