@@ -354,22 +354,31 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     p.out = out;
     p.rsum = r;
     p.divide = divide ? 1 : 0;
-    // Tensor cores where the operand rows fit the single-CTA layout (up to 256
-    // bytes) and dv <= 256; the CUDA-core kernel otherwise or with FS_APPLY_SIMT=1.
-    const int dv_pad = (dv + 15) / 16 * 16;
+    // Tensor cores for dv <= 256: on CTA pairs for the 512-byte operand rows
+    // (and at every width with FS_APPLY_PAIR=1), on one CTA for rows of up to
+    // 256 bytes where its plan fits.  The CUDA-core kernel otherwise, for the
+    // fp32 SIMT precision, or with FS_APPLY_SIMT=1.
     const int vpl = v_bf16 ? 1 : 2;
-    int kslots = 0, stages = 0;
     const char *force_simt = getenv("FS_APPLY_SIMT");
-    const size_t smem = (h->prec != FS_PREC_F32_SIMT && !h->pair && h->row_bytes <= 256 && dv <= 256 &&
-                         !(force_simt && atoi(force_simt) != 0))
-                            ? fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages)
-                            : 0;
+    const bool tc_ok = h->prec != FS_PREC_F32_SIMT && dv <= 256 && !(force_simt && atoi(force_simt) != 0);
+    bool use_pair = h->pair;
+    if (const char *env = getenv("FS_APPLY_PAIR")) use_pair = atoi(env) != 0;
+    int dv_pad = use_pair ? (dv + 31) / 32 * 32 : (dv + 15) / 16 * 16;
+    int kslots = 0, stages = 0;
+    size_t smem = 0;
+    if (tc_ok && use_pair)
+        smem = fs::apply_tc2_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
+    if (tc_ok && smem == 0 && !h->pair && h->row_bytes <= 256) {
+        use_pair = false;
+        dv_pad = (dv + 15) / 16 * 16;
+        smem = fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
+    }
     if (smem == 0) {
         h->last_apply = 2;
         FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
         return FS_OK;
     }
-    h->last_apply = 1;
+    h->last_apply = use_pair ? 3 : 1;
     p.row_bytes = h->row_bytes;
     p.swz = h->swz;
     p.plane_bytes = h->plane_bytes;
@@ -395,6 +404,7 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
         cuuint64_t gstride[1] = {(cuuint64_t)p.cols_rows * 2};
         cuuint32_t box[2] = {64, (cuuint32_t)dv_pad};
         cuuint32_t estr[2] = {1, 1};
+        if (use_pair) box[1] = (cuuint32_t)(dv_pad / 2);  // each CTA of a pair loads half the columns of V
         CUresult r2 = fn ? fn(&map_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vt, gdim, gstride, box, estr,
                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
@@ -402,9 +412,20 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
         if (r2 != CUDA_SUCCESS) st = fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed for V (%d)", (int)r2);
     }
     if (e == cudaSuccess && st == FS_OK) {
-        e = fs::launch_apply_tc(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r,
-                                fdir ? &h->mapY_r : &h->mapX_r, &map_v, smem, h->stream);
-        g_launches.fetch_add(1, std::memory_order_relaxed);
+        if (use_pair) {
+            // each CTA of a pair loads a 64-point half of every 128-column tile of K
+            CUtensorMap map_k2{};
+            st = encode_map(h, &map_k2, fdir ? h->packY : h->packX, D.batch * p.cols_rows, 64);
+            if (st == FS_OK) {
+                e = fs::launch_apply_tc2(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r, &map_k2, &map_v,
+                                         smem, h->stream);
+                g_launches.fetch_add(1, std::memory_order_relaxed);
+            }
+        } else {
+            e = fs::launch_apply_tc(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r,
+                                    fdir ? &h->mapY_r : &h->mapX_r, &map_v, smem, h->stream);
+            g_launches.fetch_add(1, std::memory_order_relaxed);
+        }
     }
     cudaFreeAsync(vt, h->stream);
     if (st != FS_OK) return st;

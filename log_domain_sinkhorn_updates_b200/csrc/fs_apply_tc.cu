@@ -149,10 +149,13 @@ __global__ void __launch_bounds__(kAThreads, 1)
     const uint32_t tmem_o = tmem_base + 256u;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producers ----------------
+        // Lane 0 streams Q, the K tiles and the bias slices; lane 1 streams the
+        // V~ halves.  Each waits only on its own rings, so a V~ stage that is
+        // still being read never holds back the next K tile.
         if (lane == 0) {
             bool ok = true;
-            int k_issued = 0, v_issued = 0, b_issued = 0;
+            int k_issued = 0, b_issued = 0;
             mbar_expect_tx(qfull, (uint32_t)kBlockRows * p.row_bytes);
             for (int a = 0; a < atoms; ++a)
                 tma_load_2d(saddr(sQ) + a * kBlockRows * swz, &map_q, saddr(qfull), a * box_inner,
@@ -172,8 +175,6 @@ __global__ void __launch_bounds__(kAThreads, 1)
                     k_issued = i + 1;
                 }
                 if (!ok) break;
-                // the bias slice before the V~ planes: the group that frees the
-                // stages this tile's planes wait for needs this tile's bias first
                 const int j = t % kABias;
                 if (t >= kABias && !mbar_wait(bempty + j, ((uint32_t)(t / kABias) & 1u) ^ 1u, p.timeout_ns)) {
                     ok = false;
@@ -183,6 +184,23 @@ __global__ void __launch_bounds__(kAThreads, 1)
                 bulk_load(saddr(sBias + j * kTS), p.col_bias + (size_t)bz * p.cols_stride + col0, kTS * 4,
                           saddr(bfull + j));
                 b_issued = t + 1;
+            }
+            if (!ok) {
+                atomicOr(p.err, kDevErrTimeout);
+                *abort_flag = 1;
+            }
+            // never leave with copies in flight
+            mbar_wait(qfull, 0, p.timeout_ns);
+            for (int i = max(0, k_issued - KS); i < k_issued; ++i)
+                mbar_wait(kfull + (i % KS), (uint32_t)(i / KS) & 1u, p.timeout_ns);
+            for (int t = max(0, b_issued - kABias); t < b_issued; ++t)
+                mbar_wait(bfull + (t % kABias), (uint32_t)(t / kABias) & 1u, p.timeout_ns);
+        } else if (lane == 1) {
+            bool ok = true;
+            int v_issued = 0;
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const int col0 = t * kTS;
+                if (*abort_flag) break;
                 for (int half = 0; half < 2; ++half) {
                     const int hh = 2 * t + half, s = hh % NS;
                     if (hh >= NS && !mbar_wait(stfree + s, ((uint32_t)(hh / NS) & 1u) ^ 1u, p.timeout_ns)) {
@@ -201,13 +219,8 @@ __global__ void __launch_bounds__(kAThreads, 1)
                 atomicOr(p.err, kDevErrTimeout);
                 *abort_flag = 1;
             }
-            mbar_wait(qfull, 0, p.timeout_ns);
-            for (int i = max(0, k_issued - KS); i < k_issued; ++i)
-                mbar_wait(kfull + (i % KS), (uint32_t)(i / KS) & 1u, p.timeout_ns);
             for (int i = max(0, v_issued - NS); i < v_issued; ++i)
                 mbar_wait(vfull + (i % NS), (uint32_t)(i / NS) & 1u, p.timeout_ns);
-            for (int t = max(0, b_issued - kABias); t < b_issued; ++t)
-                mbar_wait(bfull + (t % kABias), (uint32_t)(t / kABias) & 1u, p.timeout_ns);
         }
         __syncwarp();
     } else if (warp == 1) {

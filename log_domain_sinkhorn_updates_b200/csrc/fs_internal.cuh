@@ -175,6 +175,12 @@ cudaError_t launch_vt_pack(const void *V, bool bf16, int batch, int m, int dv, i
                            void *out, cudaStream_t s);
 cudaError_t launch_apply_tc(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
                             const void *map_v, size_t smem, cudaStream_t s);
+// The CTA-pair transport application (fs_apply_tc2.cu): plan for dv_pad a
+// multiple of 32 (at most 256), and the launch (map_k: 64-row boxes; rows_pad /
+// 128 must be even).
+size_t apply_tc2_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages);
+cudaError_t launch_apply_tc2(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
+                             const void *map_v, size_t smem, cudaStream_t s);
 // A kernel whose one bounded mbarrier wait nothing ever completes: after
 // timeout_ns it raises kDevErrTimeout and returns (fs_tc_common usage check).
 cudaError_t launch_wait_probe(unsigned long long timeout_ns, int *err, cudaStream_t s);

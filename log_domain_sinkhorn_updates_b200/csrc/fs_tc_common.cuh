@@ -169,6 +169,12 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *b, uint32_t parity, 
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
     asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
+// Arrive on an mbarrier of another CTA of the cluster, releasing at cluster
+// scope what this thread wrote before (shared-memory operands that the peer's
+// tensor-core instructions will read, after fence.proxy.async).
+__device__ __forceinline__ void mbar_arrive_cluster_release(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
 // TMA box load into this CTA's shared memory whose completion is counted on
 // an mbarrier of either CTA of the pair (here: the pair's first CTA).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *map, uint32_t cluster_bar, int x, int y) {

@@ -15,8 +15,10 @@ exp2f adds 2^-21, and the fp32 sum over m terms adds m 2^-24.  Hence
 
 The tensor-core path also splits P/a_i and V into bf16 hi + lo pairs, which
 carry 2^-16 each and drop a term of 2^-16 relative size, so its bound adds
-2^-14.  Every test runs both paths: the tensor-core default and the CUDA-core
-validation kernel (FS_APPLY_SIMT=1).
+2^-14.  Every test runs three paths: the one-CTA tensor-core kernel
+(FS_APPLY_PAIR=0), the tensor-core kernel on CTA pairs (FS_APPLY_PAIR=1; the
+default for 512-byte operand rows) and the CUDA-core validation kernel
+(FS_APPLY_SIMT=1).
 """
 import numpy as np
 import pytest
@@ -70,8 +72,13 @@ def _rel_bound(Xo, Yo, loga, logb, f, g, eps, cost):
     return np.log(2.0) * 2.0 ** -23 * M + 2.0 ** -21 + len(Yo) * 2.0 ** -24
 
 
-PATHS = {"tc": "0", "simt": "1"}
-SPLIT = {"tc": 2.0 ** -14, "simt": 0.0}
+PATHS = {"tc": ("0", "0"), "tc_pair": ("0", "1"), "simt": ("1", "0")}  # (FS_APPLY_SIMT, FS_APPLY_PAIR)
+SPLIT = {"tc": 2.0 ** -14, "tc_pair": 2.0 ** -14, "simt": 0.0}
+
+
+def _set_path(monkeypatch, path):
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
+    monkeypatch.setenv("FS_APPLY_PAIR", PATHS[path][1])
 
 
 def _assert_path(fs, h, path, dv):
@@ -82,6 +89,8 @@ def _assert_path(fs, h, path, dv):
     ran = fs.fs_get_info(h)["last_apply_path"]
     if path == "simt":
         assert ran == "simt", ran
+    elif path == "tc_pair":  # the pair's plan fits every operand width here up to dv = 256
+        assert ran == "tc_pair", ran
     elif dv <= 128:
         assert ran == "tc", ran
     else:
@@ -94,7 +103,7 @@ def _assert_path(fs, h, path, dv):
 @pytest.mark.parametrize("dv", [1, 5, 33, 70, 256])
 def test_transport_apply_parity(cuda_device, name, dv, path, monkeypatch):
     import torch
-    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
+    _set_path(monkeypatch, path)
     fs = _fs()
     prob = make_problem(name, **SMALL[name])
     X, Y, a_d, b_d = device_inputs(prob)
@@ -124,7 +133,7 @@ def test_transport_apply_parity(cuda_device, name, dv, path, monkeypatch):
 @pytest.mark.parametrize("name", ["tiny", "middim", "highdim", "batched"])
 def test_barycentric_map_and_grad_parity(cuda_device, name, path, monkeypatch):
     import torch
-    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
+    _set_path(monkeypatch, path)
     fs = _fs()
     prob = make_problem(name, **SMALL[name])
     X, Y, a_d, b_d = device_inputs(prob)
@@ -154,7 +163,7 @@ def test_barycentric_map_and_grad_parity(cuda_device, name, path, monkeypatch):
 @pytest.mark.parametrize("path", list(PATHS))
 def test_transport_apply_cosine_parity(cuda_device, path, monkeypatch):
     import torch
-    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
+    _set_path(monkeypatch, path)
     fs = _fs()
     prob = make_problem("middim", n=1000, m=900)
     X, Y, a_d, b_d = device_inputs(prob)
@@ -187,7 +196,7 @@ def test_transposed_apply_and_grad_y_parity(cuda_device, name, path, monkeypatch
     second half) against the oracle, whose transposed forms exchange the two
     clouds' roles (C is symmetric)."""
     import torch
-    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
+    _set_path(monkeypatch, path)
     fs = _fs()
     prob = make_problem(name, **SMALL[name])
     X, Y, a_d, b_d = device_inputs(prob)
@@ -226,7 +235,7 @@ def test_transport_apply_edge_shapes(cuda_device, n, m, d, path, monkeypatch):
     128-row blocks, the 128-column tiles and their 64-column halves (one valid
     column in the last tile, whole halves of padding)."""
     import torch
-    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path])
+    _set_path(monkeypatch, path)
     fs = _fs()
     rng = np.random.default_rng(n * 1000 + m + d)
     Xo = rng.standard_normal((n, d))
@@ -291,3 +300,49 @@ def test_transport_apply_tf32_kind(cuda_device, name, prec):
         err = (np.abs(out[k] - oo) / (rel[:, None] * absw)).max()
         print(f"{prec} {name}[{k}] worst err / bound = {err:.3f}")
         assert err <= 1.0
+
+
+@pytest.mark.parametrize("case", ["f32-d128-auto", "f32-d64-3xtf32", "cosine-d128-auto", "bf16-d256-auto"])
+def test_transport_apply_wide_rows_on_cta_pairs(cuda_device, case):
+    """Handles whose packed operand rows are 512 bytes run their passes on CTA pairs; their
+    transport application must run on the tensor cores too, by default, within the same
+    bound: fp32 clouds at d = 128 (3xF16), 3xTF32 at d = 64, the cosine cost at d = 128,
+    and bf16 clouds at d = 256 (one plane of 256 values).  Every one of these forms the
+    score to about fp32 accuracy, which the bound assumes (one-pass TF32 does not)."""
+    import torch
+    fs = _fs()
+    kind, dim, prec = case.split("-")
+    name = "middim" if dim == "d64" else "highdim"
+    prob = make_problem(name, **SMALL[name], **({"d": 256} if dim == "d256" else {}))
+    cost = "cosine" if kind == "cosine" else "sqeuclidean"
+    if kind == "bf16":
+        X, Y, a_d, b_d = device_inputs(prob)
+    else:
+        # fp32 inputs (for highdim, the recipe's bf16 values, exactly)
+        X = torch.from_numpy(prob.X[0].astype(np.float32))[None].to(cuda_device)
+        Y = torch.from_numpy(prob.Y[0].astype(np.float32))[None].to(cuda_device)
+        _, _, a_d, b_d = device_inputs(prob)
+    kw = {} if prec == "auto" else {"prec": prec}
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps, cost=cost, **kw)
+    info = fs.fs_get_info(h)
+    assert info["cta_pair"] == 1 and info["row_bytes"] == 512, info
+    f32, g32 = _potentials(prob, cost)
+    rng = np.random.default_rng(321)
+    for dv in (1, 64, 130):
+        V = rng.standard_normal((1, prob.m, dv)).astype(np.float32)
+        out = torch.empty(1, prob.n, dv, device=cuda_device)
+        r = torch.empty(1, prob.n, device=cuda_device)
+        fs.fs_transport_apply(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device),
+                              torch.from_numpy(V).to(cuda_device), out, r)
+        fs.fs_sync(h)
+        assert fs.fs_get_info(h)["last_apply_path"] == "tc_pair"
+        Xo, Yo, loga, logb = oracle_arrays(prob)[0]
+        fk, gk = f32[0].astype(np.float64), g32[0].astype(np.float64)
+        oo, ro = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, V[0].astype(np.float64), cost=cost)
+        absw, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(V[0]).astype(np.float64),
+                                         cost=cost)
+        rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, cost) + 2.0 ** -14
+        err = np.abs(out.cpu().numpy()[0] - oo) / (rel[:, None] * absw)
+        rerr = np.abs(r.cpu().numpy()[0] - ro) / (rel * ro)
+        print(f"{case} dv={dv}: worst err / bound = {err.max():.3f}, row sums {rerr.max():.3f}")
+        assert err.max() <= 1.0 and rerr.max() <= 1.0
