@@ -52,9 +52,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline sample duration")
-    ap.add_argument("--op", choices=["solve", "transport"], default="solve",
+    ap.add_argument("--op", choices=["solve", "transport", "hvp"], default="solve",
                     help="solve: the Sinkhorn solve (the headline); transport: the barycentric map at the "
-                         "converged potentials (transport application, tensor-core kernel)")
+                         "converged potentials (transport application, tensor-core kernel); hvp: the streaming "
+                         "Hessian-vector product of the EOT cost in X at the converged potentials (batch 1)")
     return ap.parse_args()
 
 
@@ -336,12 +337,73 @@ def run_transport(args):
     return 0
 
 
+def run_hvp(args):
+    """fs_hvp_x at the workload's converged potentials in a seeded direction, conjugate
+    gradients to a relative residual of 1e-6: one product per step, timed with CUDA events
+    (the product synchronises once per CG step; its host waits are inside the timed region)."""
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    import log_domain_sinkhorn_updates_b200 as fs
+    prob = make_problem(args.workload, n=args.n, m=args.m, batch=1)
+    n, m, d = prob.n, prob.m, prob.d
+    if prob.dtype == "bf16":
+        X = torch.from_numpy(prob.X_dev.view(np.int16)).view(torch.bfloat16).to(dev)
+        Y = torch.from_numpy(prob.Y_dev.view(np.int16)).view(torch.bfloat16).to(dev)
+    else:
+        X, Y = torch.from_numpy(prob.X_dev).to(dev), torch.from_numpy(prob.Y_dev).to(dev)
+    a = None if prob.a_dev is None else torch.from_numpy(prob.a_dev).to(dev)
+    b = None if prob.b_dev is None else torch.from_numpy(prob.b_dev).to(dev)
+    h = fs.fs_create(X, Y, a, b, eps=prob.eps)
+    f = torch.zeros(1, n, device=dev)
+    g = torch.zeros(1, m, device=dev)
+    fs.fs_solve(h, f, g, args.iters or prob.iters)
+    V = torch.from_numpy(np.random.default_rng(200).standard_normal((1, n, d)).astype(np.float32)).to(dev)
+    out = torch.empty(1, n, d, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    its = 0
+    for _ in range(args.warmup):
+        its = fs.fs_hvp_x(h, f, g, X, Y, V, out, max_cg_iters=500, cg_rtol=1e-6)
+    fs.fs_sync(h)
+    sampler = ClockSampler(gpu_identifier(torch, dev))
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    launches0 = fs.fs_kernel_launches()
+    tot = 0.0
+    for _ in range(args.steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        its = fs.fs_hvp_x(h, f, g, X, Y, V, out, max_cg_iters=500, cg_rtol=1e-6)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        tot += e0.elapsed_time(e1)
+    launches = fs.fs_kernel_launches() - launches0
+    clocks = sampler.stop()
+    info = fs.fs_get_info(h)
+    line = {
+        "metric": "streaming Hessian-vector product of the EOT cost in X (ms per product, CG to 1e-6)",
+        "value": tot / args.steps, "unit": "ms", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot / args.steps, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if info["prec"] == "bf16" else "f32", "data": "synthetic",
+        "config": workload_config(prob, args.iters or prob.iters, {
+            "op": "fs_hvp_x", "cg_steps": int(its), "fused_term": bool(info["last_hvp_fused"]),
+            "precision": info["prec"], "step": "fs_hvp_x at the potentials of the solve (solve untimed)",
+            "half_iters_per_step": 0, "l2": "not flushed (a product is tens of passes over the same operands)"}),
+        "cpu_baseline": None, "e2e": None, "clocks": clocks, "gpu_launches": int(launches),
+    }
+    fs.fs_destroy(h)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "transport":
         return run_transport(args)
+    if args.op == "hvp":
+        return run_hvp(args)
 
     import torch
     import torch.distributed as dist

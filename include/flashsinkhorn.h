@@ -128,6 +128,11 @@ typedef struct {
                                the last alternating fs_solve reduced in its final pass (f and g were
                                that solve's output, unchanged bit for bit); 0: it streamed its own
                                measure passes */
+    int last_hvp_fused;     /* 1: the handle's last fs_hvp_x formed its transport-matrix term
+                               sum_j P_ij (v_i.y_j) y_j in one tensor-core pass (bf16 operands, or the
+                               3xF16 / 3xTF32 splits, rows up to 256 bytes); 0: as d / nq transport
+                               applications of width nq d (other operands, FS_HVP_FUSED=0, or
+                               FS_APPLY_SIMT=1) */
 } fs_info;
 
 /*

@@ -41,7 +41,8 @@ class FsInfo(ctypes.Structure):
                 ("block_cols", ctypes.c_int), ("splits_f", ctypes.c_int), ("splits_g", ctypes.c_int),
                 ("launches_update", ctypes.c_int), ("launches_solve_iter", ctypes.c_int),
                 ("device_bytes", ctypes.c_size_t), ("cta_pair", ctypes.c_int), ("last_apply_path", ctypes.c_int),
-                ("last_solve_graph", ctypes.c_int), ("last_measure_fused", ctypes.c_int)]
+                ("last_solve_graph", ctypes.c_int), ("last_measure_fused", ctypes.c_int),
+                ("last_hvp_fused", ctypes.c_int)]
 
     def as_dict(self):
         d = {k: getattr(self, k) for k, _ in self._fields_}

@@ -61,6 +61,7 @@ struct fs_handle {
     bool meas_ok = false;            // meas_cache holds the f-direction measure at the snapshot
     std::vector<double> meas_cache;  // [batch][8] as in h->red
     int last_measure_fused = 0;
+    int last_hvp_fused = 0;  // 1: the last fs_hvp_x formed sum_j P_ij (v_i.y_j) y_j in one fused pass
     std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
     int host_err[4] = {0, 0, 0, 0};
     CUtensorMap mapX_r{}, mapX_c{}, mapY_r{}, mapY_c{};  // row-side (128-row box) / column-side (256-row box)
@@ -516,6 +517,110 @@ bool capture_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule sche
     h->gkernels = t_captured;
     return true;
 }
+// MV_i = sum_j P_ij (v_i . y_j) y_j in one pass over the plan (fs_hvp_tc.cu), batch 1,
+// squared Euclidean cost; *done = false (and nothing enqueued) where the handle's
+// operands have no fused form or its plan does not fit.
+fs_status hvp_fused_term(fs_handle *h, const float *f, const float *g, const void *Y, const float *V, float *MV,
+                         bool *done) {
+    *done = false;
+    const fs_desc &D = h->desc;
+    if (h->prec == FS_PREC_F32_SIMT || h->pair || D.batch != 1 || D.cost != FS_COST_SQEUCLIDEAN) return FS_OK;
+    const int umode = fs::hvp_w_mode(h->prec, h->plane_bytes, h->row_bytes);
+    if (umode == 0) return FS_OK;
+    const bool bf16 = D.dtype == FS_BF16;
+    const int vpl = bf16 ? 1 : 2;
+    const int dv_pad = (D.d + 15) / 16 * 16;
+    int kslots = 0, stages = 0;
+    const size_t smem = fs::hvp_w_plan(h->row_bytes, umode, dv_pad, vpl, &kslots, &stages);
+    if (smem == 0 || dv_pad > 256) return FS_OK;
+    const size_t n = (size_t)D.n;
+    size_t off = 0;
+    auto carve = [&](size_t bytes) {
+        const size_t o = off;
+        off += align256(bytes);
+        return o;
+    };
+    const size_t o_u = carve((umode == 2 ? 2 : 1) * (size_t)h->n_pad * h->row_bytes);
+    const size_t o_norm = carve((size_t)h->n_stride * 4);
+    const size_t o_vt = carve((size_t)vpl * dv_pad * h->m_pad * 2);
+    const size_t o_mx = carve(16);
+    cudaMemPool_t pool;
+    uint8_t *blk = nullptr;
+    FS_CUDA(h, device_pool(h->device, &pool));
+    FS_CUDA(h, cudaMallocFromPoolAsync((void **)&blk, off, pool, h->stream));
+    auto run = [&]() -> fs_status {
+        cudaStream_t s = h->stream;
+        FS_LAUNCH(h, run_bias(h, g, true));  // the f-direction column bias from g
+        float uscale = 1.f;
+        if (umode == 1) {
+            if (h->pack_mode == fs::kPack3xF16) {  // U's own power-of-two scale, as for X and Y
+                float *mx = reinterpret_cast<float *>(blk + o_mx);
+                float host = 0.f;
+                FS_LAUNCH(h, fs::launch_maxabs(V, false, D.n, D.d, 1, nullptr, mx, s));
+                FS_CUDA(h, cudaMemcpyAsync(&host, mx, sizeof(float), cudaMemcpyDeviceToHost, s));
+                FS_CUDA(h, cudaStreamSynchronize(s));
+                if (host > 0.f && std::isfinite(host))
+                    uscale = std::ldexp(1.f, 14 - (int)std::ceil(std::log2((double)host)));
+            }
+            FS_LAUNCH(h, fs::launch_pack(V, false, D.n, h->n_pad, D.d, 1, nullptr, uscale, h->pack_mode, h->d_p,
+                                         h->row_elems, blk + o_u, reinterpret_cast<float *>(blk + o_norm), h->n_stride,
+                                         h->err, s, false));
+        } else {
+            FS_LAUNCH(h, fs::launch_u_split(V, D.n, h->n_pad, D.d, h->row_elems, blk + o_u, s));
+        }
+        FS_LAUNCH(h, fs::launch_vt_pack(Y, bf16, 1, D.m, D.d, h->m_pad, dv_pad, vpl, blk + o_vt, s));
+        CUtensorMap map_u{}, map_v{};
+        fs_status st = encode_map(h, &map_u, blk + o_u, (umode == 2 ? 2 : 1) * h->n_pad, kBlockRows);
+        if (st != FS_OK) return st;
+        auto fn = encode_fn();
+        cuuint64_t gdim[2] = {(cuuint64_t)h->m_pad, (cuuint64_t)vpl * dv_pad};
+        cuuint64_t gstride[1] = {(cuuint64_t)h->m_pad * 2};
+        cuuint32_t box[2] = {64, (cuuint32_t)dv_pad};
+        cuuint32_t estr[2] = {1, 1};
+        const CUresult r2 = fn ? fn(&map_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, blk + o_vt, gdim, gstride, box, estr,
+                                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
+                               : CUDA_ERROR_NOT_SUPPORTED;
+        if (r2 != CUDA_SUCCESS) return fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed for Y~ (%d)", (int)r2);
+        fs::ApplyParams p{};
+        p.rows = D.n;
+        p.rows_pad = h->n_pad;
+        p.rows_stride = h->n_stride;
+        p.cols = D.m;
+        p.cols_rows = h->m_pad;
+        p.cols_stride = h->m_stride;
+        p.d = D.d;
+        p.d_p = h->d_p;
+        p.row_elems = h->row_elems;
+        p.pack_mode = h->pack_mode;
+        p.dv = D.d;
+        p.scale = fs::kLog2ed / (double)D.eps;
+        p.pot_row = f;
+        p.row_norm = h->xn;
+        p.row_logw2 = h->la2;
+        p.col_bias = h->bias_col;
+        p.out = MV;
+        p.row_bytes = h->row_bytes;
+        p.swz = h->swz;
+        p.plane_bytes = h->plane_bytes;
+        p.dv_pad = dv_pad;
+        p.kslots = kslots;
+        p.stages = stages;
+        p.sscale = h->sscale;
+        p.timeout_ns = h->timeout_ns;
+        p.err = h->err;
+        // K holds 2 kscale (y - t) and U holds uscale v: v . (y - t) = S' / (2 kscale uscale)
+        const float cw = (float)(1.0 / (2.0 * (double)h->kscale * (double)uscale));
+        FS_LAUNCH(h, fs::launch_hvp_w(p, h->prec, umode, vpl, cw, V, bf16 ? nullptr : h->center, &h->mapX_r, &map_u,
+                                      &h->mapY_r, &map_v, smem, s));
+        return FS_OK;
+    };
+    const fs_status st = run();
+    cudaFreeAsync(blk, h->stream);
+    if (st == FS_OK) *done = true;
+    return st;
+}
+
 }  // namespace
 
 extern "C" {
@@ -664,14 +769,24 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
         FS_LAUNCH(h, fs::hvp_dgy(Y, bf16, x, (int)m, (int)d, dgY, s));
         s2 = apply(h, f, g, dgY, false, (int)d, Q1, nullptr, false, true);
         if (s2 != FS_OK) return s2;
-        // sum_j P_ij (y_j.v_i) y_j, nq columns of y at a time
-        FS_CUDA(h, cudaMemsetAsync(MV, 0, n * d * 4, s));
-        for (int k0 = 0; k0 < (int)d; k0 += nq) {
-            const int q = (int)d - k0 < nq ? (int)d - k0 : nq;
-            FS_LAUNCH(h, fs::hvp_ychunk(Y, bf16, (int)m, (int)d, k0, q, Vc, s));
-            s2 = apply(h, f, g, Vc, false, q * (int)d, Oc, nullptr, false, true);
+        // sum_j P_ij (y_j.v_i) y_j: in one fused pass where the handle's operands
+        // allow it (tensor cores), else nq columns of y at a time
+        bool fused = false;
+        const char *env_fused = getenv("FS_HVP_FUSED"), *env_simt = getenv("FS_APPLY_SIMT");
+        if (!(env_fused && atoi(env_fused) == 0) && !(env_simt && atoi(env_simt) != 0)) {
+            s2 = hvp_fused_term(h, f, g, Y, V, MV, &fused);
             if (s2 != FS_OK) return s2;
-            FS_LAUNCH(h, fs::hvp_mv_acc(V, Oc, (int)n, (int)d, k0, q, MV, s));
+        }
+        h->last_hvp_fused = fused ? 1 : 0;
+        if (!fused) {
+            FS_CUDA(h, cudaMemsetAsync(MV, 0, n * d * 4, s));
+            for (int k0 = 0; k0 < (int)d; k0 += nq) {
+                const int q = (int)d - k0 < nq ? (int)d - k0 : nq;
+                FS_LAUNCH(h, fs::hvp_ychunk(Y, bf16, (int)m, (int)d, k0, q, Vc, s));
+                s2 = apply(h, f, g, Vc, false, q * (int)d, Oc, nullptr, false, true);
+                if (s2 != FS_OK) return s2;
+                FS_LAUNCH(h, fs::hvp_mv_acc(V, Oc, (int)n, (int)d, k0, q, MV, s));
+            }
         }
         FS_LAUNCH(h, fs::hvp_final(X, bf16, V, PY, r, df, Pdg, Q1, MV, (int)n, (int)d, D.eps, out, s));
         return FS_OK;
@@ -1138,6 +1253,7 @@ fs_status fs_get_info(const fs_handle *h, fs_info *info) {
     info->last_apply_path = h->last_apply;
     info->last_solve_graph = h->last_solve_graph;
     info->last_measure_fused = h->last_measure_fused;
+    info->last_hvp_fused = h->last_hvp_fused;
     return FS_OK;
 }
 

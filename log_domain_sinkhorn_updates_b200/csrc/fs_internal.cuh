@@ -209,6 +209,14 @@ cudaError_t launch_lse_tc2(const PassParams &p, int batch, bool measure, int pre
                            const void *map_cols, size_t smem_bytes, cudaStream_t s);
 size_t tc2_smem_bytes(int row_bytes, int stages, bool measure);
 int tc2_max_stages(int row_bytes, bool measure);
+// The fused transport-matrix term of the HVP (fs_hvp_tc.cu): which U packing the
+// handle's precision takes (0: none), the plan, the bf16 hi/lo split of U, the launch.
+int hvp_w_mode(int prec, int plane_bytes, int row_bytes);
+size_t hvp_w_plan(int row_bytes, int umode, int dv_pad, int vpl, int *kslots, int *stages);
+cudaError_t launch_u_split(const float *V, int rows, int rows_pad, int d, int row_elems, void *out, cudaStream_t s);
+cudaError_t launch_hvp_w(const ApplyParams &p, int prec, int umode, int vpl, float cw, const float *dirv,
+                         const float *center, const void *map_q, const void *map_u, const void *map_k,
+                         const void *map_v, size_t smem, cudaStream_t s);
 // Record msg as this thread's handle-less error (what fs_last_error(NULL) returns).
 void set_thread_error(const char *msg);
 // Add `count` kernels launched outside fs_api.cu to what fs_kernel_launches reports.

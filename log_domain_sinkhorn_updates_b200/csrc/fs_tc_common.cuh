@@ -238,7 +238,8 @@ struct RowGeom {
 template <int KIND>
 __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t accum);
-template <int KIND, int NPASS, int KS, int AROWS, bool PAIR = false>
+// ONTO: accumulate onto what D holds already (else the first MMA starts D afresh).
+template <int KIND, int NPASS, int KS, int AROWS, bool PAIR = false, bool ONTO = false>
 __device__ __forceinline__ void issue_s_tile(uint32_t d_tmem, uint64_t adesc, const uint64_t (&bdesc)[4],
                                              uint32_t idesc) {
     using G = RowGeom<NPASS, KS>;
@@ -249,10 +250,11 @@ __device__ __forceinline__ void issue_s_tile(uint32_t d_tmem, uint64_t adesc, co
         const int bo = (pass == 2 ? G::kPlane : 0) + 32 * k;
         const uint64_t ad = adesc + (uint64_t)(((ao / G::kSwz) * (AROWS * G::kSwz) + ao % G::kSwz) >> 4);
         const uint64_t bd = bdesc[bo / G::kSwz] + (uint64_t)((bo % G::kSwz) >> 4);
+        const uint32_t acc = (ONTO || i > 0) ? 1u : 0u;
         if constexpr (PAIR)
-            tc_mma_pair<KIND>(d_tmem, ad, bd, idesc, i > 0 ? 1u : 0u);
+            tc_mma_pair<KIND>(d_tmem, ad, bd, idesc, acc);
         else
-            tc_mma<KIND>(d_tmem, ad, bd, idesc, i > 0 ? 1u : 0u);
+            tc_mma<KIND>(d_tmem, ad, bd, idesc, acc);
     }
 }
 

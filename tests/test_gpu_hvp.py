@@ -15,8 +15,11 @@ final combination subtracts (all of them are plan-weighted averages of
   application carries the 2^-14 product error, which the solve amplifies by the
   conditioning of the reduced system (at most 16 here).
 The cases include the recipes' own dimensions, d = 64 (3xF16 operands) and
-d = 128 (bf16 operands), where the transport-matrix product runs in column
-blocks on the tensor cores.
+d = 128 (bf16 operands).  Three paths each: the tensor-core default, where the
+transport-matrix term sum_j P_ij (v_i . y_j) y_j is one fused pass (a second
+score v_i . y_j against the same K tile); the same term as d / nq transport
+applications of column blocks of y (FS_HVP_FUSED=0); and the CUDA-core
+validation kernels (FS_APPLY_SIMT=1).
 """
 import numpy as np
 import pytest
@@ -39,11 +42,15 @@ CASES = {
 }
 
 
-@pytest.mark.parametrize("path", ["tc", "simt"])
+PATHS = {"tc": ("0", "1"), "tc_blocked": ("0", "0"), "simt": ("1", "0")}  # (FS_APPLY_SIMT, FS_HVP_FUSED)
+
+
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", list(CASES))
 def test_hvp_x_parity(cuda_device, name, path, monkeypatch):
     import torch
-    monkeypatch.setenv("FS_APPLY_SIMT", "1" if path == "simt" else "0")
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
+    monkeypatch.setenv("FS_HVP_FUSED", PATHS[path][1])
     import log_domain_sinkhorn_updates_b200 as fs
     from helpers import device_inputs
     prob = make_problem(name.split("-")[0], **CASES[name])
@@ -58,8 +65,10 @@ def test_hvp_x_parity(cuda_device, name, path, monkeypatch):
     its = fs.fs_hvp_x(h, torch.from_numpy(f32[None]).to(cuda_device), torch.from_numpy(g32[None]).to(cuda_device),
                       X, Y, torch.from_numpy(V[None]).to(cuda_device), out, max_cg_iters=500, cg_rtol=1e-7)
     fs.fs_sync(h)
-    if path == "tc":
-        assert fs.fs_get_info(h)["last_apply_path"] in ("tc", "tc_pair")
+    info = fs.fs_get_info(h)
+    if path != "simt":
+        assert info["last_apply_path"] in ("tc", "tc_pair")
+    assert info["last_hvp_fused"] == (1 if path == "tc" else 0), info
     H = out.cpu().numpy()[0]
     Ho = dense.hvp_x(Xo, Yo, loga, logb, f32.astype(np.float64), g32.astype(np.float64), prob.eps,
                      V.astype(np.float64))
