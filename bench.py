@@ -52,6 +52,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline sample duration")
+    ap.add_argument("--shard", choices=["replicas", "rows"], default="replicas",
+                    help="multi-GPU mode of --op solve: replicas (each rank solves its own copy of the workload, "
+                         "weak scaling) or rows (one problem, rows and columns split over the ranks, the "
+                         "potentials all-gathered after every half-iteration; strong scaling)")
     ap.add_argument("--op", choices=["solve", "transport", "hvp"], default="solve",
                     help="solve: the Sinkhorn solve (the headline); transport: the barycentric map at the "
                          "converged potentials (transport application, tensor-core kernel); hvp: the streaming "
@@ -396,10 +400,87 @@ def run_hvp(args):
     return 0
 
 
+def run_row_sharded(args):
+    """One problem per job, its rows split over the ranks (log_domain_sinkhorn_updates_b200.sharded):
+    each rank updates its share of f, then of g, and the slices are all-gathered (NCCL) after
+    every half-iteration.  value = the problem's entries per half-iteration x 2 iters / the
+    slowest rank's device time ("scaling": "strong")."""
+    import torch
+    import torch.distributed as dist
+    from log_domain_sinkhorn_updates_b200.sharded import DistGather, FsShard, LocalGather, shard_ranges, \
+        solve_row_sharded
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import log_domain_sinkhorn_updates_b200 as fs
+    prob = make_problem(args.workload, n=args.n, m=args.m, batch=args.batch)
+    iters = args.iters or prob.iters
+    B, n, m = prob.batch, prob.n, prob.m
+    if prob.dtype == "bf16":
+        X = torch.from_numpy(prob.X_dev.view(np.int16)).view(torch.bfloat16).to(dev)
+        Y = torch.from_numpy(prob.Y_dev.view(np.int16)).view(torch.bfloat16).to(dev)
+    else:
+        X, Y = torch.from_numpy(prob.X_dev).to(dev), torch.from_numpy(prob.Y_dev).to(dev)
+    a = None if prob.a_dev is None else torch.from_numpy(prob.a_dev).to(dev)
+    b = None if prob.b_dev is None else torch.from_numpy(prob.b_dev).to(dev)
+    rr, _ = shard_ranges(n, world)
+    cc, _ = shard_ranges(m, world)
+    shard = FsShard(X, Y, a, b, prob.eps, rr[rank], cc[rank])
+    gather = DistGather() if world > 1 else LocalGather()
+    for _ in range(args.warmup):
+        solve_row_sharded([shard], gather, n, m, B, world, 2, device=dev)
+    sampler = ClockSampler(gpu_identifier(torch, dev))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    launches0 = fs.fs_kernel_launches()
+    stream = torch.cuda.current_stream(dev)
+    tot = 0.0
+    f = g = None
+    for _ in range(args.steps):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        f, g = solve_row_sharded([shard], gather, n, m, B, world, iters, device=dev)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        tot += e0.elapsed_time(e1)
+    launches = fs.fs_kernel_launches() - launches0
+    clocks = sampler.stop()
+    tot = max_over_ranks([tot], dev)[0]
+    value = args.steps * 2 * iters * B * n * m / (tot / 1e3)
+    shard.close()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot / args.steps, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": prob.dtype, "data": "synthetic",
+        "config": workload_config(prob, iters, {
+            "step": f"row-sharded fs_update_f / fs_update_g x {iters}, all-gather after every half-iteration",
+            "parallelism": f"rows x{world}", "l2": "not flushed (the shards stay resident)"}),
+        "cpu_baseline": None, "e2e": None, "clocks": clocks, "gpu_launches": int(launches),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.shard == "rows" and args.op == "solve":
+        return run_row_sharded(args)
     if args.op == "transport":
         return run_transport(args)
     if args.op == "hvp":
