@@ -15,10 +15,12 @@
 // 512-byte operand rows (fp32 clouds at d = 128 in 3xF16 or TF32, 3xTF32 at
 // d = 64) run on the tensor cores too.
 //
-// Roles and data flow are those of the one-CTA kernel (warp 0 TMA producer,
-// warp 1 TMEM allocator and, in the pair's first CTA, MMA issuer, warps 2..9
-// two softmax groups taking the even and the odd tiles).  Synchronisation of
-// the pair:
+// Roles and data flow are those of the one-CTA kernel (warp 0 the Q / K / bias
+// producer, warp 10 the V~ producer, warp 1 TMEM allocator and, in the pair's
+// first CTA, MMA issuer, warps 2..9 two softmax groups taking the even and the
+// odd tiles).  The V~ producer has a warp of its own: sharing warp 0 with the
+// K producer measured 1 % slower at n = m = 65536, d = 128.  Synchronisation
+// of the pair:
 //  * the TMA copies of both CTAs (Q, K halves, V~ halves) count on the first
 //    CTA's barriers, where the MMA issuer waits;
 //  * every MMA completion is committed to both CTAs at once (multicast commit):
@@ -38,7 +40,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kP2Threads = 320;
+constexpr int kP2Threads = 352;
 constexpr int kP2TS = 128;          // columns per tile (N of the S product)
 constexpr int kP2KRows = 64;        // K rows of a tile held by each CTA
 constexpr int kP2TH = 64;           // columns per half (K of one P V product)
@@ -151,9 +153,9 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 
     if (warp == 0) {
         // ---------------- TMA producers (both CTAs) ----------------
-        // Lane 0 streams Q, this CTA's K halves and the bias slices; lane 1 this
-        // CTA's V~ halves.  Each waits only on its own rings, so a V~ stage that
-        // is still being read never holds back the next K tile.
+        // Warp 0 streams Q, this CTA's K halves and the bias slices; warp 10
+        // this CTA's V~ halves.  Each waits only on its own rings, so a V~ stage
+        // that is still being read never holds back the next K tile.
         if (lane == 0) {
             bool ok = true;
             int k_issued = 0, b_issued = 0;
@@ -201,7 +203,10 @@ __global__ void __launch_bounds__(kP2Threads, 1)
             }
             for (int t = max(0, b_issued - kP2Bias); t < b_issued; ++t)
                 mbar_wait(bfull + (t % kP2Bias), (uint32_t)(t / kP2Bias) & 1u, p.timeout_ns);
-        } else if (lane == 1) {
+        }
+        __syncwarp();
+    } else if (warp == 10) {
+        if (lane == 0) {
             bool ok = true;
             int v_issued = 0;
             for (int t = 0; ok && t < ntiles; ++t) {
@@ -327,7 +332,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
             mbar_wait(ofull, 0, p.timeout_ns);
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 2 && warp < 10) {
         // ---------------- softmax groups (both CTAs) ----------------
         const int q = warp & 3;
         const int grp = (warp - 2) >> 2;
