@@ -264,17 +264,32 @@ def barycentric_projection(X, Y, loga, logb, f, g, eps, cost="sqeuclidean"):
     return out / r[:, None]
 
 
-def grad_x(X, Y, loga, logb, f, g, eps):
+def grad_x(X, Y, loga, logb, f, g, eps, cost="sqeuclidean"):
     """Gradient of the entropic OT cost with respect to the positions X at the
-    potentials (f, g), squared-Euclidean cost: sum_j P_ij dC_ij/dx_i =
-    2 (r_i x_i - sum_j P_ij y_j).  At optimal potentials this is the gradient of
-    the optimal value (envelope theorem)."""
-    out, r = transport_apply(X, Y, loga, logb, f, g, eps, Y)
-    return 2.0 * (r[:, None] * np.asarray(X, dtype=np.float64) - out)
+    potentials (f, g): sum_j P_ij dC_ij/dx_i.  At optimal potentials this is the
+    gradient of the optimal value (envelope theorem).
+
+    * squared Euclidean, dC/dx = 2 (x - y): 2 (r_i x_i - sum_j P_ij y_j);
+    * cosine, C = 1 - x.y / (|x| |y|), dC/dx = -(y^ - (x^.y^) x^) / |x| with
+      x^ = x / |x|, y^ = y / |y| (the part of y^ orthogonal to x, over |x|):
+      -(b_i - (x^_i.b_i) x^_i) / |x_i| with b_i = sum_j P_ij y^_j, the per-pair
+      gradients being linear in y^_j.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    if cost == "cosine":
+        Y = np.asarray(Y, dtype=np.float64)
+        Yh = Y / np.linalg.norm(Y, axis=1)[:, None]
+        bsum, _ = transport_apply(X, Y, loga, logb, f, g, eps, Yh, cost)
+        nx = np.linalg.norm(X, axis=1)
+        Xh = X / nx[:, None]
+        return -(bsum - np.sum(Xh * bsum, axis=1)[:, None] * Xh) / nx[:, None]
+    out, r = transport_apply(X, Y, loga, logb, f, g, eps, Y, cost)
+    return 2.0 * (r[:, None] * X - out)
 
 
-def grad_y(X, Y, loga, logb, f, g, eps):
-    """Gradient of the entropic OT cost with respect to the positions Y at (f, g),
-    squared-Euclidean cost: 2 (c_j y_j - sum_i P_ij x_i) -- grad_x with the roles
-    of the two clouds (and weights, potentials) exchanged, C being symmetric."""
-    return grad_x(Y, X, logb, loga, g, f, eps)
+def grad_y(X, Y, loga, logb, f, g, eps, cost="sqeuclidean"):
+    """Gradient of the entropic OT cost with respect to the positions Y at (f, g):
+    grad_x with the roles of the two clouds (and weights, potentials) exchanged,
+    both costs being symmetric in x and y (squared Euclidean: 2 (c_j y_j -
+    sum_i P_ij x_i))."""
+    return grad_x(Y, X, logb, loga, g, f, eps, cost)

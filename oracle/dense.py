@@ -103,28 +103,65 @@ def two_by_two_plan(C, a1, b1, eps):
     return np.array([[p, a1 - p], [b1 - p, 1.0 - a1 - b1 + p]])
 
 
-def hvp_x(X, Y, loga, logb, f, g, eps, V):
-    """Hessian-vector product of the entropic OT cost with respect to the positions X
-    (squared Euclidean cost) at optimal potentials (f, g), in direction V [n, d].
+def cost_grad_x(X, Y, cost="sqeuclidean"):
+    """Per-pair gradients dC_ij/dx_i [n, m, d], written out from the definition of C:
+    2 (x_i - y_j) for the squared Euclidean cost; for the cosine cost,
+    d/dx (1 - x.y/(|x| |y|)) = -(y^ - (x^.y^) x^) / |x| (x^ = x/|x|, y^ = y/|y|)."""
+    X = np.asarray(X, dtype=np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+    if cost == "cosine":
+        nx = np.linalg.norm(X, axis=1)
+        Xh, Yh = X / nx[:, None], Y / np.linalg.norm(Y, axis=1)[:, None]
+        s = Xh @ Yh.T
+        return -(Yh[None, :, :] - s[:, :, None] * Xh[:, None, :]) / nx[:, None, None]
+    return 2.0 * (X[:, None, :] - Y[None, :, :])
 
-    The gradient is G_i = 2 sum_j P_ij (x_i - y_j).  Moving X along V changes P
-    directly through C (dC_ij = 2 (x_i - y_j).v_i) and through the potentials,
-    whose response (df, dg) keeps both marginals fixed:
+
+def cost_hess_x(X, Y, V, cost="sqeuclidean"):
+    """Per-pair Hessian-vector products (d^2 C_ij/dx_i^2) v_i [n, m, d].  Squared
+    Euclidean: 2 v_i.  Cosine, differentiating the gradient above once more
+    along v (s = x^.y^, |x| = rho):
+      [ (y^.v) x^ + s v + (x^.v) y^ - 3 s (x^.v) x^ ] / rho^2."""
+    X = np.asarray(X, dtype=np.float64)
+    Y = np.asarray(Y, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    n, m = X.shape[0], Y.shape[0]
+    if cost == "cosine":
+        nx = np.linalg.norm(X, axis=1)
+        Xh, Yh = X / nx[:, None], Y / np.linalg.norm(Y, axis=1)[:, None]
+        s = Xh @ Yh.T                                  # [n, m]
+        yv = V @ Yh.T                                  # y^_j . v_i
+        xv = np.sum(Xh * V, axis=1)                    # x^_i . v_i
+        H = (yv[:, :, None] * Xh[:, None, :] + s[:, :, None] * V[:, None, :] +
+             xv[:, None, None] * Yh[None, :, :] - 3.0 * (s * xv[:, None])[:, :, None] * Xh[:, None, :])
+        return H / (nx ** 2)[:, None, None]
+    return np.broadcast_to(2.0 * V[:, None, :], (n, m, X.shape[1])).copy()
+
+
+def hvp_x(X, Y, loga, logb, f, g, eps, V, cost="sqeuclidean"):
+    """Hessian-vector product of the entropic OT cost with respect to the positions X
+    at optimal potentials (f, g), in direction V [n, d].
+
+    The gradient is G_i = sum_j P_ij D_ij, D_ij = dC_ij/dx_i (2 (x_i - y_j) for
+    the squared Euclidean cost).  Moving X along V changes P directly through C
+    (dC_ij = D_ij.v_i) and through the potentials, whose response (df, dg) keeps
+    both marginals fixed:
         r_i df_i + (P dg)_i   = sum_j P_ij dC_ij
         (P^T df)_j + c_j dg_j = sum_i P_ij dC_ij
     (a singular system: (k, -k) is free and does not change the result).  Then
-        dG_i = 2 r_i v_i + (2/eps) sum_j P_ij (df_i + dg_j - dC_ij)(x_i - y_j).
-    Everything here is dense (tiny inputs only): P materialised, the linear
-    system solved by least squares.
+        dG_i = sum_j P_ij (d^2 C_ij/dx_i^2) v_i + (1/eps) sum_j P_ij (df_i + dg_j - dC_ij) D_ij
+    (2 r_i v_i for the first sum at the squared Euclidean cost).  Everything here
+    is dense (tiny inputs only): P and the per-pair derivatives materialised,
+    the linear system solved by least squares.
     """
     X = np.asarray(X, dtype=np.float64)
     Y = np.asarray(Y, dtype=np.float64)
     V = np.asarray(V, dtype=np.float64)
-    P = plan(cost_matrix(X, Y), np.asarray(loga, float), np.asarray(logb, float), np.asarray(f, float),
+    P = plan(cost_matrix(X, Y, cost), np.asarray(loga, float), np.asarray(logb, float), np.asarray(f, float),
              np.asarray(g, float), eps)
     n, m = P.shape
-    D = X[:, None, :] - Y[None, :, :]                 # x_i - y_j
-    dC = 2.0 * np.einsum("ijk,ik->ij", D, V)          # 2 (x_i - y_j).v_i
+    D = cost_grad_x(X, Y, cost)
+    dC = np.einsum("ijk,ik->ij", D, V)
     r, c = P.sum(axis=1), P.sum(axis=0)
     A = np.zeros((n + m, n + m))
     A[:n, :n] = np.diag(r)
@@ -135,4 +172,4 @@ def hvp_x(X, Y, loga, logb, f, g, eps, V):
     sol = np.linalg.lstsq(A, rhs, rcond=None)[0]
     df, dg = sol[:n], sol[n:]
     W = P * (df[:, None] + dg[None, :] - dC)
-    return 2.0 * r[:, None] * V + (2.0 / eps) * np.einsum("ij,ijk->ik", W, D)
+    return np.einsum("ij,ijk->ik", P, cost_hess_x(X, Y, V, cost)) + np.einsum("ij,ijk->ik", W, D) / eps

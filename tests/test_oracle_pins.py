@@ -337,7 +337,8 @@ def test_transport_apply_matches_dense_plan(cost):
     np.testing.assert_allclose(ones[:, 0], oracle.marginals(X, Y, loga, logb, f, g, eps, cost=cost)[0], rtol=1e-12)
 
 
-def test_grad_x_matches_finite_differences_of_the_optimal_value():
+@pytest.mark.parametrize("cost", ["sqeuclidean", "cosine"])
+def test_grad_x_matches_finite_differences_of_the_optimal_value(cost):
     """At optimal potentials the entropic OT value (the dual) has gradient
     sum_j P_ij dC_ij/dx_i with respect to x_i (envelope theorem)."""
     rng = np.random.default_rng(72)
@@ -349,11 +350,11 @@ def test_grad_x_matches_finite_differences_of_the_optimal_value():
     loga, logb = np.log(a / a.sum()), np.log(b / b.sum())
 
     def value(Xv):
-        f, g = oracle.solve(Xv, Y, loga, logb, eps, 400)
-        return oracle.costs(Xv, Y, loga, logb, f, g, eps)["dual"], f, g
+        f, g = oracle.solve(Xv, Y, loga, logb, eps, 400, cost=cost)
+        return oracle.costs(Xv, Y, loga, logb, f, g, eps, cost=cost)["dual"], f, g
 
     _, f, g = value(X)
-    G = oracle.grad_x(X, Y, loga, logb, f, g, eps)
+    G = oracle.grad_x(X, Y, loga, logb, f, g, eps, cost=cost)
     h = 1e-5
     for i in range(n):
         for k in range(d):
@@ -379,7 +380,8 @@ def test_barycentric_projection_tends_to_the_optimal_assignment():
     assert np.abs(T - Y[cols]).max() < 1e-2
 
 
-def test_grad_y_matches_finite_differences_of_the_optimal_value():
+@pytest.mark.parametrize("cost", ["sqeuclidean", "cosine"])
+def test_grad_y_matches_finite_differences_of_the_optimal_value(cost):
     rng = np.random.default_rng(73)
     n, m, d, eps = 5, 6, 2, 0.4
     X = rng.standard_normal((n, d))
@@ -389,11 +391,11 @@ def test_grad_y_matches_finite_differences_of_the_optimal_value():
     loga, logb = np.log(a / a.sum()), np.log(b / b.sum())
 
     def value(Yv):
-        f, g = oracle.solve(X, Yv, loga, logb, eps, 500)
-        return oracle.costs(X, Yv, loga, logb, f, g, eps)["dual"], f, g
+        f, g = oracle.solve(X, Yv, loga, logb, eps, 500, cost=cost)
+        return oracle.costs(X, Yv, loga, logb, f, g, eps, cost=cost)["dual"], f, g
 
     _, f, g = value(Y)
-    G = oracle.grad_y(X, Y, loga, logb, f, g, eps)
+    G = oracle.grad_y(X, Y, loga, logb, f, g, eps, cost=cost)
     h = 1e-5
     for j in range(m):
         for k in range(d):
@@ -407,7 +409,8 @@ def test_grad_y_matches_finite_differences_of_the_optimal_value():
 # ---- streaming HVP (Metodologia section 3: Hessian-vector products of the EOT
 # loss as sequences of transport-vector and transport-matrix products)
 
-def test_hvp_x_matches_finite_differences_of_the_gradient():
+@pytest.mark.parametrize("cost", ["sqeuclidean", "cosine"])
+def test_hvp_x_matches_finite_differences_of_the_gradient(cost):
     """dense.hvp_x against central differences of the gradient at re-converged
     potentials: (G(X + hV) - G(X - hV)) / 2h."""
     rng = np.random.default_rng(74)
@@ -420,24 +423,61 @@ def test_hvp_x_matches_finite_differences_of_the_gradient():
     V = rng.standard_normal((n, d))
 
     def grad(Xv):
-        f, g = oracle.solve(Xv, Y, loga, logb, eps, 800)
-        return oracle.grad_x(Xv, Y, loga, logb, f, g, eps), f, g
+        f, g = oracle.solve(Xv, Y, loga, logb, eps, 800, cost=cost)
+        return oracle.grad_x(Xv, Y, loga, logb, f, g, eps, cost=cost), f, g
 
     _, f, g = grad(X)
-    H = dense.hvp_x(X, Y, loga, logb, f, g, eps, V)
+    H = dense.hvp_x(X, Y, loga, logb, f, g, eps, V, cost=cost)
     h = 1e-5
     fd = (grad(X + h * V)[0] - grad(X - h * V)[0]) / (2 * h)
     np.testing.assert_allclose(H, fd, rtol=1e-6, atol=1e-8)
 
 
-def test_hvp_x_is_symmetric():
+@pytest.mark.parametrize("cost", ["sqeuclidean", "cosine"])
+def test_hvp_x_is_symmetric(cost):
     """<W, H V> = <V, H W>: the Hessian is symmetric."""
     rng = np.random.default_rng(75)
     n, m, d, eps = 6, 8, 2, 0.5
     X = rng.standard_normal((n, d))
     Y = rng.standard_normal((m, d))
     loga, logb = np.full(n, -np.log(n)), np.full(m, -np.log(m))
-    f, g = oracle.solve(X, Y, loga, logb, eps, 800)
+    f, g = oracle.solve(X, Y, loga, logb, eps, 800, cost=cost)
     V, W = rng.standard_normal((n, d)), rng.standard_normal((n, d))
-    assert abs(np.sum(W * dense.hvp_x(X, Y, loga, logb, f, g, eps, V)) -
-               np.sum(V * dense.hvp_x(X, Y, loga, logb, f, g, eps, W))) <= 1e-10
+    assert abs(np.sum(W * dense.hvp_x(X, Y, loga, logb, f, g, eps, V, cost=cost)) -
+               np.sum(V * dense.hvp_x(X, Y, loga, logb, f, g, eps, W, cost=cost))) <= 1e-10
+
+
+@pytest.mark.parametrize("cost", ["sqeuclidean", "cosine"])
+def test_per_pair_cost_derivatives_match_finite_differences(cost):
+    """dense.cost_grad_x and dense.cost_hess_x (the per-pair first and second
+    derivatives the HVP is built from) against central differences of the cost
+    matrix itself and of cost_grad_x."""
+    rng = np.random.default_rng(76)
+    X = rng.standard_normal((4, 3))
+    Y = rng.standard_normal((5, 3))
+    V = rng.standard_normal((4, 3))
+    h = 1e-6
+    D = dense.cost_grad_x(X, Y, cost)
+    for k in range(3):
+        E = np.zeros_like(X)
+        E[:, k] = h
+        fd = (dense.cost_matrix(X + E, Y, cost) - dense.cost_matrix(X - E, Y, cost)) / (2 * h)
+        np.testing.assert_allclose(D[:, :, k], fd, rtol=1e-7, atol=1e-9)
+    fdH = (dense.cost_grad_x(X + h * V, Y, cost) - dense.cost_grad_x(X - h * V, Y, cost)) / (2 * h)
+    np.testing.assert_allclose(dense.cost_hess_x(X, Y, V, cost), fdH, rtol=1e-6, atol=1e-8)
+
+
+def test_cosine_gradient_is_tangent_and_scales_inversely():
+    """The cosine cost depends on x only through x / |x|: its gradient with
+    respect to x_i is orthogonal to x_i, and scaling a point by s > 0 scales its
+    gradient by 1 / s (the potentials do not change)."""
+    rng = np.random.default_rng(77)
+    X = rng.standard_normal((6, 3))
+    Y = rng.standard_normal((7, 3))
+    loga, logb = np.full(6, -np.log(6)), np.full(7, -np.log(7))
+    f, g = oracle.solve(X, Y, loga, logb, 0.3, 500, cost="cosine")
+    G = oracle.grad_x(X, Y, loga, logb, f, g, 0.3, cost="cosine")
+    assert np.abs(np.sum(G * X, axis=1)).max() <= 1e-13
+    s = np.array([0.5, 2.0, 3.0, 1.0, 7.0, 0.25])
+    G2 = oracle.grad_x(X * s[:, None], Y, loga, logb, f, g, 0.3, cost="cosine")
+    np.testing.assert_allclose(G2, G / s[:, None], rtol=1e-12, atol=1e-15)
