@@ -250,11 +250,15 @@ FS_API fs_status fs_transport_apply(fs_handle *h, const float *f, const float *g
  * packed form); out: device fp32 [batch][n][d].  Asynchronous. */
 FS_API fs_status fs_barycentric_map(fs_handle *h, const float *f, const float *g, const void *Y, float *out);
 
-/* Gradient of the entropic OT cost with respect to the positions X at (f, g),
- * squared Euclidean cost: grad_i = sum_j P_ij 2 (x_i - y_j) = 2 (r_i x_i -
- * sum_j P_ij y_j) (at optimal potentials, the gradient of the optimal value).
- * X, Y: the caller's device clouds in the handle's dtype; grad: device fp32
- * [batch][n][d].  FS_ERR_UNSUPPORTED for the cosine cost.  Asynchronous. */
+/* Gradient of the entropic OT cost with respect to the positions X at (f, g):
+ * grad_i = sum_j P_ij dC_ij/dx_i (at optimal potentials, the gradient of the
+ * optimal value).  Squared Euclidean cost: 2 (r_i x_i - sum_j P_ij y_j).
+ * Cosine cost (dC/dx = -(y^ - (x^.y^) x^) / |x|, x^ = x / |x|):
+ * -(b_i - (x^_i.b_i) x^_i) / |x_i| with b_i = sum_j P_ij y^_j, one transport
+ * application of Y's unit rows (an fp32 copy of them is taken from the
+ * device's memory pool for the call).  X, Y: the caller's device clouds in
+ * the handle's dtype (the ones the handle was created from); grad: device
+ * fp32 [batch][n][d].  Asynchronous. */
 FS_API fs_status fs_grad_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
                            float *grad);
 
@@ -265,30 +269,37 @@ FS_API fs_status fs_grad_x(fs_handle *h, const float *f, const float *g, const v
 FS_API fs_status fs_transport_apply_t(fs_handle *h, const float *f, const float *g, const float *U, int du,
                                       float *out, float *c);
 
-/* Gradient of the entropic OT cost with respect to the positions Y at (f, g),
- * squared Euclidean cost: grad_j = sum_i P_ij 2 (y_j - x_i) = 2 (c_j y_j -
- * sum_i P_ij x_i).  With fs_grad_x and the potentials themselves (the
- * gradients with respect to the weights a and b, up to the constant fixed by
- * sum a = sum b = 1) this is the backward pass of the EOT loss.  X, Y: the
- * caller's device clouds in the handle's dtype; grad: device fp32
- * [batch][m][d].  FS_ERR_UNSUPPORTED for the cosine cost.  Asynchronous. */
+/* Gradient of the entropic OT cost with respect to the positions Y at (f, g):
+ * fs_grad_x with the clouds' roles exchanged (both costs are symmetric).
+ * Squared Euclidean cost: 2 (c_j y_j - sum_i P_ij x_i); cosine cost:
+ * -(b_j - (y^_j.b_j) y^_j) / |y_j| with b_j = sum_i P_ij x^_i.  With fs_grad_x
+ * and the potentials themselves (the gradients with respect to the weights a
+ * and b, up to the constant fixed by sum a = sum b = 1) this is the backward
+ * pass of the EOT loss.  X, Y: the caller's device clouds in the handle's
+ * dtype; grad: device fp32 [batch][m][d].  Asynchronous. */
 FS_API fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
                            float *grad);
 
 /*
  * Hessian-vector product of the entropic OT cost with respect to the positions
- * X, squared Euclidean cost, at optimal device potentials (f, g), in the
- * direction V (device fp32 [n][d]); out: device fp32 [n][d].  Streaming
+ * X, at optimal device potentials (f, g), in the
+ * direction V (device fp32 [batch][n][d]); out: device fp32 [batch][n][d].  Streaming
  * ("FlashSinkhorn: IO-aware EOT on GPU", Metodologia section 3): a sequence of
  * transport-vector and transport-matrix products, O((n + m) d) memory.  The
  * potentials' response solves
  *   [diag(c) - P^T diag(1/r) P] dg = w - P^T (u / r)
  * by conjugate gradients (each step one transport-vector product each way),
  * stopped after max_cg_iters steps or when the residual falls below
- * cg_rtol times its start; *cg_iters_done (may be NULL) receives the steps.
- * One problem only (batch = 1).  X, Y: the caller's device clouds in the
- * handle's dtype.  Synchronises the stream once per CG step.
- * Errors: FS_ERR_INVALID_ARG, FS_ERR_UNSUPPORTED (cosine cost, batch > 1).
+ * cg_rtol times its start.  Each problem of a batch runs its own CG (its own
+ * scalars and stopping test; a problem that has converged takes no further
+ * steps while the others continue); *cg_iters_done (may be NULL) receives the
+ * most steps any problem took.  The cosine cost takes the same sequence on
+ * Y's unit rows y^ and the direction's part orthogonal to each x_i, over |x_i|
+ * (its change of C is -y^_j.v~_i), with the second derivative of the cosine
+ * distance in the final combination; its transport-matrix term is always the
+ * column-block form (fs_get_info's last_hvp_fused = 0).  X, Y: the caller's
+ * device clouds in the handle's dtype.  Synchronises the stream once per CG
+ * step.  Errors: FS_ERR_INVALID_ARG, FS_ERR_UNSUPPORTED (batch > 65535).
  */
 FS_API fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
                           const float *V, float *out, int max_cg_iters, double cg_rtol, int *cg_iters_done);

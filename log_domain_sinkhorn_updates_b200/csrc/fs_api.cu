@@ -524,7 +524,7 @@ fs_status hvp_fused_term(fs_handle *h, const float *f, const float *g, const voi
                          bool *done) {
     *done = false;
     const fs_desc &D = h->desc;
-    if (h->prec == FS_PREC_F32_SIMT || h->pair || D.batch != 1 || D.cost != FS_COST_SQEUCLIDEAN) return FS_OK;
+    if (h->prec == FS_PREC_F32_SIMT || h->pair || D.cost != FS_COST_SQEUCLIDEAN) return FS_OK;
     const int umode = fs::hvp_w_mode(h->prec, h->plane_bytes, h->row_bytes);
     if (umode == 0) return FS_OK;
     const bool bf16 = D.dtype == FS_BF16;
@@ -533,16 +533,16 @@ fs_status hvp_fused_term(fs_handle *h, const float *f, const float *g, const voi
     int kslots = 0, stages = 0;
     const size_t smem = fs::hvp_w_plan(h->row_bytes, umode, dv_pad, vpl, &kslots, &stages);
     if (smem == 0 || dv_pad > 256) return FS_OK;
-    const size_t n = (size_t)D.n;
+    const int B = D.batch;
     size_t off = 0;
     auto carve = [&](size_t bytes) {
         const size_t o = off;
         off += align256(bytes);
         return o;
     };
-    const size_t o_u = carve((umode == 2 ? 2 : 1) * (size_t)h->n_pad * h->row_bytes);
-    const size_t o_norm = carve((size_t)h->n_stride * 4);
-    const size_t o_vt = carve((size_t)vpl * dv_pad * h->m_pad * 2);
+    const size_t o_u = carve((umode == 2 ? 2 : 1) * (size_t)B * h->n_pad * h->row_bytes);
+    const size_t o_norm = carve((size_t)B * h->n_stride * 4);
+    const size_t o_vt = carve((size_t)B * vpl * dv_pad * h->m_pad * 2);
     const size_t o_mx = carve(16);
     cudaMemPool_t pool;
     uint8_t *blk = nullptr;
@@ -556,24 +556,24 @@ fs_status hvp_fused_term(fs_handle *h, const float *f, const float *g, const voi
             if (h->pack_mode == fs::kPack3xF16) {  // U's own power-of-two scale, as for X and Y
                 float *mx = reinterpret_cast<float *>(blk + o_mx);
                 float host = 0.f;
-                FS_LAUNCH(h, fs::launch_maxabs(V, false, D.n, D.d, 1, nullptr, mx, s));
+                FS_LAUNCH(h, fs::launch_maxabs(V, false, D.n, D.d, B, nullptr, mx, s));
                 FS_CUDA(h, cudaMemcpyAsync(&host, mx, sizeof(float), cudaMemcpyDeviceToHost, s));
                 FS_CUDA(h, cudaStreamSynchronize(s));
                 if (host > 0.f && std::isfinite(host))
                     uscale = std::ldexp(1.f, 14 - (int)std::ceil(std::log2((double)host)));
             }
-            FS_LAUNCH(h, fs::launch_pack(V, false, D.n, h->n_pad, D.d, 1, nullptr, uscale, h->pack_mode, h->d_p,
+            FS_LAUNCH(h, fs::launch_pack(V, false, D.n, h->n_pad, D.d, B, nullptr, uscale, h->pack_mode, h->d_p,
                                          h->row_elems, blk + o_u, reinterpret_cast<float *>(blk + o_norm), h->n_stride,
                                          h->err, s, false));
         } else {
-            FS_LAUNCH(h, fs::launch_u_split(V, D.n, h->n_pad, D.d, h->row_elems, blk + o_u, s));
+            FS_LAUNCH(h, fs::launch_u_split(V, B, D.n, h->n_pad, D.d, h->row_elems, blk + o_u, s));
         }
-        FS_LAUNCH(h, fs::launch_vt_pack(Y, bf16, 1, D.m, D.d, h->m_pad, dv_pad, vpl, blk + o_vt, s));
+        FS_LAUNCH(h, fs::launch_vt_pack(Y, bf16, B, D.m, D.d, h->m_pad, dv_pad, vpl, blk + o_vt, s));
         CUtensorMap map_u{}, map_v{};
-        fs_status st = encode_map(h, &map_u, blk + o_u, (umode == 2 ? 2 : 1) * h->n_pad, kBlockRows);
+        fs_status st = encode_map(h, &map_u, blk + o_u, (umode == 2 ? 2 : 1) * B * h->n_pad, kBlockRows);
         if (st != FS_OK) return st;
         auto fn = encode_fn();
-        cuuint64_t gdim[2] = {(cuuint64_t)h->m_pad, (cuuint64_t)vpl * dv_pad};
+        cuuint64_t gdim[2] = {(cuuint64_t)h->m_pad, (cuuint64_t)B * vpl * dv_pad};
         cuuint64_t gstride[1] = {(cuuint64_t)h->m_pad * 2};
         cuuint32_t box[2] = {64, (cuuint32_t)dv_pad};
         cuuint32_t estr[2] = {1, 1};
@@ -611,7 +611,7 @@ fs_status hvp_fused_term(fs_handle *h, const float *f, const float *g, const voi
         p.err = h->err;
         // K holds 2 kscale (y - t) and U holds uscale v: v . (y - t) = S' / (2 kscale uscale)
         const float cw = (float)(1.0 / (2.0 * (double)h->kscale * (double)uscale));
-        FS_LAUNCH(h, fs::launch_hvp_w(p, h->prec, umode, vpl, cw, V, bf16 ? nullptr : h->center, &h->mapX_r, &map_u,
+        FS_LAUNCH(h, fs::launch_hvp_w(p, B, h->prec, umode, vpl, cw, V, bf16 ? nullptr : h->center, &h->mapX_r, &map_u,
                                       &h->mapY_r, &map_v, smem, s));
         return FS_OK;
     };
@@ -638,10 +638,34 @@ fs_status fs_barycentric_map(fs_handle *h, const float *f, const float *g, const
     return apply(h, f, g, Y, h->desc.dtype == FS_BF16, h->desc.d, out, nullptr, true);
 }
 
+// Cosine-cost gradient with respect to the `own` cloud (X for the f direction):
+// b = P (other)^ (the transport application of the other cloud's unit rows, from
+// a pool scratch), then grad = -(b - (own^.b) own^) / |own|, row by row.
+static fs_status cosine_grad(fs_handle *h, const float *f, const float *g, const void *own, const void *other, bool fdir,
+                      float *grad) {
+    const fs_desc &D = h->desc;
+    const bool bf16 = D.dtype == FS_BF16;
+    const size_t own_rows = (size_t)D.batch * (fdir ? D.n : D.m), other_rows = (size_t)D.batch * (fdir ? D.m : D.n);
+    FS_CUDA(h, cudaSetDevice(h->device));
+    cudaMemPool_t pool;
+    float *unit = nullptr;
+    FS_CUDA(h, device_pool(h->device, &pool));
+    FS_CUDA(h, cudaMallocFromPoolAsync((void **)&unit, other_rows * D.d * 4, pool, h->stream));
+    auto run = [&]() -> fs_status {
+        FS_LAUNCH(h, fs::cos_unit_rows(other, bf16, other_rows, D.d, unit, h->stream));
+        fs_status st = apply(h, f, g, unit, false, D.d, grad, nullptr, false, fdir);
+        if (st != FS_OK) return st;
+        FS_LAUNCH(h, fs::cos_grad(own, bf16, grad, own_rows, D.d, grad, h->stream));
+        return FS_OK;
+    };
+    const fs_status st = run();
+    cudaFreeAsync(unit, h->stream);
+    return st;
+}
+
 fs_status fs_grad_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y, float *grad) {
     if (!h || !f || !g || !X || !Y || !grad) return fail(h, FS_ERR_INVALID_ARG, "null argument");
-    if (h->desc.cost != FS_COST_SQEUCLIDEAN)
-        return fail(h, FS_ERR_UNSUPPORTED, "fs_grad_x is defined for the squared Euclidean cost");
+    if (h->desc.cost == FS_COST_COSINE) return cosine_grad(h, f, g, X, Y, true, grad);
     const fs_desc &D = h->desc;
     const bool bf16 = D.dtype == FS_BF16;
     fs_status st = apply(h, f, g, Y, bf16, D.d, grad, h->rsum, false);  // grad <- P Y, rsum <- P 1
@@ -658,8 +682,7 @@ fs_status fs_transport_apply_t(fs_handle *h, const float *f, const float *g, con
 
 fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const void *X, const void *Y, float *grad) {
     if (!h || !f || !g || !X || !Y || !grad) return fail(h, FS_ERR_INVALID_ARG, "null argument");
-    if (h->desc.cost != FS_COST_SQEUCLIDEAN)
-        return fail(h, FS_ERR_UNSUPPORTED, "fs_grad_y is defined for the squared Euclidean cost");
+    if (h->desc.cost == FS_COST_COSINE) return cosine_grad(h, f, g, Y, X, false, grad);
     const fs_desc &D = h->desc;
     const bool bf16 = D.dtype == FS_BF16;
     fs_status st = apply(h, f, g, X, bf16, D.d, grad, h->rsum, false, false);  // grad <- P^T X, rsum <- P^T 1
@@ -673,19 +696,28 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     if (!h || !f || !g || !X || !Y || !V || !out || max_cg_iters < 1 || !(cg_rtol > 0.0))
         return fail(h, FS_ERR_INVALID_ARG, "bad argument");
     const fs_desc &D = h->desc;
-    if (D.cost != FS_COST_SQEUCLIDEAN)
-        return fail(h, FS_ERR_UNSUPPORTED, "fs_hvp_x is defined for the squared Euclidean cost");
-    if (D.batch != 1) return fail(h, FS_ERR_UNSUPPORTED, "fs_hvp_x takes one problem (batch = 1)");
+    if (D.batch > 65535) return fail(h, FS_ERR_UNSUPPORTED, "fs_hvp_x takes at most 65535 problems");
     FS_CUDA(h, cudaSetDevice(h->device));
-    const size_t n = (size_t)D.n, m = (size_t)D.m, d = (size_t)D.d;
+    // Each problem of the batch is its own solve, laid out problem after problem:
+    // the row-wise steps run over B n rows (B m columns) at once, the reductions
+    // and the CG scalars are per problem.
+    const int B = D.batch;
+    const size_t n1 = (size_t)D.n, m1 = (size_t)D.m, d = (size_t)D.d;
+    const size_t n = (size_t)B * n1, m = (size_t)B * m1;
+    // The cosine cost runs the same sequence on the unit rows Y^ (fp32) and the
+    // projected direction v~ (fs_cosine.cu), with its own first and last steps.
+    const bool cosine = D.cost == FS_COST_COSINE;
     const bool bf16 = D.dtype == FS_BF16;
     // Columns of y folded into one transport-matrix product (width nq d, fp32):
     // as many as keep the width within 256 and, where the handle's operands
     // suit the tensor-core application, within its shared-memory plan.
     int nq = d >= 256 ? 1 : (int)(256 / d);
-    if (h->prec != FS_PREC_F32_SIMT && !h->pair && h->row_bytes <= 256) {
+    if (h->prec != FS_PREC_F32_SIMT) {
         int ks = 0, stg = 0;
-        while (nq > 1 && fs::apply_tc_plan(h->row_bytes, (nq * (int)d + 15) / 16 * 16, 2, &ks, &stg) == 0) --nq;
+        if (h->pair)  // the CTA-pair application, fp32 columns in two bf16 planes
+            while (nq > 1 && fs::apply_tc2_plan(h->row_bytes, (nq * (int)d + 31) / 32 * 32, 2, &ks, &stg) == 0) --nq;
+        else if (h->row_bytes <= 256)
+            while (nq > 1 && fs::apply_tc_plan(h->row_bytes, (nq * (int)d + 15) / 16 * 16, 2, &ks, &stg) == 0) --nq;
     }
     // scratch, O((n + m) d), from the pool for this call
     size_t off = 0;
@@ -699,64 +731,81 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     const size_t o_res = carve(m), o_p = carve(m), o_Ap = carve(m), o_Pdg = carve(n), o_df = carve(n);
     const size_t o_dgY = carve(m * d), oQ1 = carve(n * d), oMV = carve(n * d), o_ones = carve(n);
     const size_t oVc = carve(m * nq * d), oOc = carve(n * nq * d);
-    const size_t o_part = carve(2 * 4096), o_sc = carve(2 * 8);
+    const size_t o_part = carve((size_t)B * 2 * 4096), o_sc = carve((size_t)B * 2 * 5);
+    const size_t o_Yh = carve(cosine ? m * d : 1), o_Vt = carve(cosine ? n * d : 1);
     cudaMemPool_t pool;
     uint8_t *blk = nullptr;
     FS_CUDA(h, device_pool(h->device, &pool));
     FS_CUDA(h, cudaMallocFromPoolAsync((void **)&blk, off, pool, h->stream));
     auto F = [&](size_t o) { return reinterpret_cast<float *>(blk + o); };
     double *part = reinterpret_cast<double *>(blk + o_part);
-    double *sc = reinterpret_cast<double *>(blk + o_sc);  // [0] rr, [1] p.Ap, [2] rr_new, [3] sum, [4] z.z
+    double *sc = reinterpret_cast<double *>(blk + o_sc);  // [k][B]: k = 0 rr, 1 p.Ap, 2 rr_new, 3 sum, 4 z.z
+    double *rr_d = sc, *pap_d = sc + B, *rrn_d = sc + 2 * B, *sum_d = sc + 3 * B, *zz_d = sc + 4 * B;
+    const double tol2 = cg_rtol * cg_rtol;
     float *PY = F(oPY), *r = F(o_r), *c = F(o_c), *W1 = F(oW1), *Tm = F(oT), *u = F(o_u), *w = F(o_w);
     float *tn = F(o_tn), *tm = F(o_tm), *z = F(o_z), *x = F(o_x), *res = F(o_res), *p = F(o_p), *Ap = F(o_Ap);
     float *Pdg = F(o_Pdg), *df = F(o_df), *dgY = F(o_dgY), *Q1 = F(oQ1), *MV = F(oMV), *ones = F(o_ones);
-    float *Vc = F(oVc), *Oc = F(oOc);
+    float *Vc = F(oVc), *Oc = F(oOc), *Yh = F(o_Yh), *Vt = F(o_Vt);
+    // the column cloud the transport products see (Y, or its unit rows), and the
+    // direction the transport-matrix term contracts with (v, or v~)
+    const void *Yop = cosine ? (const void *)Yh : Y;
+    const bool ybf = cosine ? false : bf16;
+    const float *Vop = cosine ? Vt : V;
     cudaStream_t s = h->stream;
     fs_status st = FS_OK;
     int it = 0;
     auto run = [&]() -> fs_status {
         // transport products that do not depend on the CG solution
-        fs_status s2 = apply(h, f, g, Y, bf16, (int)d, PY, r, false, true);  // P Y, r = P 1
+        if (cosine) FS_LAUNCH(h, fs::cos_unit_rows(Y, bf16, m, (int)d, Yh, s));
+        fs_status s2 = apply(h, f, g, Yop, ybf, (int)d, PY, r, false, true);  // P Y (P Y^), r = P 1
         if (s2 != FS_OK) return s2;
         FS_LAUNCH(h, fs::launch_fill(ones, n, 1.f, s));
         s2 = apply(h, f, g, ones, false, 1, tm, c, false, false);  // c = P^T 1
         if (s2 != FS_OK) return s2;
-        FS_LAUNCH(h, fs::hvp_prep(X, bf16, V, PY, r, (int)n, (int)d, u, W1, s));
-        s2 = apply(h, f, g, W1, false, (int)d + 1, Tm, nullptr, false, false);  // P^T [V | x.v]
+        if (cosine)
+            FS_LAUNCH(h, fs::cos_hvp_prep(X, bf16, V, PY, n, (int)d, u, W1, Vt, s));
+        else
+            FS_LAUNCH(h, fs::hvp_prep(X, bf16, V, PY, r, (int)n, (int)d, u, W1, s));
+        s2 = apply(h, f, g, W1, false, (int)d + 1, Tm, nullptr, false, false);  // P^T [v | x.v] (P^T [v~ | 0])
         if (s2 != FS_OK) return s2;
-        FS_LAUNCH(h, fs::hvp_w(Y, bf16, Tm, (int)m, (int)d, w, s));
+        FS_LAUNCH(h, fs::hvp_w(Yop, ybf, Tm, (int)m, (int)d, cosine ? 1.f : 2.f, w, s));
         FS_LAUNCH(h, fs::hvp_vec(n, u, r, 1.f, nullptr, 0.f, true, tn, s));  // u / r
         s2 = apply(h, f, g, tn, false, 1, tm, nullptr, false, false);        // P^T (u / r)
         if (s2 != FS_OK) return s2;
         FS_LAUNCH(h, fs::hvp_vec(m, w, nullptr, 1.f, tm, -1.f, false, z, s));  // z = w - P^T (u / r)
-        FS_LAUNCH(h, fs::hvp_dot(m, z, nullptr, part, sc + 3, s));
-        FS_LAUNCH(h, fs::hvp_center(m, sc + 3, z, s));
-        // CG on [diag(c) - P^T diag(1/r) P] dg = z, iterates kept orthogonal to 1
+        FS_LAUNCH(h, fs::hvp_dot(B, m1, z, nullptr, part, sum_d, s));
+        FS_LAUNCH(h, fs::hvp_center(B, m1, sum_d, z, s));
+        // CG on [diag(c) - P^T diag(1/r) P] dg = z, iterates kept orthogonal to 1;
+        // a problem stops once rr <= tol2 z.z, the others run on
         FS_CUDA(h, cudaMemsetAsync(x, 0, m * 4, s));
         FS_CUDA(h, cudaMemcpyAsync(res, z, m * 4, cudaMemcpyDeviceToDevice, s));
         FS_CUDA(h, cudaMemcpyAsync(p, z, m * 4, cudaMemcpyDeviceToDevice, s));
-        FS_LAUNCH(h, fs::hvp_dot(m, z, z, part, sc + 0, s));
-        FS_LAUNCH(h, fs::hvp_dot(m, z, z, part, sc + 4, s));
-        double host[5];
-        FS_CUDA(h, cudaMemcpyAsync(host, sc, 5 * 8, cudaMemcpyDeviceToHost, s));
+        FS_LAUNCH(h, fs::hvp_dot(B, m1, z, z, part, rr_d, s));
+        FS_LAUNCH(h, fs::hvp_dot(B, m1, z, z, part, zz_d, s));
+        std::vector<double> rr((size_t)B), zz((size_t)B);
+        FS_CUDA(h, cudaMemcpyAsync(rr.data(), rr_d, (size_t)B * 8, cudaMemcpyDeviceToHost, s));
+        FS_CUDA(h, cudaMemcpyAsync(zz.data(), zz_d, (size_t)B * 8, cudaMemcpyDeviceToHost, s));
         FS_CUDA(h, cudaStreamSynchronize(s));
-        const double zz = host[4];
-        double rr = host[0];
-        while (it < max_cg_iters && rr > cg_rtol * cg_rtol * zz && zz > 0.0) {
+        auto any_running = [&]() {
+            for (int b = 0; b < B; ++b)
+                if (rr[b] > tol2 * zz[b] && zz[b] > 0.0) return true;
+            return false;
+        };
+        while (it < max_cg_iters && any_running()) {
             s2 = apply(h, f, g, p, false, 1, tn, nullptr, false, true);  // P p
             if (s2 != FS_OK) return s2;
             FS_LAUNCH(h, fs::hvp_vec(n, tn, r, 1.f, nullptr, 0.f, true, tn, s));  // / r
             s2 = apply(h, f, g, tn, false, 1, tm, nullptr, false, false);       // P^T (P p / r)
             if (s2 != FS_OK) return s2;
             FS_LAUNCH(h, fs::hvp_vec(m, p, c, 1.f, tm, -1.f, false, Ap, s));  // c o p - ...
-            FS_LAUNCH(h, fs::hvp_dot(m, Ap, nullptr, part, sc + 3, s));
-            FS_LAUNCH(h, fs::hvp_center(m, sc + 3, Ap, s));
-            FS_LAUNCH(h, fs::hvp_dot(m, p, Ap, part, sc + 1, s));
-            FS_LAUNCH(h, fs::hvp_cg_step(m, sc + 0, sc + 1, p, Ap, x, res, s));
-            FS_LAUNCH(h, fs::hvp_dot(m, res, res, part, sc + 2, s));
-            FS_LAUNCH(h, fs::hvp_cg_dir(m, sc + 2, sc + 0, res, p, s));
-            FS_CUDA(h, cudaMemcpyAsync(sc + 0, sc + 2, 8, cudaMemcpyDeviceToDevice, s));
-            FS_CUDA(h, cudaMemcpyAsync(&rr, sc + 2, 8, cudaMemcpyDeviceToHost, s));
+            FS_LAUNCH(h, fs::hvp_dot(B, m1, Ap, nullptr, part, sum_d, s));
+            FS_LAUNCH(h, fs::hvp_center(B, m1, sum_d, Ap, s));
+            FS_LAUNCH(h, fs::hvp_dot(B, m1, p, Ap, part, pap_d, s));
+            FS_LAUNCH(h, fs::hvp_cg_step(B, m1, rr_d, pap_d, zz_d, tol2, p, Ap, x, res, s));
+            FS_LAUNCH(h, fs::hvp_dot(B, m1, res, res, part, rrn_d, s));
+            FS_LAUNCH(h, fs::hvp_cg_dir(B, m1, rrn_d, rr_d, zz_d, tol2, res, p, s));
+            FS_CUDA(h, cudaMemcpyAsync(rr_d, rrn_d, (size_t)B * 8, cudaMemcpyDeviceToDevice, s));
+            FS_CUDA(h, cudaMemcpyAsync(rr.data(), rrn_d, (size_t)B * 8, cudaMemcpyDeviceToHost, s));
             FS_CUDA(h, cudaStreamSynchronize(s));
             ++it;
         }
@@ -766,7 +815,7 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
         FS_LAUNCH(h, fs::hvp_vec(n, u, nullptr, 1.f, Pdg, -1.f, false, df, s));
         FS_LAUNCH(h, fs::hvp_vec(n, df, r, 1.f, nullptr, 0.f, true, df, s));
         // P (dg o Y)
-        FS_LAUNCH(h, fs::hvp_dgy(Y, bf16, x, (int)m, (int)d, dgY, s));
+        FS_LAUNCH(h, fs::hvp_dgy(Yop, ybf, x, (int)m, (int)d, dgY, s));
         s2 = apply(h, f, g, dgY, false, (int)d, Q1, nullptr, false, true);
         if (s2 != FS_OK) return s2;
         // sum_j P_ij (y_j.v_i) y_j: in one fused pass where the handle's operands
@@ -782,13 +831,16 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
             FS_CUDA(h, cudaMemsetAsync(MV, 0, n * d * 4, s));
             for (int k0 = 0; k0 < (int)d; k0 += nq) {
                 const int q = (int)d - k0 < nq ? (int)d - k0 : nq;
-                FS_LAUNCH(h, fs::hvp_ychunk(Y, bf16, (int)m, (int)d, k0, q, Vc, s));
+                FS_LAUNCH(h, fs::hvp_ychunk(Yop, ybf, (int)m, (int)d, k0, q, Vc, s));
                 s2 = apply(h, f, g, Vc, false, q * (int)d, Oc, nullptr, false, true);
                 if (s2 != FS_OK) return s2;
-                FS_LAUNCH(h, fs::hvp_mv_acc(V, Oc, (int)n, (int)d, k0, q, MV, s));
+                FS_LAUNCH(h, fs::hvp_mv_acc(Vop, Oc, (int)n, (int)d, k0, q, MV, s));
             }
         }
-        FS_LAUNCH(h, fs::hvp_final(X, bf16, V, PY, r, df, Pdg, Q1, MV, (int)n, (int)d, D.eps, out, s));
+        if (cosine)
+            FS_LAUNCH(h, fs::cos_hvp_final(X, bf16, V, PY, df, Q1, MV, n, (int)d, D.eps, out, s));
+        else
+            FS_LAUNCH(h, fs::hvp_final(X, bf16, V, PY, r, df, Pdg, Q1, MV, (int)n, (int)d, D.eps, out, s));
         return FS_OK;
     };
     st = run();

@@ -12,6 +12,11 @@
 //   [diag(c) - P^T diag(1/r) P] dg = w - P^T (u / r),   df = (u - P dg) / r
 //   (H V)_i = 2 r_i v_i + (2/eps) [ df_i (r_i x_i - (P Y)_i) + (P dg)_i x_i - (P (dg o Y))_i
 //             - 2 ( (x_i.v_i)(r_i x_i - (P Y)_i) - x_i ((P Y)_i.v_i) + sum_j P_ij (y_j.v_i) y_j ) ]
+//
+// A batch of independent problems is laid out problem after problem ([batch][n]
+// and [batch][n][d]), so the row-wise kernels run over batch x n rows as they
+// are; the reductions and the conjugate-gradient updates take one problem per
+// blockIdx.y, each with its own scalars.
 #include <cuda_bf16.h>
 
 #include "fs_internal.cuh"
@@ -54,13 +59,14 @@ __global__ void prep_kernel(const T *X, const float *V, const float *PY, const f
     }
 }
 
-// w_j = 2 (T_j[d] - y_j . T_j[0:d]),  T = P^T W1  ([m][d+1])
+// w_j = alpha (T_j[d] - y_j . T_j[0:d]),  T = P^T W1  ([m][d+1]); alpha = 2 for the
+// squared Euclidean cost (W1 = [v | x.v]), 1 for the cosine cost (W1 = [v~ | 0], Y = Y^)
 template <typename T>
-__global__ void w_kernel(const T *Y, const float *Tm, int m, int d, float *w) {
+__global__ void w_kernel(const T *Y, const float *Tm, int m, int d, float alpha, float *w) {
     GRID_LOOP(j, (size_t)m) {
         float s = 0.f;
         for (int k = 0; k < d; ++k) s = fmaf(ldv(Y, j * d + k), Tm[j * (d + 1) + k], s);
-        w[j] = 2.f * (Tm[j * (d + 1) + d] - s);
+        w[j] = alpha * (Tm[j * (d + 1) + d] - s);
     }
 }
 
@@ -74,52 +80,73 @@ __global__ void vec_kernel(size_t n, const float *x, const float *a, float alpha
     }
 }
 
-// Deterministic dot product: fixed-order block trees, then one block over the partials.
-__global__ void dot_partial_kernel(size_t n, const float *x, const float *y, double *part) {
+// Problem b = blockIdx.y owns the segment [b len, (b + 1) len) of every vector.
+#define SEG_LOOP(i, len) for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < (len); i += (size_t)gridDim.x * blockDim.x)
+
+// Deterministic per-problem dot products: fixed-order block trees over each
+// problem's segment (part[b][blockIdx.x]), then one block per problem over its partials.
+__global__ void dot_partial_kernel(size_t len, const float *x, const float *y, double *part) {
     __shared__ double sh[256];
+    const size_t base = (size_t)blockIdx.y * len;
     double s = 0.0;
-    GRID_LOOP(i, n) s += (double)x[i] * (double)(y ? y[i] : 1.f);
+    SEG_LOOP(i, len) s += (double)x[base + i] * (double)(y ? y[base + i] : 1.f);
     sh[threadIdx.x] = s;
     __syncthreads();
     for (int k = 128; k > 0; k >>= 1) {
         if ((int)threadIdx.x < k) sh[threadIdx.x] += sh[threadIdx.x + k];
         __syncthreads();
     }
-    if (threadIdx.x == 0) part[blockIdx.x] = sh[0];
+    if (threadIdx.x == 0) part[(size_t)blockIdx.y * gridDim.x + blockIdx.x] = sh[0];
 }
 __global__ void dot_final_kernel(int nb, const double *part, double *out) {
     __shared__ double sh[256];
+    const double *pb = part + (size_t)blockIdx.x * nb;
     double s = 0.0;
-    for (int i = threadIdx.x; i < nb; i += 256) s += part[i];
+    for (int i = threadIdx.x; i < nb; i += 256) s += pb[i];
     sh[threadIdx.x] = s;
     __syncthreads();
     for (int k = 128; k > 0; k >>= 1) {
         if ((int)threadIdx.x < k) sh[threadIdx.x] += sh[threadIdx.x + k];
         __syncthreads();
     }
-    if (threadIdx.x == 0) *out = sh[0];
+    if (threadIdx.x == 0) out[blockIdx.x] = sh[0];
 }
 
-// x -= s / n (s: a device double), keeping CG iterates orthogonal to the constant vector
-__global__ void center_vec_kernel(size_t n, const double *s, float *x) {
-    const float mean = (float)(*s / (double)n);
-    GRID_LOOP(i, n) x[i] -= mean;
+// x_b -= s_b / len (s: device doubles, one per problem), keeping each problem's
+// CG iterates orthogonal to the constant vector
+__global__ void center_vec_kernel(size_t len, const double *s, float *x) {
+    const size_t base = (size_t)blockIdx.y * len;
+    const float mean = (float)(s[blockIdx.y] / (double)len);
+    SEG_LOOP(i, len) x[base + i] -= mean;
+}
+
+// A problem's CG is still running while rr > tol2 zz (zz = z.z, the right-hand
+// side's square norm); the host's loop test is the same comparison.
+__device__ __forceinline__ bool cg_active(const double *rr, const double *zz, double tol2, int b) {
+    return rr[b] > tol2 * zz[b] && zz[b] > 0.0;
 }
 
 // CG update on the device, from device scalars rr (r.r) and pap (p.Ap):
-//   alpha = rr / pap;  x += alpha p;  res -= alpha Ap
-__global__ void cg_step_kernel(size_t n, const double *rr, const double *pap, const float *p, const float *Ap,
-                               float *x, float *res) {
-    const float alpha = (float)(*rr / *pap);
-    GRID_LOOP(i, n) {
-        x[i] = fmaf(alpha, p[i], x[i]);
-        res[i] = fmaf(-alpha, Ap[i], res[i]);
+//   alpha = rr / pap;  x += alpha p;  res -= alpha Ap   (problems still running)
+__global__ void cg_step_kernel(size_t len, const double *rr, const double *pap, const double *zz, double tol2,
+                               const float *p, const float *Ap, float *x, float *res) {
+    const int b = blockIdx.y;
+    if (!cg_active(rr, zz, tol2, b)) return;
+    const size_t base = (size_t)b * len;
+    const float alpha = (float)(rr[b] / pap[b]);
+    SEG_LOOP(i, len) {
+        x[base + i] = fmaf(alpha, p[base + i], x[base + i]);
+        res[base + i] = fmaf(-alpha, Ap[base + i], res[base + i]);
     }
 }
-// p = res + (rr_new / rr) p
-__global__ void cg_dir_kernel(size_t n, const double *rr_new, const double *rr, const float *res, float *p) {
-    const float beta = (float)(*rr_new / *rr);
-    GRID_LOOP(i, n) p[i] = fmaf(beta, p[i], res[i]);
+// p = res + (rr_new / rr) p   (problems still running, judged on rr before the step)
+__global__ void cg_dir_kernel(size_t len, const double *rr_new, const double *rr, const double *zz, double tol2,
+                              const float *res, float *p) {
+    const int b = blockIdx.y;
+    if (!cg_active(rr, zz, tol2, b)) return;
+    const size_t base = (size_t)b * len;
+    const float beta = (float)(rr_new[b] / rr[b]);
+    SEG_LOOP(i, len) p[base + i] = fmaf(beta, p[base + i], res[base + i]);
 }
 
 // out_jk = dg_j y_jk
@@ -179,11 +206,11 @@ cudaError_t hvp_prep(const void *X, bool bf16, const float *V, const float *PY, 
         prep_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const float *>(X), V, PY, r, n, d, u, W1);
     return cudaGetLastError();
 }
-cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float *w, cudaStream_t s) {
+cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float alpha, float *w, cudaStream_t s) {
     if (bf16)
-        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), Tm, m, d, w);
+        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), Tm, m, d, alpha, w);
     else
-        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const float *>(Y), Tm, m, d, w);
+        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const float *>(Y), Tm, m, d, alpha, w);
     return cudaGetLastError();
 }
 cudaError_t hvp_vec(size_t n, const float *x, const float *a, float alpha, const float *y, float beta, bool div,
@@ -191,24 +218,28 @@ cudaError_t hvp_vec(size_t n, const float *x, const float *a, float alpha, const
     vec_kernel<<<blocks_for(n), 256, 0, s>>>(n, x, a, alpha, y, beta, div, out);
     return cudaGetLastError();
 }
-// *out = x.y (y null: sum of x); part holds at least 4096 doubles.
-cudaError_t hvp_dot(size_t n, const float *x, const float *y, double *part, double *out, cudaStream_t s) {
-    const int nb = blocks_for(n);
-    dot_partial_kernel<<<nb, 256, 0, s>>>(n, x, y, part);
-    dot_final_kernel<<<1, 256, 0, s>>>(nb, part, out);
+// out[b] = x_b.y_b (y null: sum of x_b) for the batch problems' segments of
+// length len; part holds at least batch x 4096 doubles.
+cudaError_t hvp_dot(int batch, size_t len, const float *x, const float *y, double *part, double *out,
+                    cudaStream_t s) {
+    const int nb = blocks_for(len);
+    dot_partial_kernel<<<dim3(nb, batch), 256, 0, s>>>(len, x, y, part);
+    dot_final_kernel<<<batch, 256, 0, s>>>(nb, part, out);
+    count_launches(1);  // the caller's launch macro counts the first
     return cudaGetLastError();
 }
-cudaError_t hvp_center(size_t n, const double *sum, float *x, cudaStream_t s) {
-    center_vec_kernel<<<blocks_for(n), 256, 0, s>>>(n, sum, x);
+cudaError_t hvp_center(int batch, size_t len, const double *sum, float *x, cudaStream_t s) {
+    center_vec_kernel<<<dim3(blocks_for(len), batch), 256, 0, s>>>(len, sum, x);
     return cudaGetLastError();
 }
-cudaError_t hvp_cg_step(size_t n, const double *rr, const double *pap, const float *p, const float *Ap, float *x,
-                        float *res, cudaStream_t s) {
-    cg_step_kernel<<<blocks_for(n), 256, 0, s>>>(n, rr, pap, p, Ap, x, res);
+cudaError_t hvp_cg_step(int batch, size_t len, const double *rr, const double *pap, const double *zz, double tol2,
+                        const float *p, const float *Ap, float *x, float *res, cudaStream_t s) {
+    cg_step_kernel<<<dim3(blocks_for(len), batch), 256, 0, s>>>(len, rr, pap, zz, tol2, p, Ap, x, res);
     return cudaGetLastError();
 }
-cudaError_t hvp_cg_dir(size_t n, const double *rr_new, const double *rr, const float *res, float *p, cudaStream_t s) {
-    cg_dir_kernel<<<blocks_for(n), 256, 0, s>>>(n, rr_new, rr, res, p);
+cudaError_t hvp_cg_dir(int batch, size_t len, const double *rr_new, const double *rr, const double *zz, double tol2,
+                       const float *res, float *p, cudaStream_t s) {
+    cg_dir_kernel<<<dim3(blocks_for(len), batch), 256, 0, s>>>(len, rr_new, rr, zz, tol2, res, p);
     return cudaGetLastError();
 }
 cudaError_t hvp_dgy(const void *Y, bool bf16, const float *dg, int m, int d, float *out, cudaStream_t s) {

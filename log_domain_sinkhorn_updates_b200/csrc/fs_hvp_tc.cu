@@ -24,6 +24,11 @@
 // Warp roles as in the transport kernel: warp 0 lane 0 streams Q, U, K and
 // the bias slices, lane 1 the Y~ halves; warp 1 allocates TMEM and issues the
 // MMAs; warps 2..9 are the two softmax groups.  Every wait is bounded.
+//
+// A batch of independent problems runs as blockIdx.z: problem bz's rows of
+// Q and U start at bz rows_pad (U's hi and lo tiles are each batch x rows_pad
+// rows), its K rows at bz cols_rows, its Y~ planes at bz vpl dv_pad, its
+// centre at bz d.
 #include <cuda_bf16.h>
 
 #include "fs_tc_common.cuh"
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rb = blockIdx.x;
+    const int rb = blockIdx.x, bz = blockIdx.z;
     const int ntiles = (p.cols + kWTS - 1) / kWTS;
     const int njobs = 2 * ntiles;
     const uint32_t tmem_cols = 512u;  // [S | S'] x 2 jobs in [0, 256), O' from 256
@@ -143,10 +148,11 @@ __global__ void __launch_bounds__(kWThreads, 1)
             int k_issued = 0, b_issued = 0;
             mbar_expect_tx(qfull, (uint32_t)(1 + kUTiles) * kBlockRows * kRowBytes);
             for (int a = 0; a < kAtoms; ++a) {
-                tma_load_2d(saddr(sQ) + a * kBlockRows * kSwz, &map_q, saddr(qfull), a * box_inner, rb * kBlockRows);
+                tma_load_2d(saddr(sQ) + a * kBlockRows * kSwz, &map_q, saddr(qfull), a * box_inner,
+                            bz * p.rows_pad + rb * kBlockRows);
                 for (int u = 0; u < kUTiles; ++u)
                     tma_load_2d(saddr(sU) + (u * kAtoms + a) * kBlockRows * kSwz, &map_u, saddr(qfull), a * box_inner,
-                                u * p.rows_pad + rb * kBlockRows);
+                                (u * (int)gridDim.z + bz) * p.rows_pad + rb * kBlockRows);
             }
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int col0 = t * kWTS;
@@ -158,7 +164,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
                         break;
                     }
                     mbar_expect_tx(kfull + s, kslot_bytes);
-                    tma_load_2d(saddr(sK + (size_t)s * kslot_bytes), &map_k, saddr(kfull + s), a * box_inner, col0);
+                    tma_load_2d(saddr(sK + (size_t)s * kslot_bytes), &map_k, saddr(kfull + s), a * box_inner,
+                                bz * p.cols_rows + col0);
                     k_issued = i + 1;
                 }
                 if (!ok) break;
@@ -168,7 +175,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
                     break;
                 }
                 mbar_expect_tx(bfull + j, kWTS * 4);
-                bulk_load(saddr(sBias + j * kWTS), p.col_bias + col0, kWTS * 4, saddr(bfull + j));
+                bulk_load(saddr(sBias + j * kWTS), p.col_bias + (size_t)bz * p.cols_stride + col0, kWTS * 4,
+                          saddr(bfull + j));
                 b_issued = t + 1;
             }
             if (!ok) {
@@ -193,7 +201,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
                 uint8_t *sv = sSt + (size_t)s * L.stage + 2 * kWPBytes;
                 mbar_expect_tx(vfull + s, (uint32_t)VPL * vplane_bytes);
                 for (int pl = 0; pl < VPL; ++pl)
-                    tma_load_2d(saddr(sv + pl * vplane_bytes), &map_v, saddr(vfull + s), jb * kWJ, pl * p.dv_pad);
+                    tma_load_2d(saddr(sv + pl * vplane_bytes), &map_v, saddr(vfull + s), jb * kWJ,
+                                (bz * VPL + pl) * p.dv_pad);
                 v_issued = jb + 1;
             }
             if (!ok) {
@@ -294,12 +303,14 @@ __global__ void __launch_bounds__(kWThreads, 1)
         const int rl = q * 32 + lane;
         const int row = rb * kBlockRows + rl;
         const bool valid = row < p.rows;
-        const float alpha = valid ? (float)(((double)p.pot_row[row] - (double)p.row_norm[row]) * p.scale) : -INFINITY;
+        const size_t grow = (size_t)bz * p.rows + row;         // row in [batch][rows] arrays
+        const size_t prow = (size_t)bz * p.rows_stride + row;  // row in the handle's padded per-point arrays
+        const float alpha = valid ? (float)(((double)p.pot_row[grow] - (double)p.row_norm[prow]) * p.scale) : -INFINITY;
         const float c = (float)(p.scale * (double)p.sscale);
         // w_ij = S'_ij cw + v_i . t (t: the centre the operands are packed around)
         float bw = 0.f;
         if (valid && center)
-            for (int k = 0; k < p.d; ++k) bw = fmaf(dirv[(size_t)row * p.d + k], center[k], bw);
+            for (int k = 0; k < p.d; ++k) bw = fmaf(dirv[grow * p.d + k], center[(size_t)bz * p.d + k], bw);
         const uint64_t cc = pack2(c, c), aa = pack2(alpha, alpha), cwp = pack2(cw, cw), bwp = pack2(bw, bw);
         const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
         const uint32_t prow_off = (uint32_t)((rl >> 3) * 1024 + (rl & 7) * 128);
@@ -383,14 +394,14 @@ __global__ void __launch_bounds__(kWThreads, 1)
         if (grp == 0) {
             const bool done = mbar_wait(ofull, 0, p.timeout_ns) && !*abort_flag;
             tc_fence_after();
-            const float a_i = valid ? (float)exp2((double)p.row_logw2[row]) : 0.f;
+            const float a_i = valid ? (float)exp2((double)p.row_logw2[prow]) : 0.f;
             for (int c0 = 0; c0 < p.dv_pad; c0 += 32) {
                 uint32_t o[32];
                 tmem_ld32(lane_base + 256u + (uint32_t)c0, o);
                 tmem_ld_wait();
                 if (done && valid)
                     for (int k = 0; k < 32 && c0 + k < p.dv; ++k)
-                        p.out[(size_t)row * p.dv + c0 + k] = __uint_as_float(o[k]) * a_i;
+                        p.out[grow * p.dv + c0 + k] = __uint_as_float(o[k]) * a_i;
             }
         }
     }
@@ -404,13 +415,16 @@ __global__ void __launch_bounds__(kWThreads, 1)
     }
 }
 
-// U = bf16 hi and lo tiles of the direction: out[0][r][k] = bf16(v), out[1][r][k] =
-// bf16(v - hi), rows r < rows_pad, row_elems per row (zero beyond d and rows).
-__global__ void u_split_kernel(const float *V, int rows, int rows_pad, int d, int row_elems, __nv_bfloat16 *out) {
-    const size_t total = (size_t)rows_pad * row_elems;
+// U = bf16 hi and lo tiles of the direction V [batch][rows][d]: out[0][bz][r][k] =
+// bf16(v), out[1][bz][r][k] = bf16(v - hi), rows r < rows_pad, row_elems per row
+// (zero beyond d and rows).
+__global__ void u_split_kernel(const float *V, int batch, int rows, int rows_pad, int d, int row_elems,
+                               __nv_bfloat16 *out) {
+    const size_t total = (size_t)batch * rows_pad * row_elems;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
-        const int r = (int)(i / row_elems), k = (int)(i % row_elems);
-        const float v = (r < rows && k < d) ? V[(size_t)r * d + k] : 0.f;
+        const size_t rr = i / row_elems;
+        const int bz = (int)(rr / rows_pad), r = (int)(rr % rows_pad), k = (int)(i % row_elems);
+        const float v = (r < rows && k < d) ? V[((size_t)bz * rows + r) * d + k] : 0.f;
         const __nv_bfloat16 h = __float2bfloat16_rn(v);
         out[i] = h;
         out[total + i] = __float2bfloat16_rn(v - __bfloat162float(h));
@@ -418,20 +432,20 @@ __global__ void u_split_kernel(const float *V, int rows, int rows_pad, int d, in
 }
 
 template <int KIND, int NPASS, int KS, int UMODE>
-cudaError_t launch_w(const ApplyParams &p, int vpl, float cw, const float *dirv, const float *center,
+cudaError_t launch_w(const ApplyParams &p, int batch, int vpl, float cw, const float *dirv, const float *center,
                      const void *mq, const void *mu, const void *mk, const void *mv, size_t smem, cudaStream_t s) {
     if (vpl == 1) {
         auto kern = hvp_w_kernel<KIND, NPASS, KS, UMODE, 1>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<p.rows_pad / kBlockRows, kWThreads, smem, s>>>(
+        kern<<<dim3(p.rows_pad / kBlockRows, 1, batch), kWThreads, smem, s>>>(
             *static_cast<const CUtensorMap *>(mq), *static_cast<const CUtensorMap *>(mu),
             *static_cast<const CUtensorMap *>(mk), *static_cast<const CUtensorMap *>(mv), p, cw, dirv, center);
     } else {
         auto kern = hvp_w_kernel<KIND, NPASS, KS, UMODE, 2>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<p.rows_pad / kBlockRows, kWThreads, smem, s>>>(
+        kern<<<dim3(p.rows_pad / kBlockRows, 1, batch), kWThreads, smem, s>>>(
             *static_cast<const CUtensorMap *>(mq), *static_cast<const CUtensorMap *>(mu),
             *static_cast<const CUtensorMap *>(mk), *static_cast<const CUtensorMap *>(mv), p, cw, dirv, center);
     }
@@ -471,33 +485,35 @@ size_t hvp_w_plan(int row_bytes, int umode, int dv_pad, int vpl, int *kslots, in
     return 0;
 }
 
-cudaError_t launch_u_split(const float *V, int rows, int rows_pad, int d, int row_elems, void *out, cudaStream_t s) {
-    const size_t total = (size_t)rows_pad * row_elems;
+cudaError_t launch_u_split(const float *V, int batch, int rows, int rows_pad, int d, int row_elems, void *out,
+                           cudaStream_t s) {
+    const size_t total = (size_t)batch * rows_pad * row_elems;
     size_t g = (total + 255) / 256;
     if (g > 148 * 16) g = 148 * 16;
-    u_split_kernel<<<(unsigned)g, 256, 0, s>>>(V, rows, rows_pad, d, row_elems, static_cast<__nv_bfloat16 *>(out));
+    u_split_kernel<<<(unsigned)g, 256, 0, s>>>(V, batch, rows, rows_pad, d, row_elems,
+                                               static_cast<__nv_bfloat16 *>(out));
     return cudaGetLastError();
 }
 
 // prec: 1 = bf16 (umode 2), 3 = 3xTF32, 4 = 3xF16 (umode 1); p: the application's
-// parameters in the f direction (batch 1), p.dv = d, p.out = MV [n][d].
-cudaError_t launch_hvp_w(const ApplyParams &p, int prec, int umode, int vpl, float cw, const float *dirv,
+// parameters in the f direction, p.dv = d, p.out = MV [batch][n][d].
+cudaError_t launch_hvp_w(const ApplyParams &p, int batch, int prec, int umode, int vpl, float cw, const float *dirv,
                          const float *center, const void *map_q, const void *map_u, const void *map_k,
                          const void *map_v, size_t smem, cudaStream_t s) {
     const int ks = p.plane_bytes / 32;
     if (prec == 1 && umode == 2) {
-        if (ks == 1) return launch_w<0, 1, 1, 2>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
-        if (ks == 2) return launch_w<0, 1, 2, 2>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
-        if (ks == 4) return launch_w<0, 1, 4, 2>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
-        if (ks == 8) return launch_w<0, 1, 8, 2>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 1) return launch_w<0, 1, 1, 2>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 2) return launch_w<0, 1, 2, 2>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 4) return launch_w<0, 1, 4, 2>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 8) return launch_w<0, 1, 8, 2>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
     } else if (prec == 4 && umode == 1) {
-        if (ks == 1) return launch_w<2, 3, 1, 1>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
-        if (ks == 2) return launch_w<2, 3, 2, 1>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
-        if (ks == 4) return launch_w<2, 3, 4, 1>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 1) return launch_w<2, 3, 1, 1>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 2) return launch_w<2, 3, 2, 1>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 4) return launch_w<2, 3, 4, 1>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
     } else if (prec == 3 && umode == 1) {
-        if (ks == 1) return launch_w<1, 3, 1, 1>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
-        if (ks == 2) return launch_w<1, 3, 2, 1>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
-        if (ks == 4) return launch_w<1, 3, 4, 1>(p, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 1) return launch_w<1, 3, 1, 1>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 2) return launch_w<1, 3, 2, 1>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
+        if (ks == 4) return launch_w<1, 3, 4, 1>(p, batch, vpl, cw, dirv, center, map_q, map_u, map_k, map_v, smem, s);
     }
     return cudaErrorInvalidValue;
 }

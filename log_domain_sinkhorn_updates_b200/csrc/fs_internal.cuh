@@ -187,14 +187,16 @@ cudaError_t launch_wait_probe(unsigned long long timeout_ns, int *err, cudaStrea
 // Element-wise pieces of the streaming Hessian-vector product (fs_hvp.cu).
 cudaError_t hvp_prep(const void *X, bool bf16, const float *V, const float *PY, const float *r, int n, int d,
                      float *u, float *W1, cudaStream_t s);
-cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float *w, cudaStream_t s);
+cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float alpha, float *w, cudaStream_t s);
 cudaError_t hvp_vec(size_t n, const float *x, const float *a, float alpha, const float *y, float beta, bool div,
                     float *out, cudaStream_t s);
-cudaError_t hvp_dot(size_t n, const float *x, const float *y, double *part, double *out, cudaStream_t s);
-cudaError_t hvp_center(size_t n, const double *sum, float *x, cudaStream_t s);
-cudaError_t hvp_cg_step(size_t n, const double *rr, const double *pap, const float *p, const float *Ap, float *x,
-                        float *res, cudaStream_t s);
-cudaError_t hvp_cg_dir(size_t n, const double *rr_new, const double *rr, const float *res, float *p, cudaStream_t s);
+cudaError_t hvp_dot(int batch, size_t len, const float *x, const float *y, double *part, double *out,
+                    cudaStream_t s);
+cudaError_t hvp_center(int batch, size_t len, const double *sum, float *x, cudaStream_t s);
+cudaError_t hvp_cg_step(int batch, size_t len, const double *rr, const double *pap, const double *zz, double tol2,
+                        const float *p, const float *Ap, float *x, float *res, cudaStream_t s);
+cudaError_t hvp_cg_dir(int batch, size_t len, const double *rr_new, const double *rr, const double *zz, double tol2,
+                       const float *res, float *p, cudaStream_t s);
 cudaError_t hvp_dgy(const void *Y, bool bf16, const float *dg, int m, int d, float *out, cudaStream_t s);
 cudaError_t hvp_ychunk(const void *Y, bool bf16, int m, int d, int k0, int nq, float *Vc, cudaStream_t s);
 cudaError_t hvp_mv_acc(const float *V, const float *Oc, int n, int d, int k0, int nq, float *MV, cudaStream_t s);
@@ -213,10 +215,19 @@ int tc2_max_stages(int row_bytes, bool measure);
 // handle's precision takes (0: none), the plan, the bf16 hi/lo split of U, the launch.
 int hvp_w_mode(int prec, int plane_bytes, int row_bytes);
 size_t hvp_w_plan(int row_bytes, int umode, int dv_pad, int vpl, int *kslots, int *stages);
-cudaError_t launch_u_split(const float *V, int rows, int rows_pad, int d, int row_elems, void *out, cudaStream_t s);
-cudaError_t launch_hvp_w(const ApplyParams &p, int prec, int umode, int vpl, float cw, const float *dirv,
+cudaError_t launch_u_split(const float *V, int batch, int rows, int rows_pad, int d, int row_elems, void *out,
+                           cudaStream_t s);
+cudaError_t launch_hvp_w(const ApplyParams &p, int batch, int prec, int umode, int vpl, float cw, const float *dirv,
                          const float *center, const void *map_q, const void *map_u, const void *map_k,
                          const void *map_v, size_t smem, cudaStream_t s);
+// Cosine-cost derivatives (fs_cosine.cu): unit rows p / |p| (fp32), the gradient
+// -(b - (x^.b) x^) / |x| from b = P Y^, and the HVP's first and last steps.
+cudaError_t cos_unit_rows(const void *P, bool bf16, size_t rows, int d, float *out, cudaStream_t s);
+cudaError_t cos_grad(const void *X, bool bf16, const float *b, size_t rows, int d, float *grad, cudaStream_t s);
+cudaError_t cos_hvp_prep(const void *X, bool bf16, const float *V, const float *b, size_t rows, int d, float *u,
+                         float *W1, float *Vt, cudaStream_t s);
+cudaError_t cos_hvp_final(const void *X, bool bf16, const float *V, const float *b, const float *df, const float *Q1,
+                          const float *MV, size_t rows, int d, float eps, float *out, cudaStream_t s);
 // Record msg as this thread's handle-less error (what fs_last_error(NULL) returns).
 void set_thread_error(const char *msg);
 // Add `count` kernels launched outside fs_api.cu to what fs_kernel_launches reports.

@@ -45,40 +45,117 @@ CASES = {
 PATHS = {"tc": ("0", "1"), "tc_blocked": ("0", "0"), "simt": ("1", "0")}  # (FS_APPLY_SIMT, FS_HVP_FUSED)
 
 
-@pytest.mark.parametrize("path", list(PATHS))
-@pytest.mark.parametrize("name", list(CASES))
-def test_hvp_x_parity(cuda_device, name, path, monkeypatch):
-    import torch
-    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
-    monkeypatch.setenv("FS_HVP_FUSED", PATHS[path][1])
-    import log_domain_sinkhorn_updates_b200 as fs
-    from helpers import device_inputs
-    prob = make_problem(name.split("-")[0], **CASES[name])
-    X, Y, a_d, b_d = device_inputs(prob)
-    Xo, Yo, loga, logb = oracle.problem_arrays(prob, 0)
-    f, g = oracle.solve(Xo, Yo, loga, logb, prob.eps, 400)
-    f32, g32 = f.astype(np.float32), g.astype(np.float32)
-    rng = np.random.default_rng(200)
-    V = rng.standard_normal((prob.n, prob.d)).astype(np.float32)
-    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
-    out = torch.empty(1, prob.n, prob.d, device=cuda_device)
-    its = fs.fs_hvp_x(h, torch.from_numpy(f32[None]).to(cuda_device), torch.from_numpy(g32[None]).to(cuda_device),
-                      X, Y, torch.from_numpy(V[None]).to(cuda_device), out, max_cg_iters=500, cg_rtol=1e-7)
-    fs.fs_sync(h)
-    info = fs.fs_get_info(h)
-    if path != "simt":
-        assert info["last_apply_path"] in ("tc", "tc_pair")
-    assert info["last_hvp_fused"] == (1 if path == "tc" else 0), info
-    H = out.cpu().numpy()[0]
-    Ho = dense.hvp_x(Xo, Yo, loga, logb, f32.astype(np.float64), g32.astype(np.float64), prob.eps,
-                     V.astype(np.float64))
-    P = dense.plan(dense.cost_matrix(Xo, Yo), loga, logb, f32.astype(np.float64), g32.astype(np.float64), prob.eps)
+BATCHED = {
+    # independent problems in one call, each with its own CG: the batched recipe
+    # at d = 32 (3xF16 operands) and the highdim recipe at d = 128 (bf16 operands)
+    "batched-b3": dict(batch=3, n=300, m=260),
+    "highdim-b2": dict(batch=2, n=256, m=240),
+}
+
+
+def _oracle_case(prob, k, cost="sqeuclidean"):
+    Xo, Yo, loga, logb = oracle.problem_arrays(prob, k)
+    f, g = oracle.solve(Xo, Yo, loga, logb, prob.eps, 400, cost=cost)
+    return Xo, Yo, loga, logb, f.astype(np.float32), g.astype(np.float32)
+
+
+def _check_row_bound(path, name, its, H, Xo, Yo, loga, logb, f32, g32, eps, V):
+    Ho = dense.hvp_x(Xo, Yo, loga, logb, f32.astype(np.float64), g32.astype(np.float64), eps, V.astype(np.float64))
+    P = dense.plan(dense.cost_matrix(Xo, Yo), loga, logb, f32.astype(np.float64), g32.astype(np.float64), eps)
     S = (P * dense.cost_matrix(Xo, Yo)).sum(axis=1) * np.abs(V).max(axis=1)
-    bound = 2.0 ** -14 * (2.0 / prob.eps) * S + 2.0 ** -10 * np.abs(Ho).max()
+    bound = 2.0 ** -14 * (2.0 / eps) * S + 2.0 ** -10 * np.abs(Ho).max()
     err = np.abs(H - Ho).max()
     rowerr = np.abs(H - Ho).max(axis=1)
     print(f"{path} {name}: cg steps {its}, max|dH| = {err:.3e}, worst row err / bound {(rowerr / bound).max():.3f}, "
           f"max|H| = {np.abs(Ho).max():.3e}, "
-          f"max_i |dH_i| / ((2/eps) S_i) = {(rowerr / ((2.0 / prob.eps) * S)).max():.3e}, "
+          f"max_i |dH_i| / ((2/eps) S_i) = {(rowerr / ((2.0 / eps) * S)).max():.3e}, "
           f"max|dH| / max|H| = {err / np.abs(Ho).max():.3e}")
     assert np.all(rowerr <= bound), (rowerr / bound).max()
+
+
+def _run_hvp(cuda_device, prob, cases, V, path, cost="sqeuclidean"):
+    import torch
+    import log_domain_sinkhorn_updates_b200 as fs
+    from helpers import device_inputs
+    X, Y, a_d, b_d = device_inputs(prob)
+    f_all = np.stack([c[4] for c in cases])
+    g_all = np.stack([c[5] for c in cases])
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps, cost=cost)
+    out = torch.empty(prob.batch, prob.n, prob.d, device=cuda_device)
+    its = fs.fs_hvp_x(h, torch.from_numpy(f_all).to(cuda_device), torch.from_numpy(g_all).to(cuda_device),
+                      X, Y, torch.from_numpy(V).to(cuda_device), out, max_cg_iters=500, cg_rtol=1e-7)
+    fs.fs_sync(h)
+    info = fs.fs_get_info(h)
+    fs.fs_destroy(h)
+    if path != "simt":
+        assert info["last_apply_path"] in ("tc", "tc_pair")
+    assert info["last_hvp_fused"] == (1 if path == "tc" and cost == "sqeuclidean" else 0), info
+    return out.cpu().numpy(), its
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("name", list(CASES))
+def test_hvp_x_parity(cuda_device, name, path, monkeypatch):
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
+    monkeypatch.setenv("FS_HVP_FUSED", PATHS[path][1])
+    prob = make_problem(name.split("-")[0], **CASES[name])
+    case = _oracle_case(prob, 0)
+    rng = np.random.default_rng(200)
+    V = rng.standard_normal((1, prob.n, prob.d)).astype(np.float32)
+    H, its = _run_hvp(cuda_device, prob, [case], V, path)
+    _check_row_bound(path, name, its, H[0], *case[:4], case[4], case[5], prob.eps, V[0])
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("name", list(BATCHED))
+def test_hvp_x_batched_parity(cuda_device, name, path, monkeypatch):
+    """Every problem of a batch against its own dense oracle HVP; the problems'
+    CG solves stop at different steps, and the call's count is the largest."""
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
+    monkeypatch.setenv("FS_HVP_FUSED", PATHS[path][1])
+    prob = make_problem(name.split("-")[0], **BATCHED[name])
+    cases = [_oracle_case(prob, k) for k in range(prob.batch)]
+    rng = np.random.default_rng(201)
+    V = rng.standard_normal((prob.batch, prob.n, prob.d)).astype(np.float32)
+    H, its = _run_hvp(cuda_device, prob, cases, V, path)
+    assert 1 <= its <= 500
+    for k, case in enumerate(cases):
+        _check_row_bound(path, f"{name}[{k}]", its, H[k], *case[:4], case[4], case[5], prob.eps, V[k])
+
+
+COSINE = {
+    # the cosine cost: fp32 d = 16 (3xF16, 64-byte rows), bf16 d = 128 (3xF16 at
+    # 512-byte rows, the CTA-pair kernels) and a batch of two at d = 32
+    "middim-d16": dict(n=260, m=240, d=16),
+    "highdim-d128": dict(n=256, m=240),
+    "batched-b2": dict(batch=2, n=200, m=180),
+}
+
+
+@pytest.mark.parametrize("path", ["tc_blocked", "simt"])
+@pytest.mark.parametrize("name", list(COSINE))
+def test_hvp_x_cosine_parity(cuda_device, name, path, monkeypatch):
+    """The cosine-cost HVP against the dense oracle (per-pair first and second
+    derivatives of the cosine distance).  Same form of bound as above, with
+    S_i = sum_j P_ij |D_ij|^2 max_k |v_ik| and D_ij = dC_ij/dx_i: the size of the
+    (1/eps) dC_ij D_ij terms the final combination sums (for the squared
+    Euclidean cost, |D|^2 = 4 |x - y|^2 and this is the bound above)."""
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
+    monkeypatch.setenv("FS_HVP_FUSED", PATHS[path][1])
+    prob = make_problem(name.split("-")[0], **COSINE[name])
+    cases = [_oracle_case(prob, k, "cosine") for k in range(prob.batch)]
+    rng = np.random.default_rng(202)
+    V = rng.standard_normal((prob.batch, prob.n, prob.d)).astype(np.float32)
+    H, its = _run_hvp(cuda_device, prob, cases, V, path, cost="cosine")
+    for k, (Xo, Yo, loga, logb, f32, g32) in enumerate(cases):
+        f64, g64 = f32.astype(np.float64), g32.astype(np.float64)
+        Ho = dense.hvp_x(Xo, Yo, loga, logb, f64, g64, prob.eps, V[k].astype(np.float64), cost="cosine")
+        P = dense.plan(dense.cost_matrix(Xo, Yo, "cosine"), loga, logb, f64, g64, prob.eps)
+        D2 = np.sum(dense.cost_grad_x(Xo, Yo, "cosine") ** 2, axis=2)
+        S = (P * D2).sum(axis=1) * np.abs(V[k]).max(axis=1)
+        bound = 2.0 ** -14 * S / prob.eps + 2.0 ** -10 * np.abs(Ho).max()
+        rowerr = np.abs(H[k] - Ho).max(axis=1)
+        print(f"{path} cosine {name}[{k}]: cg steps {its}, worst row err / bound {(rowerr / bound).max():.3f}, "
+              f"max|dH| / max|H| = {rowerr.max() / np.abs(Ho).max():.3e}, "
+              f"max_i |dH_i| / (S_i / eps) = {(rowerr / (S / prob.eps)).max():.3e}")
+        assert np.all(rowerr <= bound), (rowerr / bound).max()

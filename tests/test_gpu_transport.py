@@ -184,9 +184,56 @@ def test_transport_apply_cosine_parity(cuda_device, path, monkeypatch):
     err = (np.abs(out.cpu().numpy()[0] - oo) / (rel[:, None] * absw)).max()
     print(f"cosine transport err / bound {err:.3f}")
     assert err <= 1.0
-    with pytest.raises(fs.FsError):
-        fs.fs_grad_x(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device), X, Y,
-                     torch.empty(1, prob.n, prob.d, device=cuda_device))
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("name", ["tiny", "middim", "highdim", "batched"])
+def test_cosine_grad_parity(cuda_device, name, path, monkeypatch):
+    """fs_grad_x and fs_grad_y under the cosine cost against the oracle's
+    cosine gradients.  grad_i = -(b_i - (x^_i.b_i) x^_i) / |x_i| with b = P Y^:
+    b carries the transport bound (rel times P |Y^|, per component), and the
+    projection adds at most |x^_k| sum_l |db_l| |x^_l| to component k; the fp32
+    normalisation and projection add 2^-20 of the terms' sizes."""
+    import torch
+    _set_path(monkeypatch, path)
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps, cost="cosine")
+    f32, g32 = _potentials(prob, "cosine", iters=30)
+    fd, gd = torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device)
+    Gx = torch.empty(prob.batch, prob.n, prob.d, device=cuda_device)
+    fs.fs_grad_x(h, fd, gd, X, Y, Gx)
+    fs.fs_sync(h)
+    ran_x = fs.fs_get_info(h)["last_apply_path"]
+    Gy = torch.empty(prob.batch, prob.m, prob.d, device=cuda_device)
+    fs.fs_grad_y(h, fd, gd, X, Y, Gy)
+    fs.fs_sync(h)
+    Gx, Gy = Gx.cpu().numpy(), Gy.cpu().numpy()
+    if path == "simt":
+        assert ran_x == "simt"
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
+        rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "cosine") + SPLIT[path]
+        relt = _rel_bound(Yo, Xo, logb, loga, gk, fk, prob.eps, "cosine") + SPLIT[path]
+        Gxo = oracle.grad_x(Xo, Yo, loga, logb, fk, gk, prob.eps, cost="cosine")
+        Gyo = oracle.grad_y(Xo, Yo, loga, logb, fk, gk, prob.eps, cost="cosine")
+        for G, Go, own, other, lw_own, lw_oth, p_own, p_oth, rl, label in (
+                (Gx[k], Gxo, Xo, Yo, loga, logb, fk, gk, rel, "x"),
+                (Gy[k], Gyo, Yo, Xo, logb, loga, gk, fk, relt, "y")):
+            rho = np.linalg.norm(own, axis=1)
+            uh = own / rho[:, None]
+            oh = other / np.linalg.norm(other, axis=1)[:, None]
+            bsum, _ = oracle.transport_apply(own, other, lw_own, lw_oth, p_own, p_oth, prob.eps, oh, cost="cosine")
+            babs, _ = oracle.transport_apply(own, other, lw_own, lw_oth, p_own, p_oth, prob.eps, np.abs(oh),
+                                             cost="cosine")
+            e = rl[:, None] * babs
+            proj = np.sum(e * np.abs(uh), axis=1)[:, None] * np.abs(uh)
+            size = np.abs(bsum) + np.sum(np.abs(bsum * uh), axis=1)[:, None] * np.abs(uh)
+            gb = (e + proj + 2.0 ** -20 * size) / rho[:, None]
+            err = (np.abs(G - Go) / gb).max()
+            print(f"{path} {name}[{k}] cosine grad_{label} err/bound {err:.3f}")
+            assert err <= 1.0
 
 
 @pytest.mark.parametrize("path", list(PATHS))
