@@ -117,10 +117,14 @@ typedef struct {
                                512-byte operand rows, or for every width when the environment
                                variable FS_CTA_PAIR=1 (FS_CTA_PAIR=0 forbids it) */
     int last_apply_path;    /* kernel of the handle's last transport application (fs_transport_apply
-                               and the calls built on it): 1 tensor cores, one CTA per 128 rows;
-                               3 tensor cores on CTA pairs (512-byte operand rows, or any width with
-                               FS_APPLY_PAIR=1); 2 CUDA cores (dv over 256, a plan that does not
-                               fit, the f32_simt precision, or FS_APPLY_SIMT=1); 0 none yet */
+                               and the calls built on it): 4 tensor cores, one CTA per 256 rows (two
+                               128-row blocks sharing every streamed tile; dv <= 128, rows of up to
+                               256 bytes, at least one such CTA per SM, or FS_ROW_BLOCKS=2 at any
+                               size); 1 tensor cores, one CTA per 128 rows (otherwise, or with
+                               FS_ROW_BLOCKS=1); 3 tensor cores on CTA pairs
+                               (512-byte operand rows, or any width with FS_APPLY_PAIR=1); 2 CUDA
+                               cores (dv over 256, the f32_simt precision, or FS_APPLY_SIMT=1);
+                               0 none yet */
     int last_solve_graph;   /* how the handle's last fs_solve ran: 1 as a replay of its CUDA graph,
                                2 as direct launches (a large problem, FS_SOLVE_GRAPH=0, or a
                                failed capture), 0 none yet */

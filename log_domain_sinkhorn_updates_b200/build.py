@@ -20,7 +20,7 @@ LIB = os.path.join(OUT_DIR, "libflashsinkhorn.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 SOURCES = ["fs_api.cu", "fs_prep.cu", "fs_lse_tc.cu", "fs_lse_tc2.cu", "fs_lse_simt.cu", "fs_apply.cu", "fs_apply_tc.cu",
-           "fs_apply_tc2.cu", "fs_hvp_tc.cu",
+           "fs_apply_tc2.cu", "fs_apply_tc_q2.cu", "fs_hvp_tc.cu",
            "fs_hvp.cu", "fs_cosine.cu", "fs_selftest.cu", "fs_noalloc.cu"]
 HEADERS = ["fs_internal.cuh", "fs_finish.cuh", "fs_prep.cuh", "fs_tc_common.cuh"]
 

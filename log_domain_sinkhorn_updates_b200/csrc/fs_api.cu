@@ -357,8 +357,10 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     p.divide = divide ? 1 : 0;
     // Tensor cores for dv <= 256: on CTA pairs for the 512-byte operand rows
     // (and at every width with FS_APPLY_PAIR=1), on one CTA for rows of up to
-    // 256 bytes where its plan fits.  The CUDA-core kernel otherwise, for the
-    // fp32 SIMT precision, or with FS_APPLY_SIMT=1.
+    // 256 bytes where its plan fits -- two 128-row blocks per CTA sharing every
+    // streamed tile where dv <= 128 and the grid still covers the SMs.  The
+    // CUDA-core kernel otherwise, for the fp32 SIMT precision, or with
+    // FS_APPLY_SIMT=1.
     const int vpl = v_bf16 ? 1 : 2;
     const char *force_simt = getenv("FS_APPLY_SIMT");
     const bool tc_ok = h->prec != FS_PREC_F32_SIMT && dv <= 256 && !(force_simt && atoi(force_simt) != 0);
@@ -367,19 +369,30 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     int dv_pad = use_pair ? (dv + 31) / 32 * 32 : (dv + 15) / 16 * 16;
     int kslots = 0, stages = 0;
     size_t smem = 0;
+    bool use_q2 = false;
     if (tc_ok && use_pair)
         smem = fs::apply_tc2_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
     if (tc_ok && smem == 0 && !h->pair && h->row_bytes <= 256) {
         use_pair = false;
         dv_pad = (dv + 15) / 16 * 16;
-        smem = fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
+        // two blocks per CTA where that still gives every SM a CTA (else the
+        // one-block grid, twice as many CTAs, runs more of the work in parallel);
+        // FS_ROW_BLOCKS=1 forces one block, FS_ROW_BLOCKS=2 two wherever they fit
+        const char *env_rb = getenv("FS_ROW_BLOCKS");
+        const int rbk = env_rb ? atoi(env_rb) : 0;
+        const long long q2_ctas = (long long)D.batch * ((p.rows_pad + 255) / 256);
+        if (rbk == 2 || (rbk != 1 && q2_ctas >= h->sms)) {
+            smem = fs::apply_q2_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
+            use_q2 = smem != 0;
+        }
+        if (smem == 0) smem = fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
     }
     if (smem == 0) {
         h->last_apply = 2;
         FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
         return FS_OK;
     }
-    h->last_apply = use_pair ? 3 : 1;
+    h->last_apply = use_pair ? 3 : (use_q2 ? 4 : 1);
     p.row_bytes = h->row_bytes;
     p.swz = h->swz;
     p.plane_bytes = h->plane_bytes;
@@ -406,8 +419,10 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
         cuuint32_t box[2] = {64, (cuuint32_t)dv_pad};
         cuuint32_t estr[2] = {1, 1};
         if (use_pair) box[1] = (cuuint32_t)(dv_pad / 2);  // each CTA of a pair loads half the columns of V
+        if (use_q2) box[0] = 32;                          // 32-column quarters, 64-byte rows
         CUresult r2 = fn ? fn(&map_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vt, gdim, gstride, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              use_q2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
                          : CUDA_ERROR_NOT_SUPPORTED;
         if (r2 != CUDA_SUCCESS) st = fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed for V (%d)", (int)r2);
@@ -422,6 +437,10 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
                                          smem, h->stream);
                 g_launches.fetch_add(1, std::memory_order_relaxed);
             }
+        } else if (use_q2) {
+            e = fs::launch_apply_q2(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r,
+                                    fdir ? &h->mapY_r : &h->mapX_r, &map_v, smem, h->stream);
+            g_launches.fetch_add(1, std::memory_order_relaxed);
         } else {
             e = fs::launch_apply_tc(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r,
                                     fdir ? &h->mapY_r : &h->mapX_r, &map_v, smem, h->stream);

@@ -179,6 +179,11 @@ cudaError_t launch_apply_tc(const ApplyParams &p, int batch, int prec, int vpl, 
 // multiple of 32 (at most 256), and the launch (map_k: 64-row boxes; rows_pad /
 // 128 must be even).
 size_t apply_tc2_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages);
+// Two 128-row blocks per CTA sharing every streamed K tile and V~ quarter
+// (fs_apply_tc_q2.cu; dv_pad <= 128, rows of up to 256 bytes).
+size_t apply_q2_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages);
+cudaError_t launch_apply_q2(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
+                            const void *map_v, size_t smem, cudaStream_t s);
 cudaError_t launch_apply_tc2(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
                              const void *map_v, size_t smem, cudaStream_t s);
 // A kernel whose one bounded mbarrier wait nothing ever completes: after

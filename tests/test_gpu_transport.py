@@ -15,10 +15,12 @@ exp2f adds 2^-21, and the fp32 sum over m terms adds m 2^-24.  Hence
 
 The tensor-core path also splits P/a_i and V into bf16 hi + lo pairs, which
 carry 2^-16 each and drop a term of 2^-16 relative size, so its bound adds
-2^-14.  Every test runs three paths: the one-CTA tensor-core kernel
-(FS_APPLY_PAIR=0), the tensor-core kernel on CTA pairs (FS_APPLY_PAIR=1; the
-default for 512-byte operand rows) and the CUDA-core validation kernel
-(FS_APPLY_SIMT=1).
+2^-14.  Every test runs four paths: the tensor-core kernel with two 128-row
+blocks per CTA (FS_ROW_BLOCKS=2; the default for dv <= 128 and rows of up to
+256 bytes once the grid covers the SMs), the one-block tensor-core kernel
+(FS_ROW_BLOCKS=1), the tensor-core kernel on CTA
+pairs (FS_APPLY_PAIR=1; the default for 512-byte operand rows) and the
+CUDA-core validation kernel (FS_APPLY_SIMT=1).
 """
 import numpy as np
 import pytest
@@ -72,27 +74,32 @@ def _rel_bound(Xo, Yo, loga, logb, f, g, eps, cost):
     return np.log(2.0) * 2.0 ** -23 * M + 2.0 ** -21 + len(Yo) * 2.0 ** -24
 
 
-PATHS = {"tc": ("0", "0"), "tc_pair": ("0", "1"), "simt": ("1", "0")}  # (FS_APPLY_SIMT, FS_APPLY_PAIR)
-SPLIT = {"tc": 2.0 ** -14, "tc_pair": 2.0 ** -14, "simt": 0.0}
+# (FS_APPLY_SIMT, FS_APPLY_PAIR, FS_ROW_BLOCKS)
+PATHS = {"tc_q2": ("0", "0", "2"), "tc": ("0", "0", "1"), "tc_pair": ("0", "1", "2"), "simt": ("1", "0", "2")}
+SPLIT = {"tc_q2": 2.0 ** -14, "tc": 2.0 ** -14, "tc_pair": 2.0 ** -14, "simt": 0.0}
 
 
 def _set_path(monkeypatch, path):
     monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
     monkeypatch.setenv("FS_APPLY_PAIR", PATHS[path][1])
+    monkeypatch.setenv("FS_ROW_BLOCKS", PATHS[path][2])
 
 
 def _assert_path(fs, h, path, dv):
     """The kernel that ran, as the handle reports it: the CUDA-core one when it is
-    forced; the tensor-core one otherwise whenever dv <= 128, where every operand
-    width of these workloads fits its shared-memory plan; either one at larger dv,
-    where fp32 V takes two bf16 planes and the plan need not fit."""
+    forced; a tensor-core one otherwise whenever dv <= 128, where every operand
+    width of these workloads fits the shared-memory plans (the two-block kernel
+    by default, the one-block kernel with FS_ROW_BLOCKS=1); at larger dv, where
+    the two-block kernel's TMEM does not hold two accumulators, the one-block
+    kernel or (fp32 V in two bf16 planes, when its plan does not fit) the CUDA
+    cores."""
     ran = fs.fs_get_info(h)["last_apply_path"]
     if path == "simt":
         assert ran == "simt", ran
     elif path == "tc_pair":  # the pair's plan fits every operand width here up to dv = 256
         assert ran == "tc_pair", ran
     elif dv <= 128:
-        assert ran == "tc", ran
+        assert ran == path, ran
     else:
         assert ran in ("tc", "simt"), ran
     return ran
@@ -332,7 +339,7 @@ def test_transport_apply_tf32_kind(cuda_device, name, prec):
     fs.fs_transport_apply(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device),
                           torch.from_numpy(V).to(cuda_device), out, None)
     fs.fs_sync(h)
-    assert fs.fs_get_info(h)["last_apply_path"] == "tc"
+    assert fs.fs_get_info(h)["last_apply_path"] in ("tc", "tc_q2")
     out = out.cpu().numpy()
     u = 2.0 ** -21
     for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
