@@ -36,6 +36,15 @@ UNIT = "cost-entries/s"
 MUFU_EX2_PER_CLK_PER_SM = 16  # special-function-unit exp2 results per clock per SM
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "lse_tc_highdim_ncu.md")
 PROFILE_TRAFFIC_APPLY = os.path.join(ROOT, "profiles", "apply_tc_highdim_ncu.md")
+PROFILE_TRAFFIC_APPLY_Q2 = os.path.join(ROOT, "profiles", "apply_q2_highdim_ncu.md")
+# the transport kernels by the path the handle reports: (ncu summary, source file, description)
+APPLY_KERNELS = {
+    "tc_q2": (PROFILE_TRAFFIC_APPLY_Q2, "fs_apply_tc_q2.cu",
+              "apply_q2_kernel (two 128-row blocks per CTA: S = Q K^T, P~ back into TMEM, O += P~ V~)"),
+    "tc": (PROFILE_TRAFFIC_APPLY, "fs_apply_tc.cu", "apply_tc_kernel (S = Q K^T, then O += P~ V~)"),
+    "tc_pair": (None, "fs_apply_tc2.cu", "apply_tc2_kernel (CTA pairs: S = Q K^T, then O += P~ V~)"),
+    "simt": (None, "fs_apply.cu", "apply_simt_kernel (CUDA cores)"),
+}
 
 
 def parse_args():
@@ -313,6 +322,7 @@ def run_transport(args):
     flops = 2.0 * entries * (d * npass_s + d * npass_o)
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", 1590.0))
+    kprof, ksrc, kdesc = APPLY_KERNELS.get(info["last_apply_path"], (None, None, str(info["last_apply_path"])))
     line = {
         "metric": "transport application (barycentric map) cost-entries/s at the converged potentials",
         "value": replica_throughput(world, args.steps, entries, tot), "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -325,10 +335,11 @@ def run_transport(args):
         "roofline": {"bound": "tensor", "achieved": flops / app_s / 1e12, "peak": peak, "unit": "TFLOP/s",
                      "frac": flops / app_s / 1e12 / peak,
                      # the committed capture is of the full highdim workload
-                     "traffic": profile_traffic(PROFILE_TRAFFIC_APPLY, "fs_apply_tc.cu")
-                     if (args.workload, args.n, args.m, args.batch) == ("highdim", None, None, None) else None,
+                     "traffic": profile_traffic(kprof, ksrc)
+                     if kprof and (args.workload, args.n, args.m, args.batch) == ("highdim", None, None, None)
+                     else None,
                      "peak_source": peak_src,
-                     "kernel": "apply_tc_kernel (S = Q K^T, then O += P~ V~)",
+                     "kernel": kdesc,
                      "flops_per_launch": flops},
         "cpu_baseline": None, "e2e": None, "clocks": clocks, "gpu_launches": int(launches),
     }

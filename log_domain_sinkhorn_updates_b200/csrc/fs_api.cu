@@ -419,10 +419,8 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
         cuuint32_t box[2] = {64, (cuuint32_t)dv_pad};
         cuuint32_t estr[2] = {1, 1};
         if (use_pair) box[1] = (cuuint32_t)(dv_pad / 2);  // each CTA of a pair loads half the columns of V
-        if (use_q2) box[0] = 32;                          // 32-column quarters, 64-byte rows
         CUresult r2 = fn ? fn(&map_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, vt, gdim, gstride, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              use_q2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
                          : CUDA_ERROR_NOT_SUPPORTED;
         if (r2 != CUDA_SUCCESS) st = fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed for V (%d)", (int)r2);
