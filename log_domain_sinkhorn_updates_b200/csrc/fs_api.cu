@@ -743,10 +743,10 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
         off += (count * 4 + 255) / 256 * 256;
         return o;
     };
-    const size_t oPY = carve(n * d), o_r = carve(n), o_c = carve(m), oW1 = carve(n * (d + 1)), oT = carve(m * (d + 1));
-    const size_t o_u = carve(n), o_w = carve(m), o_tn = carve(n), o_tm = carve(m), o_z = carve(m), o_x = carve(m);
-    const size_t o_res = carve(m), o_p = carve(m), o_Ap = carve(m), o_Pdg = carve(n), o_df = carve(n);
-    const size_t o_dgY = carve(m * d), oQ1 = carve(n * d), oMV = carve(n * d), o_ones = carve(n);
+    const size_t oPY = carve(n * d), o_r = carve(n), o_c = carve(m), oW1 = carve(n * (d + 2)), oT = carve(m * (d + 2));
+    const size_t o_u = carve(n), o_tn = carve(n), o_tm = carve(m), o_z = carve(m), o_x = carve(m);
+    const size_t o_res = carve(m), o_p = carve(m), o_Ap = carve(m), o_df = carve(n);
+    const size_t o_dgY = carve(m * (d + 1)), oQ1 = carve(n * (d + 1)), oMV = carve(n * d);
     const size_t oVc = carve(m * nq * d), oOc = carve(n * nq * d);
     const size_t o_part = carve((size_t)B * 2 * 4096), o_sc = carve((size_t)B * 2 * 5);
     const size_t o_Yh = carve(cosine ? m * d : 1), o_Vt = carve(cosine ? n * d : 1);
@@ -759,9 +759,9 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     double *sc = reinterpret_cast<double *>(blk + o_sc);  // [k][B]: k = 0 rr, 1 p.Ap, 2 rr_new, 3 sum, 4 z.z
     double *rr_d = sc, *pap_d = sc + B, *rrn_d = sc + 2 * B, *sum_d = sc + 3 * B, *zz_d = sc + 4 * B;
     const double tol2 = cg_rtol * cg_rtol;
-    float *PY = F(oPY), *r = F(o_r), *c = F(o_c), *W1 = F(oW1), *Tm = F(oT), *u = F(o_u), *w = F(o_w);
+    float *PY = F(oPY), *r = F(o_r), *c = F(o_c), *W1 = F(oW1), *Tm = F(oT), *u = F(o_u);
     float *tn = F(o_tn), *tm = F(o_tm), *z = F(o_z), *x = F(o_x), *res = F(o_res), *p = F(o_p), *Ap = F(o_Ap);
-    float *Pdg = F(o_Pdg), *df = F(o_df), *dgY = F(o_dgY), *Q1 = F(oQ1), *MV = F(oMV), *ones = F(o_ones);
+    float *df = F(o_df), *dgY = F(o_dgY), *Q1 = F(oQ1), *MV = F(oMV);
     float *Vc = F(oVc), *Oc = F(oOc), *Yh = F(o_Yh), *Vt = F(o_Vt);
     // the column cloud the transport products see (Y, or its unit rows), and the
     // direction the transport-matrix term contracts with (v, or v~)
@@ -774,22 +774,18 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     auto run = [&]() -> fs_status {
         // transport products that do not depend on the CG solution
         if (cosine) FS_LAUNCH(h, fs::cos_unit_rows(Y, bf16, m, (int)d, Yh, s));
+        // (every application costs a full pass over the plan whatever its width, so
+        // the vectors that share a direction go through one application together)
         fs_status s2 = apply(h, f, g, Yop, ybf, (int)d, PY, r, false, true);  // P Y (P Y^), r = P 1
         if (s2 != FS_OK) return s2;
-        FS_LAUNCH(h, fs::launch_fill(ones, n, 1.f, s));
-        s2 = apply(h, f, g, ones, false, 1, tm, c, false, false);  // c = P^T 1
-        if (s2 != FS_OK) return s2;
         if (cosine)
-            FS_LAUNCH(h, fs::cos_hvp_prep(X, bf16, V, PY, n, (int)d, u, W1, Vt, s));
+            FS_LAUNCH(h, fs::cos_hvp_prep(X, bf16, V, PY, r, n, (int)d, u, W1, Vt, s));
         else
             FS_LAUNCH(h, fs::hvp_prep(X, bf16, V, PY, r, (int)n, (int)d, u, W1, s));
-        s2 = apply(h, f, g, W1, false, (int)d + 1, Tm, nullptr, false, false);  // P^T [v | x.v] (P^T [v~ | 0])
+        // P^T [v | x.v | u/r] (P^T [v~ | 0 | u/r]) and its row sums c = P^T 1
+        s2 = apply(h, f, g, W1, false, (int)d + 2, Tm, c, false, false);
         if (s2 != FS_OK) return s2;
-        FS_LAUNCH(h, fs::hvp_w(Yop, ybf, Tm, (int)m, (int)d, cosine ? 1.f : 2.f, w, s));
-        FS_LAUNCH(h, fs::hvp_vec(n, u, r, 1.f, nullptr, 0.f, true, tn, s));  // u / r
-        s2 = apply(h, f, g, tn, false, 1, tm, nullptr, false, false);        // P^T (u / r)
-        if (s2 != FS_OK) return s2;
-        FS_LAUNCH(h, fs::hvp_vec(m, w, nullptr, 1.f, tm, -1.f, false, z, s));  // z = w - P^T (u / r)
+        FS_LAUNCH(h, fs::hvp_w(Yop, ybf, Tm, (int)m, (int)d, cosine ? 1.f : 2.f, z, s));  // z = w - P^T (u / r)
         FS_LAUNCH(h, fs::hvp_dot(B, m1, z, nullptr, part, sum_d, s));
         FS_LAUNCH(h, fs::hvp_center(B, m1, sum_d, z, s));
         // CG on [diag(c) - P^T diag(1/r) P] dg = z, iterates kept orthogonal to 1;
@@ -826,15 +822,11 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
             FS_CUDA(h, cudaStreamSynchronize(s));
             ++it;
         }
-        // df = (u - P dg) / r
-        s2 = apply(h, f, g, x, false, 1, Pdg, nullptr, false, true);
-        if (s2 != FS_OK) return s2;
-        FS_LAUNCH(h, fs::hvp_vec(n, u, nullptr, 1.f, Pdg, -1.f, false, df, s));
-        FS_LAUNCH(h, fs::hvp_vec(n, df, r, 1.f, nullptr, 0.f, true, df, s));
-        // P (dg o Y)
+        // Q1 = P [dg o Y | dg] in one application; df = (u - P dg) / r
         FS_LAUNCH(h, fs::hvp_dgy(Yop, ybf, x, (int)m, (int)d, dgY, s));
-        s2 = apply(h, f, g, dgY, false, (int)d, Q1, nullptr, false, true);
+        s2 = apply(h, f, g, dgY, false, (int)d + 1, Q1, nullptr, false, true);
         if (s2 != FS_OK) return s2;
+        FS_LAUNCH(h, fs::hvp_df(n, (int)d, u, Q1, r, df, s));
         // sum_j P_ij (y_j.v_i) y_j: in one fused pass where the handle's operands
         // allow it (tensor cores), else nq columns of y at a time
         bool fused = false;
@@ -857,7 +849,7 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
         if (cosine)
             FS_LAUNCH(h, fs::cos_hvp_final(X, bf16, V, PY, df, Q1, MV, n, (int)d, D.eps, out, s));
         else
-            FS_LAUNCH(h, fs::hvp_final(X, bf16, V, PY, r, df, Pdg, Q1, MV, (int)n, (int)d, D.eps, out, s));
+            FS_LAUNCH(h, fs::hvp_final(X, bf16, V, PY, r, df, Q1, MV, (int)n, (int)d, D.eps, out, s));
         return FS_OK;
     };
     st = run();

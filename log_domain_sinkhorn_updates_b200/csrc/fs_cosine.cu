@@ -74,11 +74,11 @@ __global__ void grad_kernel(const T *X, const float *b, size_t rows, int d, floa
     }
 }
 
-// v~_i = (v_i - (x^_i.v_i) x^_i) / rho_i  -> Vt [n][d] and W1 = [v~_i | 0] [n][d+1];
-// u_i = sum_j P_ij dC_ij = -b_i.v~_i  (b = P Y^)
+// v~_i = (v_i - (x^_i.v_i) x^_i) / rho_i  -> Vt [n][d] and W1 = [v~_i | 0 | u_i / r_i] [n][d+2];
+// u_i = sum_j P_ij dC_ij = -b_i.v~_i  (b = P Y^, r = P 1)
 template <typename T>
-__global__ void hvp_prep_kernel(const T *X, const float *V, const float *b, size_t rows, int d, float *u,
-                                float *W1, float *Vt) {
+__global__ void hvp_prep_kernel(const T *X, const float *V, const float *b, const float *r, size_t rows, int d,
+                                float *u, float *W1, float *Vt) {
     ROW_LOOP(i, rows) {
         const float rho = row_norm(X, i, d), inv = 1.f / rho;
         float xv = 0.f;
@@ -87,17 +87,19 @@ __global__ void hvp_prep_kernel(const T *X, const float *V, const float *b, size
         for (int k = 0; k < d; ++k) {
             const float vt = (V[i * d + k] - xv * (ldc(X, i * d + k) * inv)) * inv;
             Vt[i * d + k] = vt;
-            W1[i * (d + 1) + k] = vt;
+            W1[i * (d + 2) + k] = vt;
             su = fmaf(b[i * d + k], vt, su);
         }
-        W1[i * (d + 1) + d] = 0.f;
         u[i] = -su;
+        W1[i * (d + 2) + d] = 0.f;
+        W1[i * (d + 2) + d + 1] = u[i] / r[i];
     }
 }
 
 // (H V)_i = [ (b_i.v_i) x^_i + s_i v_i + (x^_i.v_i) b_i - 3 s_i (x^_i.v_i) x^_i ] / rho_i^2
 //           - (1/eps) (T_i - (x^_i.T_i) x^_i) / rho_i,
 // s_i = x^_i.b_i,  T_i = df_i b_i + (P (dg o Y^))_i + sum_j P_ij (v~_i.y^_j) y^_j
+// (Q1: P [dg o Y^ | dg], [n][d+1])
 template <typename T>
 __global__ void hvp_final_kernel(const T *X, const float *V, const float *b, const float *df, const float *Q1,
                                  const float *MV, size_t rows, int d, float eps, float *out) {
@@ -106,7 +108,7 @@ __global__ void hvp_final_kernel(const T *X, const float *V, const float *b, con
         float s = 0.f, bv = 0.f, xv = 0.f, xt = 0.f;
         for (int k = 0; k < d; ++k) {
             const float xh = ldc(X, i * d + k) * inv, v = V[i * d + k], bk = b[i * d + k];
-            const float t = fmaf(df[i], bk, Q1[i * d + k] + MV[i * d + k]);
+            const float t = fmaf(df[i], bk, Q1[i * (d + 1) + k] + MV[i * d + k]);
             s = fmaf(xh, bk, s);
             bv = fmaf(bk, v, bv);
             xv = fmaf(xh, v, xv);
@@ -115,7 +117,7 @@ __global__ void hvp_final_kernel(const T *X, const float *V, const float *b, con
         const float inv2 = inv * inv, ie = 1.f / eps;
         for (int k = 0; k < d; ++k) {
             const float xh = ldc(X, i * d + k) * inv, v = V[i * d + k], bk = b[i * d + k];
-            const float t = fmaf(df[i], bk, Q1[i * d + k] + MV[i * d + k]);
+            const float t = fmaf(df[i], bk, Q1[i * (d + 1) + k] + MV[i * d + k]);
             const float second = (bv * xh + s * v + xv * bk - 3.f * s * xv * xh) * inv2;
             out[i * d + k] = second - ie * (t - xt * xh) * inv;
         }
@@ -140,13 +142,13 @@ cudaError_t cos_grad(const void *X, bool bf16, const float *b, size_t rows, int 
     return cudaGetLastError();
 }
 
-cudaError_t cos_hvp_prep(const void *X, bool bf16, const float *V, const float *b, size_t rows, int d, float *u,
-                         float *W1, float *Vt, cudaStream_t s) {
+cudaError_t cos_hvp_prep(const void *X, bool bf16, const float *V, const float *b, const float *r, size_t rows, int d,
+                         float *u, float *W1, float *Vt, cudaStream_t s) {
     if (bf16)
-        hvp_prep_kernel<<<grid_rows(rows), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(X), V, b, rows, d, u, W1,
-                                                        Vt);
+        hvp_prep_kernel<<<grid_rows(rows), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(X), V, b, r, rows, d, u,
+                                                        W1, Vt);
     else
-        hvp_prep_kernel<<<grid_rows(rows), 256, 0, s>>>(static_cast<const float *>(X), V, b, rows, d, u, W1, Vt);
+        hvp_prep_kernel<<<grid_rows(rows), 256, 0, s>>>(static_cast<const float *>(X), V, b, r, rows, d, u, W1, Vt);
     return cudaGetLastError();
 }
 

@@ -42,7 +42,7 @@ __host__ __device__ inline int blocks_for(size_t n) {
 
 #define GRID_LOOP(i, n) for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < (n); i += (size_t)gridDim.x * blockDim.x)
 
-// u_i = 2 (r_i x_i - PY_i).v_i;  W1_i = [v_i | x_i.v_i]  ([n][d+1])
+// u_i = 2 (r_i x_i - PY_i).v_i;  W1_i = [v_i | x_i.v_i | u_i / r_i]  ([n][d+2])
 template <typename T>
 __global__ void prep_kernel(const T *X, const float *V, const float *PY, const float *r, int n, int d, float *u,
                             float *W1) {
@@ -52,21 +52,23 @@ __global__ void prep_kernel(const T *X, const float *V, const float *PY, const f
             const float x = ldv(X, i * d + k), v = V[i * d + k];
             su = fmaf(r[i] * x - PY[i * d + k], v, su);
             sxv = fmaf(x, v, sxv);
-            W1[i * (d + 1) + k] = v;
+            W1[i * (d + 2) + k] = v;
         }
-        W1[i * (d + 1) + d] = sxv;
         u[i] = 2.f * su;
+        W1[i * (d + 2) + d] = sxv;
+        W1[i * (d + 2) + d + 1] = u[i] / r[i];
     }
 }
 
-// w_j = alpha (T_j[d] - y_j . T_j[0:d]),  T = P^T W1  ([m][d+1]); alpha = 2 for the
-// squared Euclidean cost (W1 = [v | x.v]), 1 for the cosine cost (W1 = [v~ | 0], Y = Y^)
+// z_j = alpha (T_j[d] - y_j . T_j[0:d]) - T_j[d+1],  T = P^T W1  ([m][d+2]): the right-hand
+// side w - P^T (u / r) of the potentials' response.  alpha = 2 for the squared Euclidean
+// cost (W1 = [v | x.v | u/r]), 1 for the cosine cost (W1 = [v~ | 0 | u/r], Y = Y^)
 template <typename T>
-__global__ void w_kernel(const T *Y, const float *Tm, int m, int d, float alpha, float *w) {
+__global__ void w_kernel(const T *Y, const float *Tm, int m, int d, float alpha, float *z) {
     GRID_LOOP(j, (size_t)m) {
         float s = 0.f;
-        for (int k = 0; k < d; ++k) s = fmaf(ldv(Y, j * d + k), Tm[j * (d + 1) + k], s);
-        w[j] = alpha * (Tm[j * (d + 1) + d] - s);
+        for (int k = 0; k < d; ++k) s = fmaf(ldv(Y, j * d + k), Tm[j * (d + 2) + k], s);
+        z[j] = alpha * (Tm[j * (d + 2) + d] - s) - Tm[j * (d + 2) + d + 1];
     }
 }
 
@@ -149,10 +151,19 @@ __global__ void cg_dir_kernel(size_t len, const double *rr_new, const double *rr
     SEG_LOOP(i, len) p[base + i] = fmaf(beta, p[base + i], res[base + i]);
 }
 
-// out_jk = dg_j y_jk
+// out_j = [dg_j y_j | dg_j]  ([m][d+1]): one application gives P (dg o Y) and P dg
 template <typename T>
 __global__ void dgy_kernel(const T *Y, const float *dg, int m, int d, float *out) {
-    GRID_LOOP(i, (size_t)m * d) out[i] = dg[i / d] * ldv(Y, i);
+    GRID_LOOP(i, (size_t)m * (d + 1)) {
+        const size_t j = i / (d + 1);
+        const int k = (int)(i % (d + 1));
+        out[i] = k < d ? dg[j] * ldv(Y, j * d + k) : dg[j];
+    }
+}
+
+// df_i = (u_i - (P dg)_i) / r_i, (P dg)_i the last column of Q = P [dg o Y | dg] ([n][d+1])
+__global__ void df_kernel(size_t n, int d, const float *u, const float *Q, const float *r, float *df) {
+    GRID_LOOP(i, n) df[i] = (u[i] - Q[i * (d + 1) + d]) / r[i];
 }
 
 // Vc_j[q d + k] = y_j[k0 + q] y_jk for q < nq  ([m][nq d])
@@ -176,10 +187,12 @@ __global__ void mv_acc_kernel(const float *V, const float *Oc, int n, int d, int
     }
 }
 
+// Q1: P [dg o Y | dg] ([n][d+1]; column d is P dg)
 template <typename T>
 __global__ void final_kernel(const T *X, const float *V, const float *PY, const float *r, const float *df,
-                             const float *Pdg, const float *Q1, const float *MV, int n, int d, float eps, float *out) {
+                             const float *Q1, const float *MV, int n, int d, float eps, float *out) {
     GRID_LOOP(i, (size_t)n) {
+        const float pdg = Q1[i * (d + 1) + d];
         float xv = 0.f, pyv = 0.f;
         for (int k = 0; k < d; ++k) {
             const float v = V[i * d + k];
@@ -189,7 +202,7 @@ __global__ void final_kernel(const T *X, const float *V, const float *PY, const 
         for (int k = 0; k < d; ++k) {
             const float x = ldv(X, i * d + k);
             const float gk = r[i] * x - PY[i * d + k];  // sum_j P_ij (x_i - y_j), component k
-            const float inner = df[i] * gk + Pdg[i] * x - Q1[i * d + k] -
+            const float inner = df[i] * gk + pdg * x - Q1[i * (d + 1) + k] -
                                 2.f * (xv * gk - x * pyv + MV[i * d + k]);
             out[i * d + k] = 2.f * r[i] * V[i * d + k] + (2.f / eps) * inner;
         }
@@ -206,11 +219,11 @@ cudaError_t hvp_prep(const void *X, bool bf16, const float *V, const float *PY, 
         prep_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const float *>(X), V, PY, r, n, d, u, W1);
     return cudaGetLastError();
 }
-cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float alpha, float *w, cudaStream_t s) {
+cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float alpha, float *z, cudaStream_t s) {
     if (bf16)
-        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), Tm, m, d, alpha, w);
+        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), Tm, m, d, alpha, z);
     else
-        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const float *>(Y), Tm, m, d, alpha, w);
+        w_kernel<<<blocks_for(m), 256, 0, s>>>(static_cast<const float *>(Y), Tm, m, d, alpha, z);
     return cudaGetLastError();
 }
 cudaError_t hvp_vec(size_t n, const float *x, const float *a, float alpha, const float *y, float beta, bool div,
@@ -244,9 +257,14 @@ cudaError_t hvp_cg_dir(int batch, size_t len, const double *rr_new, const double
 }
 cudaError_t hvp_dgy(const void *Y, bool bf16, const float *dg, int m, int d, float *out, cudaStream_t s) {
     if (bf16)
-        dgy_kernel<<<blocks_for((size_t)m * d), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), dg, m, d, out);
+        dgy_kernel<<<blocks_for((size_t)m * (d + 1)), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(Y), dg, m, d,
+                                                                   out);
     else
-        dgy_kernel<<<blocks_for((size_t)m * d), 256, 0, s>>>(static_cast<const float *>(Y), dg, m, d, out);
+        dgy_kernel<<<blocks_for((size_t)m * (d + 1)), 256, 0, s>>>(static_cast<const float *>(Y), dg, m, d, out);
+    return cudaGetLastError();
+}
+cudaError_t hvp_df(size_t n, int d, const float *u, const float *Q, const float *r, float *df, cudaStream_t s) {
+    df_kernel<<<blocks_for(n), 256, 0, s>>>(n, d, u, Q, r, df);
     return cudaGetLastError();
 }
 cudaError_t hvp_ychunk(const void *Y, bool bf16, int m, int d, int k0, int nq, float *Vc, cudaStream_t s) {
@@ -262,14 +280,13 @@ cudaError_t hvp_mv_acc(const float *V, const float *Oc, int n, int d, int k0, in
     return cudaGetLastError();
 }
 cudaError_t hvp_final(const void *X, bool bf16, const float *V, const float *PY, const float *r, const float *df,
-                      const float *Pdg, const float *Q1, const float *MV, int n, int d, float eps, float *out,
-                      cudaStream_t s) {
+                      const float *Q1, const float *MV, int n, int d, float eps, float *out, cudaStream_t s) {
     if (bf16)
-        final_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(X), V, PY, r, df, Pdg, Q1, MV,
-                                                   n, d, eps, out);
-    else
-        final_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const float *>(X), V, PY, r, df, Pdg, Q1, MV, n, d,
+        final_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(X), V, PY, r, df, Q1, MV, n, d,
                                                    eps, out);
+    else
+        final_kernel<<<blocks_for(n), 256, 0, s>>>(static_cast<const float *>(X), V, PY, r, df, Q1, MV, n, d, eps,
+                                                   out);
     return cudaGetLastError();
 }
 

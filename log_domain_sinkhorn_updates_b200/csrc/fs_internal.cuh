@@ -192,7 +192,7 @@ cudaError_t launch_wait_probe(unsigned long long timeout_ns, int *err, cudaStrea
 // Element-wise pieces of the streaming Hessian-vector product (fs_hvp.cu).
 cudaError_t hvp_prep(const void *X, bool bf16, const float *V, const float *PY, const float *r, int n, int d,
                      float *u, float *W1, cudaStream_t s);
-cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float alpha, float *w, cudaStream_t s);
+cudaError_t hvp_w(const void *Y, bool bf16, const float *Tm, int m, int d, float alpha, float *z, cudaStream_t s);
 cudaError_t hvp_vec(size_t n, const float *x, const float *a, float alpha, const float *y, float beta, bool div,
                     float *out, cudaStream_t s);
 cudaError_t hvp_dot(int batch, size_t len, const float *x, const float *y, double *part, double *out,
@@ -203,11 +203,11 @@ cudaError_t hvp_cg_step(int batch, size_t len, const double *rr, const double *p
 cudaError_t hvp_cg_dir(int batch, size_t len, const double *rr_new, const double *rr, const double *zz, double tol2,
                        const float *res, float *p, cudaStream_t s);
 cudaError_t hvp_dgy(const void *Y, bool bf16, const float *dg, int m, int d, float *out, cudaStream_t s);
+cudaError_t hvp_df(size_t n, int d, const float *u, const float *Q, const float *r, float *df, cudaStream_t s);
 cudaError_t hvp_ychunk(const void *Y, bool bf16, int m, int d, int k0, int nq, float *Vc, cudaStream_t s);
 cudaError_t hvp_mv_acc(const float *V, const float *Oc, int n, int d, int k0, int nq, float *MV, cudaStream_t s);
 cudaError_t hvp_final(const void *X, bool bf16, const float *V, const float *PY, const float *r, const float *df,
-                      const float *Pdg, const float *Q1, const float *MV, int n, int d, float eps, float *out,
-                      cudaStream_t s);
+                      const float *Q1, const float *MV, int n, int d, float eps, float *out, cudaStream_t s);
 // grad[bz][i][k] = 2 (r_i x_ik - pv[bz][i][k]) from the caller's X (fp32 or bf16).
 cudaError_t launch_grad_combine(const void *X, bool bf16, const float *r, const float *pv, int batch, int rows,
                                 int d, float *grad, cudaStream_t s);
@@ -229,8 +229,8 @@ cudaError_t launch_hvp_w(const ApplyParams &p, int batch, int prec, int umode, i
 // -(b - (x^.b) x^) / |x| from b = P Y^, and the HVP's first and last steps.
 cudaError_t cos_unit_rows(const void *P, bool bf16, size_t rows, int d, float *out, cudaStream_t s);
 cudaError_t cos_grad(const void *X, bool bf16, const float *b, size_t rows, int d, float *grad, cudaStream_t s);
-cudaError_t cos_hvp_prep(const void *X, bool bf16, const float *V, const float *b, size_t rows, int d, float *u,
-                         float *W1, float *Vt, cudaStream_t s);
+cudaError_t cos_hvp_prep(const void *X, bool bf16, const float *V, const float *b, const float *r, size_t rows, int d,
+                         float *u, float *W1, float *Vt, cudaStream_t s);
 cudaError_t cos_hvp_final(const void *X, bool bf16, const float *V, const float *b, const float *df, const float *Q1,
                           const float *MV, size_t rows, int d, float eps, float *out, cudaStream_t s);
 // Record msg as this thread's handle-less error (what fs_last_error(NULL) returns).
