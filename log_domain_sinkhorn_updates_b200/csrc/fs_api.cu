@@ -450,6 +450,26 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     FS_CUDA(h, e);
     return FS_OK;
 }
+// One-column transport application out = P v (fdir) or P^T v through the streamed
+// LSE pass's vector mode: the softmax warps accumulate sum_j 2^(z_j - m) v_j next to
+// the row's LSE state, so the column costs no P~ and no P V product, and the
+// pass runs at the LSE pass's rate (a tensor-core application of one column costs
+// as much as one of 128).  vpad: scratch of batch x (the column side's stride)
+// floats.  r (may be null) receives the row sums.  Tensor-core handles only.
+fs_status apply_vec(fs_handle *h, const float *f, const float *g, const float *v, bool fdir, float *out, float *r,
+                    float *vpad) {
+    const fs_desc &D = h->desc;
+    fs::PassParams p = make_pass(h, fdir, true);
+    FS_LAUNCH(h, fs::launch_pad_vec(v, D.batch, p.cols, p.cols_stride, vpad, h->stream));
+    FS_LAUNCH(h, run_bias(h, fdir ? g : f, fdir));
+    p.pot_in = fdir ? f : g;
+    p.col_vec = vpad;
+    p.vec_out = out;
+    p.vec_rsum = r;
+    FS_LAUNCH(h, run_pass(h, p, fdir, true));
+    return FS_OK;
+}
+
 // The launches of fs_solve, in order, on h->stream.
 fs_status enqueue_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule schedule) {
     if (schedule == FS_SCHED_ALTERNATING) {
@@ -750,6 +770,7 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     const size_t oVc = carve(m * nq * d), oOc = carve(n * nq * d);
     const size_t o_part = carve((size_t)B * 2 * 4096), o_sc = carve((size_t)B * 2 * 5);
     const size_t o_Yh = carve(cosine ? m * d : 1), o_Vt = carve(cosine ? n * d : 1);
+    const size_t o_vpad = carve((size_t)B * (h->n_stride > h->m_stride ? h->n_stride : h->m_stride));
     cudaMemPool_t pool;
     uint8_t *blk = nullptr;
     FS_CUDA(h, device_pool(h->device, &pool));
@@ -762,7 +783,15 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     float *PY = F(oPY), *r = F(o_r), *c = F(o_c), *W1 = F(oW1), *Tm = F(oT), *u = F(o_u);
     float *tn = F(o_tn), *tm = F(o_tm), *z = F(o_z), *x = F(o_x), *res = F(o_res), *p = F(o_p), *Ap = F(o_Ap);
     float *df = F(o_df), *dgY = F(o_dgY), *Q1 = F(oQ1), *MV = F(oMV);
-    float *Vc = F(oVc), *Oc = F(oOc), *Yh = F(o_Yh), *Vt = F(o_Vt);
+    float *Vc = F(oVc), *Oc = F(oOc), *Yh = F(o_Yh), *Vt = F(o_Vt), *vpad = F(o_vpad);
+    // the CG's one-column products through the LSE pass's vector mode on tensor-core
+    // handles; the CUDA-core validation path keeps the transport kernels
+    const char *env_simt0 = getenv("FS_APPLY_SIMT");
+    const bool use_vec = h->prec != FS_PREC_F32_SIMT && !(env_simt0 && atoi(env_simt0) != 0);
+    auto apply1 = [&](const float *vin, bool fdir, float *vout) -> fs_status {
+        if (use_vec) return apply_vec(h, f, g, vin, fdir, vout, nullptr, vpad);
+        return apply(h, f, g, vin, false, 1, vout, nullptr, false, fdir);
+    };
     // the column cloud the transport products see (Y, or its unit rows), and the
     // direction the transport-matrix term contracts with (v, or v~)
     const void *Yop = cosine ? (const void *)Yh : Y;
@@ -805,10 +834,10 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
             return false;
         };
         while (it < max_cg_iters && any_running()) {
-            s2 = apply(h, f, g, p, false, 1, tn, nullptr, false, true);  // P p
+            s2 = apply1(p, true, tn);  // P p
             if (s2 != FS_OK) return s2;
             FS_LAUNCH(h, fs::hvp_vec(n, tn, r, 1.f, nullptr, 0.f, true, tn, s));  // / r
-            s2 = apply(h, f, g, tn, false, 1, tm, nullptr, false, false);       // P^T (P p / r)
+            s2 = apply1(tn, false, tm);  // P^T (P p / r)
             if (s2 != FS_OK) return s2;
             FS_LAUNCH(h, fs::hvp_vec(m, p, c, 1.f, tm, -1.f, false, Ap, s));  // c o p - ...
             FS_LAUNCH(h, fs::hvp_dot(B, m1, Ap, nullptr, part, sum_d, s));

@@ -76,6 +76,19 @@ __device__ void finish_rows(const PassParams &p, int rb, int rl, float m, float 
             }
         }
         if (!p.tail_stats) return;  // uniform over the kernel: a launch parameter
+    } else if (p.col_vec) {
+        // Vector pass: w / l is the plan-weighted average of v over row i, and the
+        // row sum r_i is that of a measure pass (below), so sum_j P_ij v_j = r_i w_i / l_i.
+        if (valid) {
+            const double lw2 = (double)p.row_logw2[prow];
+            const double pot = (double)p.pot_in[(size_t)bz * p.rows + row];
+            const double r = exp2(lw2 + (pot - (double)p.row_norm[prow]) * (kLog2ed / p.eps) + lse2);
+            const double avg = (l > 0.f) ? (double)w / (double)l : 0.0;
+            p.vec_out[(size_t)bz * p.rows + row] = (float)(r * avg);
+            if (p.vec_rsum) p.vec_rsum[(size_t)bz * p.rows + row] = (float)r;
+            if (!isfinite(r) || !isfinite(avg)) atomicOr(p.err, kDevErrNonfinite);
+        }
+        return;  // uniform over the kernel: a launch parameter
     } else if (valid) {
         // Measure mode: with the current row potential pot_in, the plan's row sum is
         //   r_i = a_i exp((pot_i - pot~_i)/eps),  pot~_i = |row|^2 - eps ln2 LSE2_i,

@@ -62,6 +62,12 @@ struct PassParams {
     double *stats;             // [batch][row_blocks][4] measure partial sums
     double *tail_stats;        // update passes, or null: [batch][row_blocks][4] marginal statistics of the
                                // potential this pass writes (the plan's row sums at that potential)
+    // Measure passes with col_vec set take the plan-weighted average of a column
+    // vector instead of the cost: vec_out_i = sum_j P_ij v_j, vec_rsum_i = sum_j P_ij
+    // (may be null); no statistics.  Tensor-core passes only.
+    const float *col_vec;      // [batch][cols_stride], zero beyond cols
+    float *vec_out;            // [batch][rows]
+    float *vec_rsum;           // [batch][rows] or null
     const void *plain_rows;    // SIMT path: [batch][rows_pad][d] fp32
     const void *plain_cols;    // SIMT path: [batch][cols_rows][d] fp32
     unsigned long long timeout_ns;

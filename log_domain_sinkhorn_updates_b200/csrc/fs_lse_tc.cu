@@ -177,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_stride + col0, bias_bytes,
                           saddr(bfull + j));
                 if (MEASURE)
-                    bulk_load(saddr(sCN + j * kBlockCols), p.col_norm + (size_t)bz * p.cols_stride + col0, bias_bytes,
+                    bulk_load(saddr(sCN + j * kBlockCols),
+                              (p.col_vec ? p.col_vec : p.col_norm) + (size_t)bz * p.cols_stride + col0, bias_bytes,
                               saddr(bfull + j));
                 bias_issued = t + 1;
             }
@@ -274,7 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rl = q * 32 + lane;    // row within the block
         const int rblk = rb * QT + (QT == 2 ? grp : 0);  // this warp's 128-row block
         const float c = p.scale2;
-        const float xn = MEASURE ? p.row_norm[(size_t)bz * p.rows_stride + rblk * kBlockRows + rl] : 0.f;
+        // a vector pass weights each column by v_j alone: no row norm, no score term
+        const float xn = MEASURE && !p.col_vec ? p.row_norm[(size_t)bz * p.rows_stride + rblk * kBlockRows + rl] : 0.f;
+        const float wsscale = p.col_vec ? 0.f : p.sscale;
         float m = -INFINITY, l = 0.f, w = 0.f;
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * kBlockCols);
         bool ok = true;
@@ -320,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(sempty + grp);
                     }
-                    consume64_measure(ra, rb2, bias + 64 * qt, cnorm + 64 * qt, c, p.sscale, xn, m, l, w);
+                    consume64_measure(ra, rb2, bias + 64 * qt, cnorm + 64 * qt, c, wsscale, xn, m, l, w);
                 }
             }
             __syncwarp();

@@ -283,6 +283,22 @@ cudaError_t launch_weights(const float *w, int batch, int cnt, int cnt_pad, floa
     return cudaGetLastError();
 }
 
+// out[b][j] = v[b][j] for j < cnt, 0 up to stride: a per-point vector in the
+// padded per-point layout the streamed passes read
+__global__ void pad_vec_kernel(const float *v, int batch, int cnt, int stride, float *out) {
+    const size_t total = (size_t)batch * stride;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t b = i / stride;
+        const int j = (int)(i % stride);
+        out[i] = j < cnt ? v[b * cnt + j] : 0.f;
+    }
+}
+
+cudaError_t launch_pad_vec(const float *v, int batch, int cnt, int stride, float *out, cudaStream_t s) {
+    pad_vec_kernel<<<grid_for((size_t)batch * stride, 256), 256, 0, s>>>(v, batch, cnt, stride, out);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_fill(float *p, size_t count, float v, cudaStream_t s) {
     fill_kernel<<<grid_for(count, 256), 256, 0, s>>>(p, count, v);
     return cudaGetLastError();

@@ -27,6 +27,8 @@ cudaError_t launch_maxabs(const void *src, bool bf16, int rows, int d, int batch
 cudaError_t launch_weights(const float *w, int batch, int cnt, int cnt_pad, float *lw2, double *wstat,
                            cudaStream_t s);
 cudaError_t launch_fill(float *p, size_t count, float v, cudaStream_t s);
+// v [batch][cnt] -> out [batch][stride], zero beyond cnt.
+cudaError_t launch_pad_vec(const float *v, int batch, int cnt, int stride, float *out, cudaStream_t s);
 cudaError_t launch_bias(const float *pot, int batch, int cnt, int cnt_pad, const float *norm, const float *lw2,
                         double scale2, float *out, cudaStream_t s);
 // *flag |= 1 if the count floats at a and b differ in any bit.
