@@ -25,17 +25,16 @@
 // ring of V~ halves (64 columns, dv_pad rows per plane), the bias slices.
 //
 // Warps: 0 streams Q, the K tiles and the bias slices; 10 streams the V~
-// halves; 1 allocates TMEM and issues the MMAs; 2..5 and 6..9 are the softmax
-// groups of blocks 0 and 1, one warp per TMEM lane quadrant.  The two blocks
-// alternate (ping-pong): per tile t the issue order is block 0's P V
-// products, S_0(t + 1) once they have completed (its P~ columns are free
-// again), block 1's P V products, S_1(t + 1).  Block 1 so runs half a tile
-// behind block 0, and each block's softmax overlaps the other block's MMAs.
-// (Issuing both S products only after both blocks' P V products left both
-// softmax groups idle together while the tensor core worked: a clock64 trace
-// at n = m = 65536, d = 128 showed 7900 clk per tile then, 6740 in this
-// order.)  The issuing thread frees K slots and V~ halves itself with
-// tcgen05.commit.
+// halves; 1 allocates TMEM; 1 and 11 issue the MMAs of block 0 and of block 1
+// (one thread each); 2..5 and 6..9 are the softmax groups of blocks 0 and 1,
+// one warp per TMEM lane quadrant.  Each block's chain runs on its own:
+// S_g(t), its softmax, its P V products, and S_g(t + 1) once those have
+// completed (its P~ columns are free again); the tensor core interleaves the
+// two chains.  A K slot and a V~ half are free once both issuing threads'
+// commits after the products that read them have arrived.  (With one issuing
+// thread the two chains were serialised through it: a clock64 trace at n = m
+// = 65536, d = 128 showed 7900 clk per tile with both S products issued after
+// both blocks' P V products, and 6740 with the blocks alternating.)
 // Every wait is bounded; on expiry the kernel raises kDevErrTimeout, stops,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -47,7 +46,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kQ2Threads = 352;
+constexpr int kQ2Threads = 384;
 constexpr int kQ2TS = 128;   // columns per tile (N of the S product)
 constexpr int kQ2H = 64;     // columns per half (K of one P V product)
 constexpr int kQ2Bias = 4;   // bias-slice ring (tiles)
@@ -119,7 +118,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < KS; ++s) {
             mbar_init(kfull + s, 1);
-            mbar_init(kempty + s, 1);
+            mbar_init(kempty + s, 2);  // both blocks' S products have read the slot
         }
         for (int j = 0; j < kQ2Bias; ++j) {
             mbar_init(bfull + j, 1);
@@ -127,7 +126,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
         }
         for (int s = 0; s < NV; ++s) {
             mbar_init(vfull + s, 1);
-            mbar_init(vfree + s, 1);
+            mbar_init(vfree + s, 2);  // both blocks' P V products have read the half
         }
         mbar_init(qfull, 1);
         for (int g = 0; g < 2; ++g) {
@@ -136,7 +135,19 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
             mbar_init(pready + 2 * g + 1, 4);
             mbar_init(pfree + g, 1);
         }
-        mbar_init(ofull, 1);
+        mbar_init(ofull, 2);  // both issuing threads' last commits
+        if constexpr (PKS == 0) {  // descriptor offsets of the S products' K steps, for any width
+            const uint32_t plane = (uint32_t)p.plane_bytes;
+            const int ksteps = (int)(plane / 32u);
+            for (int i = 0; i < NPASS * ksteps; ++i) {
+                const int pass = i / ksteps, k = i % ksteps;
+                const uint32_t ao = (pass == 1 ? plane : 0u) + 32u * k;
+                const uint32_t bo = (pass == 2 ? plane : 0u) + 32u * k;
+                koff[i] = ((ao / swz) * (kBlockRows * swz) + ao % swz) >> 4;
+                koff[kQ2MaxKsteps + i] = bo / swz;
+                koff[2 * kQ2MaxKsteps + i] = (bo % swz) >> 4;
+            }
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -225,38 +236,27 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                 mbar_wait(vfull + (i % NV), (uint32_t)(i / NV) & 1u, p.timeout_ns);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == 1 || warp == 11) {
+        // ---------------- MMA issuers: warp 1 for block 0, warp 11 for block 1 ----------------
         if (lane == 0) {
+            const int g = warp == 1 ? 0 : 1;
             const uint32_t idesc_s = make_idesc<KIND, kBlockRows, kQ2TS>();
             // P~ V~: bf16 x bf16 -> fp32, M = 128, N = dv_pad, A from TMEM
             const uint32_t idesc_o = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.dv_pad >> 3) << 17) |
                                      ((uint32_t)(kBlockRows >> 4) << 24);
-            const uint32_t plane = (uint32_t)p.plane_bytes;
-            const int ksteps = (int)(plane / 32u);
-            const int nk = NPASS * ksteps;
-            if constexpr (PKS == 0) {
-                for (int i = 0; i < nk; ++i) {
-                    const int pass = i / ksteps, k = i % ksteps;
-                    const uint32_t ao = (pass == 1 ? plane : 0u) + 32u * k;
-                    const uint32_t bo = (pass == 2 ? plane : 0u) + 32u * k;
-                    koff[i] = ((ao / swz) * (kBlockRows * swz) + ao % swz) >> 4;
-                    koff[kQ2MaxKsteps + i] = bo / swz;
-                    koff[2 * kQ2MaxKsteps + i] = (bo % swz) >> 4;
-                }
-            }
-            const uint64_t adesc[2] = {make_sdesc(saddr(sQ), swz), make_sdesc(saddr(sQ) + qblock_bytes, swz)};
+            const int nk = NPASS * (p.plane_bytes / 32);
+            const uint64_t adesc = make_sdesc(saddr(sQ) + g * qblock_bytes, swz);
             // S_g(t) = Q_g K(t)^T into block g's columns
-            auto s_product = [&](const int g, const uint64_t (&bdesc)[4]) {
+            auto s_product = [&](const uint64_t (&bdesc)[4]) {
                 const uint32_t dt = tmem_base + (uint32_t)(g * kQ2TS);
                 if constexpr (PKS > 0) {
-                    issue_s_tile<KIND, NPASS, PKS, kBlockRows>(dt, adesc[g], bdesc, idesc_s);
+                    issue_s_tile<KIND, NPASS, PKS, kBlockRows>(dt, adesc, bdesc, idesc_s);
                 } else {
                     for (int i = 0; i < nk; ++i) {
                         const uint32_t ba = koff[kQ2MaxKsteps + i];
                         const uint64_t bd =
                             ba == 0 ? bdesc[0] : (ba == 1 ? bdesc[1] : (ba == 2 ? bdesc[2] : bdesc[3]));
-                        tc_mma<KIND>(dt, adesc[g] + koff[i], bd + koff[2 * kQ2MaxKsteps + i], idesc_s,
+                        tc_mma<KIND>(dt, adesc + koff[i], bd + koff[2 * kQ2MaxKsteps + i], idesc_s,
                                      i > 0 ? 1u : 0u);
                     }
                 }
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
             };
             // O_g += P~_g(t, h) V~(t, h): 4 K steps of 16 (8 TMEM columns of bf16 pairs each),
             // hi.hi + lo.hi (+ hi.lo); every offset and accumulate flag an immediate
-            auto pv_half = [&](const int g, const uint32_t vs, const int h, const uint32_t first) {
+            auto pv_half = [&](const uint32_t vs, const int h, const uint32_t first) {
                 const uint32_t to = tmem_base + 256u + (uint32_t)(g * kQ2TS);
                 const uint32_t phi = tmem_base + (uint32_t)(g * kQ2TS + h * kQ2H);
                 const uint32_t plo = phi + 32u;
@@ -296,48 +296,39 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                 uint64_t bdesc[4];
                 ok = ok && k_tile(0, bdesc);
                 if (ok) {
-                    s_product(0, bdesc);
-                    s_product(1, bdesc);
+                    s_product(bdesc);
                     for (int a = 0; a < atoms; ++a) tc_commit(saddr(kempty + (a % KS)));
                 }
             }
-            uint64_t bnext[4] = {0ull, 0ull, 0ull, 0ull};
             for (int t = 0; ok && t < ntiles; ++t) {
                 const uint32_t tp = (uint32_t)t & 1u;
-                for (int g = 0; ok && g < 2; ++g) {
-                    for (int h = 0; h < 2; ++h) {  // O_g += P~_g(t) V~(t)
-                        const int hh = 2 * t + h, s = hh % NV;
-                        if (!mbar_wait(pready + 2 * g + h, tp, p.timeout_ns) ||
-                            !mbar_wait(vfull + s, (uint32_t)(hh / NV) & 1u, p.timeout_ns) || *abort_flag) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t vs = saddr(sV + (size_t)s * L.vstage);
-                        if (t == 0 && h == 0)
-                            pv_half(g, vs, h, 0u);
-                        else
-                            pv_half(g, vs, h, 1u);
-                        if (g == 1) tc_commit(saddr(vfree + s));  // both blocks have read this V~ half
-                    }
-                    if (!ok) break;
-                    tc_commit(saddr(pfree + g));
-                    if (t + 1 >= ntiles) continue;
-                    // S_g(t + 1) as soon as block g's P~ columns are free again,
-                    // before the other block's products of tile t
-                    if (g == 0 && !k_tile(t + 1, bnext)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!mbar_wait(pfree + g, tp, p.timeout_ns) || *abort_flag) {
+                for (int h = 0; h < 2; ++h) {  // O_g += P~_g(t) V~(t)
+                    const int hh = 2 * t + h, s = hh % NV;
+                    if (!mbar_wait(pready + 2 * g + h, tp, p.timeout_ns) ||
+                        !mbar_wait(vfull + s, (uint32_t)(hh / NV) & 1u, p.timeout_ns) || *abort_flag) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    s_product(g, bnext);
-                    if (g == 1)
-                        for (int a = 0; a < atoms; ++a) tc_commit(saddr(kempty + (((t + 1) * atoms + a) % KS)));
+                    const uint32_t vs = saddr(sV + (size_t)s * L.vstage);
+                    if (t == 0 && h == 0)
+                        pv_half(vs, h, 0u);
+                    else
+                        pv_half(vs, h, 1u);
+                    tc_commit(saddr(vfree + s));
                 }
+                if (!ok) break;
+                tc_commit(saddr(pfree + g));
+                if (t + 1 >= ntiles) break;
+                // S_g(t + 1) as soon as this block's P~ columns are free again
+                uint64_t bdesc[4];
+                if (!k_tile(t + 1, bdesc) || !mbar_wait(pfree + g, tp, p.timeout_ns) || *abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                s_product(bdesc);
+                for (int a = 0; a < atoms; ++a) tc_commit(saddr(kempty + (((t + 1) * atoms + a) % KS)));
             }
             if (!ok) {
                 atomicOr(p.err, kDevErrTimeout);
@@ -347,7 +338,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
             mbar_wait(ofull, 0, p.timeout_ns);
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 2 && warp < 10) {
         // ---------------- softmax groups: group g owns row block g ----------------
         const int q = warp & 3;
         const int grp = (warp - 2) >> 2;
