@@ -224,6 +224,9 @@ fs::PassParams make_pass(const fs_handle *h, bool fdir, bool measure) {
     p.tiles_per_split = fdir ? h->tps_f : h->tps_g;
     p.col_tiles = (p.cols + kBlockCols - 1) / kBlockCols;
     p.stages = measure ? h->stages_meas : h->stages;
+    // two MMA-issuing threads for one-pass operands and short split jobs (see fs_lse_tc.cu)
+    const int npass = (h->prec == FS_PREC_3XTF32 || h->prec == FS_PREC_3XF16) ? 3 : 1;
+    p.issuers = (npass == 1 || npass * (h->plane_bytes / 32) <= 4) ? 2 : 1;
     p.eps = (double)D.eps;
     p.scale2 = (float)(fs::kLog2ed / (double)D.eps * (double)h->sscale);
     p.sscale = h->sscale;

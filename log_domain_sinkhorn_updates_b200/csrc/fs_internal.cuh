@@ -47,6 +47,8 @@ struct PassParams {
     int tiles_per_split;       // column tiles handled by one split
     int col_tiles;             // 256-column tiles covering cols
     int stages;                // pipeline depth (tensor-core path)
+    int issuers;               // MMA-issuing threads of the one-CTA tensor-core pass: 1, or 2 (one per TMEM
+                               // buffer, so the two softmax groups' score chains do not wait on each other)
     float scale2;              // log2(e)/eps, times sscale
     float sscale;              // factor from the MMA's raw score to S_ij (1 unless operands were scaled)
     double eps;

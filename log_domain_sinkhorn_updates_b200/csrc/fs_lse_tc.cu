@@ -23,8 +23,17 @@
 // Nothing of size n*m ever leaves the SM: the pass writes one potential per
 // row (fused epilogue, section 2).
 //
-// Warp roles (320 threads): warp 0 = TMA producer, warp 1 = TMEM allocator and
-// MMA issuer, warps 2..9 = softmax.  Every mbarrier wait is bounded by
+// Warp roles (352 threads): warp 0 = TMA producer, warp 1 = TMEM allocator and
+// MMA issuer, warps 2..9 = softmax, warp 10 = the second MMA issuer when
+// p.issuers = 2: warp 1 then issues the even jobs and warp 10 the odd ones, so
+// one softmax group's wait for its buffer never holds back the other group's
+// next S.  Measured per pass: bf16 at d = 128 (8 MMAs per job) 2 % faster at
+// equal clock, 3xF16 at d = 3 (3 MMAs) 2 % faster, 3xF16 at d = 32 (6 MMAs)
+// 1 % slower, 3xF16 at d = 64 (12 MMAs) 5 % slower: the two groups' MMAs
+// interleave in the pipe and both S arrive late.  So two threads issue for
+// one-pass operands and for split jobs of at most 4 MMAs.  The K slots of a
+// tile go back to the producer through a commit after each of its jobs.
+// Every mbarrier wait is bounded by
 // p.timeout_ns; on expiry the kernel raises kDevErrTimeout, stops issuing,
 // drains its own copies and MMAs, frees TMEM and returns.
 //
@@ -39,7 +48,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kTmemCols = 512;   // two 256-column fp32 accumulators
 constexpr int kMaxKsteps = 64;   // MMA instructions per tile: NPASS x (plane bytes / 32) <= 3 x 16
 constexpr int kMaxAtoms = 4;     // swizzle atoms per packed row (row_bytes <= 512)
@@ -113,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(full + s, 1);
-            mbar_init(empty + s, 1);  // the softmax group of the tile's last job
+            mbar_init(empty + s, QT);  // a commit after each of the tile's jobs
         }
         for (int j = 0; j < kBiasSlots; ++j) {
             mbar_init(bfull + j, 1);
@@ -124,7 +133,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(sfull + b, 1);
             mbar_init(sempty + b, 4);
         }
-        mbar_init(drain, 1);
+        mbar_init(drain, p.issuers == 2 ? 2 : 1);
+        {  // descriptor offsets of a tile's MMAs (A slice in the Q tile; B atom and offset)
+            const uint32_t plane = (uint32_t)p.plane_bytes;
+            const int ksteps = (int)(plane / 32u);
+            for (int i = 0; i < NPASS * ksteps; ++i) {
+                const int pass = i / ksteps, k = i % ksteps;
+                // (A plane, B plane) = (hi,hi), (lo,hi), (hi,lo)
+                const uint32_t ao = (pass == 1 ? plane : 0u) + 32u * k;
+                const uint32_t bo = (pass == 2 ? plane : 0u) + 32u * k;
+                koff[i] = ((ao / swz) * (kBlockRows * swz) + ao % swz) >> 4;
+                koff[kMaxKsteps + i] = bo / swz;
+                koff[2 * kMaxKsteps + i] = (bo % swz) >> 4;
+            }
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -194,29 +216,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_wait(bfull + (t % kBiasSlots), (uint32_t)(t / kBiasSlots) & 1u, p.timeout_ns);
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == 1 || (warp == 10 && p.issuers == 2)) {  // (the launcher admits 1 or 2)
+        // ---------------- MMA issuer(s) ----------------
+        // One thread issues every job, or (issuers = 2) warp 1 the even jobs
+        // (TMEM buffer 0) and warp 10 the odd ones (buffer 1).
         if (lane == 0) {
             const uint32_t idesc = make_idesc<KIND>();
-            // For every MMA of a tile: the A-descriptor offset of its K slice in
-            // the Q tile, and which atom (ring slot) and offset of B it reads.
-            const uint32_t plane = (uint32_t)p.plane_bytes;
-            const int ksteps = (int)(plane / 32u);
-            const int nk = NPASS * ksteps;
-            for (int i = 0; i < nk; ++i) {
-                const int pass = i / ksteps, k = i % ksteps;
-                // (A plane, B plane) = (hi,hi), (lo,hi), (hi,lo)
-                const uint32_t ao = (pass == 1 ? plane : 0u) + 32u * k;
-                const uint32_t bo = (pass == 2 ? plane : 0u) + 32u * k;
-                koff[i] = ((ao / swz) * (kBlockRows * swz) + ao % swz) >> 4;
-                koff[kMaxKsteps + i] = bo / swz;
-                koff[2 * kMaxKsteps + i] = (bo % swz) >> 4;
-            }
+            const int nk = NPASS * (p.plane_bytes / 32);
+            const int jstep = p.issuers == 2 ? 2 : 1, jb0 = warp == 1 ? 0 : 1;
             const uint64_t adesc0 = make_sdesc(saddr(sQ), swz);
             const uint32_t qstride = (uint32_t)(atoms * kBlockRows * swz) >> 4;  // one Q tile, in descriptor units
             bool ok = mbar_wait(qfull, 0, p.timeout_ns);
             uint64_t bdesc[kMaxAtoms];
-            for (int jb = 0; ok && jb < njobs; ++jb) {
+            for (int jb = jb0; ok && jb < njobs; jb += jstep) {
                 const int b = jb & 1;
                 const int t = QT == 2 ? (jb >> 1) : jb;
                 const int qt = QT == 2 ? b : 0;
@@ -224,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                if (qt == 0) {  // first job of tile t: wait for its K slots
+                if (qt == 0 || jstep == 2) {  // tile t's K slots (the first job of the tile, or each job)
 #pragma unroll
                     for (int a = 0; a < kMaxAtoms; ++a) {
                         if (a < atoms) {
@@ -249,11 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_mma<KIND>(dt, adesc + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
                     }
                 }
-                // One commit per job: it completes when the job's MMAs have read
-                // their operands and written S.  The softmax group that waits on
-                // it hands the tile's K slots back after the tile's last job.  (A
-                // commit stalls the MMA pipe, so the chain carries no other.)
+                // A commit per job for its softmax group, and one per K slot: the
+                // slot is free once every job of its tile has read it (QT arrivals).
                 tc_commit(saddr(sfull + b));
+                for (int a = 0; a < atoms; ++a) tc_commit(saddr(empty + ((t * atoms + a) % NS)));
             }
             if (!ok) {
                 atomicOr(p.err, kDevErrTimeout);
@@ -264,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(drain, 0, p.timeout_ns);
         }
         __syncwarp();
-    } else {
+    } else if (warp >= 2 && warp < 10) {
         // ---------------- softmax warps ----------------
         // Group 0 (warps 2..5) takes the even tiles, which the MMA writes to TMEM
         // buffer 0; group 1 (warps 6..9) the odd tiles in buffer 1.  The two
@@ -290,8 +301,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            if (q == 2 && lane == 0 && (QT == 1 || grp == 1))  // tile t's last job is complete: its K slots are free
-                for (int a = 0; a < atoms; ++a) mbar_arrive(empty + ((t * atoms + a) % NS));
             const float *bias = sBias + j * kBlockCols;
             if (!MEASURE) {
 #pragma unroll 1
@@ -423,6 +432,7 @@ int tc_max_stages(int row_bytes, int qt, bool measure) {
 // prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16; qt: 128-row blocks per CTA (1 or 2).
 cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int qt, const void *map_rows,
                           const void *map_cols, size_t smem, cudaStream_t s) {
+    if (p.issuers != 1 && p.issuers != 2) return cudaErrorInvalidValue;
     if (qt != 1 && qt != 2) return cudaErrorInvalidValue;
     if (prec == 1) return launch_kind<0, 1>(p, batch, measure, qt, map_rows, map_cols, smem, s);
     if (prec == 2) return launch_kind<1, 1>(p, batch, measure, qt, map_rows, map_cols, smem, s);
