@@ -124,7 +124,9 @@ typedef struct {
                                FS_ROW_BLOCKS=1); 3 tensor cores on CTA pairs
                                (512-byte operand rows, or any width with FS_APPLY_PAIR=1); 2 CUDA
                                cores (dv over 256, the f32_simt precision, or FS_APPLY_SIMT=1);
-                               0 none yet */
+                               5 one column (dv = 1) through the streamed LSE pass with the column
+                               vector as its weight (tensor-core handles; FS_APPLY_VEC=0 keeps the
+                               kernels above); 0 none yet */
     int last_solve_graph;   /* how the handle's last fs_solve ran: 1 as a replay of its CUDA graph,
                                2 as direct launches (a large problem, FS_SOLVE_GRAPH=0, or a
                                failed capture), 0 none yet */
@@ -244,7 +246,11 @@ FS_API fs_status fs_destroy(fs_handle *h);
  *   r[k][i]      = sum_j P_ij                 (device [batch][n]; may be NULL)
  * out: device fp32 [batch][n][dv].  Scores come from the handle's packed
  * operands (its precision); the exponent is formed in double and the sums in
- * fp32.  Asynchronous.  Errors: FS_ERR_INVALID_ARG (null pointer, dv < 1).
+ * fp32.  A single column (dv = 1) on a tensor-core handle runs as a streamed
+ * LSE pass that weights each column by V_j (the plan-weighted average beside
+ * the row's LSE state), at that pass's cost; it takes an fp32 scratch of the
+ * column side's length from the device's memory pool for the call.
+ * Asynchronous.  Errors: FS_ERR_INVALID_ARG (null pointer, dv < 1).
  */
 FS_API fs_status fs_transport_apply(fs_handle *h, const float *f, const float *g, const float *V, int dv,
                                     float *out, float *r);

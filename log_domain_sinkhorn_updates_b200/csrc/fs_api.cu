@@ -663,6 +663,30 @@ fs_status hvp_fused_term(fs_handle *h, const float *f, const float *g, const voi
 
 }  // namespace
 
+// A single column on a tensor-core handle goes through the LSE pass's vector mode
+// (apply_vec), unless FS_APPLY_VEC=0 or the CUDA-core path is asked for.
+static bool vec_path(const fs_handle *h, int dv) {
+    if (dv != 1 || h->prec == FS_PREC_F32_SIMT) return false;
+    const char *e = getenv("FS_APPLY_VEC");
+    if (e && atoi(e) == 0) return false;
+    const char *s = getenv("FS_APPLY_SIMT");
+    return !(s && atoi(s) != 0);
+}
+static fs_status apply_vec_alloc(fs_handle *h, const float *f, const float *g, const float *v, bool fdir,
+                                 float *out, float *r) {
+    const fs_desc &D = h->desc;
+    FS_CUDA(h, cudaSetDevice(h->device));
+    cudaMemPool_t pool;
+    float *vpad = nullptr;
+    FS_CUDA(h, device_pool(h->device, &pool));
+    FS_CUDA(h, cudaMallocFromPoolAsync((void **)&vpad, (size_t)D.batch * (fdir ? h->m_stride : h->n_stride) * 4,
+                                       pool, h->stream));
+    const fs_status st = apply_vec(h, f, g, v, fdir, out, r, vpad);
+    cudaFreeAsync(vpad, h->stream);
+    if (st == FS_OK) h->last_apply = 5;
+    return st;
+}
+
 extern "C" {
 
 // ---- transport application ("FlashSinkhorn: IO-aware EOT on GPU", Metodologia
@@ -670,6 +694,7 @@ extern "C" {
 fs_status fs_transport_apply(fs_handle *h, const float *f, const float *g, const float *V, int dv, float *out,
                              float *r) {
     if (!h || !f || !g || !V || !out || dv < 1) return fail(h, FS_ERR_INVALID_ARG, "bad argument");
+    if (vec_path(h, dv)) return apply_vec_alloc(h, f, g, V, true, out, r);
     return apply(h, f, g, V, false, dv, out, r, false);
 }
 
@@ -717,6 +742,7 @@ fs_status fs_grad_x(fs_handle *h, const float *f, const float *g, const void *X,
 fs_status fs_transport_apply_t(fs_handle *h, const float *f, const float *g, const float *U, int du, float *out,
                                float *c) {
     if (!h || !f || !g || !U || !out || du < 1) return fail(h, FS_ERR_INVALID_ARG, "bad argument");
+    if (vec_path(h, du)) return apply_vec_alloc(h, f, g, U, false, out, c);
     return apply(h, f, g, U, false, du, out, c, false, false);
 }
 

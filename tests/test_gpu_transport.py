@@ -83,6 +83,7 @@ def _set_path(monkeypatch, path):
     monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
     monkeypatch.setenv("FS_APPLY_PAIR", PATHS[path][1])
     monkeypatch.setenv("FS_ROW_BLOCKS", PATHS[path][2])
+    monkeypatch.setenv("FS_APPLY_VEC", "0")  # one-column applications through these kernels too
 
 
 def _assert_path(fs, h, path, dv):
@@ -357,13 +358,14 @@ def test_transport_apply_tf32_kind(cuda_device, name, prec):
 
 
 @pytest.mark.parametrize("case", ["f32-d128-auto", "f32-d64-3xtf32", "cosine-d128-auto", "bf16-d256-auto"])
-def test_transport_apply_wide_rows_on_cta_pairs(cuda_device, case):
+def test_transport_apply_wide_rows_on_cta_pairs(cuda_device, case, monkeypatch):
     """Handles whose packed operand rows are 512 bytes run their passes on CTA pairs; their
     transport application must run on the tensor cores too, by default, within the same
     bound: fp32 clouds at d = 128 (3xF16), 3xTF32 at d = 64, the cosine cost at d = 128,
     and bf16 clouds at d = 256 (one plane of 256 values).  Every one of these forms the
     score to about fp32 accuracy, which the bound assumes (one-pass TF32 does not)."""
     import torch
+    monkeypatch.setenv("FS_APPLY_VEC", "0")  # dv = 1 through the pair kernel too
     fs = _fs()
     kind, dim, prec = case.split("-")
     name = "middim" if dim == "d64" else "highdim"
@@ -400,3 +402,46 @@ def test_transport_apply_wide_rows_on_cta_pairs(cuda_device, case):
         rerr = np.abs(r.cpu().numpy()[0] - ro) / (rel * ro)
         print(f"{case} dv={dv}: worst err / bound = {err.max():.3f}, row sums {rerr.max():.3f}")
         assert err.max() <= 1.0 and rerr.max() <= 1.0
+
+
+@pytest.mark.parametrize("transposed", [False, True])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_one_column_through_the_lse_pass(cuda_device, name, transposed, monkeypatch):
+    """dv = 1 on a tensor-core handle runs as a streamed LSE pass weighting each
+    column by V_j (last_apply_path "lse_vec"): (P v)_i = r_i w_i / l_i with the
+    running max, fp32 sums and no bf16 split, so the CUDA-core bound applies
+    (no 2^-14 term)."""
+    import torch
+    monkeypatch.delenv("FS_APPLY_VEC", raising=False)
+    monkeypatch.delenv("FS_APPLY_SIMT", raising=False)
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    f32, g32 = _potentials(prob, "sqeuclidean")
+    rng = np.random.default_rng(555)
+    cnt_in, cnt_out = (prob.n, prob.m) if transposed else (prob.m, prob.n)
+    V = rng.standard_normal((prob.batch, cnt_in, 1)).astype(np.float32)
+    out = torch.empty(prob.batch, cnt_out, 1, device=cuda_device)
+    r = torch.empty(prob.batch, cnt_out, device=cuda_device)
+    fd, gd, Vd = (torch.from_numpy(x).to(cuda_device) for x in (f32, g32, V))
+    if transposed:
+        fs.fs_transport_apply_t(h, fd, gd, Vd, out, r)
+    else:
+        fs.fs_transport_apply(h, fd, gd, Vd, out, r)
+    fs.fs_sync(h)
+    assert fs.fs_get_info(h)["last_apply_path"] == "lse_vec"
+    out, r = out.cpu().numpy(), r.cpu().numpy()
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        fk, gk = f32[k].astype(np.float64), g32[k].astype(np.float64)
+        if transposed:  # P^T v: the transposed problem's rows are Y's points
+            args = (Yo, Xo, logb, loga, gk, fk)
+        else:
+            args = (Xo, Yo, loga, logb, fk, gk)
+        oo, ro = oracle.transport_apply(*args, prob.eps, V[k].astype(np.float64))
+        absw, _ = oracle.transport_apply(*args, prob.eps, np.abs(V[k]).astype(np.float64))
+        rel = _rel_bound(*args, prob.eps, "sqeuclidean")
+        err = (np.abs(out[k] - oo) / (rel[:, None] * absw)).max()
+        rerr = (np.abs(r[k] - ro) / (rel * ro)).max()
+        print(f"{name}[{k}] transposed={transposed}: worst err / bound {err:.3f}, row sums {rerr:.3f}")
+        assert err <= 1.0 and rerr <= 1.0
