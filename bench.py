@@ -42,6 +42,8 @@ APPLY_KERNELS = {
     "tc_q2": (PROFILE_TRAFFIC_APPLY_Q2, "fs_apply_tc_q2.cu",
               "apply_q2_kernel (two 128-row blocks per CTA: S = Q K^T, P~ back into TMEM, O += P~ V~)"),
     "tc": (PROFILE_TRAFFIC_APPLY, "fs_apply_tc.cu", "apply_tc_kernel (S = Q K^T, then O += P~ V~)"),
+    "tc_2s": (None, "fs_apply_tc_q2.cu",
+              "apply_q2_kernel, one row block (both groups on one block, alternate tiles, P~ in TMEM)"),
     "tc_pair": (None, "fs_apply_tc2.cu", "apply_tc2_kernel (CTA pairs: S = Q K^T, then O += P~ V~)"),
     "simt": (None, "fs_apply.cu", "apply_simt_kernel (CUDA cores)"),
 }

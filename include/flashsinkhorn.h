@@ -118,12 +118,16 @@ typedef struct {
                                variable FS_CTA_PAIR=1 (FS_CTA_PAIR=0 forbids it) */
     int last_apply_path;    /* kernel of the handle's last transport application (fs_transport_apply
                                and the calls built on it): 4 tensor cores, one CTA per 256 rows (two
-                               128-row blocks sharing every streamed tile; dv <= 128, rows of up to
+                               128-row blocks sharing every streamed tile; dv < 64, rows of up to
                                256 bytes, at least one such CTA per SM, or FS_ROW_BLOCKS=2 at any
-                               size); 1 tensor cores, one CTA per 128 rows (otherwise, or with
+                               size); 1 tensor cores, one CTA per 128 rows (dv over 128, or with
                                FS_ROW_BLOCKS=1); 3 tensor cores on CTA pairs
                                (512-byte operand rows, or any width with FS_APPLY_PAIR=1); 2 CUDA
                                cores (dv over 256, the f32_simt precision, or FS_APPLY_SIMT=1);
+                               6 tensor cores, one CTA per 128 rows with both softmax groups on the
+                               block, taking alternate tiles into their own TMEM columns (dv <= 128,
+                               rows of up to 256 bytes, where mode 4 is not taken; FS_ROW_BLOCKS=3
+                               at any size);
                                5 one column (dv = 1) through the streamed LSE pass with the column
                                vector as its weight (tensor-core handles; FS_APPLY_VEC=0 keeps the
                                kernels above); 0 none yet */

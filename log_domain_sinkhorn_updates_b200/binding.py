@@ -47,7 +47,7 @@ class FsInfo(ctypes.Structure):
     def as_dict(self):
         d = {k: getattr(self, k) for k, _ in self._fields_}
         d["prec"] = PRECISION_NAMES.get(d["prec"], d["prec"])
-        d["last_apply_path"] = {0: None, 1: "tc", 2: "simt", 3: "tc_pair", 4: "tc_q2", 5: "lse_vec"}.get(d["last_apply_path"],
+        d["last_apply_path"] = {0: None, 1: "tc", 2: "simt", 3: "tc_pair", 4: "tc_q2", 5: "lse_vec", 6: "tc_2s"}.get(d["last_apply_path"],
                                                                                d["last_apply_path"])
         d["last_solve_graph"] = {0: None, 1: "graph", 2: "direct"}.get(d["last_solve_graph"], d["last_solve_graph"])
         return d

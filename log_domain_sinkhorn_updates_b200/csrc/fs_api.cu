@@ -373,19 +373,25 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     int kslots = 0, stages = 0;
     size_t smem = 0;
     bool use_q2 = false;
+    int qb = 2;
     if (tc_ok && use_pair)
         smem = fs::apply_tc2_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
     if (tc_ok && smem == 0 && !h->pair && h->row_bytes <= 256) {
         use_pair = false;
         dv_pad = (dv + 15) / 16 * 16;
-        // two blocks per CTA where that still gives every SM a CTA (else the
-        // one-block grid, twice as many CTAs, runs more of the work in parallel);
-        // FS_ROW_BLOCKS=1 forces one block, FS_ROW_BLOCKS=2 two wherever they fit
+        // Two 128-row blocks per CTA for narrow V where that still gives every SM
+        // a CTA; else one block shared by both groups, which take alternate tiles
+        // (twice the CTAs).  Measured at dv = 128 (n = m = 65536): 3.33 ms shared,
+        // 3.41 two blocks; middim (dv = 64, 64 two-block CTAs): 0.299 shared, 0.352
+        // the one-block kernel; dv = 3 and dv = 32: two blocks 1-3 % faster.
+        // FS_ROW_BLOCKS=1 forces the one-block kernel of fs_apply_tc.cu, =2 two
+        // blocks, =3 one shared block, wherever they fit.
         const char *env_rb = getenv("FS_ROW_BLOCKS");
         const int rbk = env_rb ? atoi(env_rb) : 0;
         const long long q2_ctas = (long long)D.batch * ((p.rows_pad + 255) / 256);
-        if (rbk == 2 || (rbk != 1 && q2_ctas >= h->sms)) {
-            smem = fs::apply_q2_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
+        if (rbk != 1) {
+            qb = rbk == 2 ? 2 : (rbk == 3 ? 1 : (q2_ctas >= h->sms && dv < 64 ? 2 : 1));
+            smem = fs::apply_q2_plan(h->row_bytes, dv_pad, vpl, qb, &kslots, &stages);
             use_q2 = smem != 0;
         }
         if (smem == 0) smem = fs::apply_tc_plan(h->row_bytes, dv_pad, vpl, &kslots, &stages);
@@ -395,7 +401,7 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
         FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
         return FS_OK;
     }
-    h->last_apply = use_pair ? 3 : (use_q2 ? 4 : 1);
+    h->last_apply = use_pair ? 3 : (use_q2 ? (qb == 2 ? 4 : 6) : 1);
     p.row_bytes = h->row_bytes;
     p.swz = h->swz;
     p.plane_bytes = h->plane_bytes;
@@ -439,7 +445,7 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
                 g_launches.fetch_add(1, std::memory_order_relaxed);
             }
         } else if (use_q2) {
-            e = fs::launch_apply_q2(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r,
+            e = fs::launch_apply_q2(p, D.batch, h->prec, vpl, qb, fdir ? &h->mapX_r : &h->mapY_r,
                                     fdir ? &h->mapY_r : &h->mapX_r, &map_v, smem, h->stream);
             g_launches.fetch_add(1, std::memory_order_relaxed);
         } else {

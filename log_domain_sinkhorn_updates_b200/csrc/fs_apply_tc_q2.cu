@@ -53,22 +53,24 @@ constexpr int kQ2Bias = 4;   // bias-slice ring (tiles)
 constexpr int kQ2MaxKsteps = 64;
 
 struct Q2Layout {
-    uint32_t q, k, v, vstage, bias, koff, bars, misc, total;
+    uint32_t q, k, v, vstage, bias, koff, rs, bars, misc, total;
 };
 
 __host__ __device__ inline int q2swz(int row_bytes) { return row_bytes <= 32 ? 32 : (row_bytes <= 64 ? 64 : 128); }
 
 // V~ stage = [plane 0 (| plane 1)], dv_pad rows of 64 bf16 (128 bytes, 128-byte swizzle).
-__host__ __device__ inline Q2Layout q2_layout(int row_bytes, int kslots, int dv_pad, int vpl, int vstages) {
+__host__ __device__ inline Q2Layout q2_layout(int row_bytes, int kslots, int dv_pad, int vpl, int vstages,
+                                              int qb) {
     Q2Layout L;
     const uint32_t swz = (uint32_t)q2swz(row_bytes);
     L.q = 0;
-    L.k = L.q + 2u * kBlockRows * (uint32_t)row_bytes;
+    L.k = L.q + (uint32_t)qb * kBlockRows * (uint32_t)row_bytes;
     L.v = L.k + (uint32_t)kslots * kQ2TS * swz;
     L.vstage = (uint32_t)vpl * dv_pad * 128;
     L.bias = L.v + (uint32_t)vstages * L.vstage;
     L.koff = L.bias + kQ2Bias * kQ2TS * 4;
-    L.bars = L.koff + 3 * kQ2MaxKsteps * 4;
+    L.rs = L.koff + 3 * kQ2MaxKsteps * 4;  // one row block: group 1's row sums for group 0
+    L.bars = L.rs + (qb == 1 ? kBlockRows * 4 : 0);
     L.misc = L.bars + (2 * kslots + 2 * kQ2Bias + 2 * vstages + 10) * 8;
     L.total = L.misc + 16;
     return L;
@@ -76,7 +78,11 @@ __host__ __device__ inline Q2Layout q2_layout(int row_bytes, int kslots, int dv_
 
 // PKS > 0: the K-step count of an operand plane, fixed at compile time (the S
 // products are issued with immediate descriptor offsets); PKS = 0: any width.
-template <int KIND, int NPASS, int VPL, int PKS>
+// QB = 2: two row blocks, group g (and issuing thread g) owns block g and every
+// tile.  QB = 1: one row block shared by both groups; group g takes the tiles of
+// parity g into its own S / P~ columns and its own O, and group 0 adds the two O
+// at the end.
+template <int KIND, int NPASS, int VPL, int PKS, int QB>
 __global__ void __launch_bounds__(kQ2Threads, 1)
     apply_q2_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const ApplyParams p) {
@@ -89,13 +95,14 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
     const uint32_t kslot_bytes = (uint32_t)kQ2TS * swz;
     const uint32_t vplane_bytes = (uint32_t)p.dv_pad * 128u;
     const uint32_t qblock_bytes = (uint32_t)kBlockRows * p.row_bytes;
-    const Q2Layout L = q2_layout(p.row_bytes, KS, p.dv_pad, VPL, NV);
+    const Q2Layout L = q2_layout(p.row_bytes, KS, p.dv_pad, VPL, NV, QB);
 
     uint8_t *sQ = smem + L.q;
     uint8_t *sK = smem + L.k;
     uint8_t *sV = smem + L.v;
     float *sBias = reinterpret_cast<float *>(smem + L.bias);
     uint32_t *koff = reinterpret_cast<uint32_t *>(smem + L.koff);
+    float *sRs = reinterpret_cast<float *>(smem + L.rs);
     uint64_t *kfull = reinterpret_cast<uint64_t *>(smem + L.bars);
     uint64_t *kempty = kfull + KS;
     uint64_t *bfull = kempty + KS;
@@ -111,22 +118,22 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rb = blockIdx.x, bz = blockIdx.z;  // rows [256 rb, 256 rb + 256) of problem bz
+    const int rb = blockIdx.x, bz = blockIdx.z;  // rows [QB 128 rb, QB 128 (rb + 1)) of problem bz
     const int ntiles = (p.cols + kQ2TS - 1) / kQ2TS;
     const uint32_t tmem_cols = 512u;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < KS; ++s) {
             mbar_init(kfull + s, 1);
-            mbar_init(kempty + s, 2);  // both blocks' S products have read the slot
+            mbar_init(kempty + s, QB);  // the S products that read the slot
         }
         for (int j = 0; j < kQ2Bias; ++j) {
             mbar_init(bfull + j, 1);
-            mbar_init(bempty + j, 8);  // every softmax warp of both blocks reads each slice
+            mbar_init(bempty + j, 4 * QB);  // the softmax warps that read the slice
         }
         for (int s = 0; s < NV; ++s) {
             mbar_init(vfull + s, 1);
-            mbar_init(vfree + s, 2);  // both blocks' P V products have read the half
+            mbar_init(vfree + s, QB);  // the P V products that read the half
         }
         mbar_init(qfull, 1);
         for (int g = 0; g < 2; ++g) {
@@ -167,11 +174,11 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
         if (lane == 0) {
             bool ok = true;
             int k_issued = 0, b_issued = 0;
-            mbar_expect_tx(qfull, 2u * qblock_bytes);
-            for (int g = 0; g < 2; ++g)
+            mbar_expect_tx(qfull, (uint32_t)QB * qblock_bytes);
+            for (int g = 0; g < QB; ++g)
                 for (int a = 0; a < atoms; ++a)
                     tma_load_2d(saddr(sQ) + g * qblock_bytes + a * kBlockRows * swz, &map_q, saddr(qfull),
-                                a * box_inner, bz * p.rows_pad + rb * 2 * kBlockRows + g * kBlockRows);
+                                a * box_inner, bz * p.rows_pad + rb * QB * kBlockRows + g * kBlockRows);
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int col0 = t * kQ2TS;
                 if (*abort_flag) break;
@@ -237,15 +244,17 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
         }
         __syncwarp();
     } else if (warp == 1 || warp == 11) {
-        // ---------------- MMA issuers: warp 1 for block 0, warp 11 for block 1 ----------------
+        // ---------------- MMA issuers: warp 1 for group 0, warp 11 for group 1 ----------------
         if (lane == 0) {
             const int g = warp == 1 ? 0 : 1;
+            // this group's tiles: every tile of its own block (QB = 2), or the tiles of parity g
+            const int t_first = QB == 2 ? 0 : g, t_step = QB == 2 ? 1 : 2;
             const uint32_t idesc_s = make_idesc<KIND, kBlockRows, kQ2TS>();
             // P~ V~: bf16 x bf16 -> fp32, M = 128, N = dv_pad, A from TMEM
             const uint32_t idesc_o = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.dv_pad >> 3) << 17) |
                                      ((uint32_t)(kBlockRows >> 4) << 24);
             const int nk = NPASS * (p.plane_bytes / 32);
-            const uint64_t adesc = make_sdesc(saddr(sQ) + g * qblock_bytes, swz);
+            const uint64_t adesc = make_sdesc(saddr(sQ) + (QB == 2 ? g : 0) * qblock_bytes, swz);
             // S_g(t) = Q_g K(t)^T into block g's columns
             auto s_product = [&](const uint64_t (&bdesc)[4]) {
                 const uint32_t dt = tmem_base + (uint32_t)(g * kQ2TS);
@@ -292,16 +301,17 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
             };
             bool ok = mbar_wait(qfull, 0, p.timeout_ns);
             tc_fence_after();
-            {
+            if (QB == 2 || t_first < ntiles) {
                 uint64_t bdesc[4];
-                ok = ok && k_tile(0, bdesc);
+                ok = ok && k_tile(t_first, bdesc);
                 if (ok) {
                     s_product(bdesc);
-                    for (int a = 0; a < atoms; ++a) tc_commit(saddr(kempty + (a % KS)));
+                    for (int a = 0; a < atoms; ++a) tc_commit(saddr(kempty + ((t_first * atoms + a) % KS)));
                 }
             }
-            for (int t = 0; ok && t < ntiles; ++t) {
-                const uint32_t tp = (uint32_t)t & 1u;
+            for (int t = t_first; ok && t < ntiles; t += t_step) {
+                // barrier phases count this group's tiles (t = g + 2 i with one row block)
+                const uint32_t tp = (uint32_t)(QB == 2 ? t : t >> 1) & 1u;
                 for (int h = 0; h < 2; ++h) {  // O_g += P~_g(t) V~(t)
                     const int hh = 2 * t + h, s = hh % NV;
                     if (!mbar_wait(pready + 2 * g + h, tp, p.timeout_ns) ||
@@ -311,7 +321,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                     }
                     tc_fence_after();
                     const uint32_t vs = saddr(sV + (size_t)s * L.vstage);
-                    if (t == 0 && h == 0)
+                    if (t == t_first && h == 0)
                         pv_half(vs, h, 0u);
                     else
                         pv_half(vs, h, 1u);
@@ -319,16 +329,17 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                 }
                 if (!ok) break;
                 tc_commit(saddr(pfree + g));
-                if (t + 1 >= ntiles) break;
-                // S_g(t + 1) as soon as this block's P~ columns are free again
+                const int tn = t + t_step;
+                if (tn >= ntiles) break;
+                // this group's next S as soon as its P~ columns are free again
                 uint64_t bdesc[4];
-                if (!k_tile(t + 1, bdesc) || !mbar_wait(pfree + g, tp, p.timeout_ns) || *abort_flag) {
+                if (!k_tile(tn, bdesc) || !mbar_wait(pfree + g, tp, p.timeout_ns) || *abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 s_product(bdesc);
-                for (int a = 0; a < atoms; ++a) tc_commit(saddr(kempty + (((t + 1) * atoms + a) % KS)));
+                for (int a = 0; a < atoms; ++a) tc_commit(saddr(kempty + ((tn * atoms + a) % KS)));
             }
             if (!ok) {
                 atomicOr(p.err, kDevErrTimeout);
@@ -343,7 +354,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
         const int q = warp & 3;
         const int grp = (warp - 2) >> 2;
         const int rl = q * 32 + lane;
-        const int row = rb * 2 * kBlockRows + grp * kBlockRows + rl;
+        const int row = rb * QB * kBlockRows + (QB == 2 ? grp : 0) * kBlockRows + rl;
         const bool valid = row < p.rows;
         const size_t prow = (size_t)bz * p.rows_stride + row;
         const float alpha = valid ? (float)(((double)p.pot_row[(size_t)bz * p.rows + row] - (double)p.row_norm[prow]) *
@@ -354,9 +365,9 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
         const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
         float rs = 0.f;
         bool ok = true;
-        for (int t = 0; ok && t < ntiles; ++t) {
+        for (int t = QB == 2 ? 0 : grp; ok && t < ntiles; t += (QB == 2 ? 1 : 2)) {
             const int j = t % kQ2Bias;
-            if (!mbar_wait(sfull + grp, (uint32_t)t & 1u, p.timeout_ns) ||
+            if (!mbar_wait(sfull + grp, (uint32_t)(QB == 2 ? t : t >> 1) & 1u, p.timeout_ns) ||
                 !mbar_wait(bfull + j, (uint32_t)(t / kQ2Bias) & 1u, p.timeout_ns)) {
                 ok = false;
                 break;
@@ -417,20 +428,46 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
             atomicOr(p.err, kDevErrTimeout);
             *abort_flag = 1;
         }
-        const bool done = mbar_wait(ofull, 0, p.timeout_ns) && !*abort_flag;
-        tc_fence_after();
-        const float a_i = valid ? (float)exp2((double)p.row_logw2[prow]) : 0.f;
-        const float scale_o = p.divide ? 1.f / rs : a_i;
-        const uint32_t to = lane_base + 256u + (uint32_t)(grp * kQ2TS);
-        for (int c0 = 0; c0 < p.dv_pad; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(to + (uint32_t)c0, o);
-            tmem_ld_wait();
-            if (done && valid)
-                for (int k = 0; k < 32 && c0 + k < p.dv; ++k)
-                    p.out[((size_t)bz * p.rows + row) * p.dv + c0 + k] = __uint_as_float(o[k]) * scale_o;
+        if constexpr (QB == 1) {  // one row block: group 0 adds group 1's row sums and O
+            if (grp == 1) sRs[rl] = rs;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            if (grp == 0) {
+                rs += sRs[rl];
+                const bool done = mbar_wait(ofull, 0, p.timeout_ns) && !*abort_flag;
+                tc_fence_after();
+                const float a_i = valid ? (float)exp2((double)p.row_logw2[prow]) : 0.f;
+                const float scale_o = p.divide ? 1.f / rs : a_i;
+                const uint32_t to = lane_base + 256u;
+                const bool both = ntiles > 1;  // group 1's O holds at least one tile
+                for (int c0 = 0; c0 < p.dv_pad; c0 += 32) {
+                    uint32_t o[32], o1[32];
+                    tmem_ld32(to + (uint32_t)c0, o);
+                    if (both) tmem_ld32(to + (uint32_t)kQ2TS + (uint32_t)c0, o1);
+                    tmem_ld_wait();
+                    if (done && valid)
+                        for (int k = 0; k < 32 && c0 + k < p.dv; ++k)
+                            p.out[((size_t)bz * p.rows + row) * p.dv + c0 + k] =
+                                (both ? __uint_as_float(o[k]) + __uint_as_float(o1[k]) : __uint_as_float(o[k])) *
+                                scale_o;
+                }
+                if (done && valid && p.rsum) p.rsum[(size_t)bz * p.rows + row] = a_i * rs;
+            }
+        } else {
+            const bool done = mbar_wait(ofull, 0, p.timeout_ns) && !*abort_flag;
+            tc_fence_after();
+            const float a_i = valid ? (float)exp2((double)p.row_logw2[prow]) : 0.f;
+            const float scale_o = p.divide ? 1.f / rs : a_i;
+            const uint32_t to = lane_base + 256u + (uint32_t)(grp * kQ2TS);
+            for (int c0 = 0; c0 < p.dv_pad; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(to + (uint32_t)c0, o);
+                tmem_ld_wait();
+                if (done && valid)
+                    for (int k = 0; k < 32 && c0 + k < p.dv; ++k)
+                        p.out[((size_t)bz * p.rows + row) * p.dv + c0 + k] = __uint_as_float(o[k]) * scale_o;
+            }
+            if (done && valid && p.rsum) p.rsum[(size_t)bz * p.rows + row] = a_i * rs;
         }
-        if (done && valid && p.rsum) p.rsum[(size_t)bz * p.rows + row] = a_i * rs;
     }
 
     tc_fence_before();
@@ -442,11 +479,11 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
     }
 }
 
-template <int KIND, int NPASS, int VPL, int PKS>
+template <int KIND, int NPASS, int VPL, int PKS, int QB>
 cudaError_t launch_q2_one(const ApplyParams &p, int batch, const void *mq, const void *mk, const void *mv,
                           size_t smem, cudaStream_t s) {
-    dim3 grid((p.rows_pad + 2 * kBlockRows - 1) / (2 * kBlockRows), 1, batch);
-    auto kern = apply_q2_kernel<KIND, NPASS, VPL, PKS>;
+    dim3 grid((p.rows_pad + QB * kBlockRows - 1) / (QB * kBlockRows), 1, batch);
+    auto kern = apply_q2_kernel<KIND, NPASS, VPL, PKS, QB>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kQ2Threads, smem, s>>>(*static_cast<const CUtensorMap *>(mq), *static_cast<const CUtensorMap *>(mk),
@@ -455,10 +492,13 @@ cudaError_t launch_q2_one(const ApplyParams &p, int batch, const void *mq, const
 }
 
 template <int KIND, int NPASS, int PKS>
-cudaError_t launch_q2_ks(const ApplyParams &p, int batch, int vpl, const void *mq, const void *mk, const void *mv,
-                         size_t smem, cudaStream_t s) {
-    return vpl == 1 ? launch_q2_one<KIND, NPASS, 1, PKS>(p, batch, mq, mk, mv, smem, s)
-                    : launch_q2_one<KIND, NPASS, 2, PKS>(p, batch, mq, mk, mv, smem, s);
+cudaError_t launch_q2_ks(const ApplyParams &p, int batch, int vpl, int qb, const void *mq, const void *mk,
+                         const void *mv, size_t smem, cudaStream_t s) {
+    if (qb == 1)
+        return vpl == 1 ? launch_q2_one<KIND, NPASS, 1, PKS, 1>(p, batch, mq, mk, mv, smem, s)
+                        : launch_q2_one<KIND, NPASS, 2, PKS, 1>(p, batch, mq, mk, mv, smem, s);
+    return vpl == 1 ? launch_q2_one<KIND, NPASS, 1, PKS, 2>(p, batch, mq, mk, mv, smem, s)
+                    : launch_q2_one<KIND, NPASS, 2, PKS, 2>(p, batch, mq, mk, mv, smem, s);
 }
 
 template <int NPASS, int KS>
@@ -469,18 +509,19 @@ bool q2_fits(const ApplyParams &p) {
 // The usual plane widths (d = 16, 32, 64 and, one-plane modes, 128 values)
 // take the S products with compile-time offsets; others the table.
 template <int KIND, int NPASS>
-cudaError_t launch_q2_kind(const ApplyParams &p, int batch, int vpl, const void *mq, const void *mk, const void *mv,
+cudaError_t launch_q2_kind(const ApplyParams &p, int batch, int vpl, int qb, const void *mq, const void *mk,
+                           const void *mv,
                            size_t smem, cudaStream_t s) {
     const int ks = p.plane_bytes / 32;
     if (ks * 32 == p.plane_bytes) {
-        if (ks == 1 && q2_fits<NPASS, 1>(p)) return launch_q2_ks<KIND, NPASS, 1>(p, batch, vpl, mq, mk, mv, smem, s);
-        if (ks == 2 && q2_fits<NPASS, 2>(p)) return launch_q2_ks<KIND, NPASS, 2>(p, batch, vpl, mq, mk, mv, smem, s);
-        if (ks == 4 && q2_fits<NPASS, 4>(p)) return launch_q2_ks<KIND, NPASS, 4>(p, batch, vpl, mq, mk, mv, smem, s);
+        if (ks == 1 && q2_fits<NPASS, 1>(p)) return launch_q2_ks<KIND, NPASS, 1>(p, batch, vpl, qb, mq, mk, mv, smem, s);
+        if (ks == 2 && q2_fits<NPASS, 2>(p)) return launch_q2_ks<KIND, NPASS, 2>(p, batch, vpl, qb, mq, mk, mv, smem, s);
+        if (ks == 4 && q2_fits<NPASS, 4>(p)) return launch_q2_ks<KIND, NPASS, 4>(p, batch, vpl, qb, mq, mk, mv, smem, s);
         if constexpr (NPASS == 1)
             if (ks == 8 && q2_fits<NPASS, 8>(p))
-                return launch_q2_ks<KIND, NPASS, 8>(p, batch, vpl, mq, mk, mv, smem, s);
+                return launch_q2_ks<KIND, NPASS, 8>(p, batch, vpl, qb, mq, mk, mv, smem, s);
     }
-    return launch_q2_ks<KIND, NPASS, 0>(p, batch, vpl, mq, mk, mv, smem, s);
+    return launch_q2_ks<KIND, NPASS, 0>(p, batch, vpl, qb, mq, mk, mv, smem, s);
 }
 
 }  // namespace
@@ -489,14 +530,14 @@ cudaError_t launch_q2_kind(const ApplyParams &p, int batch, int vpl, const void 
 // (slots of one operand atom of a 128-column tile) and its V~ ring depth (64-
 // column halves); 0 if it does not fit or dv_pad exceeds 128 (two O
 // accumulators next to the two S / P~ blocks in TMEM).
-size_t apply_q2_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages) {
+size_t apply_q2_plan(int row_bytes, int dv_pad, int vpl, int qb, int *kslots, int *stages) {
     const size_t limit = 227 * 1024;
     if (dv_pad < 16 || dv_pad > 128 || dv_pad % 16 != 0 || row_bytes > 256) return 0;
     const int atoms = row_bytes / q2swz(row_bytes);
     // {K slots in atoms, V~ halves}, best first
     const int plans[6][2] = {{2 * atoms, 4}, {2 * atoms, 3}, {atoms, 4}, {atoms, 3}, {2 * atoms, 2}, {atoms, 2}};
     for (const auto &pl : plans) {
-        const size_t bytes = (size_t)q2_layout(row_bytes, pl[0], dv_pad, vpl, pl[1]).total + 1024;
+        const size_t bytes = (size_t)q2_layout(row_bytes, pl[0], dv_pad, vpl, pl[1], qb).total + 1024;
         if (bytes <= limit) {
             *kslots = pl[0];
             *stages = pl[1];
@@ -508,12 +549,13 @@ size_t apply_q2_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stage
 
 // prec: 1 = bf16, 2 = tf32, 3 = 3xTF32, 4 = 3xF16 (the S product); vpl: planes of V~;
 // map_v: V~ with a box of 64 columns x dv_pad rows, 128-byte swizzle.
-cudaError_t launch_apply_q2(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
-                            const void *map_v, size_t smem, cudaStream_t s) {
-    if (prec == 1) return launch_q2_kind<0, 1>(p, batch, vpl, map_q, map_k, map_v, smem, s);
-    if (prec == 2) return launch_q2_kind<1, 1>(p, batch, vpl, map_q, map_k, map_v, smem, s);
-    if (prec == 3) return launch_q2_kind<1, 3>(p, batch, vpl, map_q, map_k, map_v, smem, s);
-    return launch_q2_kind<2, 3>(p, batch, vpl, map_q, map_k, map_v, smem, s);
+cudaError_t launch_apply_q2(const ApplyParams &p, int batch, int prec, int vpl, int qb, const void *map_q,
+                            const void *map_k, const void *map_v, size_t smem, cudaStream_t s) {
+    if (qb != 1 && qb != 2) return cudaErrorInvalidValue;
+    if (prec == 1) return launch_q2_kind<0, 1>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
+    if (prec == 2) return launch_q2_kind<1, 1>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
+    if (prec == 3) return launch_q2_kind<1, 3>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
+    return launch_q2_kind<2, 3>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
 }
 
 }  // namespace fs

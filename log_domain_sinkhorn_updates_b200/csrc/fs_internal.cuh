@@ -189,9 +189,11 @@ cudaError_t launch_apply_tc(const ApplyParams &p, int batch, int prec, int vpl, 
 size_t apply_tc2_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages);
 // Two 128-row blocks per CTA sharing every streamed K tile and V~ quarter
 // (fs_apply_tc_q2.cu; dv_pad <= 128, rows of up to 256 bytes).
-size_t apply_q2_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stages);
-cudaError_t launch_apply_q2(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
-                            const void *map_v, size_t smem, cudaStream_t s);
+// qb: 128-row blocks per CTA, 2 (each group its own block) or 1 (both groups on one
+// block, alternate tiles).
+size_t apply_q2_plan(int row_bytes, int dv_pad, int vpl, int qb, int *kslots, int *stages);
+cudaError_t launch_apply_q2(const ApplyParams &p, int batch, int prec, int vpl, int qb, const void *map_q,
+                            const void *map_k, const void *map_v, size_t smem, cudaStream_t s);
 cudaError_t launch_apply_tc2(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,
                              const void *map_v, size_t smem, cudaStream_t s);
 // A kernel whose one bounded mbarrier wait nothing ever completes: after

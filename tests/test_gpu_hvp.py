@@ -88,7 +88,7 @@ def _run_hvp(cuda_device, prob, cases, V, path, cost="sqeuclidean"):
     info = fs.fs_get_info(h)
     fs.fs_destroy(h)
     if path != "simt":
-        assert info["last_apply_path"] in ("tc", "tc_q2", "tc_pair")
+        assert info["last_apply_path"] in ("tc", "tc_q2", "tc_2s", "tc_pair")
     assert info["last_hvp_fused"] == (1 if path == "tc" and cost == "sqeuclidean" else 0), info
     return out.cpu().numpy(), its
 

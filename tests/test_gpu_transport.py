@@ -15,10 +15,13 @@ exp2f adds 2^-21, and the fp32 sum over m terms adds m 2^-24.  Hence
 
 The tensor-core path also splits P/a_i and V into bf16 hi + lo pairs, which
 carry 2^-16 each and drop a term of 2^-16 relative size, so its bound adds
-2^-14.  Every test runs four paths: the tensor-core kernel with two 128-row
-blocks per CTA (FS_ROW_BLOCKS=2; the default for dv <= 128 and rows of up to
-256 bytes once the grid covers the SMs), the one-block tensor-core kernel
-(FS_ROW_BLOCKS=1), the tensor-core kernel on CTA
+2^-14.  Every test runs five paths: the tensor-core kernel with two 128-row
+blocks per CTA (FS_ROW_BLOCKS=2; the default for dv < 64 and rows of up to
+256 bytes once the grid covers the SMs), the same kernel with one block shared
+by both softmax groups taking alternate tiles (FS_ROW_BLOCKS=3; the default
+for dv of 64 to 128 and for smaller grids), the one-block tensor-core kernel
+(FS_ROW_BLOCKS=1), the
+tensor-core kernel on CTA
 pairs (FS_APPLY_PAIR=1; the default for 512-byte operand rows) and the
 CUDA-core validation kernel (FS_APPLY_SIMT=1).
 """
@@ -75,8 +78,9 @@ def _rel_bound(Xo, Yo, loga, logb, f, g, eps, cost):
 
 
 # (FS_APPLY_SIMT, FS_APPLY_PAIR, FS_ROW_BLOCKS)
-PATHS = {"tc_q2": ("0", "0", "2"), "tc": ("0", "0", "1"), "tc_pair": ("0", "1", "2"), "simt": ("1", "0", "2")}
-SPLIT = {"tc_q2": 2.0 ** -14, "tc": 2.0 ** -14, "tc_pair": 2.0 ** -14, "simt": 0.0}
+PATHS = {"tc_q2": ("0", "0", "2"), "tc_2s": ("0", "0", "3"), "tc": ("0", "0", "1"), "tc_pair": ("0", "1", "2"),
+         "simt": ("1", "0", "2")}
+SPLIT = {"tc_q2": 2.0 ** -14, "tc_2s": 2.0 ** -14, "tc": 2.0 ** -14, "tc_pair": 2.0 ** -14, "simt": 0.0}
 
 
 def _set_path(monkeypatch, path):
@@ -340,7 +344,7 @@ def test_transport_apply_tf32_kind(cuda_device, name, prec):
     fs.fs_transport_apply(h, torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device),
                           torch.from_numpy(V).to(cuda_device), out, None)
     fs.fs_sync(h)
-    assert fs.fs_get_info(h)["last_apply_path"] in ("tc", "tc_q2")
+    assert fs.fs_get_info(h)["last_apply_path"] in ("tc", "tc_q2", "tc_2s")
     out = out.cpu().numpy()
     u = 2.0 ** -21
     for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
