@@ -143,6 +143,11 @@ typedef struct {
                                3xF16 / 3xTF32 splits, rows up to 256 bytes); 0: as d / nq transport
                                applications of width nq d (other operands, FS_HVP_FUSED=0, or
                                FS_APPLY_SIMT=1) */
+    int last_apply_parts;   /* column parts of the row blocks past the last full wave in the handle's
+                               last transport application (path 6, batch 1: where those row blocks
+                               fill at most half the SMs, each is split over its column tiles into
+                               up to 8 parts of at least two tiles, and a merge kernel adds the
+                               parts; FS_APPLY_TAIL=0 turns this off); 1: no row block split */
 } fs_info;
 
 /*

@@ -42,7 +42,7 @@ class FsInfo(ctypes.Structure):
                 ("launches_update", ctypes.c_int), ("launches_solve_iter", ctypes.c_int),
                 ("device_bytes", ctypes.c_size_t), ("cta_pair", ctypes.c_int), ("last_apply_path", ctypes.c_int),
                 ("last_solve_graph", ctypes.c_int), ("last_measure_fused", ctypes.c_int),
-                ("last_hvp_fused", ctypes.c_int)]
+                ("last_hvp_fused", ctypes.c_int), ("last_apply_parts", ctypes.c_int)]
 
     def as_dict(self):
         d = {k: getattr(self, k) for k, _ in self._fields_}

@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <string>
@@ -62,6 +63,7 @@ struct fs_handle {
     std::vector<double> meas_cache;  // [batch][8] as in h->red
     int last_measure_fused = 0;
     int last_hvp_fused = 0;  // 1: the last fs_hvp_x formed sum_j P_ij (v_i.y_j) y_j in one fused pass
+    int last_apply_parts = 1;  // column parts of the split row blocks of the last application (1: none)
     std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
     int host_err[4] = {0, 0, 0, 0};
     CUtensorMap mapX_r{}, mapX_c{}, mapY_r{}, mapY_c{};  // row-side (128-row box) / column-side (256-row box)
@@ -398,10 +400,12 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     }
     if (smem == 0) {
         h->last_apply = 2;
+        h->last_apply_parts = 1;
         FS_LAUNCH(h, fs::launch_apply_simt(p, D.batch, h->stream));
         return FS_OK;
     }
     h->last_apply = use_pair ? 3 : (use_q2 ? (qb == 2 ? 4 : 6) : 1);
+    h->last_apply_parts = 1;
     p.row_bytes = h->row_bytes;
     p.swz = h->swz;
     p.plane_bytes = h->plane_bytes;
@@ -411,12 +415,40 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
     p.sscale = h->sscale;
     p.timeout_ns = h->timeout_ns;
     p.err = h->err;
-    // V~: V transposed, bf16 planes [batch][vpl][dv_pad][m_pad], from the pool for this call
-    const size_t vt_bytes = (size_t)D.batch * vpl * dv_pad * p.cols_rows * 2;
+    // One row block per CTA (one CTA per SM): the row blocks past the last full
+    // wave, where they fill at most half the SMs, are split over their column
+    // tiles into k parts of at least two tiles (one per softmax group), so the
+    // last wave takes 1/k of a CTA's time.  A second launch runs the parts, and
+    // a merge kernel adds them.  Highdim (512 row blocks, 148 SMs): the last 68
+    // in two parts each.  FS_APPLY_TAIL=0 keeps every row block whole.
+    p.main_blocks = p.rows_pad / fs::kBlockRows;
+    p.tail_k = 1;
+    size_t tail_rows = 0;
+    if (use_q2 && qb == 1 && D.batch == 1) {
+        const char *env_tail = getenv("FS_APPLY_TAIL");
+        const int blocks = p.rows_pad / fs::kBlockRows, rem = blocks % h->sms;
+        const int ntiles = (p.cols + 127) / 128;
+        int k = rem > 0 ? std::min(8, h->sms / rem) : 1;
+        k = std::min(k, ntiles / 2);
+        if (env_tail && atoi(env_tail) == 0) k = 1;
+        if (k > 1) {
+            p.tail_k = h->last_apply_parts = k;
+            p.main_blocks = blocks - rem;
+            tail_rows = (size_t)rem * fs::kBlockRows;
+        }
+    }
+    // V~: V transposed, bf16 planes [batch][vpl][dv_pad][m_pad], from the pool for
+    // this call, followed by the split row blocks' partial sums
+    const size_t vt_bytes = ((size_t)D.batch * vpl * dv_pad * p.cols_rows * 2 + 255) / 256 * 256;
+    const size_t tail_bytes = (size_t)p.tail_k * tail_rows * (dv + 1) * 4;
     cudaMemPool_t pool;
     void *vt = nullptr;
     FS_CUDA(h, device_pool(h->device, &pool));
-    FS_CUDA(h, cudaMallocFromPoolAsync(&vt, vt_bytes, pool, h->stream));
+    FS_CUDA(h, cudaMallocFromPoolAsync(&vt, vt_bytes + tail_bytes, pool, h->stream));
+    if (p.tail_k > 1) {
+        p.tail_o = reinterpret_cast<float *>(static_cast<char *>(vt) + vt_bytes);
+        p.tail_rs = p.tail_o + (size_t)p.tail_k * tail_rows * dv;
+    }
     cudaError_t e = fs::launch_vt_pack(V, v_bf16, D.batch, p.cols, dv, p.cols_rows, dv_pad, vpl, vt, h->stream);
     g_launches.fetch_add(1, std::memory_order_relaxed);
     CUtensorMap map_v{};
@@ -447,7 +479,7 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
         } else if (use_q2) {
             e = fs::launch_apply_q2(p, D.batch, h->prec, vpl, qb, fdir ? &h->mapX_r : &h->mapY_r,
                                     fdir ? &h->mapY_r : &h->mapX_r, &map_v, smem, h->stream);
-            g_launches.fetch_add(1, std::memory_order_relaxed);
+            g_launches.fetch_add(qb == 1 && p.tail_k > 1 ? (p.main_blocks > 0) + 2 : 1, std::memory_order_relaxed);
         } else {
             e = fs::launch_apply_tc(p, D.batch, h->prec, vpl, fdir ? &h->mapX_r : &h->mapY_r,
                                     fdir ? &h->mapY_r : &h->mapX_r, &map_v, smem, h->stream);
@@ -689,7 +721,10 @@ static fs_status apply_vec_alloc(fs_handle *h, const float *f, const float *g, c
                                        pool, h->stream));
     const fs_status st = apply_vec(h, f, g, v, fdir, out, r, vpad);
     cudaFreeAsync(vpad, h->stream);
-    if (st == FS_OK) h->last_apply = 5;
+    if (st == FS_OK) {
+        h->last_apply = 5;
+        h->last_apply_parts = 1;
+    }
     return st;
 }
 
@@ -1379,6 +1414,7 @@ fs_status fs_get_info(const fs_handle *h, fs_info *info) {
     info->last_solve_graph = h->last_solve_graph;
     info->last_measure_fused = h->last_measure_fused;
     info->last_hvp_fused = h->last_hvp_fused;
+    info->last_apply_parts = h->last_apply_parts;
     return FS_OK;
 }
 

@@ -81,8 +81,9 @@ __host__ __device__ inline Q2Layout q2_layout(int row_bytes, int kslots, int dv_
 // QB = 2: two row blocks, group g (and issuing thread g) owns block g and every
 // tile.  QB = 1: one row block shared by both groups; group g takes the tiles of
 // parity g into its own S / P~ columns and its own O, and group 0 adds the two O
-// at the end.
-template <int KIND, int NPASS, int VPL, int PKS, int QB>
+// at the end.  TAIL (QB = 1): CTA x takes column part x % tail_k of row block
+// main_blocks + x / tail_k and leaves its raw sums for the merge kernel.
+template <int KIND, int NPASS, int VPL, int PKS, int QB, bool TAIL>
 __global__ void __launch_bounds__(kQ2Threads, 1)
     apply_q2_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const ApplyParams p) {
@@ -118,8 +119,13 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rb = blockIdx.x, bz = blockIdx.z;  // rows [QB 128 rb, QB 128 (rb + 1)) of problem bz
+    const int bz = blockIdx.z;
     const int ntiles = (p.cols + kQ2TS - 1) / kQ2TS;
+    // rows [QB 128 rb, QB 128 (rb + 1)) of problem bz over the column tiles [tb, tb + nt)
+    const int rb = TAIL ? p.main_blocks + (int)blockIdx.x / p.tail_k : (int)blockIdx.x;
+    const int part = TAIL ? (int)blockIdx.x % p.tail_k : 0;
+    const int tb = TAIL ? part * ntiles / p.tail_k : 0;
+    const int nt = TAIL ? (part + 1) * ntiles / p.tail_k - tb : ntiles;
     const uint32_t tmem_cols = 512u;
 
     if (threadIdx.x == 0) {
@@ -179,8 +185,8 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                 for (int a = 0; a < atoms; ++a)
                     tma_load_2d(saddr(sQ) + g * qblock_bytes + a * kBlockRows * swz, &map_q, saddr(qfull),
                                 a * box_inner, bz * p.rows_pad + rb * QB * kBlockRows + g * kBlockRows);
-            for (int t = 0; ok && t < ntiles; ++t) {
-                const int col0 = t * kQ2TS;
+            for (int t = 0; ok && t < nt; ++t) {
+                const int col0 = (tb + t) * kQ2TS;
                 if (*abort_flag) break;
                 for (int a = 0; a < atoms && ok; ++a) {
                     const int i = t * atoms + a, s = i % KS;
@@ -221,7 +227,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
         if (lane == 0) {
             bool ok = true;
             int v_issued = 0;
-            for (int hh = 0; ok && hh < 2 * ntiles; ++hh) {
+            for (int hh = 0; ok && hh < 2 * nt; ++hh) {
                 if (*abort_flag) break;
                 const int s = hh % NV;
                 if (hh >= NV && !mbar_wait(vfree + s, ((uint32_t)(hh / NV) & 1u) ^ 1u, p.timeout_ns)) {
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                 uint8_t *sv = sV + (size_t)s * L.vstage;
                 mbar_expect_tx(vfull + s, (uint32_t)VPL * vplane_bytes);
                 for (int pl = 0; pl < VPL; ++pl)
-                    tma_load_2d(saddr(sv + pl * vplane_bytes), &map_v, saddr(vfull + s), hh * kQ2H,
+                    tma_load_2d(saddr(sv + pl * vplane_bytes), &map_v, saddr(vfull + s), (2 * tb + hh) * kQ2H,
                                 (bz * VPL + pl) * p.dv_pad);
                 v_issued = hh + 1;
             }
@@ -301,7 +307,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
             };
             bool ok = mbar_wait(qfull, 0, p.timeout_ns);
             tc_fence_after();
-            if (QB == 2 || t_first < ntiles) {
+            if (QB == 2 || t_first < nt) {
                 uint64_t bdesc[4];
                 ok = ok && k_tile(t_first, bdesc);
                 if (ok) {
@@ -309,7 +315,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                     for (int a = 0; a < atoms; ++a) tc_commit(saddr(kempty + ((t_first * atoms + a) % KS)));
                 }
             }
-            for (int t = t_first; ok && t < ntiles; t += t_step) {
+            for (int t = t_first; ok && t < nt; t += t_step) {
                 // barrier phases count this group's tiles (t = g + 2 i with one row block)
                 const uint32_t tp = (uint32_t)(QB == 2 ? t : t >> 1) & 1u;
                 for (int h = 0; h < 2; ++h) {  // O_g += P~_g(t) V~(t)
@@ -330,7 +336,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                 if (!ok) break;
                 tc_commit(saddr(pfree + g));
                 const int tn = t + t_step;
-                if (tn >= ntiles) break;
+                if (tn >= nt) break;
                 // this group's next S as soon as its P~ columns are free again
                 uint64_t bdesc[4];
                 if (!k_tile(tn, bdesc) || !mbar_wait(pfree + g, tp, p.timeout_ns) || *abort_flag) {
@@ -365,7 +371,7 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
         const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
         float rs = 0.f;
         bool ok = true;
-        for (int t = QB == 2 ? 0 : grp; ok && t < ntiles; t += (QB == 2 ? 1 : 2)) {
+        for (int t = QB == 2 ? 0 : grp; ok && t < nt; t += (QB == 2 ? 1 : 2)) {
             const int j = t % kQ2Bias;
             if (!mbar_wait(sfull + grp, (uint32_t)(QB == 2 ? t : t >> 1) & 1u, p.timeout_ns) ||
                 !mbar_wait(bfull + j, (uint32_t)(t / kQ2Bias) & 1u, p.timeout_ns)) {
@@ -436,21 +442,37 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
                 const bool done = mbar_wait(ofull, 0, p.timeout_ns) && !*abort_flag;
                 tc_fence_after();
                 const float a_i = valid ? (float)exp2((double)p.row_logw2[prow]) : 0.f;
-                const float scale_o = p.divide ? 1.f / rs : a_i;
-                const uint32_t to = lane_base + 256u;
-                const bool both = ntiles > 1;  // group 1's O holds at least one tile
-                for (int c0 = 0; c0 < p.dv_pad; c0 += 32) {
-                    uint32_t o[32], o1[32];
-                    tmem_ld32(to + (uint32_t)c0, o);
-                    if (both) tmem_ld32(to + (uint32_t)kQ2TS + (uint32_t)c0, o1);
-                    tmem_ld_wait();
-                    if (done && valid)
-                        for (int k = 0; k < 32 && c0 + k < p.dv; ++k)
-                            p.out[((size_t)bz * p.rows + row) * p.dv + c0 + k] =
-                                (both ? __uint_as_float(o[k]) + __uint_as_float(o1[k]) : __uint_as_float(o[k])) *
-                                scale_o;
+                if constexpr (TAIL) {  // the raw sums of this column part (two tiles or more), for the merge
+                    const uint32_t to = lane_base + 256u;
+                    const size_t tail_rows = (size_t)(gridDim.x / p.tail_k) * kBlockRows;
+                    const size_t slot = (size_t)part * tail_rows + (size_t)(blockIdx.x / p.tail_k) * kBlockRows + rl;
+                    for (int c0 = 0; c0 < p.dv_pad; c0 += 32) {
+                        uint32_t o[32], o1[32];
+                        tmem_ld32(to + (uint32_t)c0, o);
+                        tmem_ld32(to + (uint32_t)kQ2TS + (uint32_t)c0, o1);
+                        tmem_ld_wait();
+                        if (done && valid)
+                            for (int k = 0; k < 32 && c0 + k < p.dv; ++k)
+                                p.tail_o[slot * p.dv + c0 + k] = __uint_as_float(o[k]) + __uint_as_float(o1[k]);
+                    }
+                    if (done && valid) p.tail_rs[slot] = rs;
+                } else {
+                    const float scale_o = p.divide ? 1.f / rs : a_i;
+                    const uint32_t to = lane_base + 256u;
+                    const bool both = nt > 1;  // group 1's O holds at least one tile
+                    for (int c0 = 0; c0 < p.dv_pad; c0 += 32) {
+                        uint32_t o[32], o1[32];
+                        tmem_ld32(to + (uint32_t)c0, o);
+                        if (both) tmem_ld32(to + (uint32_t)kQ2TS + (uint32_t)c0, o1);
+                        tmem_ld_wait();
+                        if (done && valid)
+                            for (int k = 0; k < 32 && c0 + k < p.dv; ++k)
+                                p.out[((size_t)bz * p.rows + row) * p.dv + c0 + k] =
+                                    (both ? __uint_as_float(o[k]) + __uint_as_float(o1[k]) : __uint_as_float(o[k])) *
+                                    scale_o;
+                    }
+                    if (done && valid && p.rsum) p.rsum[(size_t)bz * p.rows + row] = a_i * rs;
                 }
-                if (done && valid && p.rsum) p.rsum[(size_t)bz * p.rows + row] = a_i * rs;
             }
         } else {
             const bool done = mbar_wait(ofull, 0, p.timeout_ns) && !*abort_flag;
@@ -479,11 +501,34 @@ __global__ void __launch_bounds__(kQ2Threads, 1)
     }
 }
 
-template <int KIND, int NPASS, int VPL, int PKS, int QB>
+// The rows of the split row blocks (batch 1): out_i = (sum over the parts of
+// their raw O_i) times 1 / r~_i (barycentric map) or a_i, and rsum_i = a_i r~_i,
+// r~_i = the sum over the parts of sum_j p~_ij.  One warp per row.
+__global__ void tail_merge_kernel(const ApplyParams p, int tail_rows) {
+    if (*p.err & kDevErrTimeout) return;  // a part gave up: its sums were never written
+    const int i = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (i >= tail_rows) return;
+    const int row = p.main_blocks * kBlockRows + i;
+    if (row >= p.rows) return;
+    float rs = 0.f;
+    for (int part = 0; part < p.tail_k; ++part) rs += p.tail_rs[(size_t)part * tail_rows + i];
+    const float a_i = (float)exp2((double)p.row_logw2[row]);
+    const float scale_o = p.divide ? 1.f / rs : a_i;
+    for (int k = lane; k < p.dv; k += 32) {
+        float o = 0.f;
+        for (int part = 0; part < p.tail_k; ++part) o += p.tail_o[((size_t)part * tail_rows + i) * p.dv + k];
+        p.out[(size_t)row * p.dv + k] = o * scale_o;
+    }
+    if (lane == 0 && p.rsum) p.rsum[row] = a_i * rs;
+}
+
+template <int KIND, int NPASS, int VPL, int PKS, int QB, bool TAIL>
 cudaError_t launch_q2_one(const ApplyParams &p, int batch, const void *mq, const void *mk, const void *mv,
                           size_t smem, cudaStream_t s) {
-    dim3 grid((p.rows_pad + QB * kBlockRows - 1) / (QB * kBlockRows), 1, batch);
-    auto kern = apply_q2_kernel<KIND, NPASS, VPL, PKS, QB>;
+    const int blocks = (p.rows_pad + QB * kBlockRows - 1) / (QB * kBlockRows);
+    // one row block per CTA: the whole row blocks, or the split ones' column parts
+    dim3 grid(QB == 2 ? blocks : (TAIL ? (blocks - p.main_blocks) * p.tail_k : p.main_blocks), 1, batch);
+    auto kern = apply_q2_kernel<KIND, NPASS, VPL, PKS, QB, TAIL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kQ2Threads, smem, s>>>(*static_cast<const CUtensorMap *>(mq), *static_cast<const CUtensorMap *>(mk),
@@ -494,11 +539,18 @@ cudaError_t launch_q2_one(const ApplyParams &p, int batch, const void *mq, const
 template <int KIND, int NPASS, int PKS>
 cudaError_t launch_q2_ks(const ApplyParams &p, int batch, int vpl, int qb, const void *mq, const void *mk,
                          const void *mv, size_t smem, cudaStream_t s) {
-    if (qb == 1)
-        return vpl == 1 ? launch_q2_one<KIND, NPASS, 1, PKS, 1>(p, batch, mq, mk, mv, smem, s)
-                        : launch_q2_one<KIND, NPASS, 2, PKS, 1>(p, batch, mq, mk, mv, smem, s);
-    return vpl == 1 ? launch_q2_one<KIND, NPASS, 1, PKS, 2>(p, batch, mq, mk, mv, smem, s)
-                    : launch_q2_one<KIND, NPASS, 2, PKS, 2>(p, batch, mq, mk, mv, smem, s);
+    if (qb == 1) {
+        // the whole row blocks, then the split ones' column parts
+        cudaError_t e = cudaSuccess;
+        if (p.main_blocks > 0)
+            e = vpl == 1 ? launch_q2_one<KIND, NPASS, 1, PKS, 1, false>(p, batch, mq, mk, mv, smem, s)
+                         : launch_q2_one<KIND, NPASS, 2, PKS, 1, false>(p, batch, mq, mk, mv, smem, s);
+        if (e != cudaSuccess || p.tail_k == 1) return e;
+        return vpl == 1 ? launch_q2_one<KIND, NPASS, 1, PKS, 1, true>(p, batch, mq, mk, mv, smem, s)
+                        : launch_q2_one<KIND, NPASS, 2, PKS, 1, true>(p, batch, mq, mk, mv, smem, s);
+    }
+    return vpl == 1 ? launch_q2_one<KIND, NPASS, 1, PKS, 2, false>(p, batch, mq, mk, mv, smem, s)
+                    : launch_q2_one<KIND, NPASS, 2, PKS, 2, false>(p, batch, mq, mk, mv, smem, s);
 }
 
 template <int NPASS, int KS>
@@ -552,10 +604,23 @@ size_t apply_q2_plan(int row_bytes, int dv_pad, int vpl, int qb, int *kslots, in
 cudaError_t launch_apply_q2(const ApplyParams &p, int batch, int prec, int vpl, int qb, const void *map_q,
                             const void *map_k, const void *map_v, size_t smem, cudaStream_t s) {
     if (qb != 1 && qb != 2) return cudaErrorInvalidValue;
-    if (prec == 1) return launch_q2_kind<0, 1>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
-    if (prec == 2) return launch_q2_kind<1, 1>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
-    if (prec == 3) return launch_q2_kind<1, 3>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
-    return launch_q2_kind<2, 3>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
+    const int blocks = p.rows_pad / kBlockRows;
+    const bool split = qb == 1 && p.tail_k > 1;
+    if (qb == 1 && (p.tail_k < 1 || p.main_blocks < 0 || p.main_blocks > blocks || (split && batch != 1)))
+        return cudaErrorInvalidValue;
+    cudaError_t e;
+    if (prec == 1)
+        e = launch_q2_kind<0, 1>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
+    else if (prec == 2)
+        e = launch_q2_kind<1, 1>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
+    else if (prec == 3)
+        e = launch_q2_kind<1, 3>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
+    else
+        e = launch_q2_kind<2, 3>(p, batch, vpl, qb, map_q, map_k, map_v, smem, s);
+    if (e != cudaSuccess || !split) return e;
+    const int tail_rows = (blocks - p.main_blocks) * kBlockRows;
+    tail_merge_kernel<<<(tail_rows * 32 + 255) / 256, 256, 0, s>>>(p, tail_rows);
+    return cudaGetLastError();
 }
 
 }  // namespace fs

@@ -161,6 +161,13 @@ struct ApplyParams {
     float sscale;                     // raw MMA score -> S_ij (3xF16 operand scaling)
     unsigned long long timeout_ns;
     int *err;
+    // one-row-block two-group kernel (fs_apply_tc_q2.cu, batch 1): row blocks from
+    // main_blocks on are split over their column tiles into tail_k parts, one CTA
+    // each; a part leaves its raw O and row sum in tail_o [tail_k][tail rows][dv]
+    // and tail_rs [tail_k][tail rows], and a merge kernel adds them.  tail_k = 1:
+    // no split (main_blocks = every row block).
+    int main_blocks, tail_k;
+    float *tail_o, *tail_rs;
 };
 
 // Launchers (defined in the .cu files); all return cudaGetLastError().
@@ -192,6 +199,8 @@ size_t apply_tc2_plan(int row_bytes, int dv_pad, int vpl, int *kslots, int *stag
 // qb: 128-row blocks per CTA, 2 (each group its own block) or 1 (both groups on one
 // block, alternate tiles).
 size_t apply_q2_plan(int row_bytes, int dv_pad, int vpl, int qb, int *kslots, int *stages);
+// With qb = 1 and p.tail_k > 1: the whole row blocks (if main_blocks > 0), the
+// split ones' column parts, then the merge kernel.
 cudaError_t launch_apply_q2(const ApplyParams &p, int batch, int prec, int vpl, int qb, const void *map_q,
                             const void *map_k, const void *map_v, size_t smem, cudaStream_t s);
 cudaError_t launch_apply_tc2(const ApplyParams &p, int batch, int prec, int vpl, const void *map_q, const void *map_k,

@@ -160,7 +160,9 @@ def test_full_size_transport_sampled(cuda_device, name):
     assert fs.fs_get_info(h)["last_apply_path"] in ("tc_q2", "tc_2s", "tc", "tc_pair")  # the kernel the bench times
     T = T.cpu().numpy()[0]
     Xo, Yo, loga, logb = oracle.problem_arrays(prob, 0)
-    rows = np.unique(np.concatenate([[0, prob.n - 1], rng.choice(prob.n, 64, replace=False)]))
+    # 64 rows anywhere, 16 of the last eighth (at highdim the row blocks split over their columns)
+    rows = np.unique(np.concatenate([[0, prob.n - 1], rng.choice(prob.n, 64, replace=False),
+                                     rng.choice(np.arange(prob.n * 7 // 8, prob.n), 16, replace=False)]))
     fk, gk = f_in[0].astype(np.float64), g_in[0].astype(np.float64)
     out, r = oracle.transport_apply(Xo[rows], Yo, loga[rows], logb, fk[rows], gk, prob.eps, Yo)
     absw, _ = oracle.transport_apply(Xo[rows], Yo, loga[rows], logb, fk[rows], gk, prob.eps, np.abs(Yo))

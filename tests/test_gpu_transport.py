@@ -141,6 +141,55 @@ def test_transport_apply_parity(cuda_device, name, dv, path, monkeypatch):
         assert err.max() <= 1.0 and rerr.max() <= 1.0
 
 
+@pytest.mark.parametrize("tail", ["1", "0"])
+@pytest.mark.parametrize("dv", [3, 64, 128])
+def test_split_row_blocks_parity(cuda_device, dv, tail, monkeypatch):
+    """More 128-row blocks than SMs in the one-row-block mode: the row blocks past
+    the last full wave are split over their column tiles, one CTA per part, and a
+    merge kernel adds the parts' sums (FS_APPLY_TAIL=0: every row block whole).
+    n = 19500 gives 154 row blocks; on 148 SMs the last 6 split into 4 parts of
+    two tiles (m = 1100: 9 tiles)."""
+    import torch
+    _set_path(monkeypatch, "tc_2s")
+    monkeypatch.setenv("FS_APPLY_TAIL", tail)
+    fs = _fs()
+    prob = make_problem("cloud3d", n=19500, m=1100)
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    f32, g32 = _potentials(prob, "sqeuclidean", iters=4)
+    rng = np.random.default_rng(300 + dv)
+    V = rng.standard_normal((1, prob.m, dv)).astype(np.float32)
+    out = torch.empty(1, prob.n, dv, device=cuda_device)
+    r = torch.empty(1, prob.n, device=cuda_device)
+    fd, gd = torch.from_numpy(f32).to(cuda_device), torch.from_numpy(g32).to(cuda_device)
+    fs.fs_transport_apply(h, fd, gd, torch.from_numpy(V).to(cuda_device), out, r)
+    fs.fs_sync(h)
+    info = fs.fs_get_info(h)
+    assert info["last_apply_path"] == "tc_2s", info
+    blocks = (prob.n + 255) // 256 * 2
+    sms = torch.cuda.get_device_properties(cuda_device).multi_processor_count
+    rem, ntiles = blocks % sms, (prob.m + 127) // 128
+    parts = min(8, sms // rem, ntiles // 2) if rem else 1
+    assert info["last_apply_parts"] == (parts if tail == "1" and parts > 1 else 1), (info, parts)
+    T = torch.empty(1, prob.n, prob.d, device=cuda_device)
+    fs.fs_barycentric_map(h, fd, gd, Y, T)
+    fs.fs_sync(h)
+    out, r, T = out.cpu().numpy()[0], r.cpu().numpy()[0], T.cpu().numpy()[0]
+    Xo, Yo, loga, logb = oracle.problem_arrays(prob, 0)
+    fk, gk = f32[0].astype(np.float64), g32[0].astype(np.float64)
+    oo, ro = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, V[0].astype(np.float64))
+    absw, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(V[0]).astype(np.float64))
+    rel = _rel_bound(Xo, Yo, loga, logb, fk, gk, prob.eps, "sqeuclidean") + SPLIT["tc_2s"]
+    err = (np.abs(out - oo) / (rel[:, None] * absw)).max()
+    rerr = (np.abs(r - ro) / (rel * ro)).max()
+    To = oracle.barycentric_projection(Xo, Yo, loga, logb, fk, gk, prob.eps)
+    py, _ = oracle.transport_apply(Xo, Yo, loga, logb, fk, gk, prob.eps, np.abs(Yo))
+    et = (np.abs(T - To) / (2 * rel[:, None] * py / ro[:, None] + 1e-6 * np.abs(To))).max()
+    print(f"split row blocks (tail={tail}, parts {info['last_apply_parts']}) dv={dv}: "
+          f"err / bound {err:.3f}, row sums {rerr:.3f}, barycentric {et:.3f}")
+    assert err <= 1.0 and rerr <= 1.0 and et <= 1.0
+
+
 @pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("name", ["tiny", "middim", "highdim", "batched"])
 def test_barycentric_map_and_grad_parity(cuda_device, name, path, monkeypatch):
