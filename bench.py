@@ -37,13 +37,16 @@ MUFU_EX2_PER_CLK_PER_SM = 16  # special-function-unit exp2 results per clock per
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "lse_tc_highdim_ncu.md")
 PROFILE_TRAFFIC_APPLY = os.path.join(ROOT, "profiles", "apply_tc_highdim_ncu.md")
 PROFILE_TRAFFIC_APPLY_Q2 = os.path.join(ROOT, "profiles", "apply_q2_highdim_ncu.md")
+PROFILE_TRAFFIC_APPLY_Q2S = os.path.join(ROOT, "profiles", "apply_q2s_highdim_ncu.md")
 # the transport kernels by the path the handle reports: (ncu summary, source file, description)
 APPLY_KERNELS = {
     "tc_q2": (PROFILE_TRAFFIC_APPLY_Q2, "fs_apply_tc_q2.cu",
               "apply_q2_kernel (two 128-row blocks per CTA: S = Q K^T, P~ back into TMEM, O += P~ V~)"),
     "tc": (PROFILE_TRAFFIC_APPLY, "fs_apply_tc.cu", "apply_tc_kernel (S = Q K^T, then O += P~ V~)"),
-    "tc_2s": (None, "fs_apply_tc_q2.cu",
-              "apply_q2_kernel, one row block (both groups on one block, alternate tiles, P~ in TMEM)"),
+    "tc_2s": (PROFILE_TRAFFIC_APPLY_Q2S, "fs_apply_tc_q2.cu",
+              "apply_q2_kernel, one row block per CTA (both groups on alternate tiles, P~ in TMEM): the whole "
+              "row blocks, then the column parts of those past the last full wave, then their merge; "
+              "traffic per application"),
     "tc_pair": (None, "fs_apply_tc2.cu", "apply_tc2_kernel (CTA pairs: S = Q K^T, then O += P~ V~)"),
     "simt": (None, "fs_apply.cu", "apply_simt_kernel (CUDA cores)"),
 }
