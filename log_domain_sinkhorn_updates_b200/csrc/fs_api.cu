@@ -67,6 +67,10 @@ struct fs_handle {
     std::vector<double> host_red;  // staging of scalar results (ordinary host memory)
     int host_err[4] = {0, 0, 0, 0};
     CUtensorMap mapX_r{}, mapX_c{}, mapY_r{}, mapY_c{};  // row-side (128-row box) / column-side (256-row box)
+    // The biases again as score-product rows (32 bytes a point, store_bias_mm), which the
+    // single-CTA update pass adds to S in one more K step, and their maps (256-row boxes).
+    void *bmm_row = nullptr, *bmm_col = nullptr;
+    CUtensorMap mapBmm_row{}, mapBmm_col{};
     int splits_f = 1, tps_f = 1, splits_g = 1, tps_g = 1;
     int stages = 2, stages_meas = 2;
     bool pair = false;  // run the passes on CTA pairs (one MMA over two SMs); FS_CTA_PAIR=1
@@ -209,6 +213,30 @@ fs_status encode_map(fs_handle *h, CUtensorMap *map, void *base, int rows_total,
     return FS_OK;
 }
 
+// The factor from a base-2 bias to raw score units (1 / scale2), and the
+// operand type of the bias rows (tf32 for the tf32 kinds, else bf16).
+float mm_inv_c(const fs_handle *h) {
+    return (float)(1.0 / (fs::kLog2ed / (double)h->desc.eps * (double)h->sscale));
+}
+int mm_tf32(const fs_handle *h) { return h->prec == FS_PREC_TF32 || h->prec == FS_PREC_3XTF32 ? 1 : 0; }
+
+// The map of a side's bias rows: rows_total rows of 32 bytes (16 bf16 or 8 fp32),
+// boxes of 256 rows, 32-byte swizzle (as the single-CTA pass's bias step reads them).
+fs_status encode_bias_map(fs_handle *h, CUtensorMap *map, void *base, int rows_total) {
+    auto fn = encode_fn();
+    if (!fn) return fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    const bool tf32 = mm_tf32(h) != 0;
+    cuuint64_t gdim[2] = {(cuuint64_t)(tf32 ? 8 : 16), (cuuint64_t)rows_total};
+    cuuint64_t gstride[1] = {32};
+    cuuint32_t box[2] = {(cuuint32_t)(tf32 ? 8 : 16), (cuuint32_t)kBlockCols};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, tf32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, gdim,
+                    gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(h, FS_ERR_CUDA, "cuTensorMapEncodeTiled failed for the bias rows (%d)", (int)r);
+    return FS_OK;
+}
+
 fs::PassParams make_pass(const fs_handle *h, bool fdir, bool measure) {
     fs::PassParams p{};
     const fs_desc &D = h->desc;
@@ -232,6 +260,8 @@ fs::PassParams make_pass(const fs_handle *h, bool fdir, bool measure) {
     p.eps = (double)D.eps;
     p.scale2 = (float)(fs::kLog2ed / (double)D.eps * (double)h->sscale);
     p.sscale = h->sscale;
+    p.mm_inv_c = mm_inv_c(h);
+    p.mm_tf32 = mm_tf32(h);
     p.col_bias = fdir ? h->bias_col : h->bias_row;
     p.row_norm = fdir ? h->xn : h->yn;
     p.row_logw2 = fdir ? h->la2 : h->lb2;
@@ -253,7 +283,8 @@ cudaError_t run_pass(fs_handle *h, const fs::PassParams &p, bool fdir, bool meas
                                   fdir ? &h->mapY_r : &h->mapX_r, measure ? h->smem_meas : h->smem, h->stream);
     const CUtensorMap *mr = fdir ? &h->mapX_r : &h->mapY_r;
     const CUtensorMap *mc = fdir ? &h->mapY_c : &h->mapX_c;
-    return fs::launch_lse_tc(p, h->desc.batch, measure, h->prec, h->qt, mr, mc,
+    const CUtensorMap *mb = fdir ? &h->mapBmm_col : &h->mapBmm_row;
+    return fs::launch_lse_tc(p, h->desc.batch, measure, h->prec, h->qt, mr, mc, mb,
                              measure ? h->smem_meas : h->smem, h->stream);
 }
 
@@ -262,8 +293,10 @@ cudaError_t run_bias(fs_handle *h, const float *pot, bool col_is_y) {
     const fs_desc &D = h->desc;
     const double scale2 = fs::kLog2ed / (double)D.eps;
     if (col_is_y)
-        return fs::launch_bias(pot, D.batch, D.m, h->m_stride, h->yn, h->lb2, scale2, h->bias_col, h->stream);
-    return fs::launch_bias(pot, D.batch, D.n, h->n_stride, h->xn, h->la2, scale2, h->bias_row, h->stream);
+        return fs::launch_bias(pot, D.batch, D.m, h->m_stride, h->yn, h->lb2, scale2, h->bias_col, h->bmm_col,
+                               mm_inv_c(h), mm_tf32(h), h->stream);
+    return fs::launch_bias(pot, D.batch, D.n, h->n_stride, h->xn, h->la2, scale2, h->bias_row, h->bmm_row,
+                           mm_inv_c(h), mm_tf32(h), h->stream);
 }
 
 fs_status update(fs_handle *h, const float *in, float *out, bool fdir, bool write_next_bias) {
@@ -271,6 +304,7 @@ fs_status update(fs_handle *h, const float *in, float *out, bool fdir, bool writ
     fs::PassParams p = make_pass(h, fdir, false);
     p.pot_out = out;
     p.next_bias = write_next_bias ? (fdir ? h->bias_row : h->bias_col) : nullptr;
+    p.next_bias_mm = write_next_bias ? (fdir ? h->bmm_row : h->bmm_col) : nullptr;
     FS_LAUNCH(h, run_pass(h, p, fdir, false));
     return FS_OK;
 }
@@ -521,10 +555,12 @@ fs_status enqueue_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule
             fs::PassParams pf = make_pass(h, true, false);
             pf.pot_out = f;
             pf.next_bias = h->bias_row;
+            pf.next_bias_mm = h->bmm_row;
             FS_LAUNCH(h, run_pass(h, pf, true, false));
             fs::PassParams pg = make_pass(h, false, false);
             pg.pot_out = g;
             pg.next_bias = h->bias_col;
+            pg.next_bias_mm = h->bmm_col;
             // the final g-pass also reduces the column marginal of the pair it leaves
             if (it == iters - 1) pg.tail_stats = h->tail_stats;
             FS_LAUNCH(h, run_pass(h, pg, false, false));
@@ -1132,6 +1168,7 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     const size_t o_xn = carve(B * h->n_stride * 4), o_yn = carve(B * h->m_stride * 4);
     const size_t o_la2 = carve(B * h->n_stride * 4), o_lb2 = carve(B * h->m_stride * 4);
     const size_t o_brow = carve(B * h->n_stride * 4), o_bcol = carve(B * h->m_stride * 4);
+    const size_t o_bmrow = carve(B * h->n_stride * 32), o_bmcol = carve(B * h->m_stride * 32);
     const size_t o_center = carve(B * D.d * 4);
     const size_t o_rsum = carve(B * max_pad * 4);
     const size_t o_part = carve(max_splits > 1 ? B * max_splits * max_pad * 16 : 16);
@@ -1167,6 +1204,8 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
     h->bias_row = reinterpret_cast<float *>(base + o_brow);
     h->rsum = reinterpret_cast<float *>(base + o_rsum);
     h->bias_col = reinterpret_cast<float *>(base + o_bcol);
+    h->bmm_row = base + o_bmrow;
+    h->bmm_col = base + o_bmcol;
     h->center = reinterpret_cast<float *>(base + o_center);
     h->part = reinterpret_cast<float4 *>(base + o_part);
     h->counters = reinterpret_cast<unsigned *>(base + o_ctr);
@@ -1223,6 +1262,8 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
         FS_LAUNCH(h, fs::launch_weights(b, D.batch, D.m, h->m_stride, h->lb2, h->wstat + 2 * B, h->stream));
         FS_LAUNCH(h, fs::launch_fill(h->bias_row, B * h->n_stride, -INFINITY, h->stream));
         FS_LAUNCH(h, fs::launch_fill(h->bias_col, B * h->m_stride, -INFINITY, h->stream));
+        FS_LAUNCH(h, fs::launch_fill_bias_mm(h->bmm_row, B * h->n_stride, mm_tf32(h), h->stream));
+        FS_LAUNCH(h, fs::launch_fill_bias_mm(h->bmm_col, B * h->m_stride, mm_tf32(h), h->stream));
         double *hw = h->host_red.data() + 2 * B * 8;
         FS_CUDA(h, cudaMemcpyAsync(hw, h->wstat, 4 * B * 8, cudaMemcpyDeviceToHost, h->stream));
         FS_CUDA(h, cudaMemcpyAsync(h->host_err, h->err, sizeof(int), cudaMemcpyDeviceToHost, h->stream));
@@ -1243,6 +1284,8 @@ fs_status fs_create(const fs_desc *desc, const void *X, const void *Y, const flo
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapX_c, h->packX, D.batch * h->n_pad, kBlockCols);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_r, h->packY, D.batch * h->m_pad, kBlockRows);
             if (s2 == FS_OK) s2 = encode_map(h, &h->mapY_c, h->packY, D.batch * h->m_pad, kBlockCols);
+            if (s2 == FS_OK) s2 = encode_bias_map(h, &h->mapBmm_row, h->bmm_row, D.batch * h->n_stride);
+            if (s2 == FS_OK) s2 = encode_bias_map(h, &h->mapBmm_col, h->bmm_col, D.batch * h->m_stride);
             if (s2 != FS_OK) return s2;
         }
         return FS_OK;

@@ -61,9 +61,12 @@ __device__ void finish_rows(const PassParams &p, int rb, int rl, float m, float 
             // The opposite pass's bias, computed from the stored float potential
             // exactly as the standalone bias kernel does, so a fused solve equals
             // the same sequence of single updates bit for bit.
-            if (p.next_bias)
-                p.next_bias[prow] =
+            if (p.next_bias) {
+                const float nb =
                     (float)__fma_rn((double)pot32 - (double)p.row_norm[prow], kLog2ed / p.eps, (double)p.row_logw2[prow]);
+                p.next_bias[prow] = nb;
+                if (p.next_bias_mm) store_bias_mm(p.next_bias_mm, prow, nb, p.mm_inv_c, p.mm_tf32);
+            }
             if (p.tail_stats) {
                 // The plan's row sum at the stored potential: the exact update is
                 // pot, the stored value pot32, so r_i = a_i exp((pot32 - pot)/eps)

@@ -17,6 +17,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace fs {
@@ -59,6 +60,9 @@ struct PassParams {
     const float *pot_in;       // [batch][rows] current row potential (measure passes)
     float *pot_out;            // [batch][rows] new row potential (update passes)
     float *next_bias;          // [batch][rows_stride] base-2 bias for the opposite pass, or null
+    void *next_bias_mm;        // with next_bias, or null: the same bias as score-product rows (store_bias_mm)
+    float mm_inv_c;            // 1 / scale2: base-2 bias -> raw score units
+    int mm_tf32;               // score-product rows in tf32 (else bf16)
     float4 *part;              // [batch][splits][rows_pad] split partials (m, l, w, -)
     unsigned *counters;        // [batch][row_blocks] arrival counters (self-resetting)
     double *stats;             // [batch][row_blocks][4] measure partial sums
@@ -108,6 +112,42 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+
+// The column bias beta_j as the tensor-core pass adds it to the score: the
+// update pass takes S'_ij = S_ij + beta_j / c from one more K step of its S
+// product, against a tile whose rows are (1, 1, 1, 0, ...), so that
+// z_ij = S'_ij c (c = scale2) needs no per-column load or add in the softmax.
+// A column's 32-byte row holds beta_j / c split into three parts exact in the
+// operand type, (hi, mid, lo, 0, ...): bf16 parts (8 significant bits each),
+// or tf32 parts (fp32 values with the low 13 mantissa bits clear, which the
+// tf32 product reads exactly); -inf (padding) is (-inf, 0, 0).
+__device__ __forceinline__ float tf32_trunc(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+__device__ __forceinline__ void store_bias_mm(void *mm, size_t j, float beta, float inv_c, int tf32) {
+    const float v = beta * inv_c;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (tf32) {
+        float p0 = v, p1 = 0.f, p2 = 0.f;
+        if (isfinite(v)) {
+            p0 = tf32_trunc(v);
+            const float r = v - p0;
+            p1 = tf32_trunc(r);
+            p2 = tf32_trunc(r - p1);
+        }
+        w = make_uint4(__float_as_uint(p0), __float_as_uint(p1), __float_as_uint(p2), 0u);
+    } else {
+        __nv_bfloat16 h0 = __float2bfloat16_rn(v), h1 = __float2bfloat16_rn(0.f), h2 = h1;
+        if (isfinite(v)) {
+            const float r = v - __bfloat162float(h0);
+            h1 = __float2bfloat16_rn(r);
+            h2 = __float2bfloat16_rn(r - __bfloat162float(h1));
+        }
+        w.x = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+        w.y = (uint32_t)__bfloat16_as_ushort(h2);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<char *>(mm) + j * 32);
+    dst[0] = w;
+    dst[1] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
@@ -175,7 +215,7 @@ cudaError_t launch_lse_simt(const PassParams &p, int batch, bool measure, cudaSt
 // Single-CTA pass; qt = 128-row blocks resident per CTA (1 or 2; rows_pad / 128
 // must be a multiple of qt).
 cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int qt,
-                          const void *map_rows, const void *map_cols, size_t smem_bytes,
+                          const void *map_rows, const void *map_cols, const void *map_bias, size_t smem_bytes,
                           cudaStream_t s);
 size_t tc_smem_bytes(int row_bytes, int qt, int stages, bool measure);
 int tc_max_stages(int row_bytes, int qt, bool measure);

@@ -18,8 +18,16 @@
 // j = g mod 2, i.e. the even or odd tiles (QT = 1) or every tile of Q tile g
 // (QT = 2).  They read S with tcgen05.ld, form
 //   z_ij = S_ij * log2(e)/eps + beta_j
-// (beta_j arrives in a separate small ring of bias slices) and update a per-row
-// online maximum and sum of 2^(z - max) in registers (online LSE, section 2).
+// and update a per-row online maximum and sum of 2^(z - max) in registers
+// (online LSE, section 2).  In the update passes the column bias enters the S
+// product itself: each job ends with one more K step, a constant tile of rows
+// (1, 1, 1, 0, ...) times the tile's bias rows (beta_j / c in three parts,
+// store_bias_mm), so TMEM holds S_ij + beta_j / c and the softmax forms
+// z - max with one packed FMA per two entries, with no bias load.  (Measured
+// without the bias work at all: 6 % less time per pass.)  The bias rows stream
+// through a ring of two tiles beside the K slots and go back to the producer
+// through the issuers' commits.  Measure passes read fp32 bias slices (and the
+// column weights) in the softmax, from a ring of their own.
 // Nothing of size n*m ever leaves the SM: the pass writes one potential per
 // row (fused epilogue, section 2).
 //
@@ -52,10 +60,12 @@ constexpr int kThreads = 352;
 constexpr int kTmemCols = 512;   // two 256-column fp32 accumulators
 constexpr int kMaxKsteps = 64;   // MMA instructions per tile: NPASS x (plane bytes / 32) <= 3 x 16
 constexpr int kMaxAtoms = 4;     // swizzle atoms per packed row (row_bytes <= 512)
-constexpr int kBiasSlots = 4;    // tiles whose bias slices may be in flight
+constexpr int kBiasSlots = 4;    // measure passes: tiles whose fp32 bias slices may be in flight
+constexpr int kBiasTiles = 2;    // update passes: tiles whose bias rows (32 bytes a column) may be in flight
+constexpr int kBiasRowBytes = 32;
 
 struct SmemLayout {
-    uint32_t q, k, bias, cnorm, merge, red, koff, bars, misc, total;
+    uint32_t q, k, bias, ones, cnorm, merge, red, koff, bars, misc, total;
 };
 
 __host__ __device__ inline int swizzle_of(int row_bytes) { return row_bytes <= 32 ? 32 : (row_bytes <= 64 ? 64 : 128); }
@@ -67,12 +77,14 @@ __host__ __device__ inline SmemLayout smem_layout(int row_bytes, int slots, bool
     L.q = 0;
     L.k = (uint32_t)(qt * kBlockRows) * row_bytes;
     L.bias = L.k + (uint32_t)slots * kBlockCols * swz;
-    L.cnorm = L.bias + kBiasSlots * kBlockCols * 4;
+    // update passes: the bias-row ring, then the tile of ones (128 rows of 32 bytes)
+    L.ones = L.bias + (measure ? kBiasSlots * kBlockCols * 4 : kBiasTiles * kBlockCols * kBiasRowBytes);
+    L.cnorm = L.ones + (measure ? 0 : kBlockRows * kBiasRowBytes);
     L.merge = L.cnorm + (measure ? kBiasSlots * kBlockCols * 4 : 0);
     L.red = L.merge + kBlockRows * 16;
     L.koff = L.red + (uint32_t)qt * 4 * kBlockRows * 8;
     L.bars = L.koff + 3 * kMaxKsteps * 4;
-    L.misc = L.bars + (2 * slots + 2 * kBiasSlots + 6) * 8;
+    L.misc = L.bars + (2 * slots + 2 * (measure ? kBiasSlots : kBiasTiles) + 6) * 8;
     L.total = L.misc + 32;
     return L;
 }
@@ -83,7 +95,7 @@ __host__ __device__ inline SmemLayout smem_layout(int row_bytes, int slots, bool
 template <int KIND, int NPASS, bool MEASURE, int QT, int KS>
 __global__ void __launch_bounds__(kThreads, 1)
     lse_tc_kernel(const __grid_constant__ CUtensorMap map_rows, const __grid_constant__ CUtensorMap map_cols,
-                  const PassParams p) {
+                  const __grid_constant__ CUtensorMap map_bias, const PassParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
 
@@ -101,11 +113,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float4 *sMerge = reinterpret_cast<float4 *>(smem + L.merge);
     double *sRed = reinterpret_cast<double *>(smem + L.red);
     uint32_t *koff = reinterpret_cast<uint32_t *>(smem + L.koff);
+    constexpr int NB = MEASURE ? kBiasSlots : kBiasTiles;  // bias ring
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);  // [NS]
     uint64_t *empty = full + NS;                                   // [NS]
-    uint64_t *bfull = empty + NS;                                  // [kBiasSlots]
-    uint64_t *bempty = bfull + kBiasSlots;                         // [kBiasSlots]
-    uint64_t *qfull = bempty + kBiasSlots;
+    uint64_t *bfull = empty + NS;                                  // [NB]
+    uint64_t *bempty = bfull + NB;                                 // [NB]
+    uint64_t *qfull = bempty + NB;
     uint64_t *sfull = qfull + 1;   // [2]
     uint64_t *sempty = sfull + 2;  // [2]
     uint64_t *drain = sempty + 2;
@@ -124,9 +137,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(full + s, 1);
             mbar_init(empty + s, QT);  // a commit after each of the tile's jobs
         }
-        for (int j = 0; j < kBiasSlots; ++j) {
+        for (int j = 0; j < NB; ++j) {
             mbar_init(bfull + j, 1);
-            mbar_init(bempty + j, 4 * QT);  // the warps of the softmax groups that read the tile
+            // measure: the softmax warps that read the slice; update: a commit after each of the tile's jobs
+            mbar_init(bempty + j, MEASURE ? 4 * QT : QT);
         }
         mbar_init(qfull, 1);
         for (int b = 0; b < 2; ++b) {
@@ -156,6 +170,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    if constexpr (!MEASURE) {
+        // The A operand of the bias step: every row (1, 1, 1, 0, ...) in both 16-byte
+        // halves, so the 32-byte swizzle (which may exchange the halves) leaves it as is.
+        const uint32_t one2 = KIND == 1 ? 0x3F800000u : 0x3F803F80u;  // two bf16 ones, or one fp32 one
+        const uint32_t w0 = one2, w1 = KIND == 1 ? 0x3F800000u : 0x3F80u, w2 = KIND == 1 ? 0x3F800000u : 0u;
+        uint32_t *ones = reinterpret_cast<uint32_t *>(smem + L.ones);
+        for (int i = threadIdx.x; i < kBlockRows * kBiasRowBytes / 4; i += blockDim.x) {
+            const int w = i & 3;  // word within a 16-byte half
+            ones[i] = w == 0 ? w0 : (w == 1 ? w1 : (w == 2 ? w2 : 0u));
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -173,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_2d(saddr(sQ) + (g * atoms + a) * kBlockRows * swz, &map_rows, saddr(qfull),
                                 a * box_inner, qrow + g * kBlockRows);
             const uint32_t bias_bytes = kBlockCols * 4;
+            const uint32_t brow_tile = kBlockCols * kBiasRowBytes;
             for (int t = 0; ok && t < ntiles; ++t) {
                 const int col0 = (tile_begin + t) * kBlockCols;
                 if (*abort_flag) break;
@@ -189,19 +216,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                     slots_issued = i + 1;
                 }
                 if (!ok) break;
-                // the tile's bias slice, after its K slots so it never delays them
-                const int j = t % kBiasSlots;
-                if (t >= kBiasSlots && !mbar_wait(bempty + j, ((uint32_t)(t / kBiasSlots) & 1u) ^ 1u, p.timeout_ns)) {
+                // the tile's bias, after its K slots so it never delays them
+                const int j = t % NB;
+                if (t >= NB && !mbar_wait(bempty + j, ((uint32_t)(t / NB) & 1u) ^ 1u, p.timeout_ns)) {
                     ok = false;
                     break;
                 }
-                mbar_expect_tx(bfull + j, bias_bytes * (MEASURE ? 2 : 1));
-                bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_stride + col0, bias_bytes,
-                          saddr(bfull + j));
-                if (MEASURE)
+                if constexpr (MEASURE) {
+                    mbar_expect_tx(bfull + j, bias_bytes * 2);
+                    bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_stride + col0,
+                              bias_bytes, saddr(bfull + j));
                     bulk_load(saddr(sCN + j * kBlockCols),
                               (p.col_vec ? p.col_vec : p.col_norm) + (size_t)bz * p.cols_stride + col0, bias_bytes,
                               saddr(bfull + j));
+                } else {  // the tile's bias rows (256 x 32 bytes, 32-byte swizzle)
+                    mbar_expect_tx(bfull + j, brow_tile);
+                    tma_load_2d(saddr(smem + L.bias + j * brow_tile), &map_bias, saddr(bfull + j), 0,
+                                bz * p.cols_stride + col0);
+                }
                 bias_issued = t + 1;
             }
             if (!ok) {
@@ -212,8 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(qfull, 0, p.timeout_ns);
             for (int i = max(0, slots_issued - NS); i < slots_issued; ++i)
                 mbar_wait(full + (i % NS), (uint32_t)(i / NS) & 1u, p.timeout_ns);
-            for (int t = max(0, bias_issued - kBiasSlots); t < bias_issued; ++t)
-                mbar_wait(bfull + (t % kBiasSlots), (uint32_t)(t / kBiasSlots) & 1u, p.timeout_ns);
+            for (int t = max(0, bias_issued - NB); t < bias_issued; ++t)
+                mbar_wait(bfull + (t % NB), (uint32_t)(t / NB) & 1u, p.timeout_ns);
         }
         __syncwarp();
     } else if (warp == 1 || (warp == 10 && p.issuers == 2)) {  // (the launcher admits 1 or 2)
@@ -226,8 +258,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int jstep = p.issuers == 2 ? 2 : 1, jb0 = warp == 1 ? 0 : 1;
             const uint64_t adesc0 = make_sdesc(saddr(sQ), swz);
             const uint32_t qstride = (uint32_t)(atoms * kBlockRows * swz) >> 4;  // one Q tile, in descriptor units
+            // the bias step: bf16 (or tf32) ones against the tile's bias rows
+            constexpr int BK = KIND == 1 ? 1 : 0;
+            const uint32_t idesc_b = make_idesc<BK>();
+            const uint64_t ones_desc = make_sdesc(saddr(smem + L.ones), (uint32_t)kBiasRowBytes);
             bool ok = mbar_wait(qfull, 0, p.timeout_ns);
-            uint64_t bdesc[kMaxAtoms];
+            uint64_t bdesc[kMaxAtoms], brow_desc = 0ull;
             for (int jb = jb0; ok && jb < njobs; jb += jstep) {
                 const int b = jb & 1;
                 const int t = QT == 2 ? (jb >> 1) : jb;
@@ -247,6 +283,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             bdesc[a] = 0ull;
                         }
                     }
+                    if constexpr (!MEASURE) {
+                        const int j = t % NB;
+                        if (!mbar_wait(bfull + j, (uint32_t)(t / NB) & 1u, p.timeout_ns)) ok = false;
+                        brow_desc = make_sdesc(saddr(smem + L.bias + j * kBlockCols * kBiasRowBytes),
+                                               (uint32_t)kBiasRowBytes);
+                    }
                 }
                 if (!ok || *abort_flag) break;
                 tc_fence_after();
@@ -261,10 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_mma<KIND>(dt, adesc + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
                     }
                 }
-                // A commit per job for its softmax group, and one per K slot: the
-                // slot is free once every job of its tile has read it (QT arrivals).
+                if constexpr (!MEASURE) tc_mma<BK>(dt, ones_desc, brow_desc, idesc_b, 1u);  // + beta_j / c
+                // A commit per job for its softmax group, and one per K slot (and
+                // bias tile): free once every job of its tile has read it (QT arrivals).
                 tc_commit(saddr(sfull + b));
                 for (int a = 0; a < atoms; ++a) tc_commit(saddr(empty + ((t * atoms + a) % NS)));
+                if constexpr (!MEASURE) tc_commit(saddr(bempty + (t % NB)));
             }
             if (!ok) {
                 atomicOr(p.err, kDevErrTimeout);
@@ -294,15 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int jb = grp; jb < njobs; jb += 2) {
             const int t = QT == 2 ? (jb >> 1) : jb;
-            const int j = t % kBiasSlots;
+            const int j = t % NB;
             if (!mbar_wait(sfull + grp, (uint32_t)(jb >> 1) & 1u, p.timeout_ns) ||
-                !mbar_wait(bfull + j, (uint32_t)(t / kBiasSlots) & 1u, p.timeout_ns)) {
+                (MEASURE && !mbar_wait(bfull + j, (uint32_t)(t / NB) & 1u, p.timeout_ns))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const float *bias = sBias + j * kBlockCols;
-            if (!MEASURE) {
+            if constexpr (!MEASURE) {
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     uint32_t r[128];
@@ -317,9 +360,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(sempty + grp);
                     }
-                    consume128(r, bias + 128 * half, c, m, l);
+                    consume128_folded(r, c, m, l);
                 }
             } else {
+                const float *bias = sBias + j * kBlockCols;
                 const float *cnorm = sCN + j * kBlockCols;
 #pragma unroll 1
                 for (int qt = 0; qt < 4; ++qt) {
@@ -334,9 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     consume64_measure(ra, rb2, bias + 64 * qt, cnorm + 64 * qt, c, wsscale, xn, m, l, w);
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bempty + j);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bempty + j);
             if (*abort_flag) break;
         }
         if (!ok) {
@@ -369,21 +413,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int KIND, int NPASS, bool MEASURE, int QT, int KS>
 cudaError_t launch_variant(const PassParams &p, int batch, const void *map_rows, const void *map_cols,
-                           size_t smem, cudaStream_t s) {
+                           const void *map_bias, size_t smem, cudaStream_t s) {
     auto kern = lse_tc_kernel<KIND, NPASS, MEASURE, QT, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.rows_pad / (QT * kBlockRows), p.splits, batch);
     kern<<<grid, kThreads, smem, s>>>(*static_cast<const CUtensorMap *>(map_rows),
-                                      *static_cast<const CUtensorMap *>(map_cols), p);
+                                      *static_cast<const CUtensorMap *>(map_cols),
+                                      *static_cast<const CUtensorMap *>(map_bias), p);
     return cudaGetLastError();
 }
 
 template <int KIND, int NPASS, int KS>
 cudaError_t launch_update(const PassParams &p, int batch, int qt, const void *map_rows, const void *map_cols,
-                          size_t smem, cudaStream_t s) {
-    return qt == 2 ? launch_variant<KIND, NPASS, false, 2, KS>(p, batch, map_rows, map_cols, smem, s)
-                   : launch_variant<KIND, NPASS, false, 1, KS>(p, batch, map_rows, map_cols, smem, s);
+                          const void *map_bias, size_t smem, cudaStream_t s) {
+    return qt == 2 ? launch_variant<KIND, NPASS, false, 2, KS>(p, batch, map_rows, map_cols, map_bias, smem, s)
+                   : launch_variant<KIND, NPASS, false, 1, KS>(p, batch, map_rows, map_cols, map_bias, smem, s);
 }
 
 // The compile-time row geometry matches the pass's packed rows.
@@ -394,22 +439,22 @@ bool fits(const Params &p) {
 
 template <int KIND, int NPASS>
 cudaError_t launch_kind(const PassParams &p, int batch, bool measure, int qt, const void *map_rows,
-                        const void *map_cols, size_t smem, cudaStream_t s) {
+                        const void *map_cols, const void *map_bias, size_t smem, cudaStream_t s) {
     if (!measure) {
         // The update passes of the usual widths issue their MMAs from compile-time
         // offsets (d = 16, 32, 64 and, for one-plane modes, 128 values per plane).
         const int ks = p.plane_bytes / 32;
         if (ks * 32 == p.plane_bytes) {
-            if (ks == 1 && fits<NPASS, 1>(p)) return launch_update<KIND, NPASS, 1>(p, batch, qt, map_rows, map_cols, smem, s);
-            if (ks == 2 && fits<NPASS, 2>(p)) return launch_update<KIND, NPASS, 2>(p, batch, qt, map_rows, map_cols, smem, s);
-            if (ks == 4 && fits<NPASS, 4>(p)) return launch_update<KIND, NPASS, 4>(p, batch, qt, map_rows, map_cols, smem, s);
+            if (ks == 1 && fits<NPASS, 1>(p)) return launch_update<KIND, NPASS, 1>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+            if (ks == 2 && fits<NPASS, 2>(p)) return launch_update<KIND, NPASS, 2>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+            if (ks == 4 && fits<NPASS, 4>(p)) return launch_update<KIND, NPASS, 4>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
             if constexpr (NPASS == 1)
-                if (ks == 8 && fits<NPASS, 8>(p)) return launch_update<KIND, NPASS, 8>(p, batch, qt, map_rows, map_cols, smem, s);
+                if (ks == 8 && fits<NPASS, 8>(p)) return launch_update<KIND, NPASS, 8>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
         }
-        return launch_update<KIND, NPASS, 0>(p, batch, qt, map_rows, map_cols, smem, s);
+        return launch_update<KIND, NPASS, 0>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
     }
-    return qt == 2 ? launch_variant<KIND, NPASS, true, 2, 0>(p, batch, map_rows, map_cols, smem, s)
-                   : launch_variant<KIND, NPASS, true, 1, 0>(p, batch, map_rows, map_cols, smem, s);
+    return qt == 2 ? launch_variant<KIND, NPASS, true, 2, 0>(p, batch, map_rows, map_cols, map_bias, smem, s)
+                   : launch_variant<KIND, NPASS, true, 1, 0>(p, batch, map_rows, map_cols, map_bias, smem, s);
 }
 
 }  // namespace
@@ -429,15 +474,17 @@ int tc_max_stages(int row_bytes, int qt, bool measure) {
     return best;
 }
 
-// prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16; qt: 128-row blocks per CTA (1 or 2).
+// prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16; qt: 128-row blocks per CTA (1 or 2);
+// map_bias: the column side's bias rows (update passes; store_bias_mm in the
+// operand type of prec, 32-byte swizzle, boxes of 256 rows).
 cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int qt, const void *map_rows,
-                          const void *map_cols, size_t smem, cudaStream_t s) {
+                          const void *map_cols, const void *map_bias, size_t smem, cudaStream_t s) {
     if (p.issuers != 1 && p.issuers != 2) return cudaErrorInvalidValue;
     if (qt != 1 && qt != 2) return cudaErrorInvalidValue;
-    if (prec == 1) return launch_kind<0, 1>(p, batch, measure, qt, map_rows, map_cols, smem, s);
-    if (prec == 2) return launch_kind<1, 1>(p, batch, measure, qt, map_rows, map_cols, smem, s);
-    if (prec == 3) return launch_kind<1, 3>(p, batch, measure, qt, map_rows, map_cols, smem, s);
-    return launch_kind<2, 3>(p, batch, measure, qt, map_rows, map_cols, smem, s);
+    if (prec == 1) return launch_kind<0, 1>(p, batch, measure, qt, map_rows, map_cols, map_bias, smem, s);
+    if (prec == 2) return launch_kind<1, 1>(p, batch, measure, qt, map_rows, map_cols, map_bias, smem, s);
+    if (prec == 3) return launch_kind<1, 3>(p, batch, measure, qt, map_rows, map_cols, map_bias, smem, s);
+    return launch_kind<2, 3>(p, batch, measure, qt, map_rows, map_cols, map_bias, smem, s);
 }
 
 }  // namespace fs

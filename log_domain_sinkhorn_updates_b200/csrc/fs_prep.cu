@@ -192,14 +192,21 @@ __global__ void fill_kernel(float *p, size_t count, float v) {
 
 // out_j = ((pot_j - |col_j|^2) log2(e)/eps + log2 w_j), -inf on padding.
 __global__ void bias_kernel(const float *pot, int cnt, int cnt_pad, int batch, const float *norm, const float *lw2,
-                            double scale2, float *out) {
+                            double scale2, float *out, void *mm, float mm_inv_c, int mm_tf32) {
     const size_t total = (size_t)batch * cnt_pad;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
         const int bz = (int)(i / cnt_pad), j = (int)(i % cnt_pad);
         float v = -INFINITY;
         if (j < cnt) v = (float)__fma_rn((double)pot[(size_t)bz * cnt + j] - (double)norm[i], scale2, (double)lw2[i]);
         out[i] = v;
+        if (mm) store_bias_mm(mm, i, v, mm_inv_c, mm_tf32);
     }
+}
+
+// Every bias row of a side as a padding column's: (-inf, 0, 0, ...).
+__global__ void fill_bias_mm_kernel(void *mm, size_t count, int tf32) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (size_t)gridDim.x * blockDim.x)
+        store_bias_mm(mm, i, -INFINITY, 1.f, tf32);
 }
 
 // out[bz][0..3] = sum over row blocks of the measure statistics (fixed order);
@@ -305,9 +312,14 @@ cudaError_t launch_fill(float *p, size_t count, float v, cudaStream_t s) {
 }
 
 cudaError_t launch_bias(const float *pot, int batch, int cnt, int cnt_pad, const float *norm, const float *lw2,
-                        double scale2, float *out, cudaStream_t s) {
+                        double scale2, float *out, void *mm, float mm_inv_c, int mm_tf32, cudaStream_t s) {
     bias_kernel<<<grid_for((size_t)batch * cnt_pad, 256), 256, 0, s>>>(pot, cnt, cnt_pad, batch, norm, lw2, scale2,
-                                                                      out);
+                                                                      out, mm, mm_inv_c, mm_tf32);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fill_bias_mm(void *mm, size_t count, int tf32, cudaStream_t s) {
+    fill_bias_mm_kernel<<<grid_for(count, 256), 256, 0, s>>>(mm, count, tf32);
     return cudaGetLastError();
 }
 

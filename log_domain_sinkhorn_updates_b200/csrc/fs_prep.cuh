@@ -29,8 +29,13 @@ cudaError_t launch_weights(const float *w, int batch, int cnt, int cnt_pad, floa
 cudaError_t launch_fill(float *p, size_t count, float v, cudaStream_t s);
 // v [batch][cnt] -> out [batch][stride], zero beyond cnt.
 cudaError_t launch_pad_vec(const float *v, int batch, int cnt, int stride, float *out, cudaStream_t s);
+// out [batch][cnt_pad]: the base-2 bias of the pass whose columns are this side,
+// -inf beyond cnt; mm (may be null): the same as score-product rows
+// (store_bias_mm, 32 bytes per column).
 cudaError_t launch_bias(const float *pot, int batch, int cnt, int cnt_pad, const float *norm, const float *lw2,
-                        double scale2, float *out, cudaStream_t s);
+                        double scale2, float *out, void *mm, float mm_inv_c, int mm_tf32, cudaStream_t s);
+// count bias rows (32 bytes each) set to a padding column's.
+cudaError_t launch_fill_bias_mm(void *mm, size_t count, int tf32, cudaStream_t s);
 // *flag |= 1 if the count floats at a and b differ in any bit.
 cudaError_t launch_differs(const float *a, const float *b, size_t count, int *flag, cudaStream_t s);
 cudaError_t launch_finalize(const double *stats, int batch, int row_blocks, const float *col_pot,

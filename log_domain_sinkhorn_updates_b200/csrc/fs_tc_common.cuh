@@ -301,6 +301,25 @@ __device__ __forceinline__ float sum_exp2(const float (&z)[CNT], float ref) {
     return ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
 }
 
+// The block's max taken, (m, l) moved to max(m, block max) and the block's
+// exponentials added against it (the rare path of the folds below).
+template <int CNT>
+__device__ __forceinline__ void rescale_block(const float (&z)[CNT], float &m, float &l) {
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int k = 0; k < CNT; k += 8) {
+        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k], z[k + 1]);
+        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 2], z[k + 3]);
+        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 4], z[k + 5]);
+        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 6], z[k + 7]);
+    }
+    const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    if (tmax == -INFINITY) return;  // nothing but padding so far
+    const float mnew = fmaxf(m, tmax);
+    l = (m == -INFINITY ? 0.f : l * ex2_approx(m - mnew)) + sum_exp2<CNT>(z, mnew);
+    m = mnew;
+}
+
 // Fold CNT scores (raw fp32 bits from TMEM) into a row's online state (m, l):
 // z = S * c + beta.  The first block of a row takes two passes (max, then
 // exponentials).  Later blocks take their exponentials against the running max
@@ -342,23 +361,47 @@ __device__ __forceinline__ void consume(const uint32_t (&r)[CNT], const float *b
             return;
         }
     }
-    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-    for (int k = 0; k < CNT; k += 8) {
-        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k], z[k + 1]);
-        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 2], z[k + 3]);
-        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 4], z[k + 5]);
-        mx[(k / 8) & 3] = max3(mx[(k / 8) & 3], z[k + 6], z[k + 7]);
-    }
-    const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-    if (tmax == -INFINITY) return;  // nothing but padding so far
-    const float mnew = fmaxf(m, tmax);
-    l = (m == -INFINITY ? 0.f : l * ex2_approx(m - mnew)) + sum_exp2<CNT>(z, mnew);
-    m = mnew;
+    rescale_block<CNT>(z, m, l);
 }
 __device__ __forceinline__ void consume128(const uint32_t (&r)[128], const float *bias, float c, float &m,
                                            float &l) {
     consume<128>(r, bias, c, m, l);
+}
+
+// The same fold for scores that already hold the column bias (the update
+// pass's S product adds beta_j / c, store_bias_mm): z = S' c, and the common
+// case is one packed FMA (S' c - max) per two entries, then the exponentials.
+template <int CNT>
+__device__ __forceinline__ void consume_folded(const uint32_t (&r)[CNT], float c, float &m, float &l) {
+    const uint64_t cc = pack2(c, c);
+    if (m != -INFINITY) {
+        const uint64_t mneg = pack2(-m, -m);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+        for (int k = 0; k < CNT; k += 2) {
+            float d0, d1;
+            unpack2(fma2(pack2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), cc, mneg), d0, d1);
+            acc[(k / 2) & 3] = add2(acc[(k / 2) & 3], pack2(ex2_approx(d0), ex2_approx(d1)));
+        }
+        float a0, a1, a2, a3, a4, a5, a6, a7;
+        unpack2(acc[0], a0, a1);
+        unpack2(acc[1], a2, a3);
+        unpack2(acc[2], a4, a5);
+        unpack2(acc[3], a6, a7);
+        const float s = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+        if (s <= kLazySum) {
+            l += s;
+            return;
+        }
+    }
+    float z[CNT];
+#pragma unroll
+    for (int k = 0; k < CNT; k += 2)
+        unpack2(fma2(pack2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), cc, 0ull), z[k], z[k + 1]);
+    rescale_block<CNT>(z, m, l);
+}
+__device__ __forceinline__ void consume128_folded(const uint32_t (&r)[128], float c, float &m, float &l) {
+    consume_folded<128>(r, c, m, l);
 }
 
 // Measure-mode fold over 64 columns (two 32-column TMEM loads): besides (m, l)
