@@ -601,7 +601,8 @@ def main():
         "tensor": {"achieved": flops / pass_s / 1e12, "peak": float(peaks.get("bf16_tflops", 1590.0)),
                    "unit": "TFLOP/s", "frac": flops / pass_s / 1e12 / float(peaks.get("bf16_tflops", 1590.0)),
                    "peak_source": peak_src},
-        "algorithmic_bytes_per_launch": (n + m) * B * (d * (2 if prob.dtype == "bf16" else 4) + 12),
+        # per point: its operand row, norm, log-weight and potential, and its 32-byte bias row
+        "algorithmic_bytes_per_launch": (n + m) * B * (d * (2 if prob.dtype == "bf16" else 4) + 44),
     }
     if clocks and clocks.get("sm_mhz"):
         roofline["frac_at_median_clock"] = ex2_rate / (sms * MUFU_EX2_PER_CLK_PER_SM * clocks["sm_mhz"] * 1e6)
