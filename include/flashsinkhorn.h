@@ -378,8 +378,8 @@ FS_API fs_status fs_solve_host(const fs_desc *desc, const void *X_host, const vo
  * on a device share the array and it keeps the last call's contents (each call
  * writes everything it reads), so calls that overlap on the GPU race -- order
  * them on one stream.  The first call on each device, with that device
- * current, looks up the array's device address and sets a kernel attribute:
- * make it before any stream capture begins.  The address is kept per device
+ * current, looks up the array's device address and sets a kernel attribute.
+ * The address is kept per device
  * for the life of the process; after cudaDeviceReset it is stale, so do not
  * call this entry point on a device that has been reset.  Errors: return
  * codes, message in fs_last_error(NULL).

@@ -23,8 +23,7 @@
 //    race and corrupt each other's results; order them on one stream or
 //    synchronise between them;
 //  * the first call on each device looks up the array's device address
-//    (cudaGetSymbolAddress) and sets the kernel's shared-memory limit; make
-//    that first call before any stream capture begins.  The address is kept
+//    (cudaGetSymbolAddress) and sets the kernel's shared-memory limit.  The address is kept
 //    per device index for the life of the process; after cudaDeviceReset the
 //    kept address refers to the old context, so do not use this entry point
 //    after resetting a device.
