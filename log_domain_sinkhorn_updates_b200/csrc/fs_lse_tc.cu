@@ -60,9 +60,15 @@ constexpr int kThreads = 352;
 constexpr int kTmemCols = 512;   // two 256-column fp32 accumulators
 constexpr int kMaxKsteps = 64;   // MMA instructions per tile: NPASS x (plane bytes / 32) <= 3 x 16
 constexpr int kMaxAtoms = 4;     // swizzle atoms per packed row (row_bytes <= 512)
-constexpr int kBiasSlots = 4;    // measure passes: tiles whose fp32 bias slices may be in flight
-constexpr int kBiasTiles = 2;    // update passes: tiles whose bias rows (32 bytes a column) may be in flight
+constexpr int kBiasSlots = 4;    // measure passes: tiles whose fp32 column slices may be in flight
+constexpr int kBiasTiles = 2;    // update and vector passes: tiles whose bias rows (32 bytes a column) may be in flight
 constexpr int kBiasRowBytes = 32;
+
+// Pass modes: an update; a measure pass with statistics; a measure pass that
+// weights each column by v_j (col_vec).  The update and vector passes add the
+// bias inside the S product; the statistics pass needs S itself (C_ij from it)
+// and reads fp32 bias slices.
+constexpr int kUpdate = 0, kStats = 1, kVector = 2;
 
 struct SmemLayout {
     uint32_t q, k, bias, ones, cnorm, merge, red, koff, bars, misc, total;
@@ -71,20 +77,22 @@ struct SmemLayout {
 __host__ __device__ inline int swizzle_of(int row_bytes) { return row_bytes <= 32 ? 32 : (row_bytes <= 64 ? 64 : 128); }
 
 // slots: K ring slots of kBlockCols rows x one swizzle atom each; qt: resident Q tiles.
-__host__ __device__ inline SmemLayout smem_layout(int row_bytes, int slots, bool measure, int qt) {
+__host__ __device__ inline SmemLayout smem_layout(int row_bytes, int slots, int mode, int qt) {
     SmemLayout L;
     const uint32_t swz = (uint32_t)swizzle_of(row_bytes);
+    const bool fold = mode != kStats;
     L.q = 0;
     L.k = (uint32_t)(qt * kBlockRows) * row_bytes;
+    // the bias-row ring and the tile of ones (128 rows of 32 bytes) of the bias step
     L.bias = L.k + (uint32_t)slots * kBlockCols * swz;
-    // update passes: the bias-row ring, then the tile of ones (128 rows of 32 bytes)
-    L.ones = L.bias + (measure ? kBiasSlots * kBlockCols * 4 : kBiasTiles * kBlockCols * kBiasRowBytes);
-    L.cnorm = L.ones + (measure ? 0 : kBlockRows * kBiasRowBytes);
-    L.merge = L.cnorm + (measure ? kBiasSlots * kBlockCols * 4 : 0);
+    L.ones = L.bias + (fold ? kBiasTiles * kBlockCols * kBiasRowBytes : 0);
+    // the fp32 column slices of measure passes: bias (statistics) and |y|^2 or v
+    L.cnorm = L.ones + (fold ? kBlockRows * kBiasRowBytes : 0) + (mode == kStats ? kBiasSlots * kBlockCols * 4 : 0);
+    L.merge = L.cnorm + (mode != kUpdate ? kBiasSlots * kBlockCols * 4 : 0);
     L.red = L.merge + kBlockRows * 16;
-    L.koff = L.red + (uint32_t)qt * 4 * kBlockRows * 8;
+    L.koff = L.red + (mode == kVector ? 0u : (uint32_t)qt * 4 * kBlockRows * 8);  // a vector pass keeps no statistics
     L.bars = L.koff + 3 * kMaxKsteps * 4;
-    L.misc = L.bars + (2 * slots + 2 * (measure ? kBiasSlots : kBiasTiles) + 6) * 8;
+    L.misc = L.bars + (2 * slots + 2 * kBiasTiles + 2 * kBiasSlots + 6) * 8;
     L.total = L.misc + 32;
     return L;
 }
@@ -92,7 +100,7 @@ __host__ __device__ inline SmemLayout smem_layout(int row_bytes, int slots, bool
 // KS > 0: the plane's K-step count, fixed at compile time (the MMAs of a job
 // are issued with immediate descriptor offsets); KS = 0: any width, offsets
 // from a table in shared memory.
-template <int KIND, int NPASS, bool MEASURE, int QT, int KS>
+template <int KIND, int NPASS, int MODE, int QT, int KS>
 __global__ void __launch_bounds__(kThreads, 1)
     lse_tc_kernel(const __grid_constant__ CUtensorMap map_rows, const __grid_constant__ CUtensorMap map_cols,
                   const __grid_constant__ CUtensorMap map_bias, const PassParams p) {
@@ -104,21 +112,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int atoms = p.row_bytes / p.swz;
     const uint32_t slot_bytes = (uint32_t)kBlockCols * swz;
     const int box_inner = p.swz / (KIND == 1 ? 4 : 2);
-    const SmemLayout L = smem_layout(p.row_bytes, NS, MEASURE, QT);
+    constexpr bool MEASURE = MODE != kUpdate;
+    constexpr bool FOLD = MODE != kStats;  // the bias enters the S product
+    const SmemLayout L = smem_layout(p.row_bytes, NS, MODE, QT);
 
     uint8_t *sQ = smem + L.q;
     uint8_t *sK = smem + L.k;
-    float *sBias = reinterpret_cast<float *>(smem + L.bias);
-    float *sCN = reinterpret_cast<float *>(smem + L.cnorm);
+    float *sBias = reinterpret_cast<float *>(smem + L.ones);  // statistics passes: fp32 bias slices
+    float *sCN = reinterpret_cast<float *>(smem + L.cnorm);   // measure passes: |y|^2 or v slices
     float4 *sMerge = reinterpret_cast<float4 *>(smem + L.merge);
     double *sRed = reinterpret_cast<double *>(smem + L.red);
     uint32_t *koff = reinterpret_cast<uint32_t *>(smem + L.koff);
-    constexpr int NB = MEASURE ? kBiasSlots : kBiasTiles;  // bias ring
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bars);  // [NS]
     uint64_t *empty = full + NS;                                   // [NS]
-    uint64_t *bfull = empty + NS;                                  // [NB]
-    uint64_t *bempty = bfull + NB;                                 // [NB]
-    uint64_t *qfull = bempty + NB;
+    uint64_t *rfull = empty + NS;                                  // [kBiasTiles] bias rows landed
+    uint64_t *rempty = rfull + kBiasTiles;                         // [kBiasTiles] read by every job of the tile
+    uint64_t *cfull = rempty + kBiasTiles;                         // [kBiasSlots] column slices landed
+    uint64_t *cempty = cfull + kBiasSlots;                         // [kBiasSlots] read by the softmax warps
+    uint64_t *qfull = cempty + kBiasSlots;
     uint64_t *sfull = qfull + 1;   // [2]
     uint64_t *sempty = sfull + 2;  // [2]
     uint64_t *drain = sempty + 2;
@@ -137,10 +148,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(full + s, 1);
             mbar_init(empty + s, QT);  // a commit after each of the tile's jobs
         }
-        for (int j = 0; j < NB; ++j) {
-            mbar_init(bfull + j, 1);
-            // measure: the softmax warps that read the slice; update: a commit after each of the tile's jobs
-            mbar_init(bempty + j, MEASURE ? 4 * QT : QT);
+        for (int j = 0; j < kBiasTiles; ++j) {
+            mbar_init(rfull + j, 1);
+            mbar_init(rempty + j, QT);  // a commit after each of the tile's jobs
+        }
+        for (int j = 0; j < kBiasSlots; ++j) {
+            mbar_init(cfull + j, 1);
+            mbar_init(cempty + j, 4 * QT);  // the warps of the softmax groups that read the tile
         }
         mbar_init(qfull, 1);
         for (int b = 0; b < 2; ++b) {
@@ -170,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    if constexpr (!MEASURE) {
+    if constexpr (FOLD) {
         // The A operand of the bias step: every row (1, 1, 1, 0, ...) in both 16-byte
         // halves, so the 32-byte swizzle (which may exchange the halves) leaves it as is.
         const uint32_t one2 = KIND == 1 ? 0x3F800000u : 0x3F803F80u;  // two bf16 ones, or one fp32 one
@@ -191,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- TMA producer ----------------
         if (lane == 0) {
             bool ok = true;
-            int slots_issued = 0, bias_issued = 0;
+            int slots_issued = 0, rows_issued = 0, slices_issued = 0;
             const int qrow = bz * p.rows_pad + rb * (QT * kBlockRows);
             mbar_expect_tx(qfull, (uint32_t)(QT * kBlockRows) * p.row_bytes);
             for (int g = 0; g < QT; ++g)
@@ -216,25 +230,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                     slots_issued = i + 1;
                 }
                 if (!ok) break;
-                // the tile's bias, after its K slots so it never delays them
-                const int j = t % NB;
-                if (t >= NB && !mbar_wait(bempty + j, ((uint32_t)(t / NB) & 1u) ^ 1u, p.timeout_ns)) {
-                    ok = false;
-                    break;
-                }
-                if constexpr (MEASURE) {
-                    mbar_expect_tx(bfull + j, bias_bytes * 2);
-                    bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_stride + col0,
-                              bias_bytes, saddr(bfull + j));
-                    bulk_load(saddr(sCN + j * kBlockCols),
-                              (p.col_vec ? p.col_vec : p.col_norm) + (size_t)bz * p.cols_stride + col0, bias_bytes,
-                              saddr(bfull + j));
-                } else {  // the tile's bias rows (256 x 32 bytes, 32-byte swizzle)
-                    mbar_expect_tx(bfull + j, brow_tile);
-                    tma_load_2d(saddr(smem + L.bias + j * brow_tile), &map_bias, saddr(bfull + j), 0,
+                // the tile's bias rows and column slices, after its K slots so they never delay them
+                if constexpr (FOLD) {  // bias rows: 256 x 32 bytes, 32-byte swizzle
+                    const int j = t % kBiasTiles;
+                    if (t >= kBiasTiles &&
+                        !mbar_wait(rempty + j, ((uint32_t)(t / kBiasTiles) & 1u) ^ 1u, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(rfull + j, brow_tile);
+                    tma_load_2d(saddr(smem + L.bias + j * brow_tile), &map_bias, saddr(rfull + j), 0,
                                 bz * p.cols_stride + col0);
+                    rows_issued = t + 1;
                 }
-                bias_issued = t + 1;
+                if constexpr (MEASURE) {  // fp32 slices: bias and |y|^2 (statistics), or v (vector)
+                    const int j = t % kBiasSlots;
+                    if (t >= kBiasSlots &&
+                        !mbar_wait(cempty + j, ((uint32_t)(t / kBiasSlots) & 1u) ^ 1u, p.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(cfull + j, bias_bytes * (MODE == kStats ? 2 : 1));
+                    if constexpr (MODE == kStats) {
+                        bulk_load(saddr(sBias + j * kBlockCols), p.col_bias + (size_t)bz * p.cols_stride + col0,
+                                  bias_bytes, saddr(cfull + j));
+                        bulk_load(saddr(sCN + j * kBlockCols), p.col_norm + (size_t)bz * p.cols_stride + col0,
+                                  bias_bytes, saddr(cfull + j));
+                    } else {
+                        bulk_load(saddr(sCN + j * kBlockCols), p.col_vec + (size_t)bz * p.cols_stride + col0,
+                                  bias_bytes, saddr(cfull + j));
+                    }
+                    slices_issued = t + 1;
+                }
             }
             if (!ok) {
                 atomicOr(p.err, kDevErrTimeout);
@@ -244,8 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(qfull, 0, p.timeout_ns);
             for (int i = max(0, slots_issued - NS); i < slots_issued; ++i)
                 mbar_wait(full + (i % NS), (uint32_t)(i / NS) & 1u, p.timeout_ns);
-            for (int t = max(0, bias_issued - NB); t < bias_issued; ++t)
-                mbar_wait(bfull + (t % NB), (uint32_t)(t / NB) & 1u, p.timeout_ns);
+            for (int t = max(0, rows_issued - kBiasTiles); t < rows_issued; ++t)
+                mbar_wait(rfull + (t % kBiasTiles), (uint32_t)(t / kBiasTiles) & 1u, p.timeout_ns);
+            for (int t = max(0, slices_issued - kBiasSlots); t < slices_issued; ++t)
+                mbar_wait(cfull + (t % kBiasSlots), (uint32_t)(t / kBiasSlots) & 1u, p.timeout_ns);
         }
         __syncwarp();
     } else if (warp == 1 || (warp == 10 && p.issuers == 2)) {  // (the launcher admits 1 or 2)
@@ -283,9 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             bdesc[a] = 0ull;
                         }
                     }
-                    if constexpr (!MEASURE) {
-                        const int j = t % NB;
-                        if (!mbar_wait(bfull + j, (uint32_t)(t / NB) & 1u, p.timeout_ns)) ok = false;
+                    if constexpr (FOLD) {
+                        const int j = t % kBiasTiles;
+                        if (!mbar_wait(rfull + j, (uint32_t)(t / kBiasTiles) & 1u, p.timeout_ns)) ok = false;
                         brow_desc = make_sdesc(saddr(smem + L.bias + j * kBlockCols * kBiasRowBytes),
                                                (uint32_t)kBiasRowBytes);
                     }
@@ -303,12 +332,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_mma<KIND>(dt, adesc + koff[i], bd + koff[2 * kMaxKsteps + i], idesc, i > 0 ? 1u : 0u);
                     }
                 }
-                if constexpr (!MEASURE) tc_mma<BK>(dt, ones_desc, brow_desc, idesc_b, 1u);  // + beta_j / c
+                if constexpr (FOLD) tc_mma<BK>(dt, ones_desc, brow_desc, idesc_b, 1u);  // + beta_j / c
                 // A commit per job for its softmax group, and one per K slot (and
                 // bias tile): free once every job of its tile has read it (QT arrivals).
                 tc_commit(saddr(sfull + b));
                 for (int a = 0; a < atoms; ++a) tc_commit(saddr(empty + ((t * atoms + a) % NS)));
-                if constexpr (!MEASURE) tc_commit(saddr(bempty + (t % NB)));
+                if constexpr (FOLD) tc_commit(saddr(rempty + (t % kBiasTiles)));
             }
             if (!ok) {
                 atomicOr(p.err, kDevErrTimeout);
@@ -330,22 +359,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rl = q * 32 + lane;    // row within the block
         const int rblk = rb * QT + (QT == 2 ? grp : 0);  // this warp's 128-row block
         const float c = p.scale2;
-        // a vector pass weights each column by v_j alone: no row norm, no score term
-        const float xn = MEASURE && !p.col_vec ? p.row_norm[(size_t)bz * p.rows_stride + rblk * kBlockRows + rl] : 0.f;
-        const float wsscale = p.col_vec ? 0.f : p.sscale;
+        const float xn = MODE == kStats ? p.row_norm[(size_t)bz * p.rows_stride + rblk * kBlockRows + rl] : 0.f;
         float m = -INFINITY, l = 0.f, w = 0.f;
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(grp * kBlockCols);
         bool ok = true;
         for (int jb = grp; jb < njobs; jb += 2) {
             const int t = QT == 2 ? (jb >> 1) : jb;
-            const int j = t % NB;
+            const int j = t % kBiasSlots;
             if (!mbar_wait(sfull + grp, (uint32_t)(jb >> 1) & 1u, p.timeout_ns) ||
-                (MEASURE && !mbar_wait(bfull + j, (uint32_t)(t / NB) & 1u, p.timeout_ns))) {
+                (MEASURE && !mbar_wait(cfull + j, (uint32_t)(t / kBiasSlots) & 1u, p.timeout_ns))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            if constexpr (!MEASURE) {
+            if constexpr (FOLD) {
 #pragma unroll 1
                 for (int half = 0; half < 2; ++half) {
                     uint32_t r[128];
@@ -360,7 +387,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(sempty + grp);
                     }
-                    consume128_folded(r, c, m, l);
+                    if constexpr (MODE == kUpdate)
+                        consume128_folded(r, c, m, l);
+                    else  // w = sum_j 2^(z_j - m) v_j beside (m, l)
+                        consume128_vec_folded(r, sCN + j * kBlockCols + 128 * half, c, m, l, w);
+                }
+                if constexpr (MODE == kVector) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(cempty + j);
                 }
             } else {
                 const float *bias = sBias + j * kBlockCols;
@@ -376,10 +410,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(sempty + grp);
                     }
-                    consume64_measure(ra, rb2, bias + 64 * qt, cnorm + 64 * qt, c, wsscale, xn, m, l, w);
+                    consume64_measure(ra, rb2, bias + 64 * qt, cnorm + 64 * qt, c, p.sscale, xn, m, l, w);
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bempty + j);
+                if (lane == 0) mbar_arrive(cempty + j);
             }
             if (*abort_flag) break;
         }
@@ -411,10 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int KIND, int NPASS, bool MEASURE, int QT, int KS>
+template <int KIND, int NPASS, int MODE, int QT, int KS>
 cudaError_t launch_variant(const PassParams &p, int batch, const void *map_rows, const void *map_cols,
                            const void *map_bias, size_t smem, cudaStream_t s) {
-    auto kern = lse_tc_kernel<KIND, NPASS, MEASURE, QT, KS>;
+    auto kern = lse_tc_kernel<KIND, NPASS, MODE, QT, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.rows_pad / (QT * kBlockRows), p.splits, batch);
@@ -424,43 +458,54 @@ cudaError_t launch_variant(const PassParams &p, int batch, const void *map_rows,
     return cudaGetLastError();
 }
 
-template <int KIND, int NPASS, int KS>
-cudaError_t launch_update(const PassParams &p, int batch, int qt, const void *map_rows, const void *map_cols,
-                          const void *map_bias, size_t smem, cudaStream_t s) {
-    return qt == 2 ? launch_variant<KIND, NPASS, false, 2, KS>(p, batch, map_rows, map_cols, map_bias, smem, s)
-                   : launch_variant<KIND, NPASS, false, 1, KS>(p, batch, map_rows, map_cols, map_bias, smem, s);
-}
-
 // The compile-time row geometry matches the pass's packed rows.
 template <int NPASS, int KS, typename Params>
 bool fits(const Params &p) {
     return p.row_bytes == RowGeom<NPASS, KS>::kRowBytes && p.swz == RowGeom<NPASS, KS>::kSwz;
 }
 
+template <int KIND, int NPASS, int MODE, int KS>
+cudaError_t launch_qt(const PassParams &p, int batch, int qt, const void *map_rows, const void *map_cols,
+                      const void *map_bias, size_t smem, cudaStream_t s) {
+    return qt == 2 ? launch_variant<KIND, NPASS, MODE, 2, KS>(p, batch, map_rows, map_cols, map_bias, smem, s)
+                   : launch_variant<KIND, NPASS, MODE, 1, KS>(p, batch, map_rows, map_cols, map_bias, smem, s);
+}
+
+// The update and vector passes of the usual widths issue their MMAs from
+// compile-time offsets (d = 16, 32, 64 and, for one-plane modes, 128 values per plane).
+template <int KIND, int NPASS, int MODE>
+cudaError_t launch_ks(const PassParams &p, int batch, int qt, const void *map_rows, const void *map_cols,
+                      const void *map_bias, size_t smem, cudaStream_t s) {
+    const int ks = p.plane_bytes / 32;
+    if (ks * 32 == p.plane_bytes) {
+        if (ks == 1 && fits<NPASS, 1>(p)) return launch_qt<KIND, NPASS, MODE, 1>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+        if (ks == 2 && fits<NPASS, 2>(p)) return launch_qt<KIND, NPASS, MODE, 2>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+        if (ks == 4 && fits<NPASS, 4>(p)) return launch_qt<KIND, NPASS, MODE, 4>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+        if constexpr (NPASS == 1)
+            if (ks == 8 && fits<NPASS, 8>(p)) return launch_qt<KIND, NPASS, MODE, 8>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+    }
+    return launch_qt<KIND, NPASS, MODE, 0>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+}
+
 template <int KIND, int NPASS>
 cudaError_t launch_kind(const PassParams &p, int batch, bool measure, int qt, const void *map_rows,
                         const void *map_cols, const void *map_bias, size_t smem, cudaStream_t s) {
-    if (!measure) {
-        // The update passes of the usual widths issue their MMAs from compile-time
-        // offsets (d = 16, 32, 64 and, for one-plane modes, 128 values per plane).
-        const int ks = p.plane_bytes / 32;
-        if (ks * 32 == p.plane_bytes) {
-            if (ks == 1 && fits<NPASS, 1>(p)) return launch_update<KIND, NPASS, 1>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
-            if (ks == 2 && fits<NPASS, 2>(p)) return launch_update<KIND, NPASS, 2>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
-            if (ks == 4 && fits<NPASS, 4>(p)) return launch_update<KIND, NPASS, 4>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
-            if constexpr (NPASS == 1)
-                if (ks == 8 && fits<NPASS, 8>(p)) return launch_update<KIND, NPASS, 8>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
-        }
-        return launch_update<KIND, NPASS, 0>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
-    }
-    return qt == 2 ? launch_variant<KIND, NPASS, true, 2, 0>(p, batch, map_rows, map_cols, map_bias, smem, s)
-                   : launch_variant<KIND, NPASS, true, 1, 0>(p, batch, map_rows, map_cols, map_bias, smem, s);
+    if (!measure) return launch_ks<KIND, NPASS, kUpdate>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+    if (p.col_vec) return launch_ks<KIND, NPASS, kVector>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
+    return launch_qt<KIND, NPASS, kStats, 0>(p, batch, qt, map_rows, map_cols, map_bias, smem, s);
 }
 
 }  // namespace
 
+// measure: the larger of the statistics and the vector layouts (one size serves both).
 size_t tc_smem_bytes(int row_bytes, int qt, int slots, bool measure) {
-    return (size_t)smem_layout(row_bytes, slots, measure, qt).total + 1024;  // + alignment slack
+    uint32_t total = smem_layout(row_bytes, slots, kUpdate, qt).total;
+    if (measure) {
+        const uint32_t a = smem_layout(row_bytes, slots, kStats, qt).total;
+        const uint32_t b = smem_layout(row_bytes, slots, kVector, qt).total;
+        total = a > b ? a : b;
+    }
+    return (size_t)total + 1024;  // + alignment slack
 }
 
 // The deepest K ring that fits (at most 8 slots) with qt resident Q tiles; 0
@@ -475,8 +520,8 @@ int tc_max_stages(int row_bytes, int qt, bool measure) {
 }
 
 // prec: 1 = bf16, 2 = tf32 (one pass), 3 = 3xTF32, 4 = 3xF16; qt: 128-row blocks per CTA (1 or 2);
-// map_bias: the column side's bias rows (update passes; store_bias_mm in the
-// operand type of prec, 32-byte swizzle, boxes of 256 rows).
+// map_bias: the column side's bias rows (update and vector passes; store_bias_mm
+// in the operand type of prec, 32-byte swizzle, boxes of 256 rows).
 cudaError_t launch_lse_tc(const PassParams &p, int batch, bool measure, int prec, int qt, const void *map_rows,
                           const void *map_cols, const void *map_bias, size_t smem, cudaStream_t s) {
     if (p.issuers != 1 && p.issuers != 2) return cudaErrorInvalidValue;

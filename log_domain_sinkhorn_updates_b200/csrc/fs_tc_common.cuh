@@ -404,6 +404,73 @@ __device__ __forceinline__ void consume128_folded(const uint32_t (&r)[128], floa
     consume_folded<128>(r, c, m, l);
 }
 
+// The vector pass's fold (scores holding the column bias, as above): beside
+// (m, l) it accumulates w = sum_j 2^(z_j - m) v_j, with v_j from shared memory.
+// The same lazy max; the rare path moves l and w to the new max together.
+template <int CNT>
+__device__ __forceinline__ void consume_vec_folded(const uint32_t (&r)[CNT], const float *vec, float c, float &m,
+                                                   float &l, float &w) {
+    const float4 *vq = reinterpret_cast<const float4 *>(vec);
+    const uint64_t cc = pack2(c, c);
+    if (m != -INFINITY) {
+        const uint64_t mneg = pack2(-m, -m);
+        uint64_t al[2] = {0ull, 0ull}, aw[2] = {0ull, 0ull};
+#pragma unroll
+        for (int k = 0; k < CNT; k += 4) {
+            const float4 v = vq[k / 4];
+            float d0, d1, d2, d3;
+            unpack2(fma2(pack2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), cc, mneg), d0, d1);
+            unpack2(fma2(pack2(__uint_as_float(r[k + 2]), __uint_as_float(r[k + 3])), cc, mneg), d2, d3);
+            const uint64_t e01 = pack2(ex2_approx(d0), ex2_approx(d1));
+            const uint64_t e23 = pack2(ex2_approx(d2), ex2_approx(d3));
+            al[0] = add2(al[0], e01);
+            al[1] = add2(al[1], e23);
+            aw[0] = fma2(e01, pack2(v.x, v.y), aw[0]);
+            aw[1] = fma2(e23, pack2(v.z, v.w), aw[1]);
+        }
+        float a0, a1, a2, a3;
+        unpack2(al[0], a0, a1);
+        unpack2(al[1], a2, a3);
+        const float s = (a0 + a1) + (a2 + a3);
+        if (s <= kLazySum) {
+            float w0, w1, w2, w3;
+            unpack2(aw[0], w0, w1);
+            unpack2(aw[1], w2, w3);
+            l += s;
+            w += (w0 + w1) + (w2 + w3);
+            return;
+        }
+    }
+    float z[CNT];
+#pragma unroll
+    for (int k = 0; k < CNT; k += 2)
+        unpack2(fma2(pack2(__uint_as_float(r[k]), __uint_as_float(r[k + 1])), cc, 0ull), z[k], z[k + 1]);
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int k = 0; k < CNT; k += 4) {
+        mx[(k / 4) & 3] = max3(mx[(k / 4) & 3], z[k], z[k + 1]);
+        mx[(k / 4) & 3] = max3(mx[(k / 4) & 3], z[k + 2], z[k + 3]);
+    }
+    const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+    if (tmax == -INFINITY) return;  // nothing but padding so far
+    const float mnew = fmaxf(m, tmax);
+    const float sc = m == -INFINITY ? 0.f : ex2_approx(m - mnew);
+    float sl = 0.f, sw = 0.f;
+#pragma unroll
+    for (int k = 0; k < CNT; ++k) {
+        const float e = ex2_approx(z[k] - mnew);
+        sl += e;
+        sw = fmaf(e, vec[k], sw);
+    }
+    l = l * sc + sl;
+    w = w * sc + sw;
+    m = mnew;
+}
+__device__ __forceinline__ void consume128_vec_folded(const uint32_t (&r)[128], const float *vec, float c, float &m,
+                                                      float &l, float &w) {
+    consume_vec_folded<128>(r, vec, c, m, l, w);
+}
+
 // Measure-mode fold over 64 columns (two 32-column TMEM loads): besides (m, l)
 // it accumulates w = sum_j 2^(z_j - m) C_ij with C_ij = |row|^2 + |col|^2 - S_ij
 // (S_ij = raw score * sscale), the plan-weighted cost of the row.
