@@ -19,15 +19,17 @@
 // (QT = 2).  They read S with tcgen05.ld, form
 //   z_ij = S_ij * log2(e)/eps + beta_j
 // and update a per-row online maximum and sum of 2^(z - max) in registers
-// (online LSE, section 2).  In the update passes the column bias enters the S
-// product itself: each job ends with one more K step, a constant tile of rows
-// (1, 1, 1, 0, ...) times the tile's bias rows (beta_j / c in three parts,
-// store_bias_mm), so TMEM holds S_ij + beta_j / c and the softmax forms
-// z - max with one packed FMA per two entries, with no bias load.  (Measured
-// without the bias work at all: 6 % less time per pass.)  The bias rows stream
-// through a ring of two tiles beside the K slots and go back to the producer
-// through the issuers' commits.  Measure passes read fp32 bias slices (and the
-// column weights) in the softmax, from a ring of their own.
+// (online LSE, section 2).  In the update passes (and the vector passes, which
+// weight column j by v_j) the column bias enters the S product itself: each
+// job ends with one more K step, a constant tile of rows (1, 1, 1, 0, ...)
+// times the tile's bias rows (beta_j / c in three parts, store_bias_mm), so
+// TMEM holds S_ij + beta_j / c and the softmax forms z - max with one packed
+// FMA per two entries, with no bias load.  (Measured without the bias work at
+// all: 6 % less time per pass.)  The bias rows stream through a ring of two
+// tiles beside the K slots and go back to the producer through the issuers'
+// commits.  Measure passes with statistics need S itself (C_ij from it): they
+// read fp32 bias and |y|^2 slices in the softmax, from a ring of their own,
+// from which vector passes read v.
 // Nothing of size n*m ever leaves the SM: the pass writes one potential per
 // row (fused epilogue, section 2).
 //
