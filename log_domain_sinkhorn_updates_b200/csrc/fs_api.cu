@@ -877,6 +877,7 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     const size_t o_part = carve((size_t)B * 2 * 4096), o_sc = carve((size_t)B * 2 * 5);
     const size_t o_Yh = carve(cosine ? m * d : 1), o_Vt = carve(cosine ? n * d : 1);
     const size_t o_vpad = carve((size_t)B * (h->n_stride > h->m_stride ? h->n_stride : h->m_stride));
+    const size_t o_steps = carve((size_t)B);
     cudaMemPool_t pool;
     uint8_t *blk = nullptr;
     FS_CUDA(h, device_pool(h->device, &pool));
@@ -885,6 +886,7 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     double *part = reinterpret_cast<double *>(blk + o_part);
     double *sc = reinterpret_cast<double *>(blk + o_sc);  // [k][B]: k = 0 rr, 1 p.Ap, 2 rr_new, 3 sum, 4 z.z
     double *rr_d = sc, *pap_d = sc + B, *rrn_d = sc + 2 * B, *sum_d = sc + 3 * B, *zz_d = sc + 4 * B;
+    int *steps_d = reinterpret_cast<int *>(blk + o_steps);  // [B] CG steps each problem took
     const double tol2 = cg_rtol * cg_rtol;
     float *PY = F(oPY), *r = F(o_r), *c = F(o_c), *W1 = F(oW1), *Tm = F(oT), *u = F(o_u);
     float *tn = F(o_tn), *tm = F(o_tm), *z = F(o_z), *x = F(o_x), *res = F(o_res), *p = F(o_p), *Ap = F(o_Ap);
@@ -926,6 +928,7 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
         // CG on [diag(c) - P^T diag(1/r) P] dg = z, iterates kept orthogonal to 1;
         // a problem stops once rr <= tol2 z.z, the others run on
         FS_CUDA(h, cudaMemsetAsync(x, 0, m * 4, s));
+        FS_CUDA(h, cudaMemsetAsync(steps_d, 0, (size_t)B * 4, s));
         FS_CUDA(h, cudaMemcpyAsync(res, z, m * 4, cudaMemcpyDeviceToDevice, s));
         FS_CUDA(h, cudaMemcpyAsync(p, z, m * 4, cudaMemcpyDeviceToDevice, s));
         FS_LAUNCH(h, fs::hvp_dot(B, m1, z, z, part, rr_d, s));
@@ -939,23 +942,37 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
                 if (rr[b] > tol2 * zz[b] && zz[b] > 0.0) return true;
             return false;
         };
-        while (it < max_cg_iters && any_running()) {
-            s2 = apply1(p, true, tn);  // P p
-            if (s2 != FS_OK) return s2;
-            FS_LAUNCH(h, fs::hvp_vec(n, tn, r, 1.f, nullptr, 0.f, true, tn, s));  // / r
-            s2 = apply1(tn, false, tm);  // P^T (P p / r)
-            if (s2 != FS_OK) return s2;
-            FS_LAUNCH(h, fs::hvp_vec(m, p, c, 1.f, tm, -1.f, false, Ap, s));  // c o p - ...
-            FS_LAUNCH(h, fs::hvp_dot(B, m1, Ap, nullptr, part, sum_d, s));
-            FS_LAUNCH(h, fs::hvp_center(B, m1, sum_d, Ap, s));
-            FS_LAUNCH(h, fs::hvp_dot(B, m1, p, Ap, part, pap_d, s));
-            FS_LAUNCH(h, fs::hvp_cg_step(B, m1, rr_d, pap_d, zz_d, tol2, p, Ap, x, res, s));
-            FS_LAUNCH(h, fs::hvp_dot(B, m1, res, res, part, rrn_d, s));
-            FS_LAUNCH(h, fs::hvp_cg_dir(B, m1, rrn_d, rr_d, zz_d, tol2, res, p, s));
-            FS_CUDA(h, cudaMemcpyAsync(rr_d, rrn_d, (size_t)B * 8, cudaMemcpyDeviceToDevice, s));
-            FS_CUDA(h, cudaMemcpyAsync(rr.data(), rrn_d, (size_t)B * 8, cudaMemcpyDeviceToHost, s));
+        // The host reads the stopping test back after every k steps: k = 1 for the
+        // first 16 steps, then up to 8 as the count grows, so at most an eighth
+        // more steps run than needed.  A problem that has converged keeps its
+        // iterates (the step kernels skip it), so the extra steps change nothing.
+        int enqueued = 0;
+        while (enqueued < max_cg_iters && any_running()) {
+            const int k = std::min(max_cg_iters - enqueued, std::max(1, std::min(8, enqueued / 8)));
+            for (int q = 0; q < k; ++q) {
+                s2 = apply1(p, true, tn);  // P p
+                if (s2 != FS_OK) return s2;
+                FS_LAUNCH(h, fs::hvp_vec(n, tn, r, 1.f, nullptr, 0.f, true, tn, s));  // / r
+                s2 = apply1(tn, false, tm);  // P^T (P p / r)
+                if (s2 != FS_OK) return s2;
+                FS_LAUNCH(h, fs::hvp_vec(m, p, c, 1.f, tm, -1.f, false, Ap, s));  // c o p - ...
+                FS_LAUNCH(h, fs::hvp_dot(B, m1, Ap, nullptr, part, sum_d, s));
+                FS_LAUNCH(h, fs::hvp_center(B, m1, sum_d, Ap, s));
+                FS_LAUNCH(h, fs::hvp_dot(B, m1, p, Ap, part, pap_d, s));
+                FS_LAUNCH(h, fs::hvp_cg_step(B, m1, rr_d, pap_d, zz_d, tol2, p, Ap, x, res, steps_d, s));
+                FS_LAUNCH(h, fs::hvp_dot(B, m1, res, res, part, rrn_d, s));
+                FS_LAUNCH(h, fs::hvp_cg_dir(B, m1, rrn_d, rr_d, zz_d, tol2, res, p, s));
+                FS_CUDA(h, cudaMemcpyAsync(rr_d, rrn_d, (size_t)B * 8, cudaMemcpyDeviceToDevice, s));
+            }
+            enqueued += k;
+            FS_CUDA(h, cudaMemcpyAsync(rr.data(), rr_d, (size_t)B * 8, cudaMemcpyDeviceToHost, s));
             FS_CUDA(h, cudaStreamSynchronize(s));
-            ++it;
+        }
+        {  // the most steps any problem took
+            std::vector<int> steps((size_t)B);
+            FS_CUDA(h, cudaMemcpyAsync(steps.data(), steps_d, (size_t)B * 4, cudaMemcpyDeviceToHost, s));
+            FS_CUDA(h, cudaStreamSynchronize(s));
+            for (int b = 0; b < B; ++b) it = std::max(it, steps[b]);
         }
         // Q1 = P [dg o Y | dg] in one application; df = (u - P dg) / r
         FS_LAUNCH(h, fs::hvp_dgy(Yop, ybf, x, (int)m, (int)d, dgY, s));

@@ -129,11 +129,13 @@ __device__ __forceinline__ bool cg_active(const double *rr, const double *zz, do
 }
 
 // CG update on the device, from device scalars rr (r.r) and pap (p.Ap):
-//   alpha = rr / pap;  x += alpha p;  res -= alpha Ap   (problems still running)
+//   alpha = rr / pap;  x += alpha p;  res -= alpha Ap   (problems still running,
+// each of which counts the step in steps[b])
 __global__ void cg_step_kernel(size_t len, const double *rr, const double *pap, const double *zz, double tol2,
-                               const float *p, const float *Ap, float *x, float *res) {
+                               const float *p, const float *Ap, float *x, float *res, int *steps) {
     const int b = blockIdx.y;
     if (!cg_active(rr, zz, tol2, b)) return;
+    if (blockIdx.x == 0 && threadIdx.x == 0) steps[b] += 1;
     const size_t base = (size_t)b * len;
     const float alpha = (float)(rr[b] / pap[b]);
     SEG_LOOP(i, len) {
@@ -246,8 +248,8 @@ cudaError_t hvp_center(int batch, size_t len, const double *sum, float *x, cudaS
     return cudaGetLastError();
 }
 cudaError_t hvp_cg_step(int batch, size_t len, const double *rr, const double *pap, const double *zz, double tol2,
-                        const float *p, const float *Ap, float *x, float *res, cudaStream_t s) {
-    cg_step_kernel<<<dim3(blocks_for(len), batch), 256, 0, s>>>(len, rr, pap, zz, tol2, p, Ap, x, res);
+                        const float *p, const float *Ap, float *x, float *res, int *steps, cudaStream_t s) {
+    cg_step_kernel<<<dim3(blocks_for(len), batch), 256, 0, s>>>(len, rr, pap, zz, tol2, p, Ap, x, res, steps);
     return cudaGetLastError();
 }
 cudaError_t hvp_cg_dir(int batch, size_t len, const double *rr_new, const double *rr, const double *zz, double tol2,

@@ -257,8 +257,9 @@ cudaError_t hvp_vec(size_t n, const float *x, const float *a, float alpha, const
 cudaError_t hvp_dot(int batch, size_t len, const float *x, const float *y, double *part, double *out,
                     cudaStream_t s);
 cudaError_t hvp_center(int batch, size_t len, const double *sum, float *x, cudaStream_t s);
+// steps[b] += 1 for each problem still running (its CG step count)
 cudaError_t hvp_cg_step(int batch, size_t len, const double *rr, const double *pap, const double *zz, double tol2,
-                        const float *p, const float *Ap, float *x, float *res, cudaStream_t s);
+                        const float *p, const float *Ap, float *x, float *res, int *steps, cudaStream_t s);
 cudaError_t hvp_cg_dir(int batch, size_t len, const double *rr_new, const double *rr, const double *zz, double tol2,
                        const float *res, float *p, cudaStream_t s);
 cudaError_t hvp_dgy(const void *Y, bool bf16, const float *dg, int m, int d, float *out, cudaStream_t s);
