@@ -68,6 +68,42 @@ def test_single_update_parity(cuda_device, name, prec):
         assert max(ef, eg) <= tol[k] / 4, (name, prec, k, ef, eg, tol[k])
 
 
+@pytest.mark.parametrize("name", ["tiny", "middim", "cloud3d", "batched"])
+def test_single_update_tf32_within_its_rounding_bound(cuda_device, name):
+    """One-pass TF32 (operands rounded to 10 mantissa bits, the column bias added
+    inside the S product in tf32 parts) is not fp32-accurate; it must stay within
+    what its operand rounding allows.  With q = x - t and k = 2(y - t) each
+    rounded to relative 2^-11, |S~_ij - S_ij| <= 2^-10 |q_i| |k_j| (Cauchy-
+    Schwarz), and the LSE moves by at most the largest change of its arguments,
+    so |f~_i - f_i| <= 2^-10 |q_i| max_j |k_j| (and symmetrically for g), plus the
+    fp32 bar of the accurate modes."""
+    import torch
+    fs = _fs()
+    prob = make_problem(name, **SMALL[name])
+    X, Y, a, b = device_inputs(prob)
+    h = fs.fs_create(X, Y, a, b, eps=prob.eps, prec="tf32")
+    rng = np.random.default_rng(78)
+    g_in = np.stack([smooth_potential(rng, prob.m, 0.5) for _ in range(prob.batch)])
+    f_in = np.stack([smooth_potential(rng, prob.n, 0.5) for _ in range(prob.batch)])
+    f = torch.empty(prob.batch, prob.n, device=cuda_device)
+    g = torch.empty(prob.batch, prob.m, device=cuda_device)
+    fs.fs_update_f(h, torch.from_numpy(g_in).to(cuda_device), f)
+    fs.fs_update_g(h, torch.from_numpy(f_in).to(cuda_device), g)
+    fs.fs_sync(h)
+    f, g = f.cpu().numpy(), g.cpu().numpy()
+    bar = 1e-4 * max_cost(prob) / 4
+    for k, (Xo, Yo, loga, logb) in enumerate(oracle_arrays(prob)):
+        t = 0.5 * (Xo.mean(axis=0) + Yo.mean(axis=0))
+        qn = np.linalg.norm(Xo - t, axis=1)
+        kn = 2 * np.linalg.norm(Yo - t, axis=1)
+        fo = oracle.update_f(Xo, Yo, logb, g_in[k].astype(np.float64), prob.eps)
+        go = oracle.update_g(Xo, Yo, loga, f_in[k].astype(np.float64), prob.eps)
+        ef = np.abs(f[k] - fo) / (2.0 ** -10 * qn * kn.max() + bar[k])
+        eg = np.abs(g[k] - go) / (2.0 ** -10 * kn * qn.max() + bar[k])
+        print(f"tf32 {name}[{k}] worst err / bound: f {ef.max():.3f}, g {eg.max():.3f}")
+        assert ef.max() <= 1.0 and eg.max() <= 1.0, (name, k, ef.max(), eg.max())
+
+
 def test_unsupported_row_width_is_reported(cuda_device):
     """3xTF32 rows of d = 65 (640 bytes) exceed the 512-byte operand rows of the tensor-core pass."""
     import torch
