@@ -356,7 +356,12 @@ fs_status tail_matches(fs_handle *h, const float *f, const float *g, bool *same)
     return FS_OK;
 }
 }  // namespace
-void fs::count_launches(unsigned count) { g_launches.fetch_add(count, std::memory_order_relaxed); }
+void fs::count_launches(unsigned count) {
+    if (t_capturing)
+        t_captured += (int)count;
+    else
+        g_launches.fetch_add(count, std::memory_order_relaxed);
+}
 
 namespace {
 // fdir: out_i = sum_j P_ij V_j over the X side's rows (V indexed by Y's points);
@@ -532,11 +537,11 @@ fs_status apply(fs_handle *h, const float *f, const float *g, const void *V, boo
 // as much as one of 128).  vpad: scratch of batch x (the column side's stride)
 // floats.  r (may be null) receives the row sums.  Tensor-core handles only.
 fs_status apply_vec(fs_handle *h, const float *f, const float *g, const float *v, bool fdir, float *out, float *r,
-                    float *vpad) {
+                    float *vpad, bool bias_ready = false) {
     const fs_desc &D = h->desc;
     fs::PassParams p = make_pass(h, fdir, true);
     FS_LAUNCH(h, fs::launch_pad_vec(v, D.batch, p.cols, p.cols_stride, vpad, h->stream));
-    FS_LAUNCH(h, run_bias(h, fdir ? g : f, fdir));
+    if (!bias_ready) FS_LAUNCH(h, run_bias(h, fdir ? g : f, fdir));
     p.pot_in = fdir ? f : g;
     p.col_vec = vpad;
     p.vec_out = out;
@@ -588,19 +593,24 @@ fs_status enqueue_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule
 // Capture enqueue_solve into h->gexec on the handle's private stream.  Returns
 // false (with no error left pending and the stream usable) if the capture or
 // the instantiation fails; the caller then launches directly.
+// The handle's stream for graph captures (and its two events), created once.
+bool ensure_graph_stream(fs_handle *h) {
+    if (h->gstream) return true;
+    if (cudaStreamCreateWithFlags(&h->gstream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->gev_in, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h->gev_out, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
 bool capture_solve(fs_handle *h, float *f, float *g, int iters, fs_schedule schedule) {
     if (h->gexec) {
         cudaGraphExecDestroy(h->gexec);
         h->gexec = nullptr;
     }
-    if (!h->gstream) {
-        if (cudaStreamCreateWithFlags(&h->gstream, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&h->gev_in, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&h->gev_out, cudaEventDisableTiming) != cudaSuccess) {
-            cudaGetLastError();
-            return false;
-        }
-    }
+    if (!ensure_graph_stream(h)) return false;
     if (cudaStreamBeginCapture(h->gstream, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
         cudaGetLastError();
         return false;
@@ -896,8 +906,9 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
     // handles; the CUDA-core validation path keeps the transport kernels
     const char *env_simt0 = getenv("FS_APPLY_SIMT");
     const bool use_vec = h->prec != FS_PREC_F32_SIMT && !(env_simt0 && atoi(env_simt0) != 0);
+    // (inside the CG both directions' biases are already in place: f and g do not change)
     auto apply1 = [&](const float *vin, bool fdir, float *vout) -> fs_status {
-        if (use_vec) return apply_vec(h, f, g, vin, fdir, vout, nullptr, vpad);
+        if (use_vec) return apply_vec(h, f, g, vin, fdir, vout, nullptr, vpad, true);
         return apply(h, f, g, vin, false, 1, vout, nullptr, false, fdir);
     };
     // the column cloud the transport products see (Y, or its unit rows), and the
@@ -942,32 +953,93 @@ fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, 
                 if (rr[b] > tol2 * zz[b] && zz[b] > 0.0) return true;
             return false;
         };
+        if (use_vec) {  // the biases of both directions, once for the whole CG
+            FS_LAUNCH(h, run_bias(h, g, true));
+            FS_LAUNCH(h, run_bias(h, f, false));
+        }
+        // k CG steps on h->stream (the stream the lambdas see)
+        auto enqueue_steps = [&](int k) -> fs_status {
+            const cudaStream_t st = h->stream;
+            for (int q = 0; q < k; ++q) {
+                fs_status s3 = apply1(p, true, tn);  // P p
+                if (s3 != FS_OK) return s3;
+                FS_LAUNCH(h, fs::hvp_vec(n, tn, r, 1.f, nullptr, 0.f, true, tn, st));  // / r
+                s3 = apply1(tn, false, tm);  // P^T (P p / r)
+                if (s3 != FS_OK) return s3;
+                FS_LAUNCH(h, fs::hvp_vec(m, p, c, 1.f, tm, -1.f, false, Ap, st));  // c o p - ...
+                FS_LAUNCH(h, fs::hvp_dot(B, m1, Ap, nullptr, part, sum_d, st));
+                FS_LAUNCH(h, fs::hvp_center(B, m1, sum_d, Ap, st));
+                FS_LAUNCH(h, fs::hvp_dot(B, m1, p, Ap, part, pap_d, st));
+                FS_LAUNCH(h, fs::hvp_cg_step(B, m1, rr_d, pap_d, zz_d, tol2, p, Ap, x, res, steps_d, st));
+                FS_LAUNCH(h, fs::hvp_dot(B, m1, res, res, part, rrn_d, st));
+                FS_LAUNCH(h, fs::hvp_cg_dir(B, m1, rrn_d, rr_d, zz_d, tol2, res, p, st));
+                FS_CUDA(h, cudaMemcpyAsync(rr_d, rrn_d, (size_t)B * 8, cudaMemcpyDeviceToDevice, st));
+            }
+            return FS_OK;
+        };
+        // Blocks of kCgBlock steps replay one CUDA graph, captured at the first
+        // such block on the handle's graph stream (its buffers are this call's);
+        // if the capture fails they are launched directly.
+        constexpr int kCgBlock = 8;
+        cudaGraphExec_t cg_exec = nullptr;
+        int cg_kernels = 0;
+        bool cg_tried = false;
+        auto capture_block = [&]() -> bool {
+            cg_tried = true;
+            if (!ensure_graph_stream(h)) return false;
+            if (cudaStreamBeginCapture(h->gstream, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+                cudaGetLastError();
+                return false;
+            }
+            const cudaStream_t user = h->stream;
+            const std::string saved_error = h->last_error;
+            h->stream = h->gstream;
+            t_capturing = true;
+            t_captured = 0;
+            const fs_status s3 = enqueue_steps(kCgBlock);
+            t_capturing = false;
+            h->stream = user;
+            h->last_error = saved_error;
+            cudaGraph_t graph = nullptr;
+            const cudaError_t ec = cudaStreamEndCapture(h->gstream, &graph);
+            const bool good = s3 == FS_OK && ec == cudaSuccess && graph != nullptr &&
+                              cudaGraphInstantiate(&cg_exec, graph, 0) == cudaSuccess;
+            if (graph) cudaGraphDestroy(graph);
+            if (!good) {
+                cudaGetLastError();
+                cg_exec = nullptr;
+                return false;
+            }
+            cg_kernels = t_captured;
+            return true;
+        };
         // The host reads the stopping test back after every k steps: k = 1 for the
         // first 16 steps, then up to 8 as the count grows, so at most an eighth
         // more steps run than needed.  A problem that has converged keeps its
         // iterates (the step kernels skip it), so the extra steps change nothing.
         int enqueued = 0;
+        fs_status cg_st = FS_OK;
         while (enqueued < max_cg_iters && any_running()) {
-            const int k = std::min(max_cg_iters - enqueued, std::max(1, std::min(8, enqueued / 8)));
-            for (int q = 0; q < k; ++q) {
-                s2 = apply1(p, true, tn);  // P p
-                if (s2 != FS_OK) return s2;
-                FS_LAUNCH(h, fs::hvp_vec(n, tn, r, 1.f, nullptr, 0.f, true, tn, s));  // / r
-                s2 = apply1(tn, false, tm);  // P^T (P p / r)
-                if (s2 != FS_OK) return s2;
-                FS_LAUNCH(h, fs::hvp_vec(m, p, c, 1.f, tm, -1.f, false, Ap, s));  // c o p - ...
-                FS_LAUNCH(h, fs::hvp_dot(B, m1, Ap, nullptr, part, sum_d, s));
-                FS_LAUNCH(h, fs::hvp_center(B, m1, sum_d, Ap, s));
-                FS_LAUNCH(h, fs::hvp_dot(B, m1, p, Ap, part, pap_d, s));
-                FS_LAUNCH(h, fs::hvp_cg_step(B, m1, rr_d, pap_d, zz_d, tol2, p, Ap, x, res, steps_d, s));
-                FS_LAUNCH(h, fs::hvp_dot(B, m1, res, res, part, rrn_d, s));
-                FS_LAUNCH(h, fs::hvp_cg_dir(B, m1, rrn_d, rr_d, zz_d, tol2, res, p, s));
-                FS_CUDA(h, cudaMemcpyAsync(rr_d, rrn_d, (size_t)B * 8, cudaMemcpyDeviceToDevice, s));
+            const int k = std::min(max_cg_iters - enqueued, std::max(1, std::min(kCgBlock, enqueued / 8)));
+            if (k == kCgBlock && (cg_exec || (!cg_tried && capture_block()))) {
+                if (cudaGraphLaunch(cg_exec, s) != cudaSuccess) {
+                    cg_st = fail(h, FS_ERR_CUDA, "CUDA graph launch of the CG steps failed");
+                    break;
+                }
+                g_launches.fetch_add((unsigned long long)cg_kernels, std::memory_order_relaxed);
+            } else {
+                cg_st = enqueue_steps(k);
+                if (cg_st != FS_OK) break;
             }
             enqueued += k;
-            FS_CUDA(h, cudaMemcpyAsync(rr.data(), rr_d, (size_t)B * 8, cudaMemcpyDeviceToHost, s));
-            FS_CUDA(h, cudaStreamSynchronize(s));
+            if (cudaMemcpyAsync(rr.data(), rr_d, (size_t)B * 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+                cudaStreamSynchronize(s) != cudaSuccess) {
+                cg_st = fail(h, FS_ERR_CUDA, "CG stopping test: %s", cudaGetErrorString(cudaGetLastError()));
+                break;
+            }
         }
+        if (cg_exec) cudaGraphExecDestroy(cg_exec);
+        if (cg_st != FS_OK) return cg_st;
         {  // the most steps any problem took
             std::vector<int> steps((size_t)B);
             FS_CUDA(h, cudaMemcpyAsync(steps.data(), steps_d, (size_t)B * 4, cudaMemcpyDeviceToHost, s));
