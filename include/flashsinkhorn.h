@@ -317,8 +317,12 @@ FS_API fs_status fs_grad_y(fs_handle *h, const float *f, const float *g, const v
  * (its change of C is -y^_j.v~_i), with the second derivative of the cosine
  * distance in the final combination; its transport-matrix term is always the
  * column-block form (fs_get_info's last_hvp_fused = 0).  X, Y: the caller's
- * device clouds in the handle's dtype.  Synchronises the stream once per CG
- * step.  Errors: FS_ERR_INVALID_ARG, FS_ERR_UNSUPPORTED (batch > 65535).
+ * device clouds in the handle's dtype.  The host reads the stopping test
+ * back after every k steps (k = 1 for the first 16, then up to 8; the steps a
+ * converged problem sits through leave its iterates unchanged), synchronising
+ * the stream each time; blocks of 8 steps replay one CUDA graph captured on the
+ * handle's graph stream.  Errors: FS_ERR_INVALID_ARG, FS_ERR_UNSUPPORTED
+ * (batch > 65535).
  */
 FS_API fs_status fs_hvp_x(fs_handle *h, const float *f, const float *g, const void *X, const void *Y,
                           const float *V, float *out, int max_cg_iters, double cg_rtol, int *cg_iters_done);
