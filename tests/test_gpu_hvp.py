@@ -73,7 +73,7 @@ def _check_row_bound(path, name, its, H, Xo, Yo, loga, logb, f32, g32, eps, V):
     assert np.all(rowerr <= bound), (rowerr / bound).max()
 
 
-def _run_hvp(cuda_device, prob, cases, V, path, cost="sqeuclidean"):
+def _run_hvp(cuda_device, prob, cases, V, path, cost="sqeuclidean", max_cg_iters=500, cg_rtol=1e-7):
     import torch
     import log_domain_sinkhorn_updates_b200 as fs
     from helpers import device_inputs
@@ -83,7 +83,7 @@ def _run_hvp(cuda_device, prob, cases, V, path, cost="sqeuclidean"):
     h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps, cost=cost)
     out = torch.empty(prob.batch, prob.n, prob.d, device=cuda_device)
     its = fs.fs_hvp_x(h, torch.from_numpy(f_all).to(cuda_device), torch.from_numpy(g_all).to(cuda_device),
-                      X, Y, torch.from_numpy(V).to(cuda_device), out, max_cg_iters=500, cg_rtol=1e-7)
+                      X, Y, torch.from_numpy(V).to(cuda_device), out, max_cg_iters=max_cg_iters, cg_rtol=cg_rtol)
     fs.fs_sync(h)
     info = fs.fs_get_info(h)
     fs.fs_destroy(h)
@@ -121,6 +121,23 @@ def test_hvp_x_batched_parity(cuda_device, name, path, monkeypatch):
     assert 1 <= its <= 500
     for k, case in enumerate(cases):
         _check_row_bound(path, f"{name}[{k}]", its, H[k], *case[:4], case[4], case[5], prob.eps, V[k])
+
+
+@pytest.mark.parametrize("path", ["tc", "simt"])
+def test_hvp_x_long_cg_in_graph_blocks(cuda_device, path, monkeypatch):
+    """A CG held to a residual fp32 cannot reach (1e-12) runs to its step limit:
+    past the first 64 steps it goes in blocks of 8 that replay one captured CUDA
+    graph.  The result must stay within the same bound, and the call must report
+    the limit as its step count."""
+    monkeypatch.setenv("FS_APPLY_SIMT", PATHS[path][0])
+    monkeypatch.setenv("FS_HVP_FUSED", PATHS[path][1])
+    prob = make_problem("middim", n=260, m=240, d=16)
+    case = _oracle_case(prob, 0)
+    rng = np.random.default_rng(202)
+    V = rng.standard_normal((1, prob.n, prob.d)).astype(np.float32)
+    H, its = _run_hvp(cuda_device, prob, [case], V, path, max_cg_iters=96, cg_rtol=1e-12)
+    assert its == 96, its
+    _check_row_bound(path, "middim long CG", its, H[0], *case[:4], case[4], case[5], prob.eps, V[0])
 
 
 COSINE = {
