@@ -180,3 +180,53 @@ def test_full_size_transport_sampled(cuda_device, name):
     err = (np.abs(T[rows] - To) / (2 * rel[:, None] * absw / r[:, None] + 1e-6 * np.abs(To))).max()
     print(f"{name} full-size barycentric map, sampled rows: worst err / bound = {err:.3f}")
     assert err <= 1.0
+
+
+@pytest.mark.parametrize("name", ["highdim", "middim", "cloud3d"])
+def test_full_size_one_column_sampled(cuda_device, name):
+    """A one-column transport application on the full workload: the streamed LSE
+    pass that weights column j by v_j (the form the HVP's conjugate gradient
+    runs, with the bias inside the S product), checked at sampled rows that the
+    oracle computes one by one.  Potentials as in the barycentric-map test; the
+    bound is the transport bound without the bf16 split term (fp32 sums, no P~
+    split), as at small sizes."""
+    import torch
+    fs = _fs()
+    prob = make_problem(name)
+    X, Y, a_d, b_d = device_inputs(prob)
+    h = fs.fs_create(X, Y, a_d, b_d, eps=prob.eps)
+    rng = np.random.default_rng(778)
+    g_in = smooth_potential(rng, prob.m, 0.05)[None]
+    if name == "highdim":
+        f_in = smooth_potential(rng, prob.n, 0.05)[None]
+    else:
+        Xo, Yo, _, logb = oracle.problem_arrays(prob, 0)
+        f_in = oracle.update_f(Xo, Yo, logb, g_in[0].astype(np.float64), prob.eps).astype(np.float32)[None]
+    v = rng.standard_normal((1, prob.m, 1)).astype(np.float32)
+    fd, gd, vd = (torch.from_numpy(x).to(cuda_device) for x in (f_in, g_in, v))
+    out = torch.empty(1, prob.n, 1, device=cuda_device)
+    r = torch.empty(1, prob.n, device=cuda_device)
+    fs.fs_transport_apply(h, fd, gd, vd, out, r)
+    fs.fs_sync(h)
+    assert fs.fs_get_info(h)["last_apply_path"] == "lse_vec"
+    out, r = out.cpu().numpy()[0, :, 0], r.cpu().numpy()[0]
+    Xo, Yo, loga, logb = oracle.problem_arrays(prob, 0)
+    rows = np.unique(np.concatenate([[0, prob.n - 1], rng.choice(prob.n, 64, replace=False)]))
+    fk, gk = f_in[0].astype(np.float64), g_in[0].astype(np.float64)
+    oo, ro = oracle.transport_apply(Xo[rows], Yo, loga[rows], logb, fk[rows], gk, prob.eps, v[0].astype(np.float64))
+    absw, _ = oracle.transport_apply(Xo[rows], Yo, loga[rows], logb, fk[rows], gk, prob.eps,
+                                     np.abs(v[0]).astype(np.float64))
+    xs_t = 0.5 * (Xo.mean(0) + Yo.mean(0))
+    xs, ys = Xo[rows] - xs_t, Yo - xs_t
+    LOG2E = 1.0 / np.log(2.0)
+    alpha = loga[rows] * LOG2E + (fk[rows] - (xs ** 2).sum(1)) * LOG2E / prob.eps
+    beta = logb * LOG2E + (gk - (ys ** 2).sum(1)) * LOG2E / prob.eps
+    M = np.abs(alpha) + np.abs(beta).max() + (2 * prob.d + 2) * 2 * np.sqrt((xs ** 2).sum(1)) * \
+        np.sqrt((ys ** 2).sum(1)).max() * LOG2E / prob.eps
+    rel = np.log(2.0) * 2.0 ** -23 * M + 2.0 ** -21 + prob.m * 2.0 ** -24
+    err = (np.abs(out[rows] - oo[:, 0]) / (rel * absw[:, 0])).max()
+    rerr = (np.abs(r[rows] - ro) / (rel * ro)).max()
+    print(f"{name} full-size one-column application, sampled rows: worst err / bound = {err:.3f}, "
+          f"row sums {rerr:.3f}")
+    assert err <= 1.0 and rerr <= 1.0
+
